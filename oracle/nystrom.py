@@ -1,0 +1,251 @@
+"""Plain fp64 CPU oracle of the Nystromformer attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or run
+this module: only the tests, the smoke check and the CPU-baseline leg of the
+benchmark do.  It shares no code with the CUDA kernels.
+
+Every step is written in the order and notation of the pages it follows, one
+(b, h) attention head at a time, with numpy fp64 arrays and numpy's matmul as
+the only library primitive.  There is no blocking, fusion or reordering beyond
+what the definitions state.
+
+Sources (page title, then section / equation):
+  [P1] "Approximating self-attention in linear time and memory via the Nystrom
+       method" (blog post): "How can we adapt the Nystrom method to approximate
+       self-attention?" (the three softmax matrices F~, A~, B~),
+       "How do we select landmarks?" (segment means, DConv skip),
+       "How is Nystromformer implemented?" (library excerpt: landmarks by
+       reshape + mean, kernel_1/2/3, product order).
+  [P5] "Nystromformer: A Nystrom-Based Algorithm for Approximating
+       Self-Attention" (paper summary), section 3.4:
+       "Moore-Penrose Pseudoinverse Computation" (Lemma 1, Z0 initialisation),
+       "Landmark Selection: Segment-Means" (Eq. 16 and its normalisation note),
+       "Putting It Together" (Eq. 17, Algorithm 1, Figure 4 with the DConv skip),
+       "Theoretical Analysis" (Lemma 2), and section 3.2 (the five stages).
+
+Readings where the pages are silent or inconsistent (each also listed in the
+design notes):
+  * Eq. 16 prints a divide-by-m; the page itself calls that a typo.  Landmark j
+    is the mean of the l = n/m contiguous tokens [j*l, (j+1)*l).
+  * The 1/sqrt(d) scale is applied inside all three softmaxes (P1 definitions,
+    P5 Algorithm 1); the library excerpt omits it for brevity.
+  * B~ is a softmax over the n keys for every landmark row (P1 definitions,
+    library excerpt softmax over the last axis).
+  * The DConv skip is a depthwise 1-D cross-correlation along the sequence with
+    one odd-length kernel w[h, :] per head, shared by the d features of that
+    head, zero "same" padding, no bias.
+  * The output uses Z after `iters` iterations, never the exact pseudoinverse.
+  * Product order F~ (Z (B~ V)); equal in exact arithmetic to the pages' other
+    orders.
+
+Parity is pinned (see tests/test_oracle_pins.py) by: brute-force loops on tiny
+inputs, the mean-of-landmarks invariant, softmax row sums, the SVD
+pseudoinverse (numpy/LAPACK) at convergence, the closed-form one-step residual
+of Lemma 1's recurrence, the exact fixed point for a uniform kernel, Lemma 2
+(m = n) and the exactness on segment-constant Q/K against brute-force n x n
+softmax attention, and numpy.correlate for the convolution.
+"""
+
+import numpy as np
+
+__all__ = [
+    "segment_means",
+    "softmax_rows",
+    "kernel_F",
+    "kernel_A",
+    "kernel_B",
+    "pinv_init",
+    "pinv_step",
+    "iterative_pinv",
+    "depthwise_conv",
+    "nystrom_head",
+    "nystrom_forward",
+    "exact_attention_head",
+    "exact_attention",
+    "algorithmic_flops",
+    "algorithmic_bytes",
+]
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def segment_means(X, m):
+    """Landmarks by segment means ([P5] "Landmark Selection: Segment-Means",
+    Eq. 16 with the page's own 1/l correction; [P1] "How do we select
+    landmarks?").
+
+    X: [n, d].  Returns [m, d]: row j is the mean of rows j*l .. j*l + l - 1,
+    l = n / m.  n must be a multiple of m (the pages assume this, "can be
+    ensured by padding")."""
+    X = _f64(X)
+    n, d = X.shape
+    if m < 1 or n % m != 0:
+        raise ValueError("segment_means needs m >= 1 dividing n (n=%d, m=%d)" % (n, m))
+    seg = n // m
+    out = np.empty((m, d), dtype=np.float64)
+    for j in range(m):
+        out[j] = X[j * seg:(j + 1) * seg].sum(axis=0) / seg
+    return out
+
+
+def softmax_rows(S):
+    """Row-wise softmax.  The row maximum is subtracted first; that changes
+    nothing mathematically and keeps exp() finite for peaky logits."""
+    S = _f64(S)
+    E = np.exp(S - S.max(axis=1, keepdims=True))
+    return E / E.sum(axis=1, keepdims=True)
+
+
+def kernel_F(Q, Kt, scale):
+    """F~ = softmax(Q K~^T / sqrt(d)), n x m, softmax over the m landmarks
+    ([P1] definitions of F~; [P5] Algorithm 1)."""
+    return softmax_rows(_f64(Q) @ _f64(Kt).T * scale)
+
+
+def kernel_A(Qt, Kt, scale):
+    """softmax(Q~ K~^T / sqrt(d)), m x m, row-wise ([P1] definitions; [P5]
+    section 3.2 stage 2a).  Its pseudoinverse is taken by iterative_pinv."""
+    return softmax_rows(_f64(Qt) @ _f64(Kt).T * scale)
+
+
+def kernel_B(Qt, K, scale):
+    """B~ = softmax(Q~ K^T / sqrt(d)), m x n, softmax over the n keys of every
+    landmark row ([P1] definitions; [P5] Algorithm 1)."""
+    return softmax_rows(_f64(Qt) @ _f64(K).T * scale)
+
+
+def pinv_init(A):
+    """Z0 = A^T / (||A||_1 ||A||_inf) ([P5] "Moore-Penrose Pseudoinverse
+    Computation", initialisation scheme).  ||A||_1 is the largest absolute
+    column sum, ||A||_inf the largest absolute row sum."""
+    A = _f64(A)
+    norm_1 = np.abs(A).sum(axis=0).max()
+    norm_inf = np.abs(A).sum(axis=1).max()
+    return A.T / (norm_1 * norm_inf)
+
+
+def pinv_step(A, Z):
+    """One step of Lemma 1 ([P5] "Moore-Penrose Pseudoinverse Computation"):
+    Z <- 1/4 Z (13 I - A Z (15 I - A Z (7 I - A Z)))."""
+    A = _f64(A)
+    Z = _f64(Z)
+    I = np.eye(A.shape[0])
+    AZ = A @ Z
+    return 0.25 * (Z @ (13.0 * I - AZ @ (15.0 * I - AZ @ (7.0 * I - AZ))))
+
+
+def iterative_pinv(A, iters, return_all=False):
+    """Z after `iters` steps of Lemma 1 from Z0 ([P5] section 3.2 stage 3: six
+    iterations in the paper's runs).  With return_all, the list Z0..Z_iters."""
+    Z = pinv_init(A)
+    allz = [Z]
+    for _ in range(iters):
+        Z = pinv_step(A, Z)
+        allz.append(Z)
+    return allz if return_all else Z
+
+
+def depthwise_conv(V, w):
+    """DConv skip on the values ([P1] "How do we select landmarks?" DConv box;
+    [P5] Figure 4 "DConv k x 1").  V: [n, d]; w: [k], k odd, shared by the d
+    features.  C[i, c] = sum_t w[t] V[i + t - (k-1)/2, c], V = 0 outside
+    [0, n)."""
+    V = _f64(V)
+    w = _f64(w).reshape(-1)
+    k = w.shape[0]
+    if k % 2 != 1:
+        raise ValueError("conv kernel length must be odd")
+    n, d = V.shape
+    half = (k - 1) // 2
+    C = np.zeros((n, d), dtype=np.float64)
+    for t in range(k):
+        off = t - half                      # source row = i + off
+        lo = max(0, -off)
+        hi = min(n, n - off)
+        if hi > lo:
+            C[lo:hi] += w[t] * V[lo + off:hi + off]
+    return C
+
+
+def nystrom_head(Q, K, V, m, iters=6, w=None, scale=None):
+    """One attention head of the Nystrom forward pass ([P5] Eq. 17 / Algorithm
+    1 with the Figure 4 skip).  Returns a dict of every intermediate:
+    Qt, Kt (landmarks), F (n x m), A (m x m), Z (after `iters` steps),
+    B (m x n), Y = B V, W = Z Y, O = F W, C (conv skip or zeros), out = O + C."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    n, d = Q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    Qt = segment_means(Q, m)
+    Kt = segment_means(K, m)
+    F = kernel_F(Q, Kt, scale)
+    A = kernel_A(Qt, Kt, scale)
+    Z = iterative_pinv(A, iters)
+    B = kernel_B(Qt, K, scale)
+    Y = B @ V
+    W = Z @ Y
+    O = F @ W
+    C = depthwise_conv(V, w) if w is not None else np.zeros_like(V)
+    return {"Qt": Qt, "Kt": Kt, "F": F, "A": A, "Z": Z, "B": B,
+            "Y": Y, "W": W, "O": O, "C": C, "out": O + C}
+
+
+def nystrom_forward(Q, K, V, m, iters=6, conv_w=None, keep=()):
+    """Batched forward over [B, H, n, d] inputs, head by head.  conv_w is
+    [H, k] (one kernel per head) or None for no skip.  Returns out [B, H, n, d]
+    fp64 and, for each name in `keep`, that intermediate stacked to
+    [B, H, ...]."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    Bn, H, n, d = Q.shape
+    out = np.empty((Bn, H, n, d), dtype=np.float64)
+    kept = {name: [] for name in keep}
+    for b in range(Bn):
+        for h in range(H):
+            w = None if conv_w is None else _f64(conv_w)[h]
+            r = nystrom_head(Q[b, h], K[b, h], V[b, h], m, iters, w)
+            out[b, h] = r["out"]
+            for name in keep:
+                kept[name].append(r[name])
+    extra = {name: np.stack(v).reshape((Bn, H) + v[0].shape) for name, v in kept.items()}
+    return (out, extra) if keep else out
+
+
+def exact_attention_head(Q, K, V, scale=None):
+    """Standard softmax attention softmax(Q K^T / sqrt(d)) V ([P5] section 3.4,
+    "Standard Self-Attention"), forming the n x n matrix.  Used for Lemma 2
+    and for the approximation-error report only."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    if scale is None:
+        scale = 1.0 / np.sqrt(Q.shape[1])
+    return softmax_rows(Q @ K.T * scale) @ V
+
+
+def exact_attention(Q, K, V):
+    Q = _f64(Q)
+    Bn, H, n, d = Q.shape
+    out = np.empty((Bn, H, n, V.shape[-1]), dtype=np.float64)
+    for b in range(Bn):
+        for h in range(H):
+            out[b, h] = exact_attention_head(Q[b, h], K[b, h], V[b, h])
+    return out
+
+
+def algorithmic_flops(Bn, H, n, d, m, iters=6):
+    """Dense-contraction flops of one forward: per head 2nmd each for Q K~^T,
+    Q~ K^T, B~ V and F~ W, 2m^2 d each for Q~ K~^T and Z Y, and 8 m^3 per
+    pinv step (four m x m products)."""
+    per_head = 8 * n * m * d + 4 * m * m * d + iters * 8 * m ** 3
+    return Bn * H * per_head
+
+
+def algorithmic_bytes(Bn, H, n, d, elem_bytes):
+    """Q, K, V read once and the output written once."""
+    return 4 * Bn * H * n * d * elem_bytes

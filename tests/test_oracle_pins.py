@@ -1,0 +1,275 @@
+"""Pins of the fp64 oracle to facts outside itself.
+
+Each test checks the oracle against something it does not compute the same
+way: brute-force loops on tiny inputs, invariants the definitions imply,
+numpy/LAPACK routines (SVD pseudoinverse, matrix norms, correlate), closed
+forms derived by hand, Lemma 2 of the paper summary ("Theoretical Analysis")
+and brute-force n x n softmax attention.  A plausible slip anywhere in the
+oracle (a dropped term, a wrong coefficient, a softmax over the wrong axis, a
+transposed operand, dividing a segment sum by m instead of l) fails one of
+them.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import nystrom as orc
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- segment means
+
+def test_segment_means_bruteforce_loops():
+    # Plain Python loops over a tiny input (n=12, m=3, l=4).
+    rng = _rng(1)
+    n, m, d = 12, 3, 2
+    X = rng.standard_normal((n, d))
+    got = orc.segment_means(X, m)
+    seg = n // m
+    for j in range(m):
+        for c in range(d):
+            acc = 0.0
+            for t in range(seg):
+                acc += float(X[j * seg + t, c])
+            assert abs(got[j, c] - acc / seg) < 1e-15
+
+
+def test_segment_means_m_equals_n_is_identity():
+    X = _rng(2).standard_normal((16, 5))
+    assert np.array_equal(orc.segment_means(X, 16), X)
+
+
+def test_segment_means_preserve_global_mean():
+    # mean over landmarks == mean over tokens; with m != l a divide-by-m
+    # (the printed typo of Eq. 16) would scale this by l/m.
+    X = _rng(3).standard_normal((64, 7))
+    for m in (2, 4, 8, 16):
+        L = orc.segment_means(X, m)
+        np.testing.assert_allclose(L.mean(axis=0), X.mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_segment_means_constant_segments():
+    vals = _rng(4).standard_normal((4, 3))
+    X = np.repeat(vals, 5, axis=0)          # n=20, four segments of 5
+    np.testing.assert_allclose(orc.segment_means(X, 4), vals, rtol=0, atol=1e-15)
+
+
+def test_segment_means_rejects_indivisible():
+    with pytest.raises(ValueError):
+        orc.segment_means(np.zeros((10, 2)), 3)
+
+
+# ---------------------------------------------------------------- softmax kernels
+
+def test_softmax_kernels_row_sums_and_axes():
+    rng = _rng(5)
+    n, m, d = 48, 6, 8
+    Q = rng.standard_normal((n, d)) * 3
+    K = rng.standard_normal((n, d)) * 3
+    Qt, Kt = orc.segment_means(Q, m), orc.segment_means(K, m)
+    s = 1 / math.sqrt(d)
+    F = orc.kernel_F(Q, Kt, s)
+    A = orc.kernel_A(Qt, Kt, s)
+    B = orc.kernel_B(Qt, K, s)
+    assert F.shape == (n, m) and A.shape == (m, m) and B.shape == (m, n)
+    for M in (F, A, B):
+        assert np.all(M > 0)
+        np.testing.assert_allclose(M.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    # B is normalised over the n keys: its columns do not sum to one.
+    assert abs(B.sum(axis=0) - 1).max() > 1e-3
+    # entries against the textbook softmax written with exp / sum per entry
+    i, j = 7, 3
+    z = [math.exp(s * float(Q[i] @ Kt[t])) for t in range(m)]
+    assert abs(F[i, j] - z[j] / sum(z)) < 1e-14
+    z = [math.exp(s * float(Qt[j] @ K[t])) for t in range(n)]
+    assert abs(B[j, i] - z[i] / sum(z)) < 1e-14
+
+
+def test_softmax_is_shift_invariant_and_handles_peaky_logits():
+    S = _rng(6).standard_normal((5, 9)) * 400.0      # exp would overflow unshifted
+    P = orc.softmax_rows(S)
+    assert np.all(np.isfinite(P))
+    np.testing.assert_allclose(P, orc.softmax_rows(S + 123.0), rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- pseudoinverse
+
+def test_pinv_init_uses_the_matrix_norms():
+    A = _rng(7).random((6, 6))
+    Z0 = orc.pinv_init(A)
+    c = np.linalg.norm(A, 1) * np.linalg.norm(A, np.inf)   # LAPACK-side norms
+    np.testing.assert_allclose(Z0 * c, A.T, rtol=1e-15, atol=0)
+    # a row-stochastic kernel has ||A||_inf = 1 exactly
+    S = orc.kernel_A(_rng(8).standard_normal((6, 4)), _rng(9).standard_normal((6, 4)), 0.5)
+    assert abs(np.linalg.norm(S, np.inf) - 1.0) < 1e-15
+
+
+def test_pinv_one_step_residual_closed_form():
+    # With E = I - A Z, one step of Lemma 1 gives exactly
+    # I - A Z' = E^3 (3I + E) / 4 (expand x(13 - 15x + 7x^2 - x^3)/4 at
+    # x = 1 - e).  A wrong coefficient or a dropped product breaks it.
+    rng = _rng(10)
+    for m in (3, 8, 17):
+        A = rng.standard_normal((m, m))
+        Z = rng.standard_normal((m, m)) * 0.3
+        I = np.eye(m)
+        E = I - A @ Z
+        E_next = I - A @ orc.pinv_step(A, Z)
+        want = E @ E @ E @ (3 * I + E) / 4
+        np.testing.assert_allclose(E_next, want, rtol=1e-10, atol=1e-10 * np.abs(want).max())
+
+
+def test_pinv_converges_to_svd_pseudoinverse():
+    rng = _rng(11)
+    for m in (4, 8, 16):
+        Qt = rng.standard_normal((m, 8)) * 0.7
+        Kt = rng.standard_normal((m, 8)) * 0.7
+        A = orc.kernel_A(Qt, Kt, 1 / math.sqrt(8))
+        Z = orc.iterative_pinv(A, 40)
+        ref = np.linalg.pinv(A)                # SVD route
+        assert np.abs(Z - ref).max() <= 1e-10 * np.abs(ref).max()
+
+
+def test_pinv_of_singular_kernel_matches_svd():
+    # two identical landmark queries give two identical rows: rank m-1
+    rng = _rng(12)
+    m = 6
+    Qt = rng.standard_normal((m, 4)) * 0.5
+    Qt[3] = Qt[1]
+    Kt = rng.standard_normal((m, 4)) * 0.5
+    A = orc.kernel_A(Qt, Kt, 0.5)
+    assert np.linalg.matrix_rank(A) == m - 1
+    # Z0 ~ A^T keeps Z off the null space in exact arithmetic; rounding noise
+    # there grows by 13/4 per step once converged, so stop soon after.
+    Z = orc.iterative_pinv(A, 13)
+    ref = np.linalg.pinv(A, rcond=1e-12)
+    assert np.abs(Z - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_pinv_uniform_kernel_is_a_fixed_point():
+    # Q~ = 0 makes A = J/m; then Z0 = J/m = A^+ and every step keeps it.
+    for m in (1, 5, 64):
+        A = orc.kernel_A(np.zeros((m, 3)), _rng(13).standard_normal((m, 3)), 1.0)
+        J = np.full((m, m), 1.0 / m)
+        np.testing.assert_allclose(A, J, rtol=0, atol=1e-16)
+        for Z in orc.iterative_pinv(A, 6, return_all=True):
+            np.testing.assert_allclose(Z, J, rtol=0, atol=1e-15)
+
+
+def test_pinv_zero_iterations_is_the_initialisation():
+    A = _rng(14).random((5, 5))
+    np.testing.assert_array_equal(orc.iterative_pinv(A, 0), orc.pinv_init(A))
+
+
+# ---------------------------------------------------------------- conv skip
+
+def test_conv_matches_numpy_correlate():
+    rng = _rng(15)
+    for n, k in ((40, 33), (10, 33), (7, 3), (5, 1)):
+        V = rng.standard_normal((n, 3))
+        w = rng.standard_normal(k)
+        C = orc.depthwise_conv(V, w)
+        for c in range(3):
+            # full cross-correlation, then the centred n samples
+            full = np.correlate(np.pad(V[:, c], (k - 1) // 2), w, mode="valid")
+            np.testing.assert_allclose(C[:, c], full, rtol=0, atol=1e-13)
+
+
+def test_conv_kernel_one_is_a_scale():
+    V = _rng(16).standard_normal((9, 4))
+    np.testing.assert_allclose(orc.depthwise_conv(V, [0.37]), 0.37 * V, rtol=0, atol=1e-16)
+
+
+def test_conv_rejects_even_kernel():
+    with pytest.raises(ValueError):
+        orc.depthwise_conv(np.zeros((4, 2)), [1.0, 2.0])
+
+
+# ---------------------------------------------------------------- whole method
+
+def test_lemma2_m_equals_n_gives_exact_attention():
+    # Lemma 2 ("Theoretical Analysis"): landmarks equal to every token make
+    # the approximation exact once the pseudoinverse has converged.
+    rng = _rng(17)
+    n, d = 16, 8
+    Q = rng.standard_normal((n, d)) * 0.8
+    K = rng.standard_normal((n, d)) * 0.8
+    V = rng.standard_normal((n, d))
+    got = orc.nystrom_head(Q, K, V, m=n, iters=40)["out"]
+    want = orc.exact_attention_head(Q, K, V)
+    assert np.abs(got - want).max() <= 1e-10 * np.abs(want).max()
+
+
+def test_segment_constant_inputs_are_reproduced_exactly():
+    # If Q and K are constant inside every segment, F~ = A rows, B~ = A
+    # columns / l, so F~ A^+ B~ equals the exact softmax matrix for any
+    # m | n (converged pseudoinverse).  Exercises segment means, all three
+    # softmax axes and the product chain with m < n.
+    rng = _rng(18)
+    n, m, d = 24, 4, 8
+    seg = n // m
+    Q = np.repeat(rng.standard_normal((m, d)), seg, axis=0)
+    K = np.repeat(rng.standard_normal((m, d)), seg, axis=0)
+    V = rng.standard_normal((n, d))                    # V is not constant
+    got = orc.nystrom_head(Q, K, V, m=m, iters=40)["out"]
+    want = orc.exact_attention_head(Q, K, V)
+    assert np.abs(got - want).max() <= 1e-10 * np.abs(want).max()
+
+
+def test_zero_queries_average_the_values():
+    # Q = 0: F~ uniform over m, A = J/m (fixed point), B~ uniform over n,
+    # so every output row is the mean of V (plus the conv skip), at any
+    # number of iterations and any m.
+    rng = _rng(19)
+    n, d = 32, 4
+    K = rng.standard_normal((n, d)) * 2
+    V = rng.standard_normal((n, d))
+    w = rng.standard_normal(5)
+    for m in (1, 4, 32):
+        r = orc.nystrom_head(np.zeros((n, d)), K, V, m=m, iters=6, w=w)
+        want = np.tile(V.mean(axis=0), (n, 1)) + orc.depthwise_conv(V, w)
+        np.testing.assert_allclose(r["out"], want, rtol=0, atol=1e-13)
+
+
+def test_single_landmark_closed_form():
+    # m = 1: A = [1], Z = 1 at every step, F~ = 1, and each output row is the
+    # softmax-weighted mean of V with weights exp(s q~ . k_i).
+    rng = _rng(20)
+    n, d = 10, 3
+    Q = rng.standard_normal((n, d))
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d))
+    s = 1 / math.sqrt(d)
+    qbar = [sum(float(Q[i, c]) for i in range(n)) / n for c in range(d)]
+    wts = [math.exp(s * sum(qbar[c] * float(K[i, c]) for c in range(d))) for i in range(n)]
+    tot = sum(wts)
+    row = [sum(wts[i] * float(V[i, c]) for i in range(n)) / tot for c in range(d)]
+    out = orc.nystrom_head(Q, K, V, m=1, iters=6)["out"]
+    np.testing.assert_allclose(out, np.tile(row, (n, 1)), rtol=0, atol=1e-14)
+
+
+def test_linear_in_values_and_heads_independent():
+    rng = _rng(21)
+    Bn, H, n, d, m = 1, 3, 16, 4, 4
+    Q = rng.standard_normal((Bn, H, n, d))
+    K = rng.standard_normal((Bn, H, n, d))
+    V1 = rng.standard_normal((Bn, H, n, d))
+    V2 = rng.standard_normal((Bn, H, n, d))
+    o1 = orc.nystrom_forward(Q, K, V1, m)
+    o2 = orc.nystrom_forward(Q, K, V2, m)
+    o12 = orc.nystrom_forward(Q, K, 2 * V1 - V2, m)
+    np.testing.assert_allclose(o12, 2 * o1 - o2, rtol=0, atol=1e-10 * np.abs(o12).max())
+    perm = [2, 0, 1]
+    op = orc.nystrom_forward(Q[:, perm], K[:, perm], V1[:, perm], m)
+    np.testing.assert_allclose(op, o1[:, perm], rtol=0, atol=1e-15)
+
+
+def test_flop_and_byte_counts():
+    # 8nmd + 4m^2 d + 48 m^3 per head at six iterations; 4 n d e bytes
+    assert orc.algorithmic_flops(1, 1, 8192, 64, 64) == 8 * 8192 * 64 * 64 + 4 * 64 * 64 * 64 + 48 * 64 ** 3
+    assert orc.algorithmic_bytes(2, 12, 8192, 64, 2) == 2 * 12 * 8192 * 64 * 2 * 4
