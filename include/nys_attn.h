@@ -1,0 +1,190 @@
+/*
+ * nys_attn.h -- C ABI of the B200 (sm_100a) Nystromformer attention forward.
+ *
+ * The library computes, for every (batch, head) pair of [B, H, n, d] inputs,
+ *
+ *     out = F~ (Z (B~ V)) + DConv(V)
+ *
+ * where (notation of "Nystromformer: A Nystrom-Based Algorithm for
+ * Approximating Self-Attention", section 3.4, and of the blog post
+ * "Approximating self-attention in linear time and memory via the Nystrom
+ * method"):
+ *   Q~, K~  segment means of Q, K over l = n/m contiguous tokens (Eq. 16,
+ *           with the page's own divide-by-l correction; blog "How do we select
+ *           landmarks?"),
+ *   F~      = softmax(Q K~^T / sqrt(d)), n x m, softmax over the m landmarks,
+ *   A       = softmax(Q~ K~^T / sqrt(d)), m x m, row-wise,
+ *   Z       = pinv_iters steps of Lemma 1 from Z0 = A^T / (||A||_1 ||A||_inf)
+ *             ("Moore-Penrose Pseudoinverse Computation"),
+ *   B~      = softmax(Q~ K^T / sqrt(d)), m x n, softmax over the n keys,
+ *   DConv   depthwise 1-D cross-correlation of V along the sequence with one
+ *           odd-length kernel per head, shared by the d features, zero "same"
+ *           padding (Figure 4 "DConv k x 1"; blog "DConv box"),
+ * and the n x n attention matrix is never formed (Eq. 17 / Algorithm 1).
+ *
+ * Conventions for every entry point:
+ *  - Tensors Q, K, V, out are [batch][heads][seq_len][head_dim], contiguous,
+ *    row-major, all of the dtype in the descriptor; out has the same dtype.
+ *  - Pointers named *_dev are CUDA device pointers; *_host are host pointers.
+ *    The caller owns every buffer; the library keeps no global mutable state
+ *    and never frees caller memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the device.  Arguments are validated on the
+ *    host before anything is enqueued: an invalid call returns a status and
+ *    launches nothing.  Launch failures return NYS_ERR_CUDA.
+ *  - Results are bitwise reproducible run to run (fixed-order reductions, no
+ *    floating-point atomics).
+ *  - batch * heads * seq_len == 0 is valid and enqueues nothing.
+ *
+ * Supported shapes:
+ *  - NYS_F32:  1 <= head_dim <= 64, 1 <= m <= 64, m <= seq_len, m | seq_len.
+ *  - NYS_BF16: head_dim == 64, m in {32, 64, 128}, m <= seq_len, m | seq_len.
+ *  - conv_k odd, 1 <= conv_k <= 63 (or conv_w == NULL / conv_k == 0: no skip).
+ *  - 0 <= pinv_iters <= 64.
+ */
+#ifndef NYS_ATTN_H
+#define NYS_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NYS_ATTN_API __attribute__((visibility("default")))
+
+typedef enum {
+  NYS_OK = 0,
+  NYS_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum value      */
+  NYS_ERR_UNSUPPORTED = 2,   /* valid request without a kernel (d, m, dtype, k)  */
+  NYS_ERR_NOT_DIVISIBLE = 3, /* seq_len is not a multiple of num_landmarks       */
+  NYS_ERR_ALIAS = 4,         /* out overlaps Q, K, V or the workspace            */
+  NYS_ERR_WORKSPACE = 5,     /* workspace smaller than nys_attn_workspace_size   */
+  NYS_ERR_CUDA = 6,          /* a CUDA runtime call or kernel launch failed      */
+  NYS_ERR_TIMEOUT = 7        /* a bounded on-device wait gave up (see below)     */
+} nys_status;
+
+typedef enum { NYS_F32 = 0, NYS_BF16 = 1 } nys_dtype;
+
+/* Shape of the [batch][heads][seq_len][head_dim] inputs. */
+typedef struct {
+  int dtype; /* nys_dtype */
+  int batch;
+  int heads;
+  int seq_len;
+  int head_dim;
+} nys_desc;
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *nys_stream_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+NYS_ATTN_API const char *nys_status_string(nys_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+NYS_ATTN_API int nys_version(void);
+
+/* Bytes of device workspace nys_attn_forward needs for this shape.  Writes
+ * *bytes; returns the same validation status nys_attn_forward would for the
+ * shape part of its arguments. */
+NYS_ATTN_API nys_status nys_attn_workspace_size(const nys_desc *desc, int num_landmarks,
+                                                size_t *bytes);
+
+/* The forward pass (Eq. 17 / Algorithm 1 with the Figure 4 DConv skip of the
+ * paper summary).
+ *   Q_dev, K_dev, V_dev  inputs, layout above.
+ *   num_landmarks        m; seq_len must be a multiple of m (the pages pad to
+ *                        ensure this; padding is not done here).
+ *   pinv_iters           steps of Lemma 1 (the paper uses 6).
+ *   conv_w_dev           [heads][conv_k] fp32 kernel of the DConv skip, or NULL
+ *                        for no skip (then conv_k is ignored).
+ *   out_dev              output, same dtype and layout as Q; must not overlap
+ *                        any input or the workspace.
+ *   workspace_dev        device scratch of at least nys_attn_workspace_size
+ *                        bytes, 256-byte aligned, or NULL: then the call
+ *                        allocates and frees it stream-ordered
+ *                        (cudaMallocAsync / cudaFreeAsync on `stream`).
+ * The workspace holds the per-head intermediates afterwards (see
+ * nys_attn_intermediates) until the next call reuses it.
+ * NYS_ERR_TIMEOUT is reserved for kernels that wait on other blocks of the
+ * same launch; every such wait is bounded and reports through the workspace
+ * error word, read back by nys_attn_check_error. */
+NYS_ATTN_API nys_status nys_attn_forward(const void *Q_dev, const void *K_dev, const void *V_dev,
+                                         const nys_desc *desc, int num_landmarks, int pinv_iters,
+                                         const float *conv_w_dev, int conv_k, void *out_dev,
+                                         void *workspace_dev, size_t workspace_bytes,
+                                         nys_stream_t stream);
+
+/* Offsets (in bytes from the start of the workspace) of the fp32
+ * intermediates a forward leaves there, for parity checks:
+ *   q_landmarks, k_landmarks  [batch*heads][m][head_dim]   Q~, K~
+ *   z                          [batch*heads][m][m]          Z after pinv_iters
+ *   y                          [batch*heads][m][head_dim]   B~ V
+ *   w                          [batch*heads][m][head_dim]   Z (B~ V)
+ *   error_word                 one uint32: 0, or a nys_status a kernel set. */
+typedef struct {
+  size_t q_landmarks;
+  size_t k_landmarks;
+  size_t z;
+  size_t y;
+  size_t w;
+  size_t error_word;
+  size_t total;
+} nys_intermediates;
+
+NYS_ATTN_API nys_status nys_attn_intermediates(const nys_desc *desc, int num_landmarks,
+                                               nys_intermediates *layout);
+
+/* Synchronises `stream`, reads the workspace error word and clears it.
+ * Returns NYS_OK or the status a kernel recorded (e.g. NYS_ERR_TIMEOUT). */
+NYS_ATTN_API nys_status nys_attn_check_error(void *workspace_dev, const nys_desc *desc,
+                                             int num_landmarks, nys_stream_t stream);
+
+/* End-to-end variant on HOST buffers: copies Q, K, V (and conv_w) from host
+ * memory into `device_buf`, runs the forward and copies the output back into
+ * out_host, all enqueued on `stream` (asynchronous: synchronise the stream
+ * before reading out_host; pinned host memory makes the copies truly async).
+ *   Q_host, K_host, V_host  [batch][heads][seq_len][head_dim] of desc->dtype.
+ *   conv_w_host             [heads][conv_k] fp32 or NULL.
+ *   device_buf              device memory of at least
+ *                           nys_attn_host_buffer_size bytes, 256-byte aligned,
+ *                           owned by the caller (staging for the inputs,
+ *                           output, conv weights and the workspace).
+ * Bytes moved per call: 3*T in, T out (+ heads*conv_k*4 in), T = tensor size. */
+NYS_ATTN_API nys_status nys_attn_host_buffer_size(const nys_desc *desc, int num_landmarks,
+                                                  int conv_k, size_t *bytes);
+NYS_ATTN_API nys_status nys_attn_forward_host(const void *Q_host, const void *K_host,
+                                              const void *V_host, const nys_desc *desc,
+                                              int num_landmarks, int pinv_iters,
+                                              const float *conv_w_host, int conv_k,
+                                              void *out_host, void *device_buf,
+                                              size_t device_buf_bytes, nys_stream_t stream);
+
+/* nys_attn_forward with per-kernel CUDA events for live timing: records
+ * events[0] on `stream` before the first kernel and events[i + 1] right after
+ * kernel i, for the nys_attn_launch_count kernels the call enqueues.  events
+ * are caller-created cudaEvent_t handles (timing enabled); n_events must be
+ * at least launches + 1, else NYS_ERR_INVALID_ARG.  Same results as
+ * nys_attn_forward. */
+NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q_dev, const void *K_dev,
+                                               const void *V_dev, const nys_desc *desc,
+                                               int num_landmarks, int pinv_iters,
+                                               const float *conv_w_dev, int conv_k,
+                                               void *out_dev, void *workspace_dev,
+                                               size_t workspace_bytes, nys_stream_t stream,
+                                               void *const *events, int n_events);
+
+/* Number of kernel launches one nys_attn_forward call enqueues for this
+ * shape (0 for an empty problem), and a short name for each launch in
+ * order, written as a comma-separated list into names (may be NULL). */
+NYS_ATTN_API nys_status nys_attn_launch_count(const nys_desc *desc, int num_landmarks,
+                                              int conv_k, int *launches);
+NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int num_landmarks,
+                                              char *names, size_t names_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NYS_ATTN_H */

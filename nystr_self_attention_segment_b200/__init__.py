@@ -1,0 +1,147 @@
+"""B200 (sm_100a) Nystromformer attention forward behind a C ABI.
+
+Python side of the library: argument marshalling from torch tensors to the
+C entry points of include/nys_attn.h (same names).  Every step of the forward
+pass runs in the CUDA kernels of libnys_attn.so; torch only supplies device
+memory and streams.  There is no CPU path: without the built library every
+call raises.
+"""
+
+from . import _lib
+from ._lib import (NYS_BF16, NYS_F32, NysError, EXPORTS, load, make_desc,  # noqa: F401
+                   nys_attn_host_buffer_size, nys_attn_intermediates, nys_attn_launch_count,
+                   nys_attn_launch_names,
+                   nys_attn_workspace_size, nys_status_string, nys_version)
+
+__all__ = [
+    "NYS_F32", "NYS_BF16", "NysError", "load", "desc_of", "nys_attn_forward",
+    "nys_attn_forward_host", "nys_attn_workspace_size", "nys_attn_intermediates",
+    "nys_attn_host_buffer_size", "nys_attn_check_error", "nys_attn_launch_count",
+    "nys_status_string", "nys_version", "Workspace", "nys_attn_launch_names",
+    "nys_attn_forward_timed",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return NYS_F32
+    if t.dtype == torch.bfloat16:
+        return NYS_BF16
+    raise TypeError("Q/K/V must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def desc_of(Q):
+    """nys_desc of a [batch, heads, n, d] tensor."""
+    if Q.dim() != 4:
+        raise ValueError("expected [batch, heads, seq_len, head_dim], got %s" % (tuple(Q.shape),))
+    b, h, n, d = Q.shape
+    return make_desc(_dtype_code(Q), b, h, n, d)
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+class Workspace:
+    """A device workspace sized for one shape, reusable across calls."""
+
+    def __init__(self, Q, num_landmarks):
+        torch = _torch()
+        self.desc = desc_of(Q)
+        self.num_landmarks = int(num_landmarks)
+        self.nbytes = nys_attn_workspace_size(self.desc, num_landmarks)
+        # +256 so that the start can be rounded up to a 256-byte boundary
+        self.buf = torch.empty(max(self.nbytes, 1) + 256, dtype=torch.uint8, device=Q.device)
+        base = self.buf.data_ptr()
+        self.offset = (-base) % 256
+        self.ptr = base + self.offset
+
+    def region(self, name, shape):
+        """A float32 view of one intermediate (see nys_attn_intermediates)."""
+        torch = _torch()
+        lay = nys_attn_intermediates(self.desc, self.num_landmarks)
+        count = 1
+        for s in shape:
+            count *= s
+        start = self.offset + lay[name]
+        return self.buf[start:start + 4 * count].view(torch.float32).view(*shape)
+
+
+def nys_attn_forward(Q, K, V, num_landmarks, pinv_iters=6, conv_w=None, out=None,
+                     workspace=None, stream=None):
+    """out = F~ (Z (B~ V)) + DConv(V) for [batch, heads, n, d] CUDA tensors
+    (float32 or bfloat16, contiguous).  conv_w: [heads, k] float32 CUDA tensor
+    or None.  workspace: a Workspace for this shape, or None (the library then
+    allocates one stream-ordered per call).  Asynchronous on `stream`."""
+    torch = _torch()
+    for name, t in (("Q", Q), ("K", K), ("V", V)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+        if t.shape != Q.shape or t.dtype != Q.dtype:
+            raise ValueError("Q, K, V must share shape and dtype")
+    desc = desc_of(Q)
+    if out is None:
+        out = torch.empty_like(Q)
+    conv_ptr, conv_k = None, 0
+    if conv_w is not None:
+        if conv_w.dtype != torch.float32 or not conv_w.is_cuda or not conv_w.is_contiguous():
+            raise ValueError("conv_w must be a contiguous float32 CUDA tensor [heads, k]")
+        if conv_w.dim() != 2 or conv_w.shape[0] != Q.shape[1]:
+            raise ValueError("conv_w must be [heads, k]")
+        conv_ptr, conv_k = conv_w.data_ptr(), conv_w.shape[1]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.ptr, workspace.nbytes
+    st = _lib.raw_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
+                          pinv_iters, conv_ptr, conv_k, out.data_ptr(), ws_ptr, ws_bytes,
+                          _stream_ptr(stream))
+    _lib.check(st, "nys_attn_forward")
+    return out
+
+
+def nys_attn_forward_timed(Q, K, V, num_landmarks, pinv_iters, conv_w, out, workspace, events,
+                           stream=None):
+    """nys_attn_forward recording events[0] before the first kernel and
+    events[i + 1] after kernel i (torch.cuda.Event objects with timing)."""
+    desc = desc_of(Q)
+    conv_ptr, conv_k = (None, 0) if conv_w is None else (conv_w.data_ptr(), conv_w.shape[1])
+    st = _lib.raw_forward_timed(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
+                                pinv_iters, conv_ptr, conv_k, out.data_ptr(), workspace.ptr,
+                                workspace.nbytes, _stream_ptr(stream),
+                                [e.cuda_event for e in events])
+    _lib.check(st, "nys_attn_forward_timed")
+    return out
+
+
+def nys_attn_check_error(workspace, stream=None):
+    """Synchronises the stream and raises if a kernel recorded an error."""
+    st = _lib.raw_check_error(workspace.ptr, workspace.desc, workspace.num_landmarks,
+                              _stream_ptr(stream))
+    _lib.check(st, "nys_attn_check_error")
+
+
+def nys_attn_forward_host(Qh, Kh, Vh, num_landmarks, pinv_iters, conv_w_host, out_host,
+                          device_buf, stream=None):
+    """End-to-end call on HOST tensors (CPU, contiguous, ideally pinned):
+    host->device copies, the forward, and the device->host copy of the output,
+    all enqueued on `stream`.  device_buf: a CUDA uint8 tensor of at least
+    nys_attn_host_buffer_size bytes (256-byte aligned).  Returns out_host;
+    synchronise the stream before reading it."""
+    desc = desc_of(Qh)
+    conv_ptr, conv_k = None, 0
+    if conv_w_host is not None:
+        conv_ptr, conv_k = conv_w_host.data_ptr(), conv_w_host.shape[1]
+    st = _lib.raw_forward_host(Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), desc,
+                               num_landmarks, pinv_iters, conv_ptr, conv_k,
+                               out_host.data_ptr(), device_buf.data_ptr(), device_buf.numel(),
+                               _stream_ptr(stream))
+    _lib.check(st, "nys_attn_forward_host")
+    return out_host

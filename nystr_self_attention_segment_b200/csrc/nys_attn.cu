@@ -1,0 +1,409 @@
+// C ABI of the Nystrom attention forward: argument validation, workspace
+// layout and the stream-ordered launch sequence.  See include/nys_attn.h for
+// the contract of every entry point.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "simt.cuh"
+
+using namespace nys;
+
+namespace {
+
+size_t elem_size(int dtype) { return dtype == NYS_BF16 ? 2 : 4; }
+
+nys_status validate_shape(const nys_desc *desc, int m) {
+  if (!desc) return NYS_ERR_INVALID_ARG;
+  if (desc->dtype != NYS_F32 && desc->dtype != NYS_BF16) return NYS_ERR_INVALID_ARG;
+  if (desc->batch < 0 || desc->heads < 0 || desc->seq_len < 0 || desc->head_dim < 1)
+    return NYS_ERR_INVALID_ARG;
+  if (m < 1) return NYS_ERR_INVALID_ARG;
+  if ((long)desc->batch * desc->heads * desc->seq_len == 0) return NYS_OK;   // empty
+  if (m > desc->seq_len) return NYS_ERR_INVALID_ARG;
+  if (desc->seq_len % m != 0) return NYS_ERR_NOT_DIVISIBLE;
+  if (desc->dtype == NYS_F32) {
+    if (desc->head_dim > 64 || m > 64) return NYS_ERR_UNSUPPORTED;
+  } else {
+    if (desc->head_dim != 64) return NYS_ERR_UNSUPPORTED;
+    if (m != 32 && m != 64 && m != 128) return NYS_ERR_UNSUPPORTED;
+  }
+  if ((long)desc->batch * desc->heads > (1L << 24) || desc->seq_len > (1 << 24))
+    return NYS_ERR_UNSUPPORTED;
+  return NYS_OK;
+}
+
+bool is_empty(const nys_desc *desc) {
+  return (long)desc->batch * desc->heads * desc->seq_len == 0;
+}
+
+Layout make_layout(const nys_desc *desc, int m) {
+  Layout L;
+  memset(&L, 0, sizeof(L));
+  const size_t BH = (size_t)desc->batch * desc->heads;
+  const size_t n = desc->seq_len, d = desc->head_dim;
+  // key splits of the B~ V pass: enough blocks to fill the GPU twice
+  const int tile = kSimtKeyTile;
+  int ntiles = (int)((n + tile - 1) / tile);
+  int splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
+  if (splits > ntiles) splits = ntiles;
+  if (splits < 1) splits = 1;
+  int tiles_per_split = (ntiles + splits - 1) / splits;
+  splits = (ntiles + tiles_per_split - 1) / tiles_per_split;
+  L.splits = splits;
+  L.keys_per_split = tiles_per_split * tile;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.q_land = take(BH * m * d * 4);
+  L.k_land = take(BH * m * d * 4);
+  L.z = take(BH * m * m * 4);
+  L.y = take(BH * m * d * 4);
+  L.w = take(BH * m * d * 4);
+  L.err = take(256);
+  L.pmax = take(BH * splits * m * 4);
+  L.psum = take(BH * splits * m * 4);
+  L.py = take(BH * splits * m * d * 4);
+  L.scratch = take(m > 64 ? BH * 5 * m * m * 4 : 0);
+  L.q_land_bf = take(0);
+  L.k_land_bf = take(0);
+  L.w_bf = take(0);
+  L.total = off;
+  return L;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  uintptr_t x0 = (uintptr_t)a, x1 = x0 + na, y0 = (uintptr_t)b, y1 = y0 + nb;
+  return x0 < y1 && y0 < x1;
+}
+
+// Records events[i + 1] after the i-th kernel when the caller asked for
+// per-kernel timing.
+struct Marks {
+  cudaEvent_t const *ev = nullptr;
+  int n = 0, next = 1;
+  void after(cudaStream_t s) {
+    if (ev && next < n) cudaEventRecord(ev[next++], s);
+  }
+};
+
+constexpr int kSimtLaunches = 5;
+const char *kSimtNames = "seg_means,pinv,bv_partial,merge_w,out";
+
+template <typename T>
+nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc, int m,
+                       int iters, const float *conv_w, int conv_k, T *out, char *ws,
+                       const Layout &L, cudaStream_t stream, Marks &mk) {
+  const int BH = desc->batch * desc->heads;
+  const int n = desc->seq_len, d = desc->head_dim;
+  float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
+  float *z = (float *)(ws + L.z), *y = (float *)(ws + L.y), *w = (float *)(ws + L.w);
+  float *pmax = (float *)(ws + L.pmax), *psum = (float *)(ws + L.psum);
+  float *py = (float *)(ws + L.py), *scratch = (float *)(ws + L.scratch);
+  const float scale = 1.0f / sqrtf((float)d);
+  const float scale_log2 = scale * kLog2e;
+
+  {
+    long total = (long)BH * m * d;
+    dim3 grid((unsigned)((total + 255) / 256), 2);
+    seg_means_scalar<T><<<grid, 256, 0, stream>>>(Q, K, qt, kt, BH, n, d, m);
+    mk.after(stream);
+  }
+  {
+    const int use_smem = m <= 64;
+    size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
+    if (sm > 48 * 1024)
+      cudaFuncSetAttribute(pinv_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    pinv_simt<<<BH, 256, sm, stream>>>(qt, kt, z, scratch, m, d, scale, iters, use_smem);
+    mk.after(stream);
+  }
+  {
+    size_t sm = ((size_t)m * d + kSimtKeyTile * (d + 1) + kSimtKeyTile * d) * 4;
+    dim3 grid(L.splits, BH);
+    if (m <= 64) {
+      auto kern = bv_partial_simt<T, 8>;
+      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      kern<<<grid, 256, sm, stream>>>(qt, K, V, pmax, psum, py, n, d, m, L.splits,
+                                      L.keys_per_split, scale_log2);
+    } else {
+      auto kern = bv_partial_simt<T, 16>;
+      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      kern<<<grid, 256, sm, stream>>>(qt, K, V, pmax, psum, py, n, d, m, L.splits,
+                                      L.keys_per_split, scale_log2);
+    }
+    mk.after(stream);
+  }
+  {
+    size_t sm = (size_t)m * d * 4;
+    if (sm > 48 * 1024)
+      cudaFuncSetAttribute(merge_w_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    merge_w_simt<<<BH, 256, sm, stream>>>(pmax, psum, py, z, y, w, m, d, L.splits);
+    mk.after(stream);
+  }
+  {
+    size_t sm = ((size_t)m * (d + 1) + (size_t)m * d + 8 * d + (conv_w ? conv_k : 0)) * 4;
+    dim3 grid((n + kSimtOutRowsPerBlock - 1) / kSimtOutRowsPerBlock, BH);
+    const int ck = conv_w ? conv_k : 0;
+    if (m <= 64) {
+      auto kern = out_simt<T, 2>;
+      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      kern<<<grid, 256, sm, stream>>>(Q, V, kt, w, conv_w, out, n, d, m, desc->heads, ck,
+                                      scale_log2);
+    } else {
+      auto kern = out_simt<T, 4>;
+      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      kern<<<grid, 256, sm, stream>>>(Q, V, kt, w, conv_w, out, n, d, m, desc->heads, ck,
+                                      scale_log2);
+    }
+    mk.after(stream);
+  }
+  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+NYS_ATTN_API const char *nys_status_string(nys_status s) {
+  switch (s) {
+    case NYS_OK: return "NYS_OK";
+    case NYS_ERR_INVALID_ARG: return "NYS_ERR_INVALID_ARG: null pointer, negative size or bad enum";
+    case NYS_ERR_UNSUPPORTED: return "NYS_ERR_UNSUPPORTED: no kernel for this head_dim / landmarks / dtype / conv_k";
+    case NYS_ERR_NOT_DIVISIBLE: return "NYS_ERR_NOT_DIVISIBLE: seq_len is not a multiple of num_landmarks";
+    case NYS_ERR_ALIAS: return "NYS_ERR_ALIAS: output overlaps an input or the workspace";
+    case NYS_ERR_WORKSPACE: return "NYS_ERR_WORKSPACE: workspace too small";
+    case NYS_ERR_CUDA: return "NYS_ERR_CUDA: CUDA runtime or launch failure";
+    case NYS_ERR_TIMEOUT: return "NYS_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "unknown nys_status";
+}
+
+NYS_ATTN_API int nys_version(void) { return 100; }
+
+NYS_ATTN_API nys_status nys_attn_workspace_size(const nys_desc *desc, int m, size_t *bytes) {
+  if (!bytes) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  *bytes = is_empty(desc) ? 0 : make_layout(desc, m).total;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_intermediates(const nys_desc *desc, int m,
+                                               nys_intermediates *out) {
+  if (!out) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) {
+    memset(out, 0, sizeof(*out));
+    return NYS_OK;
+  }
+  Layout L = make_layout(desc, m);
+  out->q_landmarks = L.q_land;
+  out->k_landmarks = L.k_land;
+  out->z = L.z;
+  out->y = L.y;
+  out->w = L.w;
+  out->error_word = L.err;
+  out->total = L.total;
+  return NYS_OK;
+}
+
+static nys_status validate_call(const void *Q, const void *K, const void *V,
+                                const nys_desc *desc, int m, int iters, const float *conv_w,
+                                int conv_k, const void *out) {
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (iters < 0) return NYS_ERR_INVALID_ARG;
+  if (iters > kMaxIters) return NYS_ERR_UNSUPPORTED;
+  if (conv_w) {
+    if (conv_k < 1) return NYS_ERR_INVALID_ARG;
+    if (conv_k % 2 == 0) return NYS_ERR_INVALID_ARG;
+    if (conv_k > kMaxConvK) return NYS_ERR_UNSUPPORTED;
+  }
+  if (is_empty(desc)) return NYS_OK;
+  if (!Q || !K || !V || !out) return NYS_ERR_INVALID_ARG;
+  return NYS_OK;
+}
+
+static nys_status forward_impl(const void *Q, const void *K, const void *V,
+                               const nys_desc *desc, int m, int iters, const float *conv_w,
+                               int conv_k, void *out, void *workspace, size_t workspace_bytes,
+                               nys_stream_t stream_, void *const *events, int n_events) {
+  nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
+  if (st != NYS_OK) return st;
+  if (events && n_events < kSimtLaunches + 1) return NYS_ERR_INVALID_ARG;
+  if (is_empty(desc)) return NYS_OK;
+  Marks mk;
+  mk.ev = (cudaEvent_t const *)events;
+  mk.n = events ? n_events : 0;
+  cudaStream_t stream = (cudaStream_t)stream_;
+  const size_t tbytes = (size_t)desc->batch * desc->heads * desc->seq_len * desc->head_dim *
+                        elem_size(desc->dtype);
+  Layout L = make_layout(desc, m);
+  if (overlaps(out, tbytes, Q, tbytes) || overlaps(out, tbytes, K, tbytes) ||
+      overlaps(out, tbytes, V, tbytes))
+    return NYS_ERR_ALIAS;
+  if (workspace) {
+    if (workspace_bytes < L.total) return NYS_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255) != 0) return NYS_ERR_INVALID_ARG;
+    if (overlaps(out, tbytes, workspace, L.total)) return NYS_ERR_ALIAS;
+  }
+  char *ws = (char *)workspace;
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
+    owned = true;
+  }
+  if (cudaMemsetAsync(ws + L.err, 0, 4, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  if (mk.ev) cudaEventRecord(mk.ev[0], stream);
+  if (st == NYS_OK) {
+    if (desc->dtype == NYS_F32)
+      st = launch_simt<float>((const float *)Q, (const float *)K, (const float *)V, desc, m,
+                              iters, conv_w, conv_k, (float *)out, ws, L, stream, mk);
+    else
+      st = launch_simt<__nv_bfloat16>((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                                      (const __nv_bfloat16 *)V, desc, m, iters, conv_w, conv_k,
+                                      (__nv_bfloat16 *)out, ws, L, stream, mk);
+  }
+  if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && st == NYS_OK) st = NYS_ERR_CUDA;
+  return st;
+}
+
+NYS_ATTN_API nys_status nys_attn_forward(const void *Q, const void *K, const void *V,
+                                         const nys_desc *desc, int m, int iters,
+                                         const float *conv_w, int conv_k, void *out,
+                                         void *workspace, size_t workspace_bytes,
+                                         nys_stream_t stream) {
+  return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
+                      stream, nullptr, 0);
+}
+
+NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q, const void *K, const void *V,
+                                               const nys_desc *desc, int m, int iters,
+                                               const float *conv_w, int conv_k, void *out,
+                                               void *workspace, size_t workspace_bytes,
+                                               nys_stream_t stream, void *const *events,
+                                               int n_events) {
+  if (!events) return NYS_ERR_INVALID_ARG;
+  return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
+                      stream, events, n_events);
+}
+
+NYS_ATTN_API nys_status nys_attn_check_error(void *workspace, const nys_desc *desc, int m,
+                                             nys_stream_t stream_) {
+  if (!workspace) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) return NYS_OK;
+  Layout L = make_layout(desc, m);
+  cudaStream_t stream = (cudaStream_t)stream_;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, (char *)workspace + L.err, 4, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync((char *)workspace + L.err, 0, 4, stream) != cudaSuccess)
+      return NYS_ERR_CUDA;
+    return (nys_status)word;
+  }
+  return NYS_OK;
+}
+
+struct HostBufLayout {
+  size_t q, k, v, out, conv, ws, total;
+};
+
+static HostBufLayout host_layout(const nys_desc *desc, int m, int conv_k) {
+  HostBufLayout H;
+  const size_t t = (size_t)desc->batch * desc->heads * desc->seq_len * desc->head_dim *
+                   elem_size(desc->dtype);
+  size_t off = 0;
+  auto take = [&](size_t b) {
+    size_t at = off;
+    off = align256(off + b);
+    return at;
+  };
+  H.q = take(t);
+  H.k = take(t);
+  H.v = take(t);
+  H.out = take(t);
+  H.conv = take((size_t)desc->heads * (conv_k > 0 ? conv_k : 0) * 4);
+  H.ws = take(is_empty(desc) ? 0 : make_layout(desc, m).total);
+  H.total = off;
+  return H;
+}
+
+NYS_ATTN_API nys_status nys_attn_host_buffer_size(const nys_desc *desc, int m, int conv_k,
+                                                  size_t *bytes) {
+  if (!bytes) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  *bytes = host_layout(desc, m, conv_k).total;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_forward_host(const void *Qh, const void *Kh, const void *Vh,
+                                              const nys_desc *desc, int m, int iters,
+                                              const float *conv_w_h, int conv_k, void *out_h,
+                                              void *dbuf, size_t dbuf_bytes,
+                                              nys_stream_t stream_) {
+  nys_status st = validate_call(Qh, Kh, Vh, desc, m, iters, conv_w_h, conv_k, out_h);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) return NYS_OK;
+  if (!dbuf) return NYS_ERR_INVALID_ARG;
+  if (((uintptr_t)dbuf & 255) != 0) return NYS_ERR_INVALID_ARG;
+  HostBufLayout H = host_layout(desc, m, conv_w_h ? conv_k : 0);
+  if (dbuf_bytes < H.total) return NYS_ERR_WORKSPACE;
+  cudaStream_t stream = (cudaStream_t)stream_;
+  char *b = (char *)dbuf;
+  const size_t t = (size_t)desc->batch * desc->heads * desc->seq_len * desc->head_dim *
+                   elem_size(desc->dtype);
+  if (cudaMemcpyAsync(b + H.q, Qh, t, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + H.k, Kh, t, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + H.v, Vh, t, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  const float *cw = nullptr;
+  if (conv_w_h) {
+    if (cudaMemcpyAsync(b + H.conv, conv_w_h, (size_t)desc->heads * conv_k * 4,
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return NYS_ERR_CUDA;
+    cw = (const float *)(b + H.conv);
+  }
+  st = nys_attn_forward(b + H.q, b + H.k, b + H.v, desc, m, iters, cw, conv_k, b + H.out,
+                        b + H.ws, H.total - H.ws, stream_);
+  if (st != NYS_OK) return st;
+  if (cudaMemcpyAsync(out_h, b + H.out, t, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_launch_count(const nys_desc *desc, int m, int conv_k,
+                                              int *launches) {
+  (void)conv_k;
+  if (!launches) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  *launches = is_empty(desc) ? 0 : kSimtLaunches;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char *names,
+                                              size_t names_bytes) {
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  const char *src = is_empty(desc) ? "" : kSimtNames;
+  if (names) {
+    if (names_bytes < strlen(src) + 1) return NYS_ERR_INVALID_ARG;
+    strcpy(names, src);
+  }
+  return NYS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Normwise error max|gpu - oracle| / max|oracle| per head, against 1e-4 for
+the fp32 path and 2e-2 for the bf16 path.  Full-size workloads run whole on
+the GPU, in the launch configuration the benchmark times; the oracle checks a
+sample of heads (heads are independent, so a sampled head is a complete
+output).  Inputs are the seeded generator's, rounded to the device dtype
+before either side sees them."""
+import numpy as np
+import pytest
+
+import nystr_self_attention_segment_b200 as nys
+from nystr_self_attention_segment_b200.inputs import BF16, F32, WORKLOADS, make_custom, make_inputs
+from oracle import nystrom as orc
+from tests.gpu_util import TOL, normwise, run, to_dev, torch
+from tests.golden.make_golden import read as read_golden
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_heads(Bn, H, k=3):
+    idx = [(0, 0), (Bn - 1, H - 1), (Bn // 2, H // 2)]
+    out = []
+    for p in idx:
+        if p not in out:
+            out.append(p)
+    return out[:k]
+
+
+def oracle_head(x, b, h, m, iters, conv=True):
+    w = x["conv_w"][h] if (conv and x["conv_w"] is not None) else None
+    return orc.nystrom_head(x["Q"][b, h], x["K"][b, h], x["V"][b, h], m, iters, w)
+
+
+# ------------------------------------------------------------------ tiny fp32
+
+@pytest.mark.parametrize("name", ["tiny_f32_m8", "tiny_f32_m64"])
+def test_tiny_fp32_against_oracle_and_golden(name):
+    wl = WORKLOADS[name]
+    x = make_inputs(wl)
+    got, ws, _ = run(x, F32, wl.landmarks, wl.pinv_iters)
+    want = orc.nystrom_forward(x["Q"], x["K"], x["V"], wl.landmarks, wl.pinv_iters, x["conv_w"])
+    assert normwise(got, want) <= TOL["f32"]
+    _, gold = read_golden(name)
+    assert normwise(got.reshape(-1), gold["out"]) <= TOL["f32"]
+
+
+def test_tiny_fp32_m_equals_n_tracks_exact_attention_with_more_iterations():
+    # Lemma 2 on the device: m = n and a converged pseudoinverse give exact
+    # softmax attention (to fp32 rounding).
+    wl = WORKLOADS["tiny_f32_m64"]
+    x = make_inputs(wl)
+    got, _, _ = run(x, F32, 64, iters=40)
+    exact = orc.exact_attention(x["Q"], x["K"], x["V"])
+    assert normwise(got, exact) <= 1e-3
+
+
+# ------------------------------------------------------------------ bf16 workloads
+
+BF16_WORKLOADS = ["bert_n512_m64", "long_n4096_m64", "headline_n8192_m64", "headline_n8192_m32",
+                  "sweep_n1024_m128", "sweep_n2048_m128", "sweep_n4096_m128", "sweep_n8192_m128",
+                  "sweep_n16384_m128", "sweep_n32768_m128", "sweep_n65536_m128"]
+
+
+@pytest.mark.parametrize("name", BF16_WORKLOADS)
+def test_bf16_workload_against_oracle(name):
+    wl = WORKLOADS[name]
+    x = make_inputs(wl)
+    got, ws, _ = run(x, BF16, wl.landmarks, wl.pinv_iters)
+    assert np.all(np.isfinite(got))
+    errs = []
+    for b, h in sample_heads(wl.batch, wl.heads):
+        want = oracle_head(x, b, h, wl.landmarks, wl.pinv_iters)["out"]
+        errs.append(normwise(got[b, h], want))
+    assert max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("name", ["bert_n512_m64", "headline_n8192_m64", "sweep_n1024_m128"])
+def test_bf16_intermediates(name):
+    # Landmarks are fp32 sums of the same bf16 inputs; Z, Y and W are checked
+    # against the oracle's steps applied to the device's own fp32 landmarks,
+    # so that the (ill-conditioned) pseudoinverse is compared on equal inputs.
+    wl = WORKLOADS[name]
+    x = make_inputs(wl)
+    m, d = wl.landmarks, wl.head_dim
+    got, ws, _ = run(x, BF16, m, wl.pinv_iters)
+    BH = wl.bh
+    qt = ws.region("q_landmarks", (BH, m, d)).cpu().numpy().astype(np.float64)
+    kt = ws.region("k_landmarks", (BH, m, d)).cpu().numpy().astype(np.float64)
+    Zg = ws.region("z", (BH, m, m)).cpu().numpy().astype(np.float64)
+    Yg = ws.region("y", (BH, m, d)).cpu().numpy().astype(np.float64)
+    Wg = ws.region("w", (BH, m, d)).cpu().numpy().astype(np.float64)
+    s = 1 / np.sqrt(d)
+    for b, h in sample_heads(wl.batch, wl.heads):
+        i = b * wl.heads + h
+        Q, K, V = (x[t][b, h].astype(np.float64) for t in ("Q", "K", "V"))
+        assert normwise(qt[i], orc.segment_means(Q, m)) <= 1e-5
+        assert normwise(kt[i], orc.segment_means(K, m)) <= 1e-5
+        Z = orc.iterative_pinv(orc.kernel_A(qt[i], kt[i], s), wl.pinv_iters)
+        assert normwise(Zg[i], Z) <= 2e-2
+        Y = orc.kernel_B(qt[i], K, s) @ V
+        assert normwise(Yg[i], Y) <= 2e-2
+        assert normwise(Wg[i], Zg[i] @ Yg[i]) <= 1e-4
+
+
+def test_long_context_error_report_against_exact_attention():
+    # Approximation-error report on the long-context workload (two heads):
+    # the Nystrom output without the conv skip against exact n x n softmax
+    # attention.  The device must reproduce the oracle's approximation error.
+    wl = WORKLOADS["long_n4096_m64"]
+    x = make_inputs(wl, batch=1, heads=2)
+    got, _, _ = run(x, BF16, wl.landmarks, wl.pinv_iters, conv=False)
+    for h in range(2):
+        exact = orc.exact_attention_head(x["Q"][0, h], x["K"][0, h], x["V"][0, h])
+        approx = oracle_head(x, 0, h, wl.landmarks, wl.pinv_iters, conv=False)["out"]
+        e_orc = np.abs(approx - exact)
+        e_gpu = np.abs(got[0, h] - exact)
+        print("head %d: oracle max %.4g mean %.4g | gpu max %.4g mean %.4g | max|exact| %.4g"
+              % (h, e_orc.max(), e_orc.mean(), e_gpu.max(), e_gpu.mean(), np.abs(exact).max()))
+        assert abs(e_gpu.max() - e_orc.max()) <= TOL["bf16"] * np.abs(approx).max()
+
+
+# ------------------------------------------------------------------ edge cases
+
+EDGE = [
+    # (B, H, n, d, m, dtype, conv_k, iters)
+    (1, 1, 64, 64, 64, BF16, 33, 6),      # m = n, one segment per token
+    (1, 1, 32, 64, 32, BF16, 33, 6),      # sequence shorter than the conv kernel
+    (1, 2, 128, 64, 128, BF16, 0, 6),     # m = n = 128, no conv
+    (2, 3, 96, 64, 32, BF16, 33, 6),      # ragged: n not a multiple of 128
+    (1, 2, 192, 64, 64, BF16, 1, 6),      # ragged, conv kernel of one tap
+    (1, 1, 320, 64, 64, BF16, 63, 6),     # ragged, widest supported conv
+    (1, 2, 1152, 64, 128, BF16, 33, 0),   # zero pinv iterations (Z = Z0)
+    (3, 1, 640, 64, 32, BF16, 5, 6),
+    (1, 1, 24, 8, 3, F32, 3, 6),          # fp32, odd sizes
+    (2, 2, 60, 17, 12, F32, 0, 6),
+    (1, 1, 64, 64, 64, F32, 7, 2),
+]
+
+
+@pytest.mark.parametrize("B,H,n,d,m,dtype,conv_k,iters", EDGE)
+def test_edge_shapes(B, H, n, d, m, dtype, conv_k, iters):
+    x = make_custom((B, H, n, d), dtype, seed=7 * n + m, scale=1.0, conv_k=conv_k)
+    got, _, _ = run(x, dtype, m, iters, conv=conv_k > 0)
+    want = orc.nystrom_forward(x["Q"], x["K"], x["V"], m, iters, x["conv_w"] if conv_k else None)
+    for b in range(B):
+        for h in range(H):
+            assert normwise(got[b, h], want[b, h]) <= TOL[dtype], (b, h)
+
+
+def test_empty_batch_is_a_no_op():
+    t = torch()
+    Q = t.empty((0, 12, 512, 64), dtype=t.bfloat16, device="cuda")
+    out = nys.nys_attn_forward(Q, Q.clone(), Q.clone(), 64, 6, None)
+    assert out.shape == Q.shape
+
+
+def test_deterministic_and_library_workspace_and_host_entry():
+    wl = WORKLOADS["bert_n512_m64"]
+    x = make_inputs(wl, batch=2)
+    t = torch()
+    a, _, (Q, K, V, cw) = run(x, BF16, 64)
+    b, _, _ = run(x, BF16, 64)
+    c, _, _ = run(x, BF16, 64, workspace=False)        # stream-ordered library workspace
+    assert np.array_equal(a, b) and np.array_equal(a, c)
+    # end-to-end entry on host buffers gives the same bits
+    desc = nys.desc_of(Q)
+    nbytes = nys.nys_attn_host_buffer_size(desc, 64, cw.shape[1])
+    dbuf = t.empty(nbytes + 256, dtype=t.uint8, device="cuda")
+    off = (-dbuf.data_ptr()) % 256
+    dview = dbuf[off:off + nbytes]
+    Qh, Kh, Vh = (u.cpu().pin_memory() for u in (Q, K, V))
+    outh = t.empty_like(Qh).pin_memory()
+    nys.nys_attn_forward_host(Qh, Kh, Vh, 64, 6, cw.cpu(), outh, dview)
+    t.cuda.synchronize()
+    assert np.array_equal(outh.float().numpy().astype(np.float64), a)
+
+
+def test_invalid_call_leaves_output_untouched():
+    t = torch()
+    Q = to_dev(np.zeros((1, 1, 100, 64), np.float32), BF16)
+    out = t.full_like(Q, 7.0)
+    with pytest.raises(nys.NysError) as e:
+        nys.nys_attn_forward(Q, Q.clone(), Q.clone(), 64, 6, None, out=out)   # 100 % 64 != 0
+    assert e.value.name == "NYS_ERR_NOT_DIVISIBLE"
+    t.cuda.synchronize()
+    assert bool((out == 7.0).all())
