@@ -113,6 +113,9 @@ def nys_attn_forward_timed(Q, K, V, num_landmarks, pinv_iters, conv_w, out, work
     events[i + 1] after kernel i (torch.cuda.Event objects with timing)."""
     desc = desc_of(Q)
     conv_ptr, conv_k = (None, 0) if conv_w is None else (conv_w.data_ptr(), conv_w.shape[1])
+    for e in events:
+        if not e.cuda_event:          # torch creates the CUDA event on first record
+            e.record()
     st = _lib.raw_forward_timed(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
                                 pinv_iters, conv_ptr, conv_k, out.data_ptr(), workspace.ptr,
                                 workspace.nbytes, _stream_ptr(stream),

@@ -291,6 +291,8 @@ NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q, const void *K, con
                                                nys_stream_t stream, void *const *events,
                                                int n_events) {
   if (!events) return NYS_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return NYS_ERR_INVALID_ARG;
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
                       stream, events, n_events);
 }
