@@ -13,7 +13,8 @@ namespace nys {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxIters = 64;
 constexpr int kMaxConvK = 63;
-constexpr int kTargetCtas = 296;   // 2 x 148 SMs of a B200
+constexpr int kNumSms = 148;       // streaming multiprocessors of a B200
+constexpr int kTargetCtas = 296;   // 2 x 148
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -44,12 +45,14 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t code) {
 // a machine without a GPU.  All regions are 256-byte aligned.
 struct Layout {
   size_t q_land, k_land, z, y, w, err;     // parity-visible fp32 intermediates
+  size_t count;                            // per-head block counters (bf16 path)
   size_t pmax, psum, py;                   // split-n partials of B~ V
   size_t scratch;                          // per-head pinv scratch (m > 64)
   size_t q_land_bf, k_land_bf, w_bf;       // bf16 MMA operands
   size_t total;
-  int splits;                              // key splits of the B~ V pass
-  int keys_per_split;
+  int splits;                              // B~ V partials per head
+  int keys_per_split;                      // SIMT path: keys per split
+  int bv_ctas_per_head;                    // tensor-core path: CTAs per head
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

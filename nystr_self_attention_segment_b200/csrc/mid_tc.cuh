@@ -1,0 +1,418 @@
+// Middle stage of the bf16 path, one launch:
+//   blocks [0, BH)            the landmark kernel A and its pseudoinverse Z
+//                             (one head each, see pinv_tc.cuh),
+//   blocks [BH, BH*(1+S))     Y = B~ V streamed over the keys, S blocks per head
+//                             ("Nystromformer: A Nystrom-Based Algorithm for
+//                             Approximating Self-Attention", section 3.4,
+//                             Eq. 17 / Algorithm 1; B~ = softmax(Q~ K^T/sqrt(d))
+//                             over the n keys is never stored),
+// and the last block of a head to finish (counted with an atomic) merges the
+// head's S partial softmax states in a fixed order into Y and forms W = Z Y.
+//
+// B~ V block.  The 128 accumulator rows (TMEM lanes) hold G = 128 / m copies
+// of the m landmark rows; copy g handles keys g*m .. g*m + m - 1 of every
+// 128-key chunk, so every TMEM lane has work.  Per chunk:
+//   TMA  K and V chunks (128 x 64 bf16, zero past n),
+//   MMA  S = [Q~; ..; Q~] K_c^T       (M=128, N=128, K=64, operands in smem),
+//   softmax warpgroup: running max / sum per row (log2 units), P = 2^(..) as
+//        bf16 straight into TMEM (zero outside the row's key group),
+//   MMA  Y_c = P V_c                   (M=128, N=64, K=128, P read from TMEM),
+//   softmax warpgroup: acc = acc * 2^(m_old - m_new) + Y_c in registers.
+// Two softmax warpgroups take alternate chunks, each with its own TMEM
+// buffers and running state; the 2G states of a landmark are merged in the
+// block at the end, giving one partial per (block, landmark).
+// Warps: 0 TMA producer, 1 MMA issuer / TMEM owner, 4-7 and 8-11 softmax.
+#pragma once
+
+#include "pinv_tc.cuh"
+
+namespace nys {
+namespace midtc {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kStages = 3;
+constexpr int kChunk = 128;
+
+struct BvSmem {
+  uint32_t q, k[kStages], v[kStages], bars, total;
+};
+__host__ __device__ inline BvSmem bv_smem() {
+  BvSmem L;
+  uint32_t off = 0;
+  auto take = [&](uint32_t b) {
+    uint32_t at = off;
+    off += (b + 1023u) & ~1023u;
+    return at;
+  };
+  L.q = take(16384u);
+  for (int s = 0; s < kStages; ++s) {
+    L.k[s] = take(16384u);
+    L.v[s] = take(16384u);
+  }
+  L.bars = take(1024u);
+  L.total = off;
+  return L;
+}
+
+template <int M>
+__host__ __device__ constexpr uint32_t smem_bytes() {
+  // pinv operands, B~ V buffers, and the merge scratch (Z, Y, weights)
+  return 1024u + (pinvtc::Cfg<M>::total > 16384u + kStages * 32768u + 1024u
+                      ? pinvtc::Cfg<M>::total
+                      : 16384u + kStages * 32768u + 1024u);
+}
+
+struct Params {
+  pinvtc::Params pinv;
+  const float *q_land;        // [BH][m][64]
+  const float *z;             // [BH][m][m]  (pinv output)
+  float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
+  float *y, *w;               // [BH][m][64]
+  uint32_t *count;            // [BH] blocks finished per head (zeroed per call)
+  uint32_t *err;
+  int BH, n, chunks_per_head, splits;
+  float scale_log2;
+};
+
+// ------------------------------------------------------------------ B~ V body
+template <int M>
+__device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensorMap *map_v,
+                                        const Params &prm, uint8_t *smem, int bh, int split) {
+  constexpr int G = 128 / M;
+  const BvSmem L = bv_smem();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c_begin = (int)((long)split * prm.chunks_per_head / prm.splits);
+  const int c_end = (int)((long)(split + 1) * prm.chunks_per_head / prm.splits);
+  const int nch = c_end - c_begin;
+
+  uint64_t *bars = (uint64_t *)(smem + L.bars);
+  uint64_t *full = bars;                  // [kStages]
+  uint64_t *empty = bars + kStages;       // [kStages]
+  uint64_t *s_full = bars + 2 * kStages;  // [2] per softmax warpgroup
+  uint64_t *s_free = s_full + 2;
+  uint64_t *p_ready = s_free + 2;
+  uint64_t *y_full = p_ready + 2;
+  uint64_t *y_free = y_full + 2;
+  uint32_t *tmem_slot = (uint32_t *)(y_free + 2);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+  const Abort ab{abort_flag, prm.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 128);
+      mbar_init(&p_ready[b], 128);
+      mbar_init(&y_full[b], 1);
+      mbar_init(&y_free[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(map_k);
+    tma_prefetch_desc(map_v);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
+  if (threadIdx.x < 256) {
+    const float4 *qt = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
+    const int row = threadIdx.x >> 1, half = threadIdx.x & 1;   // 4 chunks each
+    float4 a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = qt[(row % M) * 16 + half * 8 + u];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      st_shared_v4(smem_u32(smem + L.q) + sw128_offset(row, half * 4 + u),
+                   pack_bf16(a[2 * u].x, a[2 * u].y), pack_bf16(a[2 * u].z, a[2 * u].w),
+                   pack_bf16(a[2 * u + 1].x, a[2 * u + 1].y),
+                   pack_bf16(a[2 * u + 1].z, a[2 * u + 1].w));
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM per softmax warpgroup w: S at 256w (128 cols), P at 256w + 128
+  // (64 cols of bf16 pairs), Y at 256w + 192 (64 cols)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nch; ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
+        const int k0 = (c_begin + i) * kChunk;
+        mbar_expect_tx(&full[s], 32768u);
+        tma_load_3d(smem + L.k[s], map_k, &full[s], 0, k0, bh);
+        tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(kFmtBF16, 128, 128, 0, 0);
+      const uint32_t id_y = make_idesc(kFmtBF16, 128, 64, 0, 1);
+      const uint32_t q_a = smem_u32(smem + L.q);
+      auto issue_pv = [&](int j) -> bool {
+        const int w = j & 1, s = j % kStages, u = j >> 1;
+        if (!mbar_wait(&p_ready[w], u & 1, ab)) return false;
+        if (!mbar_wait(&y_free[w], (u & 1) ^ 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t v_a = smem_u32(smem + L.v[s]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts(tmem + 256 * w + 192, tmem + 256 * w + 128 + 8 * k,
+                      make_sdesc(v_a + k * 2048u, 16, 1024), id_y, k > 0);
+        mma_commit(&y_full[w]);
+        mma_commit(&empty[s]);
+        return true;
+      };
+      bool ok = true;
+      for (int i = 0; i < nch && ok; ++i) {
+        const int s = i % kStages, w = i & 1, u = i >> 1;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) break;
+        if (!mbar_wait(&s_free[w], (u & 1) ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t k_a = smem_u32(smem + L.k[s]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem + 256 * w, make_sdesc(q_a + 32 * k, 16, 1024),
+                   make_sdesc(k_a + 32 * k, 16, 1024), id_s, k > 0);
+        mma_commit(&s_full[w]);
+        if (i > 0) ok = issue_pv(i - 1);
+      }
+      if (ok && nch > 0) issue_pv(nch - 1);
+    }
+  }
+  // softmax warpgroups; their running states are kept for the merge below
+  float run_max = -INFINITY, run_sum = 0.f;
+  float acc[64];
+#pragma unroll
+  for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+  const int wg = (warp >= 8) ? 1 : 0;
+  const int r = threadIdx.x & 127;          // accumulator row == TMEM lane
+  const int j = r % M, g = r / M;           // landmark, key group
+  if (warp >= 4) {
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + 256 * wg;
+    {   // P starts at zero: each row only ever writes its own key group
+      uint32_t z[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) z[e] = 0u;
+      tmem_st32(t_s + 128, z);
+      tmem_st32(t_s + 160, z);
+      tmem_st_wait();
+    }
+    for (int i = wg; i < nch; i += 2) {
+      const int u = i >> 1;
+      if (!mbar_wait(&s_full[wg], u & 1, ab)) break;
+      tc_fence_after();
+      float v[M];
+#pragma unroll
+      for (int c = 0; c < M; c += 32) tmem_ld32(t_s + g * M + c, v + c);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[wg]);
+      const int key0 = (c_begin + i) * kChunk + g * M;
+      const int valid = min(M, prm.n - key0);     // keys of this group inside [0, n)
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < M; ++c)
+        if (c < valid) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+      const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mnew = fmaxf(run_max, cmax * prm.scale_log2);
+      const bool none = (mnew == -INFINITY);
+      const float alpha = none ? 1.f : fast_exp2(run_max - mnew);
+      float ps[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+      uint32_t pk[M / 2];
+#pragma unroll
+      for (int c = 0; c < M; c += 2) {
+        const float p0 = (c < valid && !none) ? fast_exp2(fmaf(v[c], prm.scale_log2, -mnew)) : 0.f;
+        const float p1 =
+            (c + 1 < valid && !none) ? fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mnew)) : 0.f;
+        ps[(c >> 1) & 7] += p0 + p1;
+        pk[c >> 1] = pack_bf16(p0, p1);
+      }
+      const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      run_sum = run_sum * alpha + psum;
+      run_max = mnew;
+#pragma unroll
+      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + 128 + g * (M / 2) + c, pk + c);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[wg]);
+      if (!mbar_wait(&y_full[wg], u & 1, ab)) break;
+      tc_fence_after();
+      float y[64];
+      tmem_ld32(t_s + 192, y);
+      tmem_ld32(t_s + 224, y + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&y_free[wg]);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha, y[c]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();   // pipeline drained: stage buffers are free for the merge
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  // In-block merge of the 2G states of every landmark, in a fixed order.
+  float *st = (float *)(smem + L.k[0]);   // [2][128][66]: max, sum, acc[64]
+  if (warp >= 4) {
+    float *o = st + (wg * 128 + r) * 66;
+    o[0] = run_max;
+    o[1] = run_sum;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) o[2 + c] = acc[c];
+  }
+  __syncthreads();
+  if (warp >= 4 && wg == 0 && g == 0) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 2 * G; ++q) mx = fmaxf(mx, st[((q / G) * 128 + (q % G) * M + j) * 66]);
+    float f[2 * G], den = 0.f;
+#pragma unroll
+    for (int q = 0; q < 2 * G; ++q) {
+      const float *o = st + ((q / G) * 128 + (q % G) * M + j) * 66;
+      f[q] = (mx == -INFINITY) ? 0.f : fast_exp2(o[0] - mx);
+      den = fmaf(o[1], f[q], den);
+    }
+    const size_t base = ((size_t)bh * prm.splits + split) * M + j;
+    prm.pmax[base] = mx;
+    prm.psum[base] = den;
+    float4 *dst = (float4 *)(prm.py + base * 64);
+#pragma unroll 4
+    for (int c4 = 0; c4 < 16; ++c4) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 2 * G; ++q) {
+        const float *o = st + ((q / G) * 128 + (q % G) * M + j) * 66 + 2 + 4 * c4;
+        a.x = fmaf(f[q], o[0], a.x);
+        a.y = fmaf(f[q], o[1], a.y);
+        a.z = fmaf(f[q], o[2], a.z);
+        a.w = fmaf(f[q], o[3], a.w);
+      }
+      dst[c4] = a;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ merge + W
+// Y = sum_s f_s py_s / sum_s f_s psum_s with f_s = 2^(pmax_s - max), over the
+// S partials of the head in order; then W = Z Y.  All threads of the block.
+template <int M>
+__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh) {
+  const int t = threadIdx.x, nt = blockDim.x;
+  const int S = prm.splits;
+  float *zs = (float *)smem;          // [M][M + 4]
+  constexpr int ZL = M + 4;
+  float *ys = zs + M * ZL;            // [M][64]
+  float *wgt = ys + M * 64;           // [S][M]
+  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
+  for (int i = t; i < M * M / 4; i += nt) {
+    const float4 v = __ldcg(z4 + i);
+    const int row = (i * 4) / M, col = (i * 4) % M;
+    *(float4 *)(zs + row * ZL + col) = v;
+  }
+  const size_t pb = (size_t)bh * S * M;
+  for (int i = t; i < S * M; i += nt) wgt[i] = __ldcg(prm.pmax + pb + i);
+  __syncthreads();
+  if (t < M) {
+    float mx = -INFINITY;
+    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
+    float den = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float f = fast_exp2(wgt[s * M + t] - mx);
+      wgt[s * M + t] = f;
+      den = fmaf(__ldcg(prm.psum + pb + (size_t)s * M + t), f, den);
+    }
+    const float inv = 1.f / den;
+    for (int s = 0; s < S; ++s) wgt[s * M + t] *= inv;
+  }
+  __syncthreads();
+  for (int idx = t; idx < M * 16; idx += nt) {
+    const int j = idx >> 4;
+    const float4 *src = (const float4 *)(prm.py + (pb + j) * 64) + (idx & 15);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < S; s0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < S) v[u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < S) {
+          const float f = wgt[(s0 + u) * M + j];
+          a.x = fmaf(f, v[u].x, a.x);
+          a.y = fmaf(f, v[u].y, a.y);
+          a.z = fmaf(f, v[u].z, a.z);
+          a.w = fmaf(f, v[u].w, a.w);
+        }
+    }
+    ((float4 *)ys)[idx] = a;
+    ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = a;
+  }
+  __syncthreads();
+  // W = Z Y: work item = (4 rows, 4 features)
+  for (int item = t; item < (M / 4) * 16; item += nt) {
+    const int c4 = item & 15, j0 = (item >> 4) * 4;
+    float4 a[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < M; ++k) {
+      const float4 yv = ((const float4 *)ys)[k * 16 + c4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float zz = zs[(j0 + q) * ZL + k];
+        a[q].x = fmaf(zz, yv.x, a[q].x);
+        a[q].y = fmaf(zz, yv.y, a[q].y);
+        a[q].z = fmaf(zz, yv.z, a[q].z);
+        a[q].w = fmaf(zz, yv.w, a[q].w);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      ((float4 *)(prm.w + (size_t)bh * M * 64))[(j0 + q) * 16 + c4] = a[q];
+  }
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads, 1)
+mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+           const Params prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint32_t last;
+  int bh;
+  if ((int)blockIdx.x < prm.BH) {
+    bh = blockIdx.x;
+    if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh);
+  } else {
+    const int b = blockIdx.x - prm.BH;
+    bh = b / prm.splits;
+    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits);
+  }
+  // publish this block's results, then count it; the last of the head's
+  // S + 1 blocks merges
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits;
+  __syncthreads();
+  if (last) {
+    __threadfence();
+    merge_body<M>(prm, smem, bh);
+  }
+}
+
+}  // namespace midtc
+}  // namespace nys

@@ -8,6 +8,10 @@
 
 #include "common.cuh"
 #include "simt.cuh"
+#include "sm100.cuh"
+#include "mid_tc.cuh"
+#include "out_tc.cuh"
+#include "stream_bf16.cuh"
 
 using namespace nys;
 
@@ -44,16 +48,32 @@ Layout make_layout(const nys_desc *desc, int m) {
   memset(&L, 0, sizeof(L));
   const size_t BH = (size_t)desc->batch * desc->heads;
   const size_t n = desc->seq_len, d = desc->head_dim;
-  // key splits of the B~ V pass: enough blocks to fill the GPU twice
-  const int tile = kSimtKeyTile;
-  int ntiles = (int)((n + tile - 1) / tile);
-  int splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
-  if (splits > ntiles) splits = ntiles;
-  if (splits < 1) splits = 1;
-  int tiles_per_split = (ntiles + splits - 1) / splits;
-  splits = (ntiles + tiles_per_split - 1) / tiles_per_split;
+  int splits;
+  if (desc->dtype == NYS_BF16) {
+    // one B~ V CTA per SM: chunk-aligned key splits per head, times the
+    // 128 / m row copies inside a CTA
+    // one pseudoinverse block per head plus `splits` B~ V blocks per head in
+    // one wave of 148 blocks; each B~ V block leaves one merged partial
+    const int chunks = (int)((n + midtc::kChunk - 1) / midtc::kChunk);
+    int per_head = BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1;
+    if (per_head < 1) per_head = 1;
+    if (per_head > chunks) per_head = chunks;
+    L.bv_ctas_per_head = per_head;
+    splits = per_head;
+    L.keys_per_split = 0;
+  } else {
+    // key splits of the SIMT B~ V pass: enough blocks to fill the GPU twice
+    const int tile = kSimtKeyTile;
+    int ntiles = (int)((n + tile - 1) / tile);
+    splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
+    if (splits > ntiles) splits = ntiles;
+    if (splits < 1) splits = 1;
+    int tiles_per_split = (ntiles + splits - 1) / splits;
+    splits = (ntiles + tiles_per_split - 1) / tiles_per_split;
+    L.keys_per_split = tiles_per_split * tile;
+    L.bv_ctas_per_head = 0;
+  }
   L.splits = splits;
-  L.keys_per_split = tiles_per_split * tile;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t at = off;
@@ -65,11 +85,12 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.z = take(BH * m * m * 4);
   L.y = take(BH * m * d * 4);
   L.w = take(BH * m * d * 4);
-  L.err = take(256);
+  L.err = take(256 + BH * 4);    // error word, then one counter per head
+  L.count = L.err + 256;
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
   L.py = take(BH * splits * m * d * 4);
-  L.scratch = take(m > 64 ? BH * 5 * m * m * 4 : 0);
+  L.scratch = take(desc->dtype == NYS_F32 && m > 64 ? BH * 5 * m * m * 4 : 0);
   L.q_land_bf = take(0);
   L.k_land_bf = take(0);
   L.w_bf = take(0);
@@ -166,6 +187,125 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, resolved through the runtime so that the
+// library does not link libcuda (it loads on machines without a GPU).
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;   // resolved once; never changes afterwards
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// [BH][n][64] bf16 viewed as a 3-D tensor (64, n, BH); box of `rows` rows;
+// 128-byte swizzle; out-of-range rows read as zero and are not written.
+bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)n, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128, (cuuint64_t)n * 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+constexpr int kTcLaunches = 3;
+const char *kTcNames = "seg_means,mid_tc,out_tc";
+
+template <int M>
+nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
+                       const nys_desc *desc, int iters, const float *conv_w, int conv_k,
+                       __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
+                       Marks &mk) {
+  const int BH = desc->batch * desc->heads;
+  const int n = desc->seq_len;
+  float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
+  float *z = (float *)(ws + L.z), *y = (float *)(ws + L.y), *w = (float *)(ws + L.w);
+  float *pmax = (float *)(ws + L.pmax), *psum = (float *)(ws + L.psum);
+  float *py = (float *)(ws + L.py);
+  uint32_t *err = (uint32_t *)(ws + L.err);
+  uint32_t *count = (uint32_t *)(ws + L.count);
+  const float scale_log2 = 0.125f * kLog2e;   // log2(e) / sqrt(64)
+  const bool conv = conv_w != nullptr;
+  const int kconv = conv ? ((128 + conv_k - 1 + 15) / 16) * 16 : 0;
+
+  CUtensorMap mq, mkk, mv, mvh, mo;
+  if (!make_map(&mq, Q, BH, n, 128) || !make_map(&mkk, K, BH, n, 128) ||
+      !make_map(&mv, V, BH, n, 128) || !make_map(&mvh, V, BH, n, conv ? kconv : 128) ||
+      !make_map(&mo, out, BH, n, 128))
+    return NYS_ERR_CUDA;
+
+  {   // segment means of Q and K (Eq. 16)
+    const int seg = n / M;
+    const int groups = seg < 32 ? seg : 32;
+    seg_means_bf16<<<dim3(M, BH, 2), 8 * groups, 0, stream>>>(Q, K, qt, kt, n, M);
+    mk.after(stream);
+  }
+  {   // pseudoinverse || B~ V, then merge + W = Z Y
+    midtc::Params p;
+    p.pinv = pinvtc::Params{qt, kt, z, err, iters, scale_log2};
+    p.q_land = qt;
+    p.z = z;
+    p.pmax = pmax;
+    p.psum = psum;
+    p.py = py;
+    p.y = y;
+    p.w = w;
+    p.count = count;
+    p.err = err;
+    p.BH = BH;
+    p.n = n;
+    p.chunks_per_head = (n + midtc::kChunk - 1) / midtc::kChunk;
+    p.splits = L.splits;
+    p.scale_log2 = scale_log2;
+    auto kern = midtc::mid_kernel<M>;
+    const uint32_t sm = midtc::smem_bytes<M>();
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    kern<<<BH * (1 + L.splits), midtc::kThreads, sm, stream>>>(mkk, mv, p);
+    mk.after(stream);
+  }
+  {   // F~ W + DConv(V)
+    const int tph = (n + outtc::kTileRows - 1) / outtc::kTileRows;
+    int cpb = kNumSms / BH;
+    if (cpb < 1) cpb = 1;
+    if (cpb > tph) cpb = tph;
+    outtc::Params p{kt, w, conv_w, err, n, desc->heads, conv ? conv_k : 1, kconv, tph, cpb,
+                    scale_log2};
+    auto kern = outtc::out_tc_kernel<M>;
+    const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    kern<<<BH * cpb, outtc::kThreads, sm, stream>>>(mq, mvh, mo, p);
+    mk.after(stream);
+  }
+  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
+                     const nys_desc *desc, int m, int iters, const float *conv_w, int conv_k,
+                     __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
+                     Marks &mk) {
+  switch (m) {
+    case 32: return launch_tc_m<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+    case 64: return launch_tc_m<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+    case 128:
+      return launch_tc_m<128>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+  }
+  return NYS_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 extern "C" {
@@ -228,6 +368,9 @@ static nys_status validate_call(const void *Q, const void *K, const void *V,
   }
   if (is_empty(desc)) return NYS_OK;
   if (!Q || !K || !V || !out) return NYS_ERR_INVALID_ARG;
+  if (desc->dtype == NYS_BF16 &&
+      (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)out) & 15) != 0)
+    return NYS_ERR_INVALID_ARG;
   return NYS_OK;
 }
 
@@ -237,7 +380,8 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
                                nys_stream_t stream_, void *const *events, int n_events) {
   nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
   if (st != NYS_OK) return st;
-  if (events && n_events < kSimtLaunches + 1) return NYS_ERR_INVALID_ARG;
+  if (events && n_events < (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches) + 1)
+    return NYS_ERR_INVALID_ARG;
   if (is_empty(desc)) return NYS_OK;
   Marks mk;
   mk.ev = (cudaEvent_t const *)events;
@@ -260,16 +404,18 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (cudaMemsetAsync(ws + L.err, 0, 4, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.err, 0, 256 + (size_t)desc->batch * desc->heads * 4, stream) !=
+      cudaSuccess)
+    st = NYS_ERR_CUDA;
   if (mk.ev) cudaEventRecord(mk.ev[0], stream);
   if (st == NYS_OK) {
     if (desc->dtype == NYS_F32)
       st = launch_simt<float>((const float *)Q, (const float *)K, (const float *)V, desc, m,
                               iters, conv_w, conv_k, (float *)out, ws, L, stream, mk);
     else
-      st = launch_simt<__nv_bfloat16>((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
-                                      (const __nv_bfloat16 *)V, desc, m, iters, conv_w, conv_k,
-                                      (__nv_bfloat16 *)out, ws, L, stream, mk);
+      st = launch_tc((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                     (const __nv_bfloat16 *)V, desc, m, iters, conv_w, conv_k,
+                     (__nv_bfloat16 *)out, ws, L, stream, mk);
   }
   if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && st == NYS_OK) st = NYS_ERR_CUDA;
   return st;
@@ -392,7 +538,7 @@ NYS_ATTN_API nys_status nys_attn_launch_count(const nys_desc *desc, int m, int c
   if (!launches) return NYS_ERR_INVALID_ARG;
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  *launches = is_empty(desc) ? 0 : kSimtLaunches;
+  *launches = is_empty(desc) ? 0 : (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches);
   return NYS_OK;
 }
 
@@ -400,7 +546,7 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
                                               size_t names_bytes) {
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  const char *src = is_empty(desc) ? "" : kSimtNames;
+  const char *src = is_empty(desc) ? "" : (desc->dtype == NYS_BF16 ? kTcNames : kSimtNames);
   if (names) {
     if (names_bytes < strlen(src) + 1) return NYS_ERR_INVALID_ARG;
     strcpy(names, src);

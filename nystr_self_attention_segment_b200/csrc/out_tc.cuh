@@ -1,0 +1,312 @@
+// Output kernel of the bf16 path on 5th-generation tensor cores:
+//
+//   out[i] = softmax_m(s q_i . K~^T) W + sum_t w_h[t] V[i + t - (k-1)/2]
+//
+// ("Nystromformer: A Nystrom-Based Algorithm for Approximating
+// Self-Attention", section 3.4: Eq. 17 / Algorithm 1 for F~ W, Figure 4 for
+// the DConv skip).  W = Z (B~ V) comes from the workspace.
+//
+// A block owns a run of 128-row tiles of one (batch, head).  Per tile:
+//   TMA  Q tile (128 x 64 bf16) and the V tile with its conv halo
+//        (kconv = 128 + k - 1 rounded up to 16 rows; zero outside [0, n)),
+//   MMA  S = Q K~^T                 (M=128, N=m, K=64; operands in smem),
+//   MMA  O = T_h V_halo             (M=128, N=64, K=kconv; T_h in TMEM),
+//        T_h is the banded Toeplitz matrix of the head's conv kernel
+//        (T_h[r][j] = w_h[j - r]), so the depthwise conv runs on the tensor
+//        cores,
+//   softmax warpgroup: row softmax of S (one TMEM lane = one row); P (the F~
+//        tile, bf16) written into TMEM over S,
+//   MMA  O += P W                   (M=128, N=64, K=m; P read from TMEM),
+//   softmax warpgroup: O -> bf16 -> shared memory -> TMA store (clipped at n).
+// Two softmax warpgroups take alternate tiles.
+// Warps: 0 TMA producer, 1 MMA issuer / TMEM owner, 4-7 and 8-11 softmax +
+// epilogue.  TMEM: warpgroup w has S at w*(m+64) and O right after it; T_h
+// follows at 2*(m+64).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace nys {
+namespace outtc {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kStages = 3;
+constexpr int kTileRows = 128;
+constexpr int kMaxKconv = 192;
+
+struct SmemLayout {
+  uint32_t kt, w, q[kStages], v[kStages], o[2], cw, bars, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
+  SmemLayout L;
+  uint32_t off = 0;
+  auto take = [&](uint32_t b) {
+    uint32_t at = off;
+    off += (b + 1023u) & ~1023u;
+    return at;
+  };
+  L.kt = take(m * 128u);
+  L.w = take(m * 128u);
+  for (int s = 0; s < kStages; ++s) {
+    L.q[s] = take(16384u);
+    L.v[s] = take(kconv * 128u);
+  }
+  L.o[0] = take(16384u);
+  L.o[1] = take(16384u);
+  L.cw = take(256u);
+  L.bars = take(256u);
+  L.total = off + 1024u;   // slack for aligning the dynamic smem base to 1 KB
+  return L;
+}
+
+struct Params {
+  const float *k_land;     // [BH][m][64] fp32
+  const float *w;          // [BH][m][64] fp32
+  const float *conv_w;     // [H][k] or null
+  uint32_t *err;
+  int n, heads, conv_k, kconv;
+  int tiles_per_head, ctas_per_head;
+  float scale_log2;
+};
+
+template <int M>
+__global__ void __launch_bounds__(kThreads, 1)
+out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
+              const __grid_constant__ CUtensorMap map_o, const Params prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const SmemLayout L = smem_layout(M, prm.kconv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / prm.ctas_per_head;
+  const int part = blockIdx.x % prm.ctas_per_head;
+  const int head = bh % prm.heads;
+  const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
+  const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
+  const int ntiles = t_end - t_begin;
+  const bool conv = prm.conv_w != nullptr;
+  const int half = (prm.conv_k - 1) / 2;
+  constexpr uint32_t kStride = M + 64;        // TMEM columns per softmax warpgroup
+  constexpr uint32_t kT = 2 * kStride;        // Toeplitz operand columns
+
+  uint64_t *bars = (uint64_t *)(smem + L.bars);
+  uint64_t *full = bars;                   // [kStages]
+  uint64_t *empty = bars + kStages;        // [kStages]
+  uint64_t *s_full = bars + 2 * kStages;   // [2] per softmax warpgroup
+  uint64_t *p_ready = s_full + 2;
+  uint64_t *o_full = p_ready + 2;
+  uint64_t *tm_free = o_full + 2;
+  uint32_t *tmem_slot = (uint32_t *)(tm_free + 2);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+  const Abort ab{abort_flag, prm.err};
+  float *cw = (float *)(smem + L.cw);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_ready[b], 128);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&tm_free[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_o);
+    if (conv) tma_prefetch_desc(&map_v);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+
+  // ---- per-head operands: K~ (B of S, K-major) and W (B of P W, MN-major),
+  // bf16 with the 128-byte swizzle; all loads issued before the stores
+  {
+    const float4 *kt = (const float4 *)(prm.k_land + (size_t)bh * M * 64);
+    const float4 *wg = (const float4 *)(prm.w + (size_t)bh * M * 64);
+    constexpr int kItems = M * 8;           // 16-byte chunks (8 bf16) per operand
+    constexpr int kPer = (kItems + kThreads - 1) / kThreads;
+    float4 a[kPer][2], c[kPer][2];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * kThreads;
+      if (idx < kItems) {
+        a[u][0] = kt[2 * idx];
+        a[u][1] = kt[2 * idx + 1];
+        c[u][0] = wg[2 * idx];
+        c[u][1] = wg[2 * idx + 1];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * kThreads;
+      if (idx < kItems) {
+        const int row = idx >> 3, ch = idx & 7;
+        st_shared_v4(smem_u32(smem + L.kt) + sw128_offset(row, ch), pack_bf16(a[u][0].x, a[u][0].y),
+                     pack_bf16(a[u][0].z, a[u][0].w), pack_bf16(a[u][1].x, a[u][1].y),
+                     pack_bf16(a[u][1].z, a[u][1].w));
+        st_shared_v4(smem_u32(smem + L.w) + sw128_offset(row, ch), pack_bf16(c[u][0].x, c[u][0].y),
+                     pack_bf16(c[u][0].z, c[u][0].w), pack_bf16(c[u][1].x, c[u][1].y),
+                     pack_bf16(c[u][1].z, c[u][1].w));
+      }
+    }
+    if (conv && threadIdx.x < prm.conv_k) cw[threadIdx.x] = prm.conv_w[(size_t)head * prm.conv_k + threadIdx.x];
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // Toeplitz operand into TMEM: row r (lane r), columns j = halo rows
+  if (conv && warp >= 4 && warp < 8) {
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    for (int c0 = 0; c0 < prm.kconv / 2; c0 += 16) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int j0 = 2 * (c0 + e) - r, j1 = j0 + 1;
+        const float lo = (j0 >= 0 && j0 < prm.conv_k) ? cw[j0] : 0.f;
+        const float hi = (j1 >= 0 && j1 < prm.conv_k) ? cw[j1] : 0.f;
+        pk[e] = pack_bf16(lo, hi);
+      }
+      tmem_st16(tmem + lane_base + kT + c0, pk);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t bytes = 16384u + (conv ? (uint32_t)prm.kconv * 128u : 0u);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
+        const int r0 = (t_begin + i) * kTileRows;
+        mbar_expect_tx(&full[s], bytes);
+        tma_load_3d(smem + L.q[s], &map_q, &full[s], 0, r0, bh);
+        if (conv) tma_load_3d(smem + L.v[s], &map_v, &full[s], 0, r0 - half, bh);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(kFmtBF16, 128, M, 0, 0);
+      const uint32_t id_o = make_idesc(kFmtBF16, 128, 64, 0, 1);
+      const uint32_t kt_a = smem_u32(smem + L.kt), w_a = smem_u32(smem + L.w);
+      auto issue_pw = [&](int j) -> bool {
+        const int w = j & 1;
+        if (!mbar_wait(&p_ready[w], (j >> 1) & 1, ab)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < M / 16; ++k)
+          mma_bf16_ts(tmem + w * kStride + M, tmem + w * kStride + 8 * k,
+                      make_sdesc(w_a + k * 2048u, 16, 1024), id_o, (conv || k > 0) ? 1u : 0u);
+        mma_commit(&o_full[w]);
+        return true;
+      };
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int s = i % kStages, w = i & 1;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) break;
+        if (!mbar_wait(&tm_free[w], ((i >> 1) & 1) ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t q_a = smem_u32(smem + L.q[s]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem + w * kStride, make_sdesc(q_a + 32 * k, 16, 1024),
+                   make_sdesc(kt_a + 32 * k, 16, 1024), id_s, k > 0);
+        mma_commit(&s_full[w]);
+        if (conv) {
+          const uint32_t v_a = smem_u32(smem + L.v[s]);
+          for (int k = 0; k < prm.kconv / 16; ++k)
+            mma_bf16_ts(tmem + w * kStride + M, tmem + kT + 8 * k,
+                        make_sdesc(v_a + k * 2048u, 16, 1024), id_o, k > 0);
+        }
+        mma_commit(&empty[s]);
+        if (i > 0) ok = issue_pw(i - 1);
+      }
+      if (ok && ntiles > 0) issue_pw(ntiles - 1);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wg = warp >= 8 ? 1 : 0;
+    const int r = threadIdx.x & 127;                 // tile row == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + wg * kStride;
+    for (int i = wg; i < ntiles; i += 2) {
+      const int u = i >> 1;
+      if (!mbar_wait(&s_full[wg], u & 1, ab)) break;
+      tc_fence_after();
+      float v[M];
+#pragma unroll
+      for (int c = 0; c < M; c += 32) tmem_ld32(t_s + c, v + c);
+      tmem_ld_wait();
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = v[q];
+#pragma unroll
+      for (int c = 8; c < M; ++c) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+      const float moff = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         prm.scale_log2;
+      float ps[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < M; ++c) {
+        v[c] = fast_exp2(fmaf(v[c], prm.scale_log2, -moff));
+        ps[c & 7] += v[c];
+      }
+      const float inv =
+          1.f / (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+      uint32_t pk[M / 2];
+#pragma unroll
+      for (int c = 0; c < M; c += 2) pk[c >> 1] = pack_bf16(v[c] * inv, v[c + 1] * inv);
+#pragma unroll
+      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + c, pk + c);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[wg]);
+      if (!mbar_wait(&o_full[wg], u & 1, ab)) break;
+      tc_fence_after();
+      float o[64];
+      tmem_ld32(t_s + M, o);
+      tmem_ld32(t_s + M + 32, o + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&tm_free[wg]);
+      // this warpgroup's staging buffer was last used two of its tiles ago
+      if (r == 0) bulk_wait_read0();
+      named_barrier(2 + wg, 128);
+      const uint32_t o_row = smem_u32(smem + L.o[wg]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(o_row + sw128_offset(r, c), pack_bf16(o[8 * c], o[8 * c + 1]),
+                     pack_bf16(o[8 * c + 2], o[8 * c + 3]), pack_bf16(o[8 * c + 4], o[8 * c + 5]),
+                     pack_bf16(o[8 * c + 6], o[8 * c + 7]));
+      fence_async_smem();
+      named_barrier(2 + wg, 128);
+      if (r == 0) {
+        tma_store_3d(&map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh);
+        bulk_commit();
+      }
+    }
+    if (r == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace outtc
+}  // namespace nys
