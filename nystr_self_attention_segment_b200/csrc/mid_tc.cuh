@@ -21,7 +21,8 @@
 // Two softmax warpgroups take alternate chunks, each with its own TMEM
 // buffers and running state; the 2G states of a landmark are merged in the
 // block at the end, giving one partial per (block, landmark).
-// Warps: 0 TMA producer, 1 MMA issuer / TMEM owner, 4-7 and 8-11 softmax.
+// Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
+// warp 1 owns TMEM), 4-7 and 8-11 softmax.
 #pragma once
 
 #include "pinv_tc.cuh"
@@ -32,7 +33,7 @@ namespace midtc {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int kStages = 3;
+constexpr int kStages = 6;   // ~1.5 us of loads in flight per SM
 constexpr int kChunk = 128;
 
 struct BvSmem {
@@ -150,15 +151,43 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // one MMA issuer per softmax warpgroup, so that neither waits behind the
+    // other's next chunk
     if (lane == 0) {
+      const int w = warp - 1;
       const uint32_t id_s = make_idesc(kFmtBF16, 128, 128, 0, 0);
       const uint32_t id_y = make_idesc(kFmtBF16, 128, 64, 0, 1);
       const uint32_t q_a = smem_u32(smem + L.q);
-      auto issue_pv = [&](int j) -> bool {
-        const int w = j & 1, s = j % kStages, u = j >> 1;
-        if (!mbar_wait(&p_ready[w], u & 1, ab)) return false;
-        if (!mbar_wait(&y_free[w], (u & 1) ^ 1, ab)) return false;
+      // S of this warpgroup's next chunk is issued as soon as the warpgroup
+      // has read the previous S, ahead of the P V of the current chunk
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % kStages, u = i >> 1;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) return false;
+        if (!mbar_wait(&s_free[w], (u & 1) ^ 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t k_a = smem_u32(smem + L.k[s]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem + 256 * w, make_sdesc(q_a + 32 * k, 16, 1024),
+                   make_sdesc(k_a + 32 * k, 16, 1024), id_s, k > 0);
+        mma_commit(&s_full[w]);
+        return true;
+      };
+      bool ok = w < nch ? issue_s(w) : true;
+      for (int i = w; i < nch && ok; i += 2) {
+        const int s = i % kStages, u = i >> 1;
+        // next S early only if its chunk has landed and S is free; never
+        // hold this chunk's P V behind a load
+        const int nx = i + 2, un = nx >> 1;
+        bool s_done = false;
+        if (nx < nch && mbar_ready(&full[nx % kStages], (nx / kStages) & 1) &&
+            mbar_ready(&s_free[w], (un & 1) ^ 1)) {
+          if (!(ok = issue_s(nx))) break;
+          s_done = true;
+        }
+        if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
+        if (!mbar_wait(&y_free[w], (u & 1) ^ 1, ab)) break;
         tc_fence_after();
         const uint32_t v_a = smem_u32(smem + L.v[s]);
 #pragma unroll
@@ -167,23 +196,8 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
                       make_sdesc(v_a + k * 2048u, 16, 1024), id_y, k > 0);
         mma_commit(&y_full[w]);
         mma_commit(&empty[s]);
-        return true;
-      };
-      bool ok = true;
-      for (int i = 0; i < nch && ok; ++i) {
-        const int s = i % kStages, w = i & 1, u = i >> 1;
-        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) break;
-        if (!mbar_wait(&s_free[w], (u & 1) ^ 1, ab)) break;
-        tc_fence_after();
-        const uint32_t k_a = smem_u32(smem + L.k[s]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tmem + 256 * w, make_sdesc(q_a + 32 * k, 16, 1024),
-                   make_sdesc(k_a + 32 * k, 16, 1024), id_s, k > 0);
-        mma_commit(&s_full[w]);
-        if (i > 0) ok = issue_pv(i - 1);
+        if (nx < nch && !s_done && !(ok = issue_s(nx))) break;
       }
-      if (ok && nch > 0) issue_pv(nch - 1);
     }
   }
   // softmax warpgroups; their running states are kept for the merge below
@@ -309,67 +323,115 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 
 // ------------------------------------------------------------------ merge + W
 // Y = sum_s f_s py_s / sum_s f_s psum_s with f_s = 2^(pmax_s - max), over the
-// S partials of the head in order; then W = Z Y.  All threads of the block.
+// S partials of the head in order; then W = Z Y.  All 384 threads; every
+// global load of a phase is issued before its results are used.
 template <int M>
 __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh) {
-  const int t = threadIdx.x, nt = blockDim.x;
+  const int t = threadIdx.x;
+  constexpr int NT = kThreads;
   const int S = prm.splits;
+  constexpr int ZL = M + 4;           // padded row of Z
   float *zs = (float *)smem;          // [M][M + 4]
-  constexpr int ZL = M + 4;
   float *ys = zs + M * ZL;            // [M][64]
   float *wgt = ys + M * 64;           // [S][M]
-  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
-  for (int i = t; i < M * M / 4; i += nt) {
-    const float4 v = __ldcg(z4 + i);
-    const int row = (i * 4) / M, col = (i * 4) % M;
-    *(float4 *)(zs + row * ZL + col) = v;
+  float *psm = wgt + S * M;           // [S][M]
+  float *den = psm + S * M;           // [M]
+  float *part = den + M;              // [2][M / 4 * 16][16]: k-half partial sums of W
+  {
+    constexpr int kZ4 = M * M / 4;
+    constexpr int kPer = (kZ4 + NT - 1) / NT;
+    const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
+    float4 v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u)
+      if (t + u * NT < kZ4) v[u] = __ldcg(z4 + t + u * NT);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = t + u * NT;
+      if (i < kZ4) *(float4 *)(zs + (i * 4 / M) * ZL + (i * 4) % M) = v[u];
+    }
   }
   const size_t pb = (size_t)bh * S * M;
-  for (int i = t; i < S * M; i += nt) wgt[i] = __ldcg(prm.pmax + pb + i);
+  for (int i = t; i < S * M; i += NT) {
+    const float a = __ldcg(prm.pmax + pb + i), b = __ldcg(prm.psum + pb + i);
+    wgt[i] = a;
+    psm[i] = b;
+  }
   __syncthreads();
   if (t < M) {
     float mx = -INFINITY;
     for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
-    float den = 0.f;
+    float d = 0.f;
     for (int s = 0; s < S; ++s) {
       const float f = fast_exp2(wgt[s * M + t] - mx);
       wgt[s * M + t] = f;
-      den = fmaf(__ldcg(prm.psum + pb + (size_t)s * M + t), f, den);
+      d = fmaf(psm[s * M + t], f, d);
     }
-    const float inv = 1.f / den;
-    for (int s = 0; s < S; ++s) wgt[s * M + t] *= inv;
+    den[t] = 1.f / d;
   }
   __syncthreads();
-  for (int idx = t; idx < M * 16; idx += nt) {
-    const int j = idx >> 4;
-    const float4 *src = (const float4 *)(prm.py + (pb + j) * 64) + (idx & 15);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  // Y: item = (landmark, 4 features); each thread takes up to 3 items per
+  // round and issues all their partial loads before accumulating them in
+  // partial order
+  constexpr int kIpt = 3;
+  for (int base = 0; base < M * 16; base += NT * kIpt) {
+    float4 a[kIpt];
+#pragma unroll
+    for (int q = 0; q < kIpt; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < S; s0 += 8) {
-      float4 v[8];
+      float4 v[kIpt][8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (s0 + u < S) v[u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
+      for (int q = 0; q < kIpt; ++q) {
+        const int idx = base + q * NT + t;
+        if (idx < M * 16) {
+          const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (s0 + u < S) {
-          const float f = wgt[(s0 + u) * M + j];
-          a.x = fmaf(f, v[u].x, a.x);
-          a.y = fmaf(f, v[u].y, a.y);
-          a.z = fmaf(f, v[u].z, a.z);
-          a.w = fmaf(f, v[u].w, a.w);
+          for (int u = 0; u < 8; ++u)
+            if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
         }
+      }
+#pragma unroll
+      for (int q = 0; q < kIpt; ++q) {
+        const int idx = base + q * NT + t;
+        if (idx < M * 16) {
+          const int j = idx >> 4;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (s0 + u < S) {
+              const float f = wgt[(s0 + u) * M + j];
+              a[q].x = fmaf(f, v[q][u].x, a[q].x);
+              a[q].y = fmaf(f, v[q][u].y, a[q].y);
+              a[q].z = fmaf(f, v[q][u].z, a[q].z);
+              a[q].w = fmaf(f, v[q][u].w, a[q].w);
+            }
+        }
+      }
     }
-    ((float4 *)ys)[idx] = a;
-    ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = a;
+#pragma unroll
+    for (int q = 0; q < kIpt; ++q) {
+      const int idx = base + q * NT + t;
+      if (idx < M * 16) {
+        const float inv = den[idx >> 4];
+        const float4 y = make_float4(a[q].x * inv, a[q].y * inv, a[q].z * inv, a[q].w * inv);
+        ((float4 *)ys)[idx] = y;
+        ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = y;
+      }
+    }
   }
   __syncthreads();
-  // W = Z Y: work item = (4 rows, 4 features)
-  for (int item = t; item < (M / 4) * 16; item += nt) {
+  // W = Z Y.  Work item = (4 rows, 4 features, half of k): M / 4 * 16 * 2
+  // items (M = 64: 512) over 384 threads; the two k halves are added in
+  // order (first half + second half) through shared memory.
+  constexpr int kItems = (M / 4) * 16;
+  for (int it = t; it < 2 * kItems; it += NT) {
+    const int kh = it / kItems, item = it % kItems;
     const int c4 = item & 15, j0 = (item >> 4) * 4;
     float4 a[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < M; ++k) {
+    const int k0 = kh * (M / 2);
+#pragma unroll 4
+    for (int k = k0; k < k0 + M / 2; ++k) {
       const float4 yv = ((const float4 *)ys)[k * 16 + c4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -380,9 +442,18 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
         a[q].w = fmaf(zz, yv.w, a[q].w);
       }
     }
+    float4 *pp = (float4 *)(part + (size_t)(kh * kItems + item) * 16);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      ((float4 *)(prm.w + (size_t)bh * M * 64))[(j0 + q) * 16 + c4] = a[q];
+    for (int q = 0; q < 4; ++q) pp[q] = a[q];
+  }
+  __syncthreads();
+  for (int idx = t; idx < M * 16; idx += NT) {   // idx = row * 16 + c4
+    const int j = idx >> 4, c4 = idx & 15;
+    const int item = (j >> 2) * 16 + c4, q = j & 3;
+    const float4 lo = ((const float4 *)(part + (size_t)item * 16))[q];
+    const float4 hi = ((const float4 *)(part + (size_t)(kItems + item) * 16))[q];
+    ((float4 *)(prm.w + (size_t)bh * M * 64))[idx] =
+        make_float4(lo.x + hi.x, lo.y + hi.y, lo.z + hi.z, lo.w + hi.w);
   }
 }
 

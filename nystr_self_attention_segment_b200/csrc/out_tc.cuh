@@ -19,9 +19,9 @@
 //   MMA  O += P W                   (M=128, N=64, K=m; P read from TMEM),
 //   softmax warpgroup: O -> bf16 -> shared memory -> TMA store (clipped at n).
 // Two softmax warpgroups take alternate tiles.
-// Warps: 0 TMA producer, 1 MMA issuer / TMEM owner, 4-7 and 8-11 softmax +
-// epilogue.  TMEM: warpgroup w has S at w*(m+64) and O right after it; T_h
-// follows at 2*(m+64).
+// Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
+// warp 1 owns TMEM), 4-7 and 8-11 softmax + epilogue.  TMEM: warpgroup w has
+// S at w*(m+64) and O right after it; T_h follows at 2*(m+64).
 #pragma once
 
 #include "sm100.cuh"
@@ -32,7 +32,7 @@ namespace outtc {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kTileRows = 128;
 constexpr int kMaxKconv = 192;
 
@@ -194,28 +194,21 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         if (conv) tma_load_3d(smem + L.v[s], &map_v, &full[s], 0, r0 - half, bh);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // one per softmax warpgroup, so that neither waits behind the other
     if (lane == 0) {
+      const int w = warp - 1;
       const uint32_t id_s = make_idesc(kFmtBF16, 128, M, 0, 0);
       const uint32_t id_o = make_idesc(kFmtBF16, 128, 64, 0, 1);
       const uint32_t kt_a = smem_u32(smem + L.kt), w_a = smem_u32(smem + L.w);
-      auto issue_pw = [&](int j) -> bool {
-        const int w = j & 1;
-        if (!mbar_wait(&p_ready[w], (j >> 1) & 1, ab)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < M / 16; ++k)
-          mma_bf16_ts(tmem + w * kStride + M, tmem + w * kStride + 8 * k,
-                      make_sdesc(w_a + k * 2048u, 16, 1024), id_o, (conv || k > 0) ? 1u : 0u);
-        mma_commit(&o_full[w]);
-        return true;
-      };
-      bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int s = i % kStages, w = i & 1;
-        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) break;
-        if (!mbar_wait(&tm_free[w], ((i >> 1) & 1) ^ 1, ab)) break;
+      // S of the next tile goes out right after P W of the current one (the
+      // tensor pipe runs one issuer's MMAs in order, so it cannot overwrite
+      // P before P W has read it); only the conv into O waits for the
+      // epilogue to release O.
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % kStages;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) return false;
         tc_fence_after();
         const uint32_t q_a = smem_u32(smem + L.q[s]);
 #pragma unroll
@@ -223,6 +216,13 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           mma_bf16(tmem + w * kStride, make_sdesc(q_a + 32 * k, 16, 1024),
                    make_sdesc(kt_a + 32 * k, 16, 1024), id_s, k > 0);
         mma_commit(&s_full[w]);
+        return true;
+      };
+      bool ok = w < ntiles ? issue_s(w) : true;
+      for (int i = w; i < ntiles && ok; i += 2) {
+        const int s = i % kStages, u = i >> 1;
+        if (!mbar_wait(&tm_free[w], (u & 1) ^ 1, ab)) break;
+        tc_fence_after();
         if (conv) {
           const uint32_t v_a = smem_u32(smem + L.v[s]);
           for (int k = 0; k < prm.kconv / 16; ++k)
@@ -230,9 +230,15 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
                         make_sdesc(v_a + k * 2048u, 16, 1024), id_o, k > 0);
         }
         mma_commit(&empty[s]);
-        if (i > 0) ok = issue_pw(i - 1);
+        if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < M / 16; ++k)
+          mma_bf16_ts(tmem + w * kStride + M, tmem + w * kStride + 8 * k,
+                      make_sdesc(w_a + k * 2048u, 16, 1024), id_o, (conv || k > 0) ? 1u : 0u);
+        mma_commit(&o_full[w]);
+        if (i + 2 < ntiles) ok = issue_s(i + 2);
       }
-      if (ok && ntiles > 0) issue_pw(ntiles - 1);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue

@@ -1,5 +1,5 @@
 // Landmark kernel and iterative pseudoinverse on 5th-generation tensor cores
-// (tf32 inputs, fp32 accumulation in TMEM), one CTA per (batch, head).
+// (tf32 inputs, fp32 accumulation in TMEM), one block per (batch, head).
 //
 // "Nystromformer: A Nystrom-Based Algorithm for Approximating
 // Self-Attention", section 3.4, "Moore-Penrose Pseudoinverse Computation":
@@ -22,10 +22,20 @@
 // P_0 = A A^T / (||A||_1 ||A||_inf).  Equal to the printed recurrence in exact
 // arithmetic; only rounding differs (tf32 operands, fp32 accumulation).
 //
-// 128 threads; thread r owns accumulator row r (TMEM lane r) and writes that
-// row of the next operands.  Both operands are K-major with the 128-byte
-// swizzle (32 fp32 per swizzle row); B operands are written transposed
-// because an MN-major tf32 B operand reads as zero on this hardware.
+// Each stage is one full-width MMA batch (at N = 64 an MMA instruction costs
+// about as much as at N = 32, so products are not split); after it, two
+// threads per accumulator row (one column half each) turn the product into
+// the next operands.
+//
+// Operands are K-major with the 128-byte swizzle (32 fp32 per swizzle row);
+// B operands are written transposed (element (k, n) at row n) because an
+// MN-major tf32 B operand reads as zero on this hardware.  (X is symmetric
+// in exact arithmetic, but substituting its rows for its columns lets the
+// tf32 rounding asymmetry of P feed back through the iteration; the peaky
+// headline workload then misses 2e-2, so the transpose is exact.)
+//
+// Threads: 0..255; thread t owns accumulator row t % 128 (TMEM lane t % 128)
+// and column half t / 128 (m = 32 uses one half); thread 0 issues the MMAs.
 #pragma once
 
 #include "sm100.cuh"
@@ -35,10 +45,12 @@ namespace pinvtc {
 
 using namespace sm100;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
 template <int M>
 struct Cfg {
+  static constexpr int kHalves = M >= 64 ? 2 : 1;      // column halves
+  static constexpr int kCols = M / kHalves;            // columns per half
   static constexpr uint32_t kAop = (M / 32) * 16384u;   // 128 rows x M (K-major)
   static constexpr uint32_t kBop = (M / 32) * M * 128u; // M rows x M (K-major)
   static constexpr uint32_t kQop = 2 * 16384u;          // 128 rows x 64 features
@@ -75,8 +87,9 @@ __device__ __forceinline__ float to_tf32(float x) {
 }
 
 // byte offset of element (row, k) of a K-major operand with `slab`-byte slabs
-__device__ __forceinline__ uint32_t kmaj_off(uint32_t slab, int row, int k) {
-  return (uint32_t)(k >> 5) * slab + sw128_offset(row, (k & 31) >> 2) + (k & 3) * 4u;
+__host__ __device__ __forceinline__ uint32_t kmaj_off(uint32_t slab, int row, int k) {
+  return (uint32_t)(k >> 5) * slab + (uint32_t)row * 128u +
+         ((((uint32_t)(k & 31) >> 2) ^ ((uint32_t)row & 7u)) << 4) + (k & 3) * 4u;
 }
 
 // Row `row`, columns c0..c0+31 (c0 a multiple of 32) of a K-major operand.
@@ -88,6 +101,7 @@ __device__ __forceinline__ void put_kmaj32(uint32_t base, uint32_t slab, int row
                  __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
                  __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
 }
+
 // Row `k` of a matrix X, columns n0..n0+31, into the K-major B operand of X
 // (M rows of 128-byte swizzled slabs): element (k, n) goes to row n, column
 // k.  The 32 threads of a warp hold 32 consecutive k, so every store
@@ -101,21 +115,20 @@ __device__ __forceinline__ void put_bT32(uint32_t base, int k, int n0, const flo
                  "r"(__float_as_uint(v[e]))
                  : "memory");
 }
-__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return __uint_as_float(v);
-}
 
-// Runs on threads 0..127 of a block (4 warps, one per TMEM lane quarter);
-// synchronises them with named barrier 1 only, so other warps of the block
-// may do something else meanwhile.  smem: Cfg<M>::total bytes, 1 KB aligned.
-__device__ __forceinline__ void sync128() { named_barrier(1, 128); }
+// Runs on threads 0..255 of a block and synchronises them with named barrier
+// 1 only, so other warps of the block may do something else meanwhile.
+// smem: Cfg<M>::total bytes, 1 KB aligned.
+__device__ __forceinline__ void sync_pinv() { named_barrier(1, kThreads); }
 
 template <int M>
 __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int bh) {
   using C = Cfg<M>;
+  constexpr int NC = C::kCols;
   const int t = threadIdx.x, warp = t >> 5;
+  const int r = t & 127, h = t >> 7;                // accumulator row, column half
+  const bool active = h < C::kHalves;
+  const int c_lo = h * NC;                          // first column of this thread's half
   uint64_t *bar = (uint64_t *)(smem + C::bars);
   uint32_t *tmem_slot = (uint32_t *)(bar + 1);
   volatile uint32_t *abort_flag = tmem_slot + 1;
@@ -127,12 +140,12 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, C::kTmemCols);
-  sync128();
 
   const uint32_t aop = smem_u32(smem + C::aop), zop = smem_u32(smem + C::zop);
   const uint32_t bop = smem_u32(smem + C::bop);
   const uint32_t qh = smem_u32(smem + C::qh), ql = smem_u32(smem + C::ql);
   const uint32_t kh = smem_u32(smem + C::kh), kl = smem_u32(smem + C::kl);
+  const float *aop_f = (const float *)(smem + C::aop);
 
   // ---- landmarks -> hi/lo tf32 operands (all loads issued before the stores)
   {
@@ -174,16 +187,17 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
   }
   fence_async_smem();
   tc_fence_before();
-  sync128();
+  sync_pinv();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t idesc = make_idesc(kFmtTF32, 128, M, 0, 0);   // both operands K-major
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   uint32_t phase = 0;
 
-  // D (+)= A B^T over K = kk, A slabs of 16 KB (128 rows), B slabs of b_slab
+  // D (+)= A B^T over K = kk; A slabs of 16 KB (128 rows), B slabs of
+  // b_slab bytes; N = M columns
   auto issue = [&](uint32_t a_base, uint32_t d_col, uint32_t b_base, uint32_t b_slab, int kk,
                    bool acc0) {
+    const uint32_t idesc = make_idesc(kFmtTF32, 128, M, 0, 0);
     for (int k = 0; k < kk / 8; ++k) {
       const uint64_t ad = make_sdesc(a_base + (k >> 2) * 16384u + (k & 3) * 32u, 16, 1024);
       const uint64_t bd = make_sdesc(b_base + (k >> 2) * b_slab + (k & 3) * 32u, 16, 1024);
@@ -196,10 +210,12 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
     tc_fence_after();
     return done;
   };
+  // makes prior shared-memory operand writes visible to the tensor cores and
+  // synchronises the operand threads
   auto sync_operands = [&]() {
     fence_async_smem();
     tc_fence_before();
-    sync128();
+    sync_pinv();
     tc_fence_after();
   };
   auto ld32 = [&](uint32_t col, float *v) {
@@ -220,45 +236,46 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
   }
   bool ok = wait_mma();
   float *zg = prm.z_out + (size_t)bh * M * M;
-  // ---- row softmax in registers; A rows into the K-major operand
-  if (ok && t < M) {
+  // ---- row softmax in registers (one thread per row); A into the A operand
+  if (ok && h == 0 && r < M) {
     float v[M];
 #pragma unroll
     for (int c = 0; c < M; c += 32) tmem_ld32(tmem + lane_base + c, v + c);
     tmem_ld_wait();
-    float mx = -INFINITY;
+    float mx[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-    for (int j = 0; j < M; ++j) mx = fmaxf(mx, v[j]);
-    const float moff = mx * prm.scale_log2;
-    float s = 0.f;
+    for (int j = 4; j < M; ++j) mx[j & 3] = fmaxf(mx[j & 3], v[j]);
+    const float moff = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * prm.scale_log2;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < M; ++j) {
-      v[j] = exp2f(fmaf(v[j], prm.scale_log2, -moff));
-      s += v[j];
+      v[j] = fast_exp2(fmaf(v[j], prm.scale_log2, -moff));
+      s[j & 3] += v[j];
     }
-    const float inv = 1.f / s;
-    float rs = 0.f;
+    const float inv = 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < M; ++j) {
       v[j] *= inv;
-      rs += fabsf(v[j]);
+      rs[j & 3] += fabsf(v[j]);
     }
-    red[M + t] = rs;
+    red[M + r] = (rs[0] + rs[1]) + (rs[2] + rs[3]);
 #pragma unroll
-    for (int c = 0; c < M; c += 32) put_kmaj32(aop, 16384u, t, c, v + c);
+    for (int c = 0; c < M; c += 32) put_kmaj32(aop, 16384u, r, c, v + c);
   }
   if (M < 128)   // A-operand rows M..127 are zero (they also pad P)
     for (int idx = t; idx < (128 - M) * (M / 4); idx += kThreads) {
       const int row = M + idx / (M / 4), k = (idx % (M / 4)) * 4;
       st_shared_v4(aop + kmaj_off(16384u, row, k), 0, 0, 0, 0);
     }
-  sync128();
+  sync_pinv();
   if (t < M) {   // column sums: a warp reads 32 consecutive columns of one row
-    float cs = 0.f;
-    for (int i = 0; i < M; ++i) cs += fabsf(ld_shared_f32(aop + kmaj_off(16384u, i, t)));
-    red[t] = cs;
+    float cs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int i = 0; i < M; ++i) cs[i & 3] += fabsf(aop_f[kmaj_off(16384u, i, t) >> 2]);
+    red[t] = (cs[0] + cs[1]) + (cs[2] + cs[3]);
   }
-  sync128();
+  sync_pinv();
   float n1 = 0.f, ninf = 0.f;
   for (int i = 0; i < M; ++i) {
     n1 = fmaxf(n1, red[i]);
@@ -267,8 +284,10 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
   const float c0 = 1.f / (n1 * ninf);
 
   if (prm.iters == 0) {   // Z = Z0 = c0 A^T
-    if (t < M)
-      for (int j = 0; j < M; ++j) zg[(size_t)t * M + j] = c0 * ld_shared_f32(aop + kmaj_off(16384u, j, t));
+    for (int idx = t; idx < M * M; idx += kThreads) {
+      const int i = idx / M, j = idx % M;
+      zg[idx] = c0 * aop_f[kmaj_off(16384u, j, i) >> 2];
+    }
   } else if (ok) {
     const uint32_t z_a = M == 128 ? zop : aop;   // Z rows: own buffer, or rows M.. of aop
     const int z_row0 = M == 128 ? 0 : M;
@@ -281,54 +300,43 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
     ok = wait_mma();
     // Z0 rows (c0 times the columns of A); A stays in rows 0..M-1 until P0
     // replaces it below, after this barrier
-    if (ok && t < M)
-      for (int cb = 0; cb < M; cb += 32) {
+    if (ok && active && r < M)
+      for (int cb = c_lo; cb < c_lo + NC; cb += 32) {
         float v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = c0 * ld_shared_f32(aop + kmaj_off(16384u, cb + e, t));
-        put_kmaj32(z_a, 16384u, z_row0 + t, cb, v);
+        for (int e = 0; e < 32; ++e) v[e] = c0 * aop_f[kmaj_off(16384u, cb + e, r) >> 2];
+        put_kmaj32(z_a, 16384u, z_row0 + r, cb, v);
       }
-    sync128();
-    if (ok && t < M)   // P0 rows and X1 = 7I - P0
-      for (int cb = 0; cb < M; cb += 32) {
+    sync_pinv();
+    if (ok && active && r < M)   // P0 rows and X1 = 7I - P0
+      for (int cb = c_lo; cb < c_lo + NC; cb += 32) {
         float v[32];
         ld32(cb, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] *= c0;
-        put_kmaj32(aop, 16384u, t, cb, v);
-        diag_minus(v, cb, t, 7.f);
-        put_bT32<M>(bop, t, cb, v);
+        put_kmaj32(aop, 16384u, r, cb, v);
+        diag_minus(v, cb, r, 7.f);
+        put_bT32<M>(bop, r, cb, v);
       }
     for (int it = 0; it < prm.iters && ok; ++it) {
       const bool last = it + 1 == prm.iters;
-      // T2 = P X1  ->  X3 = 15I - T2
-      sync_operands();
-      if (t == 0) {
-        issue(aop, 0, bop, M * 128u, M, false);
-        mma_commit(bar);
-      }
-      if (!(ok = wait_mma())) break;
-      if (t < M)
-        for (int cb = 0; cb < M; cb += 32) {
-          float v[32];
-          ld32(cb, v);
-          diag_minus(v, cb, t, 15.f);
-          put_bT32<M>(bop, t, cb, v);
+      // T2 = P X1  ->  X3 = 15I - T2 ;  T4 = P X3  ->  X5 = 13I - T4
+      for (int stage = 0; stage < 2 && ok; ++stage) {
+        sync_operands();
+        if (t == 0) {
+          issue(aop, 0, bop, M * 128u, M, false);
+          mma_commit(bar);
         }
-      // T4 = P X3  ->  X5 = 13I - T4
-      sync_operands();
-      if (t == 0) {
-        issue(aop, 0, bop, M * 128u, M, false);
-        mma_commit(bar);
+        if (!(ok = wait_mma())) break;
+        if (active && r < M)
+          for (int cb = c_lo; cb < c_lo + NC; cb += 32) {
+            float v[32];
+            ld32(cb, v);
+            diag_minus(v, cb, r, stage == 0 ? 15.f : 13.f);
+            put_bT32<M>(bop, r, cb, v);
+          }
       }
-      if (!(ok = wait_mma())) break;
-      if (t < M)
-        for (int cb = 0; cb < M; cb += 32) {
-          float v[32];
-          ld32(cb, v);
-          diag_minus(v, cb, t, 13.f);
-          put_bT32<M>(bop, t, cb, v);
-        }
+      if (!ok) break;
       // [P'; Z'] = 1/4 [P; Z] X5
       sync_operands();
       if (t == 0) {
@@ -338,39 +346,39 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
       }
       if (!(ok = wait_mma())) break;
       if (M <= 64) {
-        if (t < 2 * M)
-          for (int cb = 0; cb < M; cb += 32) {
+        if (active && r < 2 * M)
+          for (int cb = c_lo; cb < c_lo + NC; cb += 32) {
             float v[32];
             ld32(cb, v);
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= 0.25f;
-            if (t >= M && last) {
-              float4 *dst = (float4 *)(zg + (size_t)(t - M) * M + cb);
+            if (r >= M && last) {
+              float4 *dst = (float4 *)(zg + (size_t)(r - M) * M + cb);
 #pragma unroll
               for (int q = 0; q < 8; ++q)
                 dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
-            put_kmaj32(aop, 16384u, t, cb, v);
-            if (t < M) {
-              diag_minus(v, cb, t, 7.f);
-              put_bT32<M>(bop, t, cb, v);
+            put_kmaj32(aop, 16384u, r, cb, v);
+            if (r < M) {
+              diag_minus(v, cb, r, 7.f);
+              put_bT32<M>(bop, r, cb, v);
             }
           }
       } else {
-        for (int cb = 0; cb < M; cb += 32) {
+        for (int cb = c_lo; cb < c_lo + NC; cb += 32) {
           float v[32];
           ld32(cb, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= 0.25f;
-          put_kmaj32(aop, 16384u, t, cb, v);
-          diag_minus(v, cb, t, 7.f);
-          put_bT32<M>(bop, t, cb, v);
+          put_kmaj32(aop, 16384u, r, cb, v);
+          diag_minus(v, cb, r, 7.f);
+          put_bT32<M>(bop, r, cb, v);
           ld32(128 + cb, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= 0.25f;
-          put_kmaj32(zop, 16384u, t, cb, v);
+          put_kmaj32(zop, 16384u, r, cb, v);
           if (last) {
-            float4 *dst = (float4 *)(zg + (size_t)t * M + cb);
+            float4 *dst = (float4 *)(zg + (size_t)r * M + cb);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -380,18 +388,11 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
     }
   }
   tc_fence_before();
-  sync128();
+  sync_pinv();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
-}
-
-template <int M>
-__global__ void __launch_bounds__(kThreads, 1) pinv_tc_kernel(const Params prm) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  pinv_body<M>(prm, smem, blockIdx.x);
 }
 
 }  // namespace pinvtc
