@@ -106,11 +106,23 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 // Records events[i + 1] after the i-th kernel when the caller asked for
 // per-kernel timing.
+// Inside a stream capture the records become external event nodes of the
+// graph, so that a replayed graph still times every kernel.
 struct Marks {
   cudaEvent_t const *ev = nullptr;
   int n = 0, next = 1;
+  static void record(cudaEvent_t e, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else
+      cudaEventRecord(e, s);
+  }
+  void first(cudaStream_t s) {
+    if (ev) record(ev[0], s);
+  }
   void after(cudaStream_t s) {
-    if (ev && next < n) cudaEventRecord(ev[next++], s);
+    if (ev && next < n) record(ev[next++], s);
   }
 };
 
@@ -407,7 +419,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
   if (cudaMemsetAsync(ws + L.err, 0, 256 + (size_t)desc->batch * desc->heads * 4, stream) !=
       cudaSuccess)
     st = NYS_ERR_CUDA;
-  if (mk.ev) cudaEventRecord(mk.ev[0], stream);
+  mk.first(stream);
   if (st == NYS_OK) {
     if (desc->dtype == NYS_F32)
       st = launch_simt<float>((const float *)Q, (const float *)K, (const float *)V, desc, m,
