@@ -26,8 +26,9 @@
  *  - Tensors Q, K, V, out are [batch][heads][seq_len][head_dim], contiguous,
  *    row-major, all of the dtype in the descriptor; out has the same dtype.
  *  - Pointers named *_dev are CUDA device pointers; *_host are host pointers.
- *    The caller owns every buffer; the library keeps no global mutable state
- *    and never frees caller memory.
+ *    The caller owns every buffer and the library never frees caller memory.
+ *    The only global mutable state is the fixed scratch array of
+ *    nys_attn_forward_static (used by that entry point alone).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and never synchronise the device.  Arguments are validated on the
  *    host before anything is enqueued: an invalid call returns a status and
@@ -174,6 +175,39 @@ NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q_dev, const void *K_
                                                void *out_dev, void *workspace_dev,
                                                size_t workspace_bytes, nys_stream_t stream,
                                                void *const *events, int n_events);
+
+/* Size of the fixed device scratch array nys_attn_forward_static uses. */
+#define NYS_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* nys_attn_forward without any device allocation: for callers that cannot
+ * allocate device memory -- hosts that own the whole device memory pool and
+ * forbid side allocations, paths where cudaMalloc's implicit device
+ * synchronisation is not acceptable, code held to a memory budget fixed at
+ * start-up.  (The paper has no counterpart; this is a deployment variant.)
+ *
+ * The scratch the forward needs (landmarks, Z, B~ V partials, W, error word
+ * and counters) lives in one file-scope __device__ array of
+ * NYS_STATIC_SCRATCH_BYTES in this library; every device that loads the
+ * library holds it until the process exits.  The caller still passes the
+ * inputs and the output (same arguments and layout as nys_attn_forward,
+ * without the workspace).
+ *  - A problem whose workspace (nys_attn_workspace_size) exceeds
+ *    NYS_STATIC_SCRATCH_BYTES is rejected with NYS_ERR_WORKSPACE before
+ *    anything is enqueued.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last
+ *    call's contents (the intermediates of nys_attn_intermediates, at the
+ *    same offsets); what must start at zero is cleared by each call.  Calls
+ *    that overlap on the GPU (different streams, or host threads without
+ *    ordering) race on the array: order them.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
+NYS_ATTN_API nys_status nys_attn_forward_static(const void *Q_dev, const void *K_dev,
+                                                const void *V_dev, const nys_desc *desc,
+                                                int num_landmarks, int pinv_iters,
+                                                const float *conv_w_dev, int conv_k,
+                                                void *out_dev, nys_stream_t stream);
 
 /* Number of kernel launches one nys_attn_forward call enqueues for this
  * shape (0 for an empty problem), and a short name for each launch in

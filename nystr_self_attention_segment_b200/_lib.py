@@ -38,7 +38,11 @@ EXPORTS = (
     "nys_attn_launch_count",
     "nys_attn_forward_timed",
     "nys_attn_launch_names",
+    "nys_attn_forward_static",
 )
+
+# Size of the fixed scratch array of nys_attn_forward_static (see the header).
+NYS_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class NysError(RuntimeError):
@@ -97,6 +101,8 @@ def load():
                                            ctypes.POINTER(P), I]
     lib.nys_attn_launch_names.restype = I
     lib.nys_attn_launch_names.argtypes = [D, I, ctypes.c_char_p, S]
+    lib.nys_attn_forward_static.restype = I
+    lib.nys_attn_forward_static.argtypes = [P, P, P, D, I, I, P, I, P, P]
     _LIB = lib
     return lib
 
@@ -177,6 +183,14 @@ def raw_forward_host(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_
                                         int(num_landmarks), int(pinv_iters), conv_ptr,
                                         int(conv_k), out_ptr, dbuf_ptr,
                                         ctypes.c_size_t(dbuf_bytes), stream_ptr)
+
+
+def raw_forward_static(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_ptr, conv_k,
+                       out_ptr, stream_ptr):
+    """nys_attn_forward_static: no workspace, no allocation."""
+    return load().nys_attn_forward_static(q_ptr, k_ptr, v_ptr, ctypes.byref(desc),
+                                          int(num_landmarks), int(pinv_iters), conv_ptr,
+                                          int(conv_k), out_ptr, stream_ptr)
 
 
 def raw_check_error(ws_ptr, desc, num_landmarks, stream_ptr):

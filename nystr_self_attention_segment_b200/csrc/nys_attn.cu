@@ -6,6 +6,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
@@ -440,6 +442,54 @@ NYS_ATTN_API nys_status nys_attn_forward(const void *Q, const void *K, const voi
                                          nys_stream_t stream) {
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
                       stream, nullptr, 0);
+}
+
+// ---------------------------------------------------------------------------
+// nys_attn_forward_static: the forward with its scratch in a fixed device
+// array instead of a caller-provided or stream-ordered workspace, for callers
+// that cannot allocate device memory (see the header).  The array lives in
+// this library's module: every device that loads the library holds it until
+// the process exits.  Host code cannot pass the array's name to a kernel (on
+// the host it is only a stand-in for the symbol), so its device address is
+// looked up with cudaGetSymbolAddress once per device, on that device's first
+// call, with that device current.
+static __device__ __align__(256) unsigned char g_static_scratch[NYS_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void *g_static_addr[kMaxDevices];            // device address per device, once resolved
+std::mutex g_static_mu;
+
+nys_status static_scratch(void **addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NYS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NYS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return NYS_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *addr = g_static_addr[dev];
+  return NYS_OK;
+}
+}  // namespace
+
+NYS_ATTN_API nys_status nys_attn_forward_static(const void *Q, const void *K, const void *V,
+                                                const nys_desc *desc, int m, int iters,
+                                                const float *conv_w, int conv_k, void *out,
+                                                nys_stream_t stream) {
+  nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) return NYS_OK;
+  if (make_layout(desc, m).total > (size_t)NYS_STATIC_SCRATCH_BYTES)
+    return NYS_ERR_WORKSPACE;   // the problem needs more scratch than the fixed array holds
+  void *ws = nullptr;
+  st = static_scratch(&ws);
+  if (st != NYS_OK) return st;
+  // the error word and the per-head counters are cleared by forward_impl
+  return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, ws,
+                      (size_t)NYS_STATIC_SCRATCH_BYTES, stream, nullptr, 0);
 }
 
 NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q, const void *K, const void *V,
