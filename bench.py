@@ -54,6 +54,26 @@ def peaks():
             "source": "fallback"}
 
 
+# ----------------------------------------------------------------- ranks
+
+def max_over_ranks(x, world, device):
+    """The max of a per-rank float over all ranks: one all-reduce, outside any
+    timed region (identity for a single process)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, ms_per_step):
+    """Whole-job tokens/s: every rank processes its own batch (weak scaling),
+    and the step takes as long as the slowest rank."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 def cpu_baseline(wl, seconds):
@@ -226,10 +246,7 @@ def run_ours(args, rank, world):
     total_ms = t_start.elapsed_time(t_end)
     per_kernel = [sum(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(K)) / K
                   for j in range(nl)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     # end to end through the host-buffer entry point (copies in the timed region)
     hb = nys.nys_attn_host_buffer_size(desc, m, wl.conv_k)
@@ -252,17 +269,14 @@ def run_ours(args, rank, world):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     if rank != 0:
         return None
     pk = peaks()
     ms = total_ms / K
     tokens = wl.tokens * world
-    value = tokens / (ms / 1e3)
+    value = job_throughput(wl.tokens, world, ms)
     # per-kernel algorithmic bytes (inputs read once + outputs written once)
     T = tensor_bytes
     kbytes = {"seg_means": 2 * T, "bv_partial": 2 * T, "out": 3 * T,
