@@ -25,6 +25,7 @@
 // warp 1 owns TMEM), 4-7 and 8-11 softmax.
 #pragma once
 
+#include "pinv_pow.cuh"
 #include "pinv_tc.cuh"
 
 namespace nys {
@@ -35,6 +36,7 @@ using namespace sm100;
 constexpr int kThreads = 384;
 constexpr int kStages = 6;   // ~1.5 us of loads in flight per SM
 constexpr int kChunk = 128;
+constexpr int kMaxSplits = 16;   // B~ V partials per head (bounds the merge scratch)
 
 struct BvSmem {
   uint32_t q, k[kStages], v[kStages], bars, total;
@@ -58,11 +60,36 @@ __host__ __device__ inline BvSmem bv_smem() {
 }
 
 template <int M>
+struct MergeCfg {
+  static constexpr int KS = M / 32;                       // 32-column slabs along K
+  static constexpr uint32_t kSlabA = 128u * 128u;         // Z: 128 rows x 32 fp32
+  static constexpr uint32_t kSlabB = 64u * 128u;          // Y^T: 64 feature rows x 32 fp32
+  static constexpr uint32_t zh = 0, zl = zh + KS * kSlabA;
+  static constexpr uint32_t yh = zl + KS * kSlabA, yl = yh + KS * kSlabB;
+  static constexpr uint32_t ys = zl;                      // Y staging [M][68] fp32 (over zl,
+                                                          // which is written after it is read)
+  static constexpr uint32_t wgt = yl + KS * kSlabB;       // [kMaxSplits][M] weights
+  static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
+  static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
+  static constexpr uint32_t bars = (den + M * 4u + 1023u) & ~1023u;
+  static constexpr uint32_t total = bars + 1024u;
+};
+
+template <int M>
+__host__ __device__ constexpr uint32_t pinv_smem() {
+  if constexpr (M <= 64) {
+    return pinvpow::Cfg<M>::total;
+  } else {
+    return pinvtc::Cfg<M>::total;
+  }
+}
+
+template <int M>
 __host__ __device__ constexpr uint32_t smem_bytes() {
   // pinv operands, B~ V buffers, and the merge scratch (Z, Y, weights)
-  return 1024u + (pinvtc::Cfg<M>::total > 16384u + kStages * 32768u + 1024u
-                      ? pinvtc::Cfg<M>::total
-                      : 16384u + kStages * 32768u + 1024u);
+  constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
+  constexpr uint32_t a = pinv_smem<M>() > bv ? pinv_smem<M>() : bv;
+  return 1024u + (a > MergeCfg<M>::total ? a : MergeCfg<M>::total);
 }
 
 struct Params {
@@ -78,9 +105,12 @@ struct Params {
 };
 
 // ------------------------------------------------------------------ B~ V body
+// tmem_in: a 512-column TMEM allocation owned by the caller, or ~0u to
+// allocate (and free) one here.
 template <int M>
 __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensorMap *map_v,
-                                        const Params &prm, uint8_t *smem, int bh, int split) {
+                                        const Params &prm, uint8_t *smem, int bh, int split,
+                                        uint32_t tmem_in) {
   constexpr int G = 128 / M;
   const BvSmem L = bv_smem();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,14 +147,18 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
     tma_prefetch_desc(map_k);
     tma_prefetch_desc(map_v);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (tmem_in != ~0u) {
+    if (threadIdx.x == 0) *tmem_slot = tmem_in;
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+  }
   // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
   if (threadIdx.x < 256) {
     const float4 *qt = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
     const int row = threadIdx.x >> 1, half = threadIdx.x & 1;   // 4 chunks each
     float4 a[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) a[u] = qt[(row % M) * 16 + half * 8 + u];
+    for (int u = 0; u < 8; ++u) a[u] = __ldcg(qt + (row % M) * 16 + half * 8 + u);
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       st_shared_v4(smem_u32(smem + L.q) + sw128_offset(row, half * 4 + u),
@@ -150,6 +184,10 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         tma_load_3d(smem + L.k[s], map_k, &full[s], 0, k0, bh);
         tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
       }
+      // consume the stage releases nobody else waits for, so that no
+      // tensor-core arrival is pending when the barriers are invalidated
+      for (int i = nch > kStages ? nch - kStages : 0; i < nch; ++i)
+        if (!mbar_wait(&empty[i % kStages], (i / kStages) & 1, ab)) break;
     }
   } else if (warp == 1 || warp == 2) {
     // one MMA issuer per softmax warpgroup, so that neither waits behind the
@@ -276,7 +314,9 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   }
   tc_fence_before();
   __syncthreads();   // pipeline drained: stage buffers are free for the merge
-  if (warp == 1) {
+  if (threadIdx.x == 0 && !*abort_flag)
+    for (int b = 0; b < 2 * kStages + 10; ++b) mbar_inval(bars + b);
+  if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -323,39 +363,82 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 
 // ------------------------------------------------------------------ merge + W
 // Y = sum_s f_s py_s / sum_s f_s psum_s with f_s = 2^(pmax_s - max), over the
-// S partials of the head in order; then W = Z Y.  All 384 threads; every
-// global load of a phase is issued before its results are used.
+// S partials of the head in order; then W = Z Y on the tensor cores as a
+// 3xTF32 product (Z hi*Y hi + Z hi*Y lo + Z lo*Y hi, about fp32 accuracy).
+// All 384 threads; every global load of a phase is issued before its results
+// are used.
+__device__ __forceinline__ uint32_t kmaj_f32(uint32_t slab, int row, int k) {
+  return (uint32_t)(k >> 5) * slab + sw128_offset(row, (k & 31) >> 2) + (k & 3) * 4u;
+}
+
+__device__ __forceinline__ float tf32_hi(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// tmem_in: a TMEM allocation of at least 64 columns owned by the caller, or
+// ~0u to allocate (and free) one here.
 template <int M>
-__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh) {
-  const int t = threadIdx.x;
+__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh,
+                                           uint32_t tmem_in) {
+  using C = MergeCfg<M>;
   constexpr int NT = kThreads;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int S = prm.splits;
-  constexpr int ZL = M + 4;           // padded row of Z
-  float *zs = (float *)smem;          // [M][M + 4]
-  float *ys = zs + M * ZL;            // [M][64]
-  float *wgt = ys + M * 64;           // [S][M]
-  float *psm = wgt + S * M;           // [S][M]
-  float *den = psm + S * M;           // [M]
-  float *part = den + M;              // [2][M / 4 * 16][16]: k-half partial sums of W
-  {
-    constexpr int kZ4 = M * M / 4;
-    constexpr int kPer = (kZ4 + NT - 1) / NT;
-    const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
-    float4 v[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u)
-      if (t + u * NT < kZ4) v[u] = __ldcg(z4 + t + u * NT);
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = t + u * NT;
-      if (i < kZ4) *(float4 *)(zs + (i * 4 / M) * ZL + (i * 4) % M) = v[u];
-    }
+  float *wgt = (float *)(smem + C::wgt);
+  float *psm = (float *)(smem + C::psm);
+  float *ysm = (float *)(smem + C::ys);
+  float *den = (float *)(smem + C::den);
+  uint64_t *bar = (uint64_t *)(smem + C::bars);
+  uint32_t *tmem_slot = (uint32_t *)(bar + 1);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+  const Abort ab{abort_flag, prm.err};
+  const uint32_t zh = smem_u32(smem + C::zh), zl = smem_u32(smem + C::zl);
+  const uint32_t yh = smem_u32(smem + C::yh), yl = smem_u32(smem + C::yl);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  const size_t pb = (size_t)bh * S * M;
-  for (int i = t; i < S * M; i += NT) {
-    const float a = __ldcg(prm.pmax + pb + i), b = __ldcg(prm.psum + pb + i);
-    wgt[i] = a;
-    psm[i] = b;
+  if (tmem_in != ~0u) {
+    if (t == 0) *tmem_slot = tmem_in;
+  } else if (warp == 0) {
+    tmem_alloc(tmem_slot, 64);
+  }
+  // Z rows (issued now for m <= 64, held in registers; written into the hi /
+  // lo K-major tf32 operands after Y, whose staging buffer overlays zl)
+  constexpr int kZ4 = M * M / 4;
+  constexpr int kZPer = (kZ4 + NT - 1) / NT;
+  constexpr bool kZEarly = M <= 64;
+  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
+  float4 zv[kZEarly ? kZPer : 1];
+  if constexpr (kZEarly) {
+#pragma unroll
+    for (int u = 0; u < kZPer; ++u)
+      if (t + u * NT < kZ4) zv[u] = __ldcg(z4 + t + u * NT);
+  }
+  auto put_z = [&](int i, float4 v) {
+    const int row = (i * 4) / M, k = (i * 4) % M;
+    const float x[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float h = tf32_hi(x[e]);
+      hi[e] = __float_as_uint(h);
+      lo[e] = __float_as_uint(tf32_hi(x[e] - h));
+    }
+    const uint32_t off = kmaj_f32(C::kSlabA, row, k);
+    st_shared_v4(zh + off, hi[0], hi[1], hi[2], hi[3]);
+    st_shared_v4(zl + off, lo[0], lo[1], lo[2], lo[3]);
+  };
+  // partial maxima and sums -> smem
+  {
+    const size_t pb = (size_t)bh * S * M;
+    for (int i = t; i < S * M; i += NT) {
+      wgt[i] = __ldcg(prm.pmax + pb + i);
+      psm[i] = __ldcg(prm.psum + pb + i);
+    }
   }
   __syncthreads();
   if (t < M) {
@@ -363,18 +446,21 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
     for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
     float d = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float f = fast_exp2(wgt[s * M + t] - mx);
+      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + t] - mx);
       wgt[s * M + t] = f;
       d = fmaf(psm[s * M + t], f, d);
     }
     den[t] = 1.f / d;
   }
   __syncthreads();
-  // Y: item = (landmark, 4 features); each thread takes up to 3 items per
-  // round and issues all their partial loads before accumulating them in
-  // partial order
+  // Y: item = (landmark j, 4 features); per round a thread takes up to kIpt
+  // items and loads their partials (in batches of 8) before summing them.
+  // Y goes to global memory (fp32) and, transposed, into the hi / lo B
+  // operands (element (k = landmark j, n = feature c) at row c, column j).
+  constexpr int kItems = M * 16;
   constexpr int kIpt = 3;
-  for (int base = 0; base < M * 16; base += NT * kIpt) {
+  const size_t pb = (size_t)bh * S * M;
+  for (int base = 0; base < kItems; base += NT * kIpt) {
     float4 a[kIpt];
 #pragma unroll
     for (int q = 0; q < kIpt; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -383,7 +469,7 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
 #pragma unroll
       for (int q = 0; q < kIpt; ++q) {
         const int idx = base + q * NT + t;
-        if (idx < M * 16) {
+        if (idx < kItems) {
           const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
@@ -393,7 +479,7 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
 #pragma unroll
       for (int q = 0; q < kIpt; ++q) {
         const int idx = base + q * NT + t;
-        if (idx < M * 16) {
+        if (idx < kItems) {
           const int j = idx >> 4;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
@@ -410,50 +496,80 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
 #pragma unroll
     for (int q = 0; q < kIpt; ++q) {
       const int idx = base + q * NT + t;
-      if (idx < M * 16) {
-        const float inv = den[idx >> 4];
+      if (idx < kItems) {
+        const int j = idx >> 4;
+        const float inv = den[j];
         const float4 y = make_float4(a[q].x * inv, a[q].y * inv, a[q].z * inv, a[q].w * inv);
-        ((float4 *)ys)[idx] = y;
         ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = y;
+        *(float4 *)(ysm + j * 68 + (idx & 15) * 4) = y;
       }
     }
   }
   __syncthreads();
-  // W = Z Y.  Work item = (4 rows, 4 features, half of k): M / 4 * 16 * 2
-  // items (M = 64: 512) over 384 threads; the two k halves are added in
-  // order (first half + second half) through shared memory.
-  constexpr int kItems = (M / 4) * 16;
-  for (int it = t; it < 2 * kItems; it += NT) {
-    const int kh = it / kItems, item = it % kItems;
-    const int c4 = item & 15, j0 = (item >> 4) * 4;
-    float4 a[4];
+  // Y^T into the hi / lo B operands: item = (feature c, 4 landmarks), one
+  // 16-byte store per operand (element (k = landmark, n = feature) at row c)
+  for (int it = t; it < 16 * M; it += NT) {
+    const int c = it & 63, j0 = (it >> 6) * 4;
+    uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int k0 = kh * (M / 2);
-#pragma unroll 4
-    for (int k = k0; k < k0 + M / 2; ++k) {
-      const float4 yv = ((const float4 *)ys)[k * 16 + c4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float zz = zs[(j0 + q) * ZL + k];
-        a[q].x = fmaf(zz, yv.x, a[q].x);
-        a[q].y = fmaf(zz, yv.y, a[q].y);
-        a[q].z = fmaf(zz, yv.z, a[q].z);
-        a[q].w = fmaf(zz, yv.w, a[q].w);
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float y = ysm[(j0 + e) * 68 + c];
+      const float h = tf32_hi(y);
+      hi[e] = __float_as_uint(h);
+      lo[e] = __float_as_uint(tf32_hi(y - h));
     }
-    float4 *pp = (float4 *)(part + (size_t)(kh * kItems + item) * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) pp[q] = a[q];
+    const uint32_t off = kmaj_f32(C::kSlabB, c, j0);
+    st_shared_v4(yh + off, hi[0], hi[1], hi[2], hi[3]);
+    st_shared_v4(yl + off, lo[0], lo[1], lo[2], lo[3]);
   }
+  __syncthreads();   // staging (over zl) consumed
+  if constexpr (kZEarly) {
+#pragma unroll
+    for (int u = 0; u < kZPer; ++u)
+      if (t + u * NT < kZ4) put_z(t + u * NT, zv[u]);
+  } else {
+    for (int i = t; i < kZ4; i += NT) put_z(i, __ldcg(z4 + i));
+  }
+  fence_async_smem();
+  tc_fence_before();
   __syncthreads();
-  for (int idx = t; idx < M * 16; idx += NT) {   // idx = row * 16 + c4
-    const int j = idx >> 4, c4 = idx & 15;
-    const int item = (j >> 2) * 16 + c4, q = j & 3;
-    const float4 lo = ((const float4 *)(part + (size_t)item * 16))[q];
-    const float4 hi = ((const float4 *)(part + (size_t)(kItems + item) * 16))[q];
-    ((float4 *)(prm.w + (size_t)bh * M * 64))[idx] =
-        make_float4(lo.x + hi.x, lo.y + hi.y, lo.z + hi.z, lo.w + hi.w);
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (t == 0) {
+    const uint32_t idesc = make_idesc(kFmtTF32, 128, 64, 0, 0);
+    // descriptors advance by 32 bytes (2 address units) per K step of 8 and by
+    // a slab per 4 steps
+    auto prod = [&](uint32_t A, uint32_t B, bool first) {
+      const uint64_t da = make_sdesc(A, 16, 1024), db = make_sdesc(B, 16, 1024);
+#pragma unroll
+      for (int k = 0; k < M / 8; ++k)
+        mma_tf32(tmem, da + (k >> 2) * (C::kSlabA >> 4) + (k & 3) * 2u,
+                 db + (k >> 2) * (C::kSlabB >> 4) + (k & 3) * 2u, idesc, (first && k == 0) ? 0u : 1u);
+    };
+    prod(zh, yh, true);
+    prod(zh, yl, false);
+    prod(zl, yh, false);
+    mma_commit(bar);
+  }
+  // W rows from TMEM: warp w reads lanes 32 (w % 4).. and columns 32 (w / 4)..
+  const int row = (warp & 3) * 32 + lane, cg = warp >> 2;
+  const bool reader = (warp & 3) * 32 < M && cg < 2;
+  if (reader && mbar_wait(bar, 0, ab)) {
+    tc_fence_after();
+    float w[32];
+    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + cg * 32, w);
+    tmem_ld_wait();
+    float4 *dst = (float4 *)(prm.w + ((size_t)bh * M + row) * 64 + cg * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      dst[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0 && !*abort_flag) mbar_inval(bar);
+  if (warp == 0 && tmem_in == ~0u) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 
@@ -463,15 +579,26 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
            const Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint32_t last;
+  __shared__ uint32_t last, tmem_base;
+  // one TMEM allocation for every body this block runs (an allocation
+  // relinquishes the block's permit to allocate again)
+  if ((threadIdx.x >> 5) == 1) tmem_alloc(&tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
   int bh;
   if ((int)blockIdx.x < prm.BH) {
     bh = blockIdx.x;
-    if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh);
+    if constexpr (M <= 64) {
+      if (threadIdx.x < pinvpow::kThreads) pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
+    } else {
+      if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
+    }
   } else {
     const int b = blockIdx.x - prm.BH;
     bh = b / prm.splits;
-    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits);
+    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem);
   }
   // publish this block's results, then count it; the last of the head's
   // S + 1 blocks merges
@@ -481,7 +608,13 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   __syncthreads();
   if (last) {
     __threadfence();
-    merge_body<M>(prm, smem, bh);
+    merge_body<M>(prm, smem, bh, tmem);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -60,6 +60,7 @@ Layout make_layout(const nys_desc *desc, int m) {
     int per_head = BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1;
     if (per_head < 1) per_head = 1;
     if (per_head > chunks) per_head = chunks;
+    if (per_head > midtc::kMaxSplits) per_head = midtc::kMaxSplits;
     L.bv_ctas_per_head = per_head;
     splits = per_head;
     L.keys_per_split = 0;

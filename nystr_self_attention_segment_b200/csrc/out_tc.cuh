@@ -72,19 +72,17 @@ struct Params {
   float scale_log2;
 };
 
+// One run of 128-row tiles [t_begin, t_end) of (batch, head) bh.  tmem_in: a
+// 512-column TMEM allocation owned by the caller, or ~0u to allocate (and
+// free) one here.  smem: smem_layout(M, kconv).total bytes, 1 KB aligned.
 template <int M>
-__global__ void __launch_bounds__(kThreads, 1)
-out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
-              const __grid_constant__ CUtensorMap map_o, const Params prm) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+__device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtensorMap *map_v,
+                                         const CUtensorMap *map_o, const Params &prm,
+                                         uint8_t *smem, int bh, int t_begin, int t_end,
+                                         uint32_t tmem_in) {
   const SmemLayout L = smem_layout(M, prm.kconv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / prm.ctas_per_head;
-  const int part = blockIdx.x % prm.ctas_per_head;
   const int head = bh % prm.heads;
-  const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
-  const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
   const int ntiles = t_end - t_begin;
   const bool conv = prm.conv_w != nullptr;
   const int half = (prm.conv_k - 1) / 2;
@@ -116,11 +114,15 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&map_q);
-    tma_prefetch_desc(&map_o);
-    if (conv) tma_prefetch_desc(&map_v);
+    tma_prefetch_desc(map_q);
+    tma_prefetch_desc(map_o);
+    if (conv) tma_prefetch_desc(map_v);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (tmem_in != ~0u) {
+    if (threadIdx.x == 0) *tmem_slot = tmem_in;
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+  }
 
   // ---- per-head operands: K~ (B of S, K-major) and W (B of P W, MN-major),
   // bf16 with the 128-byte swizzle; all loads issued before the stores
@@ -134,10 +136,10 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     for (int u = 0; u < kPer; ++u) {
       const int idx = threadIdx.x + u * kThreads;
       if (idx < kItems) {
-        a[u][0] = kt[2 * idx];
-        a[u][1] = kt[2 * idx + 1];
-        c[u][0] = wg[2 * idx];
-        c[u][1] = wg[2 * idx + 1];
+        a[u][0] = __ldcg(kt + 2 * idx);
+        a[u][1] = __ldcg(kt + 2 * idx + 1);
+        c[u][0] = __ldcg(wg + 2 * idx);
+        c[u][1] = __ldcg(wg + 2 * idx + 1);
       }
     }
 #pragma unroll
@@ -190,9 +192,13 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
         const int r0 = (t_begin + i) * kTileRows;
         mbar_expect_tx(&full[s], bytes);
-        tma_load_3d(smem + L.q[s], &map_q, &full[s], 0, r0, bh);
-        if (conv) tma_load_3d(smem + L.v[s], &map_v, &full[s], 0, r0 - half, bh);
+        tma_load_3d(smem + L.q[s], map_q, &full[s], 0, r0, bh);
+        if (conv) tma_load_3d(smem + L.v[s], map_v, &full[s], 0, r0 - half, bh);
       }
+      // consume the stage releases nobody else waits for (no tensor-core
+      // arrival may be pending when the barriers are invalidated)
+      for (int i = ntiles > kStages ? ntiles - kStages : 0; i < ntiles; ++i)
+        if (!mbar_wait(&empty[i % kStages], (i / kStages) & 1, ab)) break;
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
@@ -300,7 +306,7 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       fence_async_smem();
       named_barrier(2 + wg, 128);
       if (r == 0) {
-        tma_store_3d(&map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh);
+        tma_store_3d(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh);
         bulk_commit();
       }
     }
@@ -308,10 +314,25 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (threadIdx.x == 0 && !*abort_flag)
+    for (int b = 0; b < 2 * kStages + 8; ++b) mbar_inval(bars + b);
+  if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads, 1)
+out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
+              const __grid_constant__ CUtensorMap map_o, const Params prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int bh = blockIdx.x / prm.ctas_per_head;
+  const int part = blockIdx.x % prm.ctas_per_head;
+  const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
+  const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
+  out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u);
 }
 
 }  // namespace outtc

@@ -121,8 +121,11 @@ __device__ __forceinline__ void put_bT32(uint32_t base, int k, int n0, const flo
 // smem: Cfg<M>::total bytes, 1 KB aligned.
 __device__ __forceinline__ void sync_pinv() { named_barrier(1, kThreads); }
 
+// tmem_in: a TMEM allocation of at least Cfg<M>::kTmemCols columns owned by
+// the caller, or ~0u to allocate (and free) one here.
 template <int M>
-__device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int bh) {
+__device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int bh,
+                                          uint32_t tmem_in = ~0u) {
   using C = Cfg<M>;
   constexpr int NC = C::kCols;
   const int t = threadIdx.x, warp = t >> 5;
@@ -139,7 +142,11 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (tmem_in != ~0u) {
+    if (t == 0) *tmem_slot = tmem_in;
+  } else if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+  }
 
   const uint32_t aop = smem_u32(smem + C::aop), zop = smem_u32(smem + C::zop);
   const uint32_t bop = smem_u32(smem + C::bop);
@@ -389,7 +396,8 @@ __device__ __forceinline__ void pinv_body(const Params &prm, uint8_t *smem, int 
   }
   tc_fence_before();
   sync_pinv();
-  if (warp == 0) {
+  if (t == 0 && !*abort_flag) mbar_inval(bar);
+  if (warp == 0 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
