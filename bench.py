@@ -280,7 +280,7 @@ def run_ours(args, rank, world):
     # per-kernel algorithmic bytes (inputs read once + outputs written once)
     T = tensor_bytes
     kbytes = {"seg_means": 2 * T, "bv_partial": 2 * T, "out": 3 * T,
-              "mid_tc": 2 * T, "out_tc": 3 * T}
+              "mid_tc": 2 * T, "out_tc": 3 * T, "fused": 4 * T}
     dom = max(range(nl), key=lambda j: per_kernel[j])
     dname = names[dom] if dom < len(names) else "kernel%d" % dom
     dbytes = kbytes.get(dname)

@@ -105,6 +105,14 @@ struct Params {
 };
 
 // ------------------------------------------------------------------ B~ V body
+// Softmax over the keys with a lazily updated reference maximum: P =
+// 2^(s - m_ref) with m_ref raised only when a chunk's maximum exceeds it by
+// more than kTau (log2 units), so P <= 2^kTau and the Y accumulator (in TMEM,
+// summed by the P V MMAs) is rescaled only then.  The two softmax
+// warpgroups take turns through their exponential-heavy section (named
+// barriers 2 and 3), so one computes while the other waits on its MMAs.
+constexpr float kTau = 8.f;
+
 // tmem_in: a 512-column TMEM allocation owned by the caller, or ~0u to
 // allocate (and free) one here.
 template <int M>
@@ -125,8 +133,8 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   uint64_t *s_free = s_full + 2;
   uint64_t *p_ready = s_free + 2;
   uint64_t *y_full = p_ready + 2;
-  uint64_t *y_free = y_full + 2;
-  uint32_t *tmem_slot = (uint32_t *)(y_free + 2);
+  constexpr int kBars = 2 * kStages + 8;
+  uint32_t *tmem_slot = (uint32_t *)(bars + kBars);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
 
@@ -140,7 +148,6 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       mbar_init(&s_free[b], 128);
       mbar_init(&p_ready[b], 128);
       mbar_init(&y_full[b], 1);
-      mbar_init(&y_free[b], 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -190,59 +197,46 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         if (!mbar_wait(&empty[i % kStages], (i / kStages) & 1, ab)) break;
     }
   } else if (warp == 1 || warp == 2) {
-    // one MMA issuer per softmax warpgroup, so that neither waits behind the
-    // other's next chunk
+    // one MMA issuer per softmax warpgroup
     if (lane == 0) {
       const int w = warp - 1;
       const uint32_t id_s = make_idesc(kFmtBF16, 128, 128, 0, 0);
       const uint32_t id_y = make_idesc(kFmtBF16, 128, 64, 0, 1);
-      const uint32_t q_a = smem_u32(smem + L.q);
-      // S of this warpgroup's next chunk is issued as soon as the warpgroup
-      // has read the previous S, ahead of the P V of the current chunk
+      const uint64_t dq = make_sdesc(smem_u32(smem + L.q), 16, 1024);
       auto issue_s = [&](int i) -> bool {
-        const int s = i % kStages, u = i >> 1;
+        const int s = i % kStages;
         if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) return false;
-        if (!mbar_wait(&s_free[w], (u & 1) ^ 1, ab)) return false;
         tc_fence_after();
-        const uint32_t k_a = smem_u32(smem + L.k[s]);
+        const uint64_t dk = make_sdesc(smem_u32(smem + L.k[s]), 16, 1024);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_bf16(tmem + 256 * w, make_sdesc(q_a + 32 * k, 16, 1024),
-                   make_sdesc(k_a + 32 * k, 16, 1024), id_s, k > 0);
+          mma_bf16(tmem + 256 * w, dq + 2u * k, dk + 2u * k, id_s, k > 0);
         mma_commit(&s_full[w]);
         return true;
       };
       bool ok = w < nch ? issue_s(w) : true;
       for (int i = w; i < nch && ok; i += 2) {
         const int s = i % kStages, u = i >> 1;
-        // next S early only if its chunk has landed and S is free; never
-        // hold this chunk's P V behind a load
-        const int nx = i + 2, un = nx >> 1;
-        bool s_done = false;
-        if (nx < nch && mbar_ready(&full[nx % kStages], (nx / kStages) & 1) &&
-            mbar_ready(&s_free[w], (un & 1) ^ 1)) {
-          if (!(ok = issue_s(nx))) break;
-          s_done = true;
+        // the next S as soon as this warpgroup has read the current one
+        if (i + 2 < nch) {
+          if (!mbar_wait(&s_free[w], u & 1, ab)) break;
+          if (!(ok = issue_s(i + 2))) break;
         }
         if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
-        if (!mbar_wait(&y_free[w], (u & 1) ^ 1, ab)) break;
         tc_fence_after();
-        const uint32_t v_a = smem_u32(smem + L.v[s]);
+        const uint64_t dv = make_sdesc(smem_u32(smem + L.v[s]), 16, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          mma_bf16_ts(tmem + 256 * w + 192, tmem + 256 * w + 128 + 8 * k,
-                      make_sdesc(v_a + k * 2048u, 16, 1024), id_y, k > 0);
+          mma_bf16_ts(tmem + 256 * w + 192, tmem + 256 * w + 128 + 8 * k, dv + 128u * k, id_y,
+                      (u > 0 || k > 0) ? 1u : 0u);
         mma_commit(&y_full[w]);
         mma_commit(&empty[s]);
-        if (nx < nch && !s_done && !(ok = issue_s(nx))) break;
       }
     }
   }
   // softmax warpgroups; their running states are kept for the merge below
   float run_max = -INFINITY, run_sum = 0.f;
   float acc[64];
-#pragma unroll
-  for (int c = 0; c < 64; ++c) acc[c] = 0.f;
   const int wg = (warp >= 8) ? 1 : 0;
   const int r = threadIdx.x & 127;          // accumulator row == TMEM lane
   const int j = r % M, g = r / M;           // landmark, key group
@@ -257,9 +251,11 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       tmem_st32(t_s + 160, z);
       tmem_st_wait();
     }
-    for (int i = wg; i < nch; i += 2) {
-      const int u = i >> 1;
-      if (!mbar_wait(&s_full[wg], u & 1, ab)) break;
+    if (wg == 1 && nch > 0) named_barrier_arrive(2, 256);   // warpgroup 0 goes first
+    bool ok = true;
+    int u = 0;
+    for (int i = wg; i < nch; i += 2, ++u) {
+      if (!(ok = mbar_wait(&s_full[wg], u & 1, ab))) break;
       tc_fence_after();
       float v[M];
 #pragma unroll
@@ -269,53 +265,101 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       mbar_arrive(&s_free[wg]);
       const int key0 = (c_begin + i) * kChunk + g * M;
       const int valid = min(M, prm.n - key0);     // keys of this group inside [0, n)
+      named_barrier(2 + wg, 256);                  // this warpgroup's turn
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+      if (valid == M) {
 #pragma unroll
-      for (int c = 0; c < M; ++c)
-        if (c < valid) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+        for (int c = 0; c < M; ++c) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < M; ++c)
+          if (c < valid) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+      }
       const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float mnew = fmaxf(run_max, cmax * prm.scale_log2);
-      const bool none = (mnew == -INFINITY);
-      const float alpha = none ? 1.f : fast_exp2(run_max - mnew);
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         prm.scale_log2;
+      const bool up = cmax > run_max + kTau;
+      bool y_done = false;
+      if (__any_sync(0xffffffffu, up)) {
+        // raise the reference of the rows that need it and rescale their Y
+        // (warp-uniform: the TMEM accesses are warp-wide)
+        const float m_new = up ? cmax : run_max;
+        const float alpha = (run_max == -INFINITY) ? 0.f : fast_exp2(run_max - m_new);
+        if (u > 0) {
+          if (!(ok = mbar_wait(&y_full[wg], (u - 1) & 1, ab))) break;
+          tc_fence_after();
+          y_done = true;
+          float y[64];
+          tmem_ld32(t_s + 192, y);
+          tmem_ld32(t_s + 224, y + 32);
+          tmem_ld_wait();
+          uint32_t ys[64];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) ys[c] = __float_as_uint(y[c] * alpha);
+          tmem_st32(t_s + 192, ys);
+          tmem_st32(t_s + 224, ys + 32);
+          tmem_st_wait();
+        }
+        run_sum *= alpha;
+        run_max = m_new;
+      }
+      const float mref = run_max;
+      const bool none = (mref == -INFINITY);
       float ps[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) ps[q] = 0.f;
       uint32_t pk[M / 2];
+      if (valid == M && !none) {
 #pragma unroll
-      for (int c = 0; c < M; c += 2) {
-        const float p0 = (c < valid && !none) ? fast_exp2(fmaf(v[c], prm.scale_log2, -mnew)) : 0.f;
-        const float p1 =
-            (c + 1 < valid && !none) ? fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mnew)) : 0.f;
-        ps[(c >> 1) & 7] += p0 + p1;
-        pk[c >> 1] = pack_bf16(p0, p1);
+        for (int c = 0; c < M; c += 2) {
+          const float p0 = fast_exp2(fmaf(v[c], prm.scale_log2, -mref));
+          const float p1 = fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mref));
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < M; c += 2) {
+          const float p0 = (c < valid && !none) ? fast_exp2(fmaf(v[c], prm.scale_log2, -mref)) : 0.f;
+          const float p1 =
+              (c + 1 < valid && !none) ? fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mref)) : 0.f;
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
       }
-      const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      run_sum = run_sum * alpha + psum;
-      run_max = mnew;
+      run_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (i + 1 < nch) named_barrier_arrive(2 + (wg ^ 1), 256);   // the other's turn
+      // P is read by the previous P V of this warpgroup: wait for it
+      if (u > 0 && !y_done) {
+        if (!(ok = mbar_wait(&y_full[wg], (u - 1) & 1, ab))) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + 128 + g * (M / 2) + c, pk + c);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[wg]);
-      if (!mbar_wait(&y_full[wg], u & 1, ab)) break;
-      tc_fence_after();
-      float y[64];
-      tmem_ld32(t_s + 192, y);
-      tmem_ld32(t_s + 224, y + 32);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&y_free[wg]);
+    }
+    if (!ok) {
+      // let the other warpgroup leave a turn it may be waiting for
+      named_barrier_arrive(2 + (wg ^ 1), 256);
+    }
+    // the state: Y of this row after the last P V of this warpgroup
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = fmaf(acc[c], alpha, y[c]);
+    for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+    if (ok && u > 0 && mbar_wait(&y_full[wg], (u - 1) & 1, ab)) {
+      tc_fence_after();
+      tmem_ld32(t_s + 192, acc);
+      tmem_ld32(t_s + 224, acc + 32);
+      tmem_ld_wait();
     }
   }
   tc_fence_before();
   __syncthreads();   // pipeline drained: stage buffers are free for the merge
   if (threadIdx.x == 0 && !*abort_flag)
-    for (int b = 0; b < 2 * kStages + 10; ++b) mbar_inval(bars + b);
+    for (int b = 0; b < kBars; ++b) mbar_inval(bars + b);
   if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -432,6 +476,27 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
     st_shared_v4(zh + off, hi[0], hi[1], hi[2], hi[3]);
     st_shared_v4(zl + off, lo[0], lo[1], lo[2], lo[3]);
   };
+  // the first batch of B~ V partials (up to 8 splits) for this thread's
+  // items, loaded before the weights are known so that the merge waits on
+  // one round of global loads
+  constexpr int kItems = M * 16;
+  constexpr int kIpt = 3;
+  constexpr int kBatch = 4;   // partials per load batch
+  constexpr bool kOneRound = kItems <= NT * kIpt;
+  float4 pv[kIpt][kBatch];
+  if constexpr (kOneRound) {
+#pragma unroll
+    for (int q = 0; q < kIpt; ++q) {
+      const int idx = q * NT + t;
+      if (idx < kItems) {
+        const float4 *src =
+            (const float4 *)(prm.py + ((size_t)bh * S * M + (idx >> 4)) * 64) + (idx & 15);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (u < S) pv[q][u] = __ldcg(src + (size_t)u * M * 16);
+      }
+    }
+  }
   // partial maxima and sums -> smem
   {
     const size_t pb = (size_t)bh * S * M;
@@ -457,23 +522,23 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
   // items and loads their partials (in batches of 8) before summing them.
   // Y goes to global memory (fp32) and, transposed, into the hi / lo B
   // operands (element (k = landmark j, n = feature c) at row c, column j).
-  constexpr int kItems = M * 16;
-  constexpr int kIpt = 3;
   const size_t pb = (size_t)bh * S * M;
   for (int base = 0; base < kItems; base += NT * kIpt) {
     float4 a[kIpt];
 #pragma unroll
     for (int q = 0; q < kIpt; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < S; s0 += 8) {
-      float4 v[kIpt][8];
+    for (int s0 = 0; s0 < S; s0 += kBatch) {
+      float4 (&v)[kIpt][kBatch] = pv;
+      if (!kOneRound || s0 > 0) {
 #pragma unroll
-      for (int q = 0; q < kIpt; ++q) {
-        const int idx = base + q * NT + t;
-        if (idx < kItems) {
-          const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
+        for (int q = 0; q < kIpt; ++q) {
+          const int idx = base + q * NT + t;
+          if (idx < kItems) {
+            const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
+            for (int u = 0; u < kBatch; ++u)
+              if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
+          }
         }
       }
 #pragma unroll
@@ -482,7 +547,7 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
         if (idx < kItems) {
           const int j = idx >> 4;
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
+          for (int u = 0; u < kBatch; ++u)
             if (s0 + u < S) {
               const float f = wgt[(s0 + u) * M + j];
               a[q].x = fmaf(f, v[q][u].x, a[q].x);
@@ -591,7 +656,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   if ((int)blockIdx.x < prm.BH) {
     bh = blockIdx.x;
     if constexpr (M <= 64) {
-      if (threadIdx.x < pinvpow::kThreads) pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
+      if (threadIdx.x < pinvpow::kBarThreads) pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
     } else {
       if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
     }

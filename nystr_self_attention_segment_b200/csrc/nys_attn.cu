@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
+#include "fused.cuh"
 #include "mid_tc.cuh"
 #include "out_tc.cuh"
 #include "stream_bf16.cuh"
@@ -45,6 +46,14 @@ bool is_empty(const nys_desc *desc) {
   return (long)desc->batch * desc->heads * desc->seq_len == 0;
 }
 
+// The persistent single-launch schedule (fused.cuh) is built but not the
+// default: its task bodies still run slower there than in the three-kernel
+// pipeline.  Compile with -DNYS_FUSED=1 to use it for m <= 64.
+#ifndef NYS_FUSED
+#define NYS_FUSED 0
+#endif
+constexpr bool kUseFused = NYS_FUSED != 0;
+
 Layout make_layout(const nys_desc *desc, int m) {
   Layout L;
   memset(&L, 0, sizeof(L));
@@ -57,7 +66,10 @@ Layout make_layout(const nys_desc *desc, int m) {
     // one pseudoinverse block per head plus `splits` B~ V blocks per head in
     // one wave of 148 blocks; each B~ V block leaves one merged partial
     const int chunks = (int)((n + midtc::kChunk - 1) / midtc::kChunk);
-    int per_head = BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1;
+    // m <= 64 (fused kernel): B~ V tasks of about 8 chunks; m = 128: one
+    // wave of 148 blocks with one pseudoinverse block per head
+    int per_head = kUseFused && m <= 64 ? chunks / 8
+                                         : (BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1);
     if (per_head < 1) per_head = 1;
     if (per_head > chunks) per_head = chunks;
     if (per_head > midtc::kMaxSplits) per_head = midtc::kMaxSplits;
@@ -88,7 +100,9 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.z = take(BH * m * m * 4);
   L.y = take(BH * m * d * 4);
   L.w = take(BH * m * d * 4);
-  L.err = take(256 + BH * 4);    // error word, then one counter per head
+  // error word and task queue, then three counters per head (segment sums,
+  // pseudoinverse + B~ V tasks, W ready); all zeroed by every call
+  L.err = take(256 + BH * 12);
   L.count = L.err + 256;
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
@@ -237,8 +251,83 @@ bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
          CUDA_SUCCESS;
 }
 
-constexpr int kTcLaunches = 3;
-const char *kTcNames = "seg_means,mid_tc,out_tc";
+// launches of the bf16 path: one fused kernel, or three
+int tc_launches(int m) { return kUseFused && m <= 64 ? 1 : 3; }
+const char *tc_names(int m) {
+  return kUseFused && m <= 64 ? "fused" : "seg_means,mid_tc,out_tc";
+}
+
+// The fused persistent kernel (m <= 64).
+template <int M>
+nys_status launch_fused(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
+                        const nys_desc *desc, int iters, const float *conv_w, int conv_k,
+                        __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
+                        Marks &mk) {
+  const int BH = desc->batch * desc->heads;
+  const int n = desc->seq_len;
+  float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
+  uint32_t *err = (uint32_t *)(ws + L.err);
+  const float scale_log2 = 0.125f * kLog2e;   // log2(e) / sqrt(64)
+  const bool conv = conv_w != nullptr;
+  const int kconv = conv ? ((128 + conv_k - 1 + 15) / 16) * 16 : 0;
+  CUtensorMap mq, mkk, mv, mvh, mo;
+  if (!make_map(&mq, Q, BH, n, 128) || !make_map(&mkk, K, BH, n, 128) ||
+      !make_map(&mv, V, BH, n, 128) || !make_map(&mvh, V, BH, n, conv ? kconv : 128) ||
+      !make_map(&mo, out, BH, n, 128))
+    return NYS_ERR_CUDA;
+  fused::Params p;
+  memset(&p, 0, sizeof(p));
+  const int chunks = (n + midtc::kChunk - 1) / midtc::kChunk;
+  const int tph = (n + outtc::kTileRows - 1) / outtc::kTileRows;
+  p.mid.pinv = pinvtc::Params{qt, kt, (float *)(ws + L.z), err, iters, scale_log2};
+  p.mid.q_land = qt;
+  p.mid.z = (float *)(ws + L.z);
+  p.mid.pmax = (float *)(ws + L.pmax);
+  p.mid.psum = (float *)(ws + L.psum);
+  p.mid.py = (float *)(ws + L.py);
+  p.mid.y = (float *)(ws + L.y);
+  p.mid.w = (float *)(ws + L.w);
+  p.mid.count = nullptr;
+  p.mid.err = err;
+  p.mid.BH = BH;
+  p.mid.n = n;
+  p.mid.chunks_per_head = chunks;
+  p.mid.splits = L.splits;
+  p.mid.scale_log2 = scale_log2;
+  p.out = outtc::Params{kt, (float *)(ws + L.w), conv_w, err, n, desc->heads,
+                        conv ? conv_k : 1, kconv, tph, 1, scale_log2};
+  p.q_land = qt;
+  p.k_land = kt;
+  p.err = err;
+  p.queue = err + 1;
+  p.seg_cnt = (uint32_t *)(ws + L.count);
+  p.head_cnt = p.seg_cnt + BH;
+  p.w_ready = p.seg_cnt + 2 * BH;
+  p.BH = BH;
+  p.seg_len = n / M;
+  // about 1024 rows (128 KB) per segment-sum task
+  p.seg_per_task = 1024 / p.seg_len;
+  if (p.seg_per_task < 1) p.seg_per_task = 1;
+  if (p.seg_per_task > M) p.seg_per_task = M;
+  p.seg_tasks = (M + p.seg_per_task - 1) / p.seg_per_task;
+  p.splits = L.splits;
+  p.tiles_per_task = 8;
+  p.out_tasks = (tph + p.tiles_per_task - 1) / p.tiles_per_task;
+  p.lag_p = 1;
+  p.lag_b = 2;
+  p.lag_o = BH < 2 ? 2 : (BH / 2 + 4 < BH ? BH / 2 + 4 : BH);
+  if (p.lag_o < p.lag_b) p.lag_o = p.lag_b;
+  p.steps = BH + p.lag_o;
+  p.total = BH * (2 * p.seg_tasks + 1 + p.splits + p.out_tasks);
+  p.inv_len = 1.f / (float)p.seg_len;
+  auto kern = fused::fused_kernel<M>;
+  const uint32_t sm = fused::smem_bytes<M>(conv ? kconv : 0);
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  const int grid = p.total < kNumSms ? p.total : kNumSms;
+  kern<<<grid, fused::kThreads, sm, stream>>>(mq, mkk, mv, mvh, mo, p);
+  mk.after(stream);
+  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
 
 template <int M>
 nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
@@ -312,6 +401,10 @@ nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_
                      const nys_desc *desc, int m, int iters, const float *conv_w, int conv_k,
                      __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
                      Marks &mk) {
+  if (kUseFused) {
+    if (m == 32) return launch_fused<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+    if (m == 64) return launch_fused<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+  }
   switch (m) {
     case 32: return launch_tc_m<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
     case 64: return launch_tc_m<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
@@ -395,7 +488,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
                                nys_stream_t stream_, void *const *events, int n_events) {
   nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
   if (st != NYS_OK) return st;
-  if (events && n_events < (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches) + 1)
+  if (events && n_events < (desc->dtype == NYS_BF16 ? tc_launches(m) : kSimtLaunches) + 1)
     return NYS_ERR_INVALID_ARG;
   if (is_empty(desc)) return NYS_OK;
   Marks mk;
@@ -419,7 +512,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (cudaMemsetAsync(ws + L.err, 0, 256 + (size_t)desc->batch * desc->heads * 4, stream) !=
+  if (cudaMemsetAsync(ws + L.err, 0, 256 + (size_t)desc->batch * desc->heads * 12, stream) !=
       cudaSuccess)
     st = NYS_ERR_CUDA;
   mk.first(stream);
@@ -601,7 +694,7 @@ NYS_ATTN_API nys_status nys_attn_launch_count(const nys_desc *desc, int m, int c
   if (!launches) return NYS_ERR_INVALID_ARG;
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  *launches = is_empty(desc) ? 0 : (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches);
+  *launches = is_empty(desc) ? 0 : (desc->dtype == NYS_BF16 ? tc_launches(m) : kSimtLaunches);
   return NYS_OK;
 }
 
@@ -609,7 +702,7 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
                                               size_t names_bytes) {
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  const char *src = is_empty(desc) ? "" : (desc->dtype == NYS_BF16 ? kTcNames : kSimtNames);
+  const char *src = is_empty(desc) ? "" : (desc->dtype == NYS_BF16 ? tc_names(m) : kSimtNames);
   if (names) {
     if (names_bytes < strlen(src) + 1) return NYS_ERR_INVALID_ARG;
     strcpy(names, src);

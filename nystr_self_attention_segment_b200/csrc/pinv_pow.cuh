@@ -34,7 +34,9 @@
 // Threads 0..255: thread t owns TMEM lane r = t % 128 and column half
 // h = t / 128.  Lanes 0..m-1 carry the P chain, lanes 64..64+m-1 the Z
 // update and r_j (their MMA rows are stacked at row 64), so the two run on
-// different warps.  Thread 0 issues the MMAs.
+// different warps.  Thread 256 (warp 8) issues the MMAs: an MMA issue
+// blocks the issuing thread until the tensor pipe takes it, which must not
+// hold up a row thread.
 #pragma once
 
 #include <type_traits>
@@ -46,7 +48,8 @@ namespace pinvpow {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;       // matrix-row threads
+constexpr int kBarThreads = 288;    // plus one issuer warp (warp 8, lane 0 issues)
 
 constexpr int kSplitIters = 3;   // Lemma 1 steps with split fp16 products
 
@@ -72,10 +75,12 @@ struct Cfg {
   static constexpr uint32_t ql = qh + 128u * 128u;
   static constexpr uint32_t kh = ql + 128u * 128u;
   static constexpr uint32_t kl = kh + 64u * 128u;
-  // fp32 copy of the current P (and first of A), rows padded to M + 4
-  static constexpr int PF = M + 4;
-  static constexpr uint32_t pf = kl + 64u * 128u;
-  static constexpr uint32_t red = pf + (uint32_t)M * PF * 4u;   // [3][M]
+  // fp32 scratch over the logits operands (dead once A is formed): P by step
+  // parity (A during setup) and P2, [M][64] each with 16-byte chunks
+  // XOR-swizzled by row so that row and column accesses avoid bank conflicts
+  static constexpr uint32_t pf = qh;                     // [2][64][64] fp32
+  static constexpr uint32_t p2f = pf + 2u * 64u * 64u * 4u;
+  static constexpr uint32_t red = kl + 64u * 128u;      // [3][M]
   static constexpr uint32_t bars = (red + 3u * M * 4u + 1023u) & ~1023u;
   static constexpr uint32_t total = bars + 1024u;
   static constexpr uint32_t kTmemCols = 128;        // D at column 0, Z update at 64
@@ -111,6 +116,29 @@ __device__ __forceinline__ void put_split(uint32_t hi_base, uint32_t lo_base, in
   }
 }
 
+// fp32 [64][64] scratch, 16-byte chunks XOR-swizzled by row: element (r, c)
+__device__ __forceinline__ int sw_idx(int r, int c) {
+  return r * 64 + ((((c >> 2) ^ (r & 7)) << 2) | (c & 3));
+}
+template <int N>
+__device__ __forceinline__ void put_row(float *buf, int r, int c0, const float *v) {
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q)
+    *(float4 *)(buf + sw_idx(r, c0 + 4 * q)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+template <int N>
+__device__ __forceinline__ void get_row(const float *buf, int r, int c0, float *v) {
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 x = *(const float4 *)(buf + sw_idx(r, c0 + 4 * q));
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
   if constexpr (N == 32) {
@@ -121,7 +149,7 @@ __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
   tmem_ld_wait();
 }
 
-// Runs on threads 0..255 of a block and synchronises them with named barrier
+// Runs on threads 0..287 of a block and synchronises them with named barrier
 // 1 only.  smem: Cfg<M>::total bytes, 1 KB aligned.  Prm carries q_land,
 // k_land ([BH][m][64] fp32), z_out ([BH][m][m] fp32), err, iters and
 // scale_log2 = log2(e) / sqrt(d).
@@ -134,8 +162,10 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   constexpr int NC = C::NC;
   const int t = threadIdx.x, warp = t >> 5;
   const int r = t & 127, h = t >> 7;
-  const bool crit = r < M;                       // P chain rows
-  const bool aux = r >= 64 && r < 64 + M;        // Z update rows
+  const bool rows = t < kThreads;
+  const bool issuer = t == kThreads;
+  const bool crit = rows && r < M;               // P chain rows
+  const bool aux = rows && r >= 64 && r < 64 + M;   // Z update rows
   const int row = crit ? r : r - 64;             // matrix row of this thread
   const int c_lo = h * NC;
   uint64_t *bar_main = (uint64_t *)(smem + C::bars);
@@ -143,7 +173,8 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   uint32_t *tmem_slot = (uint32_t *)(bar_main + 2);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   float *red = (float *)(smem + C::red);         // row sums [M], column halves [2][M]
-  float *pf = (float *)(smem + C::pf);
+  float *pf0 = (float *)(smem + C::pf);          // fp32 P by step parity (A during setup)
+  float *p2f = (float *)(smem + C::p2f);         // fp32 P2 of the current step
   const Abort ab{abort_flag, prm.err};
   if (t == 0) {
     mbar_init(bar_main, 1);
@@ -166,7 +197,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   const uint32_t ph = a2h + 64u * 128u, pl = a2l + 64u * 128u;   // P at row 64 of a2
 
   // ---- landmarks -> split bf16 operands (all loads issued first)
-  {
+  if (rows) {
     constexpr int kPer = M * 8 / kThreads;      // 16-byte chunks per thread per tensor
     const float4 *qg = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
     const float4 *kg = (const float4 *)(prm.k_land + (size_t)bh * M * 64);
@@ -192,7 +223,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   }
   fence_async_smem();
   tc_fence_before();
-  named_barrier(1, kThreads);
+  named_barrier(1, kBarThreads);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -215,7 +246,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   auto sync_ops = [&]() -> bool {
     fence_async_smem();
     tc_fence_before();
-    const bool failed = named_barrier_or(1, kThreads, !ok);
+    const bool failed = named_barrier_or(1, kBarThreads, !ok);
     tc_fence_after();
     return !failed;
   };
@@ -238,18 +269,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       mma(d, a_l, b_h, idesc, kk, true);
     }
   };
-  const uint64_t dqh = make_sdesc(qh, 16, 1024), dql = make_sdesc(ql, 16, 1024);
-  const uint64_t dkh = make_sdesc(kh, 16, 1024), dkl = make_sdesc(kl, 16, 1024);
-  const uint64_t dph = make_sdesc(ph, 16, 1024), dpl = make_sdesc(pl, 16, 1024);
-  const uint64_t da2h = make_sdesc(a2h, 16, 1024), da2l = make_sdesc(a2l, 16, 1024);
-  const uint64_t duh = make_sdesc(uh, 16, 1024), dul = make_sdesc(ul, 16, 1024);
-  const uint64_t dazh = make_sdesc(azh, 16, 1024), dazl = make_sdesc(azl, 16, 1024);
-  const uint64_t dbrh = make_sdesc(brh, 16, 1024), dbrl = make_sdesc(brl, 16, 1024);
+  // operand descriptors (built where an MMA is issued)
+  auto sd = [](uint32_t a) { return make_sdesc(a, 16, 1024); };
   float *zg = prm.z_out + (size_t)bh * M * M;
 
   // ---- logits (split bf16) -> TMEM columns 0..M-1
-  if (t == 0) {
-    mma3(tmem, dqh, dql, dkh, dkl, id_bf, K64{}, true);
+  if (issuer) {
+    mma3(tmem, sd(qh), sd(ql), sd(kh), sd(kl), id_bf, K64{}, true);
     mma_commit(bar_main);
   }
   wait_main(crit && h == 0);
@@ -279,16 +305,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
     red[r] = (rs[0] + rs[1]) + (rs[2] + rs[3]);
     put_split<M, true>(ph, pl, r, 0, v);
-#pragma unroll
-    for (int q = 0; q < M / 4; ++q)
-      *(float4 *)(pf + r * C::PF + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
-                                                       v[4 * q + 3]);
+    put_row<M>(pf0, r, 0, v);
   }
   if (!sync_ops()) ok = false;
   // ---- A A^T on the tensor cores; meanwhile the Z rows take the columns of
   //      A (their Z0 rows up to c0) and their partial column sums
-  if (ok && t == 0) {
-    mma3(tmem, dph, dpl, dph, dpl, id_f16, KM{}, true);
+  if (ok && issuer) {
+    mma3(tmem, sd(ph), sd(pl), sd(ph), sd(pl), id_f16, KM{}, true);
     mma_commit(bar_main);
   }
   float acol[NC];
@@ -296,12 +319,12 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     float cs = 0.f;
 #pragma unroll
     for (int k = 0; k < NC; ++k) {
-      acol[k] = pf[(c_lo + k) * C::PF + row];
+      acol[k] = pf0[sw_idx(c_lo + k, row)];
       cs += fabsf(acol[k]);
     }
     red[M + h * M + row] = cs;
   }
-  named_barrier(1, kThreads);
+  named_barrier(1, kBarThreads);
   float n1 = 0.f, ninf = 0.f;
 #pragma unroll 8
   for (int i = 0; i < M; ++i) {
@@ -322,16 +345,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
   }
   wait_main(crit);
-  float p[NC], p2[NC];
   if (ok && crit) {   // P0 = c0 A A^T
+    float p[NC];
     ld_cols<NC>(t_d + c_lo, p);
 #pragma unroll
     for (int k = 0; k < NC; ++k) p[k] *= c0;
     put_split<NC, true>(ph, pl, row, c_lo, p);
-#pragma unroll
-    for (int q = 0; q < NC / 4; ++q)
-      *(float4 *)(pf + row * C::PF + c_lo + 4 * q) =
-          make_float4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+    put_row<NC>(pf0, row, c_lo, p);
   }
   if (!sync_ops()) ok = false;
 
@@ -339,7 +359,6 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   //      issued in stage 2 of step j (behind the chain's MMA) and read back
   //      by the Z rows in stage 1 of step j + 1; r_j alternates between two
   //      buffers by step parity.
-  float pr[NC];   // Z rows: P_j row of the same index (for r_j)
   const int iters = ok ? prm.iters : 0;
   bool good = ok;   // block-uniform: no stage failed
   const uint32_t id_z = make_idesc(kFmtBF16, 128, M, 0, 0);
@@ -347,19 +366,9 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   for (int j = 0; j < iters; ++j) {
     const bool split = j < kSplitIters, split_next = j + 1 < kSplitIters;
     // stage 1: P2 = P P
-    if (t == 0) {
-      mma3(tmem, dph, dpl, dph, dpl, id_f16, KM{}, split);
+    if (issuer) {
+      mma3(tmem, sd(ph), sd(pl), sd(ph), sd(pl), id_f16, KM{}, split);
       mma_commit(bar_main);
-    }
-    if (aux) {
-#pragma unroll
-      for (int q = 0; q < NC / 4; ++q) {
-        const float4 x = *(const float4 *)(pf + row * C::PF + c_lo + 4 * q);
-        pr[4 * q] = x.x;
-        pr[4 * q + 1] = x.y;
-        pr[4 * q + 2] = x.z;
-        pr[4 * q + 3] = x.w;
-      }
     }
     if (j >= 2) {   // Z_{j-1} back into the Z operand
       wait_z(aux);
@@ -371,45 +380,47 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
     wait_main(crit);
     if (ok && crit) {
-      float uu[NC];
+      float p2[NC], uu[NC];
       ld_cols<NC>(t_d + c_lo, p2);
+      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, uu);     // P_j
 #pragma unroll
-      for (int k = 0; k < NC; ++k) uu[k] = fmaf(7.f, p[k], -p2[k]);
+      for (int k = 0; k < NC; ++k) uu[k] = fmaf(7.f, uu[k], -p2[k]);
       put_split<NC, true>(a2h, a2l, row, c_lo, p2, split);
       put_split<NC, true>(uh, ul, row, c_lo, uu, split);
+      put_row<NC>(p2f, row, c_lo, p2);
     }
     if (!sync_ops()) {
       good = false;
       break;
     }
     // stage 2: [P2; P] U, then Z_j = Z_{j-1} r_{j-1}
-    if (t == 0) {
-      mma3(tmem, da2h, da2l, duh, dul, id_f16, KM{}, split);
+    if (issuer) {
+      mma3(tmem, sd(a2h), sd(a2l), sd(uh), sd(ul), id_f16, KM{}, split);
       mma_commit(bar_main);
       if (j > 0) {
         const uint32_t rb = ((j - 1) & 1) * (kBr >> 4);
-        mma3(tmem + 64, dazh, dazl, dbrh + rb, dbrl + rb, id_z, KM{}, true);
+        mma3(tmem + 64, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
         mma_commit(bar_z);
       }
     }
     wait_main(crit || aux);
     if (ok && crit) {   // P_{j+1} = 1/4 (13 P - 15 P2 + 7 P^3 - P^4)
-      float d[NC];
+      float d[NC], a[NC], b[NC];
       ld_cols<NC>(t_d + c_lo, d);
+      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, a);       // P_j
+      get_row<NC>(p2f, row, c_lo, b);                        // P_j^2
 #pragma unroll
-      for (int k = 0; k < NC; ++k) p[k] = 0.25f * fmaf(13.f, p[k], fmaf(-15.f, p2[k], d[k]));
-      put_split<NC, true>(ph, pl, row, c_lo, p, split_next);
-#pragma unroll
-      for (int q = 0; q < NC / 4; ++q)
-        *(float4 *)(pf + row * C::PF + c_lo + 4 * q) =
-            make_float4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+      for (int k = 0; k < NC; ++k) d[k] = 0.25f * fmaf(13.f, a[k], fmaf(-15.f, b[k], d[k]));
+      put_split<NC, true>(ph, pl, row, c_lo, d, split_next);
+      put_row<NC>(pf0 + ((j + 1) & 1) * 4096, row, c_lo, d);
     }
     if (ok && aux) {   // r_j = 1/4 (13I - 15 P + 7 P^2 - P^3)
-      float d[NC];
+      float d[NC], a[NC];
       ld_cols<NC>(t_d + c_lo, d);
+      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, a);       // P_j
 #pragma unroll
       for (int k = 0; k < NC; ++k)
-        d[k] = 0.25f * ((c_lo + k == row ? 13.f : 0.f) + fmaf(-15.f, pr[k], d[k]));
+        d[k] = 0.25f * ((c_lo + k == row ? 13.f : 0.f) + fmaf(-15.f, a[k], d[k]));
       const uint32_t rb = (j & 1) * kBr;
       put_split<NC, false>(brh + rb, brl + rb, row, c_lo, d);
     }
@@ -430,9 +441,9 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       good = sync_ops();
     }
     if (good) {
-      if (t == 0) {
+      if (issuer) {
         const uint32_t rb = ((iters - 1) & 1) * (kBr >> 4);
-        mma3(tmem + 64, dazh, dazl, dbrh + rb, dbrl + rb, id_z, KM{}, true);
+        mma3(tmem + 64, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
         mma_commit(bar_z);
       }
       wait_z(aux);
@@ -447,7 +458,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
   }
   tc_fence_before();
-  named_barrier(1, kThreads);
+  named_barrier(1, kBarThreads);
   if (t == 0 && !*abort_flag) {
     mbar_inval(bar_main);
     mbar_inval(bar_z);

@@ -302,6 +302,12 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrives on a named barrier without waiting (the producer side of a
+// bar.sync by other warps).
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Named barrier that also returns, to every participating thread, whether any
 // of them passed `flag` = true (bar.red.or), so that a block leaves a loop
 // together.
