@@ -66,12 +66,12 @@ struct MergeCfg {
   static constexpr uint32_t kSlabB = 64u * 128u;          // Y^T: 64 feature rows x 32 fp32
   static constexpr uint32_t zh = 0, zl = zh + KS * kSlabA;
   static constexpr uint32_t yh = zl + KS * kSlabA, yl = yh + KS * kSlabB;
-  static constexpr uint32_t ys = zl;                      // Y staging [M][68] fp32 (over zl,
-                                                          // which is written after it is read)
   static constexpr uint32_t wgt = yl + KS * kSlabB;       // [kMaxSplits][M] weights
   static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
   static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
-  static constexpr uint32_t bars = (den + M * 4u + 1023u) & ~1023u;
+  static constexpr uint32_t ys = (den + M * 4u + 127u) & ~127u;   // Y staging [M][68] fp32
+  static constexpr uint32_t ys_end = ys + (M <= 64 ? M * 68u * 4u : 0u);
+  static constexpr uint32_t bars = (ys_end + 1023u) & ~1023u;
   static constexpr uint32_t total = bars + 1024u;
 };
 
@@ -406,11 +406,14 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 }
 
 // ------------------------------------------------------------------ merge + W
-// Y = sum_s f_s py_s / sum_s f_s psum_s with f_s = 2^(pmax_s - max), over the
-// S partials of the head in order; then W = Z Y on the tensor cores as a
-// 3xTF32 product (Z hi*Y hi + Z hi*Y lo + Z lo*Y hi, about fp32 accuracy).
-// All 384 threads; every global load of a phase is issued before its results
-// are used.
+// Two steps, run by different blocks so that the first is off the critical
+// path:
+//   merge_y_body  Y = sum_s f_s py_s / sum_s f_s psum_s, f_s = 2^(pmax_s -
+//                 max), over the S partials of the head in order (run by the
+//                 last B~ V block of the head);
+//   w_body        W = Z Y on the tensor cores as a 3xTF32 product (Z hi*Y hi
+//                 + Z hi*Y lo + Z lo*Y hi, about fp32 accuracy), run by the
+//                 second of {pseudoinverse block, Y merge} to finish.
 __device__ __forceinline__ uint32_t kmaj_f32(uint32_t slab, int row, int k) {
   return (uint32_t)(k >> 5) * slab + sw128_offset(row, (k & 31) >> 2) + (k & 3) * 4u;
 }
@@ -421,89 +424,41 @@ __device__ __forceinline__ float tf32_hi(float x) {
   return __uint_as_float(r);
 }
 
-// tmem_in: a TMEM allocation of at least 64 columns owned by the caller, or
-// ~0u to allocate (and free) one here.
+// All 384 threads; every global load is issued before its result is used.
+// ysm: optional [M][68] fp32 staging copy of Y in shared memory (or null).
 template <int M>
-__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh,
-                                           uint32_t tmem_in) {
+__device__ __forceinline__ void merge_y_body(const Params &prm, uint8_t *smem, int bh,
+                                             float *ysm = nullptr) {
   using C = MergeCfg<M>;
   constexpr int NT = kThreads;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int t = threadIdx.x;
   const int S = prm.splits;
   float *wgt = (float *)(smem + C::wgt);
   float *psm = (float *)(smem + C::psm);
-  float *ysm = (float *)(smem + C::ys);
   float *den = (float *)(smem + C::den);
-  uint64_t *bar = (uint64_t *)(smem + C::bars);
-  uint32_t *tmem_slot = (uint32_t *)(bar + 1);
-  volatile uint32_t *abort_flag = tmem_slot + 1;
-  const Abort ab{abort_flag, prm.err};
-  const uint32_t zh = smem_u32(smem + C::zh), zl = smem_u32(smem + C::zl);
-  const uint32_t yh = smem_u32(smem + C::yh), yl = smem_u32(smem + C::yl);
-  if (t == 0) {
-    mbar_init(bar, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (tmem_in != ~0u) {
-    if (t == 0) *tmem_slot = tmem_in;
-  } else if (warp == 0) {
-    tmem_alloc(tmem_slot, 64);
-  }
-  // Z rows (issued now for m <= 64, held in registers; written into the hi /
-  // lo K-major tf32 operands after Y, whose staging buffer overlays zl)
-  constexpr int kZ4 = M * M / 4;
-  constexpr int kZPer = (kZ4 + NT - 1) / NT;
-  constexpr bool kZEarly = M <= 64;
-  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
-  float4 zv[kZEarly ? kZPer : 1];
-  if constexpr (kZEarly) {
-#pragma unroll
-    for (int u = 0; u < kZPer; ++u)
-      if (t + u * NT < kZ4) zv[u] = __ldcg(z4 + t + u * NT);
-  }
-  auto put_z = [&](int i, float4 v) {
-    const int row = (i * 4) / M, k = (i * 4) % M;
-    const float x[4] = {v.x, v.y, v.z, v.w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float h = tf32_hi(x[e]);
-      hi[e] = __float_as_uint(h);
-      lo[e] = __float_as_uint(tf32_hi(x[e] - h));
-    }
-    const uint32_t off = kmaj_f32(C::kSlabA, row, k);
-    st_shared_v4(zh + off, hi[0], hi[1], hi[2], hi[3]);
-    st_shared_v4(zl + off, lo[0], lo[1], lo[2], lo[3]);
-  };
-  // the first batch of B~ V partials (up to 8 splits) for this thread's
-  // items, loaded before the weights are known so that the merge waits on
-  // one round of global loads
+  // the first batch of partials for this thread's items, loaded before the
+  // weights are known so that the merge waits on one round of global loads
   constexpr int kItems = M * 16;
   constexpr int kIpt = 3;
   constexpr int kBatch = 4;   // partials per load batch
   constexpr bool kOneRound = kItems <= NT * kIpt;
+  const size_t pb = (size_t)bh * S * M;
   float4 pv[kIpt][kBatch];
   if constexpr (kOneRound) {
 #pragma unroll
     for (int q = 0; q < kIpt; ++q) {
       const int idx = q * NT + t;
       if (idx < kItems) {
-        const float4 *src =
-            (const float4 *)(prm.py + ((size_t)bh * S * M + (idx >> 4)) * 64) + (idx & 15);
+        const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
 #pragma unroll
         for (int u = 0; u < kBatch; ++u)
           if (u < S) pv[q][u] = __ldcg(src + (size_t)u * M * 16);
       }
     }
   }
-  // partial maxima and sums -> smem
-  {
-    const size_t pb = (size_t)bh * S * M;
-    for (int i = t; i < S * M; i += NT) {
-      wgt[i] = __ldcg(prm.pmax + pb + i);
-      psm[i] = __ldcg(prm.psum + pb + i);
-    }
+  for (int i = t; i < S * M; i += NT) {
+    wgt[i] = __ldcg(prm.pmax + pb + i);
+    psm[i] = __ldcg(prm.psum + pb + i);
   }
   __syncthreads();
   if (t < M) {
@@ -518,11 +473,6 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
     den[t] = 1.f / d;
   }
   __syncthreads();
-  // Y: item = (landmark j, 4 features); per round a thread takes up to kIpt
-  // items and loads their partials (in batches of 8) before summing them.
-  // Y goes to global memory (fp32) and, transposed, into the hi / lo B
-  // operands (element (k = landmark j, n = feature c) at row c, column j).
-  const size_t pb = (size_t)bh * S * M;
   for (int base = 0; base < kItems; base += NT * kIpt) {
     float4 a[kIpt];
 #pragma unroll
@@ -562,38 +512,106 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
     for (int q = 0; q < kIpt; ++q) {
       const int idx = base + q * NT + t;
       if (idx < kItems) {
-        const int j = idx >> 4;
-        const float inv = den[j];
+        const float inv = den[idx >> 4];
         const float4 y = make_float4(a[q].x * inv, a[q].y * inv, a[q].z * inv, a[q].w * inv);
         ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = y;
-        *(float4 *)(ysm + j * 68 + (idx & 15) * 4) = y;
+        if (ysm) *(float4 *)(ysm + (idx >> 4) * 68 + (idx & 15) * 4) = y;
       }
     }
   }
   __syncthreads();
-  // Y^T into the hi / lo B operands: item = (feature c, 4 landmarks), one
-  // 16-byte store per operand (element (k = landmark, n = feature) at row c)
-  for (int it = t; it < 16 * M; it += NT) {
-    const int c = it & 63, j0 = (it >> 6) * 4;
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float y = ysm[(j0 + e) * 68 + c];
-      const float h = tf32_hi(y);
-      hi[e] = __float_as_uint(h);
-      lo[e] = __float_as_uint(tf32_hi(y - h));
-    }
-    const uint32_t off = kmaj_f32(C::kSlabB, c, j0);
-    st_shared_v4(yh + off, hi[0], hi[1], hi[2], hi[3]);
-    st_shared_v4(yl + off, lo[0], lo[1], lo[2], lo[3]);
+}
+
+// W = Z Y from the head's Z and Y in global memory.  tmem_in: a TMEM
+// allocation of at least 64 columns owned by the caller, or ~0u to allocate
+// (and free) one here.
+// z_ready: the hi / lo Z operand is already in shared memory (written by the
+// pseudoinverse that ran in this block); ysm: Y staged in shared memory by
+// merge_y_body (or null: Y is read from global memory).
+template <int M>
+__device__ __forceinline__ void w_body(const Params &prm, uint8_t *smem, int bh,
+                                       uint32_t tmem_in, bool z_ready = false,
+                                       const float *ysm = nullptr) {
+  using C = MergeCfg<M>;
+  constexpr int NT = kThreads;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  uint64_t *bar = (uint64_t *)(smem + C::bars);
+  uint32_t *tmem_slot = (uint32_t *)(bar + 1);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+  const Abort ab{abort_flag, prm.err};
+  const uint32_t zh = smem_u32(smem + C::zh), zl = smem_u32(smem + C::zl);
+  const uint32_t yh = smem_u32(smem + C::yh), yl = smem_u32(smem + C::yl);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  __syncthreads();   // staging (over zl) consumed
-  if constexpr (kZEarly) {
+  if (tmem_in != ~0u) {
+    if (t == 0) *tmem_slot = tmem_in;
+  } else if (warp == 0) {
+    tmem_alloc(tmem_slot, 64);
+  }
+  // loads: Z rows (float4) and Y^T items (feature c, 4 landmarks) as four
+  // scalars, all issued before any is used
+  constexpr int kZ4 = M * M / 4;
+  constexpr int kZPer = (kZ4 + NT - 1) / NT;
+  constexpr int kYT = 16 * M;                 // Y^T items
+  constexpr int kYPer = (kYT + NT - 1) / NT;
+  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
+  const float *yg = prm.y + (size_t)bh * M * 64;
+  float4 zv[kZPer];
+  float yv[kYPer][4];
+  if (!z_ready) {
 #pragma unroll
     for (int u = 0; u < kZPer; ++u)
-      if (t + u * NT < kZ4) put_z(t + u * NT, zv[u]);
-  } else {
-    for (int i = t; i < kZ4; i += NT) put_z(i, __ldcg(z4 + i));
+      if (t + u * NT < kZ4) zv[u] = __ldcg(z4 + t + u * NT);
+  }
+#pragma unroll
+  for (int u = 0; u < kYPer; ++u) {
+    const int it = t + u * NT;
+    if (it < kYT) {
+      const int c = it & 63, j0 = (it >> 6) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        yv[u][e] = ysm ? ysm[(j0 + e) * 68 + c] : __ldcg(yg + (size_t)(j0 + e) * 64 + c);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kZPer; ++u) {
+    const int i = t + u * NT;
+    if (!z_ready && i < kZ4) {
+      const int row = (i * 4) / M, k = (i * 4) % M;
+      const float x[4] = {zv[u].x, zv[u].y, zv[u].z, zv[u].w};
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float h = tf32_hi(x[e]);
+        hi[e] = __float_as_uint(h);
+        lo[e] = __float_as_uint(tf32_hi(x[e] - h));
+      }
+      const uint32_t off = kmaj_f32(C::kSlabA, row, k);
+      st_shared_v4(zh + off, hi[0], hi[1], hi[2], hi[3]);
+      st_shared_v4(zl + off, lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+  // Y^T into the hi / lo B operands: element (k = landmark, n = feature) at
+  // row c, one 16-byte store per operand
+#pragma unroll
+  for (int u = 0; u < kYPer; ++u) {
+    const int it = t + u * NT;
+    if (it < kYT) {
+      const int c = it & 63, j0 = (it >> 6) * 4;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float h = tf32_hi(yv[u][e]);
+        hi[e] = __float_as_uint(h);
+        lo[e] = __float_as_uint(tf32_hi(yv[u][e] - h));
+      }
+      const uint32_t off = kmaj_f32(C::kSlabB, c, j0);
+      st_shared_v4(yh + off, hi[0], hi[1], hi[2], hi[3]);
+      st_shared_v4(yl + off, lo[0], lo[1], lo[2], lo[3]);
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -609,7 +627,8 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
 #pragma unroll
       for (int k = 0; k < M / 8; ++k)
         mma_tf32(tmem, da + (k >> 2) * (C::kSlabA >> 4) + (k & 3) * 2u,
-                 db + (k >> 2) * (C::kSlabB >> 4) + (k & 3) * 2u, idesc, (first && k == 0) ? 0u : 1u);
+                 db + (k >> 2) * (C::kSlabB >> 4) + (k & 3) * 2u, idesc,
+                 (first && k == 0) ? 0u : 1u);
     };
     prod(zh, yh, true);
     prod(zh, yl, false);
@@ -638,6 +657,16 @@ __device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int
   }
 }
 
+// Both steps in one block (used by the persistent schedule).
+template <int M>
+__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh,
+                                           uint32_t tmem_in) {
+  merge_y_body<M>(prm, smem, bh);
+  __threadfence();
+  __syncthreads();
+  w_body<M>(prm, smem, bh, tmem_in);
+}
+
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -656,7 +685,9 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   if ((int)blockIdx.x < prm.BH) {
     bh = blockIdx.x;
     if constexpr (M <= 64) {
-      if (threadIdx.x < pinvpow::kBarThreads) pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
+      if (threadIdx.x < pinvpow::kBarThreads)
+        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem + MergeCfg<M>::zh,
+                              smem + MergeCfg<M>::zl);
     } else {
       if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
     }
@@ -666,14 +697,21 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem);
   }
   // publish this block's results, then count it; the last of the head's
-  // S + 1 blocks merges
+  // S + 1 blocks merges the B~ V partials into Y and forms W = Z Y.  When the
+  // last is the pseudoinverse block (m <= 64), Z is already in its shared
+  // memory as the W operand.
   __threadfence();
   __syncthreads();
+  const bool is_pinv = (int)blockIdx.x < prm.BH;
   if (threadIdx.x == 0) last = atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits;
   __syncthreads();
   if (last) {
     __threadfence();
-    merge_body<M>(prm, smem, bh, tmem);
+    constexpr bool kStage = M <= 64;
+    float *ysm = kStage ? (float *)(smem + MergeCfg<M>::ys) : nullptr;
+    merge_y_body<M>(prm, smem, bh, ysm);
+    // the pseudoinverse leaves Z as the W operand only after at least one step
+    w_body<M>(prm, smem, bh, tmem, kStage && is_pinv && prm.pinv.iters > 0, ysm);
   }
   tc_fence_before();
   __syncthreads();
