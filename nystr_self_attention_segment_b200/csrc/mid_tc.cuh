@@ -677,6 +677,10 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   // one TMEM allocation for every body this block runs (an allocation
   // relinquishes the block's permit to allocate again)
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&tmem_base, 512);
+  // launched early (programmatic dependent launch): the landmarks come from
+  // the previous kernel
+  griddep_wait();
+  griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -696,22 +700,31 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     bh = b / prm.splits;
     bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem);
   }
-  // publish this block's results, then count it; the last of the head's
-  // S + 1 blocks merges the B~ V partials into Y and forms W = Z Y.  When the
-  // last is the pseudoinverse block (m <= 64), Z is already in its shared
-  // memory as the W operand.
+  // publish this block's results.  The last B~ V block of a head merges the
+  // partials into Y (while the pseudoinverse is still running, in general);
+  // the second of {pseudoinverse, Y merge} to finish forms W = Z Y, with Z
+  // already in shared memory as the W operand when that is the
+  // pseudoinverse block (m <= 64, at least one step).  Counters: count[bh]
+  // B~ V blocks done, count[BH + bh] inputs of W ready.
   __threadfence();
   __syncthreads();
   const bool is_pinv = (int)blockIdx.x < prm.BH;
-  if (threadIdx.x == 0) last = atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits;
+  if (threadIdx.x == 0)
+    last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
   __syncthreads();
   if (last) {
-    __threadfence();
-    constexpr bool kStage = M <= 64;
-    float *ysm = kStage ? (float *)(smem + MergeCfg<M>::ys) : nullptr;
-    merge_y_body<M>(prm, smem, bh, ysm);
-    // the pseudoinverse leaves Z as the W operand only after at least one step
-    w_body<M>(prm, smem, bh, tmem, kStage && is_pinv && prm.pinv.iters > 0, ysm);
+    if (!is_pinv) {
+      __threadfence();
+      merge_y_body<M>(prm, smem, bh);
+      __threadfence();
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      w_body<M>(prm, smem, bh, tmem, M <= 64 && is_pinv && prm.pinv.iters > 0);
+    }
   }
   tc_fence_before();
   __syncthreads();

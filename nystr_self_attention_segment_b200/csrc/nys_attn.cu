@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "simt.cuh"
@@ -251,6 +252,25 @@ bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
          CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream drains (it waits in griddep_wait before
+// reading that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // launches of the bf16 path: one fused kernel, or three
 int tc_launches(int m) { return kUseFused && m <= 64 ? 1 : 3; }
 const char *tc_names(int m) {
@@ -378,7 +398,9 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     auto kern = midtc::mid_kernel<M>;
     const uint32_t sm = midtc::smem_bytes<M>();
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    kern<<<BH * (1 + L.splits), midtc::kThreads, sm, stream>>>(mkk, mv, p);
+    if (launch_pdl(kern, dim3(BH * (1 + L.splits)), dim3(midtc::kThreads), sm, stream, mkk, mv,
+                   p) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {   // F~ W + DConv(V)
@@ -391,7 +413,9 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    kern<<<BH * cpb, outtc::kThreads, sm, stream>>>(mq, mvh, mo, p);
+    if (launch_pdl(kern, dim3(BH * cpb), dim3(outtc::kThreads), sm, stream, mq, mvh, mo, p) !=
+        cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;

@@ -332,6 +332,9 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int part = blockIdx.x % prm.ctas_per_head;
   const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
   const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
+  // launched early (programmatic dependent launch): K~ and W come from the
+  // previous kernels
+  griddep_wait();
   out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u);
 }
 

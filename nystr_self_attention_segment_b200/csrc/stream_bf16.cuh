@@ -4,7 +4,7 @@
 //    page's 1/l correction), one pass over Q and K with 16-byte loads;
 #pragma once
 
-#include "common.cuh"
+#include "sm100.cuh"
 
 namespace nys {
 
@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(256)
 seg_means_bf16(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                float *__restrict__ Qt, float *__restrict__ Kt, int n, int m) {
   __shared__ float part[32][64];
+  sm100::griddep_launch_dependents();   // the next kernel waits for this grid anyway
   const int j = blockIdx.x, bh = blockIdx.y;
   const __nv_bfloat16 *X = blockIdx.z == 0 ? Q : K;
   float *Xt = blockIdx.z == 0 ? Qt : Kt;
