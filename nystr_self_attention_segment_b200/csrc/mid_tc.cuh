@@ -115,10 +115,13 @@ constexpr float kTau = 8.f;
 
 // tmem_in: a 512-column TMEM allocation owned by the caller, or ~0u to
 // allocate (and free) one here.
+// wait_prev: launched with programmatic dependent launch; the first K / V
+// chunk loads are issued before the wait for the previous kernel, the Q~
+// operand (its result) is read after it.
 template <int M>
 __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensorMap *map_v,
                                         const Params &prm, uint8_t *smem, int bh, int split,
-                                        uint32_t tmem_in) {
+                                        uint32_t tmem_in, bool wait_prev = false) {
   constexpr int G = 128 / M;
   const BvSmem L = bv_smem();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -159,6 +162,17 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   } else if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
   }
+  __syncthreads();   // barriers initialised
+  const int pre = nch < kStages ? nch : kStages;   // chunk loads issued up front
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < pre; ++i) {
+      const int k0 = (c_begin + i) * kChunk;
+      mbar_expect_tx(&full[i], 32768u);
+      tma_load_3d(smem + L.k[i], map_k, &full[i], 0, k0, bh);
+      tma_load_3d(smem + L.v[i], map_v, &full[i], 0, k0, bh);
+    }
+  }
+  if (wait_prev) griddep_wait();
   // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
   if (threadIdx.x < 256) {
     const float4 *qt = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
@@ -183,7 +197,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < nch; ++i) {
+      for (int i = pre; i < nch; ++i) {
         const int s = i % kStages;
         if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
         const int k0 = (c_begin + i) * kChunk;
@@ -677,9 +691,9 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   // one TMEM allocation for every body this block runs (an allocation
   // relinquishes the block's permit to allocate again)
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&tmem_base, 512);
-  // launched early (programmatic dependent launch): the landmarks come from
-  // the previous kernel
-  griddep_wait();
+  // launched early (programmatic dependent launch): the bodies wait for the
+  // previous kernel before they read the landmarks; the next kernel waits
+  // for this whole grid before it reads anything this grid writes
   griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -688,6 +702,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   int bh;
   if ((int)blockIdx.x < prm.BH) {
     bh = blockIdx.x;
+    griddep_wait();
     if constexpr (M <= 64) {
       if (threadIdx.x < pinvpow::kBarThreads)
         pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem + MergeCfg<M>::zh,
@@ -698,7 +713,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   } else {
     const int b = blockIdx.x - prm.BH;
     bh = b / prm.splits;
-    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem);
+    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem, true);
   }
   // publish this block's results.  The last B~ V block of a head merges the
   // partials into Y (while the pseudoinverse is still running, in general);

@@ -76,10 +76,14 @@ struct Params {
 // 512-column TMEM allocation owned by the caller, or ~0u to allocate (and
 // free) one here.  smem: smem_layout(M, kconv).total bytes, 1 KB aligned.
 template <int M>
+// wait_prev: launched with programmatic dependent launch; everything that
+// reads only the inputs (barriers, TMEM, the Toeplitz operand, the first
+// kStages tile loads) runs before the wait for the previous kernel, the K~ /
+// W operand loads after it.
 __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtensorMap *map_v,
                                          const CUtensorMap *map_o, const Params &prm,
                                          uint8_t *smem, int bh, int t_begin, int t_end,
-                                         uint32_t tmem_in) {
+                                         uint32_t tmem_in, bool wait_prev = false) {
   const SmemLayout L = smem_layout(M, prm.kconv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = bh % prm.heads;
@@ -124,6 +128,40 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     tmem_alloc(tmem_slot, 512);
   }
 
+  if (conv && threadIdx.x < prm.conv_k)
+    cw[threadIdx.x] = prm.conv_w[(size_t)head * prm.conv_k + threadIdx.x];
+  tc_fence_before();
+  __syncthreads();   // barriers, TMEM address, conv weights
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t bytes = 16384u + (conv ? (uint32_t)prm.kconv * 128u : 0u);
+  const int pre = ntiles < kStages ? ntiles : kStages;   // tile loads issued up front
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < pre; ++i) {
+      const int r0 = (t_begin + i) * kTileRows;
+      mbar_expect_tx(&full[i], bytes);
+      tma_load_3d(smem + L.q[i], map_q, &full[i], 0, r0, bh);
+      if (conv) tma_load_3d(smem + L.v[i], map_v, &full[i], 0, r0 - half, bh);
+    }
+  }
+  // Toeplitz operand into TMEM: row r (lane r), columns j = halo rows
+  if (conv && warp >= 4 && warp < 8) {
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    for (int c0 = 0; c0 < prm.kconv / 2; c0 += 16) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int j0 = 2 * (c0 + e) - r, j1 = j0 + 1;
+        const float lo = (j0 >= 0 && j0 < prm.conv_k) ? cw[j0] : 0.f;
+        const float hi = (j1 >= 0 && j1 < prm.conv_k) ? cw[j1] : 0.f;
+        pk[e] = pack_bf16(lo, hi);
+      }
+      tmem_st16(tmem + lane_base + kT + c0, pk);
+    }
+    tmem_st_wait();
+  }
+  if (wait_prev) griddep_wait();
   // ---- per-head operands: K~ (B of S, K-major) and W (B of P W, MN-major),
   // bf16 with the 128-byte swizzle; all loads issued before the stores
   {
@@ -155,30 +193,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
                      pack_bf16(c[u][1].z, c[u][1].w));
       }
     }
-    if (conv && threadIdx.x < prm.conv_k) cw[threadIdx.x] = prm.conv_w[(size_t)head * prm.conv_k + threadIdx.x];
   }
   fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  // Toeplitz operand into TMEM: row r (lane r), columns j = halo rows
-  if (conv && warp >= 4 && warp < 8) {
-    const int r = threadIdx.x - 128;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    for (int c0 = 0; c0 < prm.kconv / 2; c0 += 16) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int j0 = 2 * (c0 + e) - r, j1 = j0 + 1;
-        const float lo = (j0 >= 0 && j0 < prm.conv_k) ? cw[j0] : 0.f;
-        const float hi = (j1 >= 0 && j1 < prm.conv_k) ? cw[j1] : 0.f;
-        pk[e] = pack_bf16(lo, hi);
-      }
-      tmem_st16(tmem + lane_base + kT + c0, pk);
-    }
-    tmem_st_wait();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -186,8 +202,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t bytes = 16384u + (conv ? (uint32_t)prm.kconv * 128u : 0u);
-      for (int i = 0; i < ntiles; ++i) {
+      for (int i = pre; i < ntiles; ++i) {
         const int s = i % kStages;
         if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
         const int r0 = (t_begin + i) * kTileRows;
@@ -332,10 +347,9 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int part = blockIdx.x % prm.ctas_per_head;
   const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
   const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
-  // launched early (programmatic dependent launch): K~ and W come from the
-  // previous kernels
-  griddep_wait();
-  out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u);
+  // launched early (programmatic dependent launch): out_body waits for the
+  // previous kernels before it reads K~ and W
+  out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u, true);
 }
 
 }  // namespace outtc
