@@ -728,9 +728,11 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
   __syncthreads();
   if (last) {
+    // a B~ V block that merges Y keeps a copy in shared memory for W
+    float *ysm = (M <= 64 && !is_pinv) ? (float *)(smem + MergeCfg<M>::ys) : nullptr;
     if (!is_pinv) {
       __threadfence();
-      merge_y_body<M>(prm, smem, bh);
+      merge_y_body<M>(prm, smem, bh, ysm);
       __threadfence();
       __syncthreads();
     }
@@ -738,7 +740,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     __syncthreads();
     if (last) {
       __threadfence();
-      w_body<M>(prm, smem, bh, tmem, M <= 64 && is_pinv && prm.pinv.iters > 0);
+      w_body<M>(prm, smem, bh, tmem, M <= 64 && is_pinv && prm.pinv.iters > 0, ysm);
     }
   }
   tc_fence_before();
