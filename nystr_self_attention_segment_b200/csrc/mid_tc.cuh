@@ -98,6 +98,7 @@ struct Params {
   const float *z;             // [BH][m][m]  (pinv output)
   float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
   float *y, *w;               // [BH][m][64]
+  uint8_t *w_op;              // [BH][m][128 B] W as the bf16 B operand of P W
   uint32_t *count;            // [BH] blocks finished per head (zeroed per call)
   uint32_t *err;
   int BH, n, chunks_per_head, splits;
@@ -661,6 +662,16 @@ __device__ __forceinline__ void w_body(const Params &prm, uint8_t *smem, int bh,
 #pragma unroll
     for (int q = 0; q < 8; ++q)
       dst[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    // and as the bf16 operand of P W: row = landmark, 16-byte chunk c at
+    // c ^ (row & 7) (the 128-byte swizzle of a 1 KB-aligned tile)
+    uint8_t *op = prm.w_op + ((size_t)bh * M + row) * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = cg * 4 + q;
+      *(uint4 *)(op + ((c ^ (row & 7)) << 4)) =
+          make_uint4(pack_bf16(w[8 * q], w[8 * q + 1]), pack_bf16(w[8 * q + 2], w[8 * q + 3]),
+                     pack_bf16(w[8 * q + 4], w[8 * q + 5]), pack_bf16(w[8 * q + 6], w[8 * q + 7]));
+    }
   }
   tc_fence_before();
   __syncthreads();

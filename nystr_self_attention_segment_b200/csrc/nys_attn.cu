@@ -111,7 +111,7 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.scratch = take(desc->dtype == NYS_F32 && m > 64 ? BH * 5 * m * m * 4 : 0);
   L.q_land_bf = take(0);
   L.k_land_bf = take(0);
-  L.w_bf = take(0);
+  L.w_bf = take(desc->dtype == NYS_BF16 ? BH * m * 128 : 0);   // W as the bf16 P W operand
   L.total = off;
   return L;
 }
@@ -307,6 +307,7 @@ nys_status launch_fused(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __
   p.mid.py = (float *)(ws + L.py);
   p.mid.y = (float *)(ws + L.y);
   p.mid.w = (float *)(ws + L.w);
+  p.mid.w_op = (uint8_t *)(ws + L.w_bf);
   p.mid.count = nullptr;
   p.mid.err = err;
   p.mid.BH = BH;
@@ -314,7 +315,7 @@ nys_status launch_fused(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __
   p.mid.chunks_per_head = chunks;
   p.mid.splits = L.splits;
   p.mid.scale_log2 = scale_log2;
-  p.out = outtc::Params{kt, (float *)(ws + L.w), conv_w, err, n, desc->heads,
+  p.out = outtc::Params{kt, (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads,
                         conv ? conv_k : 1, kconv, tph, 1, scale_log2};
   p.q_land = qt;
   p.k_land = kt;
@@ -388,6 +389,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     p.py = py;
     p.y = y;
     p.w = w;
+    p.w_op = (uint8_t *)(ws + L.w_bf);
     p.count = count;
     p.err = err;
     p.BH = BH;
@@ -408,7 +410,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     int cpb = kNumSms / BH;
     if (cpb < 1) cpb = 1;
     if (cpb > tph) cpb = tph;
-    outtc::Params p{kt, w, conv_w, err, n, desc->heads, conv ? conv_k : 1, kconv, tph, cpb,
+    outtc::Params p{kt, (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads, conv ? conv_k : 1, kconv, tph, cpb,
                     scale_log2};
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;

@@ -64,7 +64,8 @@ __host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
 
 struct Params {
   const float *k_land;     // [BH][m][64] fp32
-  const float *w;          // [BH][m][64] fp32
+  const uint8_t *w_op;     // [BH][m][128 B]: W as the bf16 B operand of P W
+                           // (row j = landmark, 64 features, 128-byte swizzle)
   const float *conv_w;     // [H][k] or null
   uint32_t *err;
   int n, heads, conv_k, kconv;
@@ -100,7 +101,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   uint64_t *p_ready = s_full + 2;
   uint64_t *o_full = p_ready + 2;
   uint64_t *tm_free = o_full + 2;
-  uint32_t *tmem_slot = (uint32_t *)(tm_free + 2);
+  uint64_t *w_ready = tm_free + 2;         // W operand in shared memory
+  uint32_t *tmem_slot = (uint32_t *)(w_ready + 1);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
   float *cw = (float *)(smem + L.cw);
@@ -116,6 +118,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       mbar_init(&o_full[b], 1);
       mbar_init(&tm_free[b], 128);
     }
+    mbar_init(w_ready, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(map_q);
@@ -161,43 +164,31 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     }
     tmem_st_wait();
   }
-  if (wait_prev) griddep_wait();
-  // ---- per-head operands: K~ (B of S, K-major) and W (B of P W, MN-major),
-  // bf16 with the 128-byte swizzle; all loads issued before the stores
+  // ---- per-head operands, bf16 with the 128-byte swizzle: K~ (B of S,
+  // K-major; written by the segment-mean kernel, which has completed once
+  // any block of the previous kernel got past its own wait, i.e. before this
+  // block could be placed on an SM) now; W (B of P W, MN-major; written by
+  // the previous kernel) by warp 3 after the wait, so that the first tiles'
+  // S, conv and softmax overlap the previous kernel's tail.  W arrives as
+  // the ready bf16 operand in one bulk copy.
+  auto put_op = [&](uint32_t base, const float4 *src, int idx) {
+    const float4 a0 = __ldcg(src + 2 * idx), a1 = __ldcg(src + 2 * idx + 1);
+    st_shared_v4(base + sw128_offset(idx >> 3, idx & 7), pack_bf16(a0.x, a0.y),
+                 pack_bf16(a0.z, a0.w), pack_bf16(a1.x, a1.y), pack_bf16(a1.z, a1.w));
+  };
   {
     const float4 *kt = (const float4 *)(prm.k_land + (size_t)bh * M * 64);
-    const float4 *wg = (const float4 *)(prm.w + (size_t)bh * M * 64);
-    constexpr int kItems = M * 8;           // 16-byte chunks (8 bf16) per operand
-    constexpr int kPer = (kItems + kThreads - 1) / kThreads;
-    float4 a[kPer][2], c[kPer][2];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int idx = threadIdx.x + u * kThreads;
-      if (idx < kItems) {
-        a[u][0] = __ldcg(kt + 2 * idx);
-        a[u][1] = __ldcg(kt + 2 * idx + 1);
-        c[u][0] = __ldcg(wg + 2 * idx);
-        c[u][1] = __ldcg(wg + 2 * idx + 1);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int idx = threadIdx.x + u * kThreads;
-      if (idx < kItems) {
-        const int row = idx >> 3, ch = idx & 7;
-        st_shared_v4(smem_u32(smem + L.kt) + sw128_offset(row, ch), pack_bf16(a[u][0].x, a[u][0].y),
-                     pack_bf16(a[u][0].z, a[u][0].w), pack_bf16(a[u][1].x, a[u][1].y),
-                     pack_bf16(a[u][1].z, a[u][1].w));
-        st_shared_v4(smem_u32(smem + L.w) + sw128_offset(row, ch), pack_bf16(c[u][0].x, c[u][0].y),
-                     pack_bf16(c[u][0].z, c[u][0].w), pack_bf16(c[u][1].x, c[u][1].y),
-                     pack_bf16(c[u][1].z, c[u][1].w));
-      }
-    }
+    for (int idx = threadIdx.x; idx < M * 8; idx += kThreads) put_op(smem_u32(smem + L.kt), kt, idx);
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (warp == 3 && lane == 0) {
+    if (wait_prev) griddep_wait();
+    mbar_expect_tx(w_ready, M * 128u);
+    bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -252,6 +243,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
         }
         mma_commit(&empty[s]);
         if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
+        if (u == 0 && !mbar_wait(w_ready, 0, ab)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < M / 16; ++k)
@@ -330,7 +322,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && !*abort_flag)
-    for (int b = 0; b < 2 * kStages + 8; ++b) mbar_inval(bars + b);
+    for (int b = 0; b < 2 * kStages + 9; ++b) mbar_inval(bars + b);
   if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
