@@ -49,7 +49,7 @@ struct Layout {
   size_t count;                            // per-head block counters (bf16 path)
   size_t pmax, psum, py;                   // split-n partials of B~ V
   size_t scratch;                          // per-head pinv scratch (m > 64)
-  size_t q_land_bf, k_land_bf, w_bf;       // bf16 MMA operands
+  size_t w_bf;                             // W as the bf16 operand of P W
   size_t total;
   int splits;                              // B~ V partials per head
   int keys_per_split;                      // SIMT path: keys per split

@@ -109,8 +109,6 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.psum = take(BH * splits * m * 4);
   L.py = take(BH * splits * m * d * 4);
   L.scratch = take(desc->dtype == NYS_F32 && m > 64 ? BH * 5 * m * m * 4 : 0);
-  L.q_land_bf = take(0);
-  L.k_land_bf = take(0);
   L.w_bf = take(desc->dtype == NYS_BF16 ? BH * m * 128 : 0);   // W as the bf16 P W operand
   L.total = off;
   return L;
