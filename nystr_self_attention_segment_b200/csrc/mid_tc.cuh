@@ -118,7 +118,8 @@ constexpr float kTau = 8.f;
 // allocate (and free) one here.
 // wait_prev: launched with programmatic dependent launch; the first K / V
 // chunk loads are issued before the wait for the previous kernel, the Q~
-// operand (its result) is read after it.
+// operand (its result) is read after it, and the next kernel may launch once
+// the wait has returned.
 template <int M>
 __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensorMap *map_v,
                                         const Params &prm, uint8_t *smem, int bh, int split,
@@ -173,7 +174,10 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       tma_load_3d(smem + L.v[i], map_v, &full[i], 0, k0, bh);
     }
   }
-  if (wait_prev) griddep_wait();
+  if (wait_prev) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
   if (threadIdx.x < 256) {
     const float4 *qt = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
@@ -703,9 +707,10 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   // relinquishes the block's permit to allocate again)
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&tmem_base, 512);
   // launched early (programmatic dependent launch): the bodies wait for the
-  // previous kernel before they read the landmarks; the next kernel waits
-  // for this whole grid before it reads anything this grid writes
-  griddep_launch_dependents();
+  // previous kernel before they read the landmarks, and only then let the
+  // next kernel launch.  So the next kernel starts after the segment-mean
+  // kernel has completed and may read K~ before its own wait; it waits for
+  // this whole grid before it reads anything this grid writes.
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -714,6 +719,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   if ((int)blockIdx.x < prm.BH) {
     bh = blockIdx.x;
     griddep_wait();
+    griddep_launch_dependents();
     if constexpr (M <= 64) {
       if (threadIdx.x < pinvpow::kBarThreads)
         pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem + MergeCfg<M>::zh,

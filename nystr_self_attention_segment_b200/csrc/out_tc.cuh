@@ -165,9 +165,9 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     tmem_st_wait();
   }
   // ---- per-head operands, bf16 with the 128-byte swizzle: K~ (B of S,
-  // K-major; written by the segment-mean kernel, which has completed once
-  // any block of the previous kernel got past its own wait, i.e. before this
-  // block could be placed on an SM) now; W (B of P W, MN-major; written by
+  // K-major; written by the segment-mean kernel, which has completed before
+  // this grid launches: every block of the previous kernel lets it launch
+  // only after its own wait for that kernel) now; W (B of P W, MN-major; written by
   // the previous kernel) by warp 3 after the wait, so that the first tiles'
   // S, conv and softmax overlap the previous kernel's tail.  W arrives as
   // the ready bf16 operand in one bulk copy.
