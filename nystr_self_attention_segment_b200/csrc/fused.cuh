@@ -272,7 +272,7 @@ __device__ __forceinline__ void run_bv(const CUtensorMap *mk, const CUtensorMap 
 }
 template <int M>
 __device__ __forceinline__ void run_merge(const Params &prm, uint8_t *smem, int bh, uint32_t tmem) {
-  midtc::merge_body<M>(prm.mid, smem, bh, tmem);
+  midtc::merge_body<M>(prm.mid, smem, bh);
 }
 
 template <int M>

@@ -61,18 +61,13 @@ __host__ __device__ inline BvSmem bv_smem() {
 
 template <int M>
 struct MergeCfg {
-  static constexpr int KS = M / 32;                       // 32-column slabs along K
-  static constexpr uint32_t kSlabA = 128u * 128u;         // Z: 128 rows x 32 fp32
-  static constexpr uint32_t kSlabB = 64u * 128u;          // Y^T: 64 feature rows x 32 fp32
-  static constexpr uint32_t zh = 0, zl = zh + KS * kSlabA;
-  static constexpr uint32_t yh = zl + KS * kSlabA, yl = yh + KS * kSlabB;
-  static constexpr uint32_t wgt = yl + KS * kSlabB;       // [kMaxSplits][M] weights
+  static constexpr int kZs = M + 4, kYs = 68;                // row strides (floats)
+  static constexpr uint32_t zs = 0;                          // Z [M][M + 4] fp32
+  static constexpr uint32_t ys = zs + M * kZs * 4u;          // Y [M][68] fp32
+  static constexpr uint32_t wgt = ys + M * kYs * 4u;         // [kMaxSplits][M] weights
   static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
   static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
-  static constexpr uint32_t ys = (den + M * 4u + 127u) & ~127u;   // Y staging [M][68] fp32
-  static constexpr uint32_t ys_end = ys + (M <= 64 ? M * 68u * 4u : 0u);
-  static constexpr uint32_t bars = (ys_end + 1023u) & ~1023u;
-  static constexpr uint32_t total = bars + 1024u;
+  static constexpr uint32_t total = den + M * 4u;
 };
 
 template <int M>
@@ -425,26 +420,17 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 }
 
 // ------------------------------------------------------------------ merge + W
-// Two steps, run by different blocks so that the first is off the critical
-// path:
-//   merge_y_body  Y = sum_s f_s py_s / sum_s f_s psum_s, f_s = 2^(pmax_s -
-//                 max), over the S partials of the head in order (run by the
-//                 last B~ V block of the head);
-//   w_body        W = Z Y on the tensor cores as a 3xTF32 product (Z hi*Y hi
-//                 + Z hi*Y lo + Z lo*Y hi, about fp32 accuracy), run by the
-//                 second of {pseudoinverse block, Y merge} to finish.
-__device__ __forceinline__ uint32_t kmaj_f32(uint32_t slab, int row, int k) {
-  return (uint32_t)(k >> 5) * slab + sw128_offset(row, (k & 31) >> 2) + (k & 3) * 4u;
-}
+// Y = sum_s f_s py_s / sum_s f_s psum_s, f_s = 2^(pmax_s - max), over the S
+// key splits of the head in split order (merge_y_body, run by the last B~ V
+// block of the head), then W = Z Y in fp32 (w_product), run by the second of
+// {pseudoinverse block, that B~ V block} to finish.
 
-__device__ __forceinline__ float tf32_hi(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
-}
-
-// All 384 threads; every global load is issued before its result is used.
-// ysm: optional [M][68] fp32 staging copy of Y in shared memory (or null).
+// All 384 threads, three phases: the S x M maxima and sums into shared
+// memory; the weights f_s and 1 / sum_s f_s psum_s of each row; then the
+// partials, a batch of up to kBatch splits of every item of a thread loaded
+// at once.  (Partials in flight during the weights phase would queue its
+// shared-memory reads behind their data.)
+// ysm: optional [M][68] fp32 copy of Y in shared memory (the W operand).
 template <int M>
 __device__ __forceinline__ void merge_y_body(const Params &prm, uint8_t *smem, int bh,
                                              float *ysm = nullptr) {
@@ -455,59 +441,58 @@ __device__ __forceinline__ void merge_y_body(const Params &prm, uint8_t *smem, i
   float *wgt = (float *)(smem + C::wgt);
   float *psm = (float *)(smem + C::psm);
   float *den = (float *)(smem + C::den);
-  // the first batch of partials for this thread's items, loaded before the
-  // weights are known so that the merge waits on one round of global loads
-  constexpr int kItems = M * 16;
-  constexpr int kIpt = 3;
-  constexpr int kBatch = 4;   // partials per load batch
-  constexpr bool kOneRound = kItems <= NT * kIpt;
   const size_t pb = (size_t)bh * S * M;
-  float4 pv[kIpt][kBatch];
-  if constexpr (kOneRound) {
+  {
+    constexpr int kPer = (kMaxSplits * M + NT - 1) / NT;
+    float a[kPer], b[kPer];
 #pragma unroll
-    for (int q = 0; q < kIpt; ++q) {
-      const int idx = q * NT + t;
-      if (idx < kItems) {
-        const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
+    for (int u = 0; u < kPer; ++u) {
+      const int i = t + u * NT;
+      if (i < S * M) {
+        a[u] = __ldcg(prm.pmax + pb + i);
+        b[u] = __ldcg(prm.psum + pb + i);
+      }
+    }
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (u < S) pv[q][u] = __ldcg(src + (size_t)u * M * 16);
+    for (int u = 0; u < kPer; ++u) {
+      const int i = t + u * NT;
+      if (i < S * M) {
+        wgt[i] = a[u];
+        psm[i] = b[u];
       }
     }
   }
-  for (int i = t; i < S * M; i += NT) {
-    wgt[i] = __ldcg(prm.pmax + pb + i);
-    psm[i] = __ldcg(prm.psum + pb + i);
-  }
   __syncthreads();
   if (t < M) {
+    const int j = t;
     float mx = -INFINITY;
-    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
+    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + j]);
     float d = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + t] - mx);
-      wgt[s * M + t] = f;
-      d = fmaf(psm[s * M + t], f, d);
+      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + j] - mx);
+      wgt[s * M + j] = f;
+      d = fmaf(psm[s * M + j], f, d);
     }
-    den[t] = 1.f / d;
+    den[j] = 1.f / d;
   }
   __syncthreads();
+  constexpr int kItems = M * 16;   // float4 items of Y
+  constexpr int kIpt = 3;          // items per thread per round
+  constexpr int kBatch = 8;        // splits per load batch
   for (int base = 0; base < kItems; base += NT * kIpt) {
     float4 a[kIpt];
 #pragma unroll
     for (int q = 0; q < kIpt; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < S; s0 += kBatch) {
-      float4 (&v)[kIpt][kBatch] = pv;
-      if (!kOneRound || s0 > 0) {
+      float4 v[kIpt][kBatch];
 #pragma unroll
-        for (int q = 0; q < kIpt; ++q) {
-          const int idx = base + q * NT + t;
-          if (idx < kItems) {
-            const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
+      for (int q = 0; q < kIpt; ++q) {
+        const int idx = base + q * NT + t;
+        if (idx < kItems) {
+          const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-              if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
-          }
+          for (int u = 0; u < kBatch; ++u)
+            if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
         }
       }
 #pragma unroll
@@ -534,178 +519,119 @@ __device__ __forceinline__ void merge_y_body(const Params &prm, uint8_t *smem, i
         const float inv = den[idx >> 4];
         const float4 y = make_float4(a[q].x * inv, a[q].y * inv, a[q].z * inv, a[q].w * inv);
         ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = y;
-        if (ysm) *(float4 *)(ysm + (idx >> 4) * 68 + (idx & 15) * 4) = y;
+        if (ysm) *(float4 *)(ysm + (idx >> 4) * C::kYs + (idx & 15) * 4) = y;
       }
     }
   }
   __syncthreads();
 }
 
-// W = Z Y from the head's Z and Y in global memory.  tmem_in: a TMEM
-// allocation of at least 64 columns owned by the caller, or ~0u to allocate
-// (and free) one here.
-// z_ready: the hi / lo Z operand is already in shared memory (written by the
-// pseudoinverse that ran in this block); ysm: Y staged in shared memory by
-// merge_y_body (or null: Y is read from global memory).
+// Z of head bh from global memory into shared memory (MergeCfg::zs); all
+// threads, every load issued before the first store.
 template <int M>
-__device__ __forceinline__ void w_body(const Params &prm, uint8_t *smem, int bh,
-                                       uint32_t tmem_in, bool z_ready = false,
-                                       const float *ysm = nullptr) {
+__device__ __forceinline__ void load_z(const Params &prm, uint8_t *smem, int bh) {
   using C = MergeCfg<M>;
-  constexpr int NT = kThreads;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  uint64_t *bar = (uint64_t *)(smem + C::bars);
-  uint32_t *tmem_slot = (uint32_t *)(bar + 1);
-  volatile uint32_t *abort_flag = tmem_slot + 1;
-  const Abort ab{abort_flag, prm.err};
-  const uint32_t zh = smem_u32(smem + C::zh), zl = smem_u32(smem + C::zl);
-  const uint32_t yh = smem_u32(smem + C::yh), yl = smem_u32(smem + C::yl);
-  if (t == 0) {
-    mbar_init(bar, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (tmem_in != ~0u) {
-    if (t == 0) *tmem_slot = tmem_in;
-  } else if (warp == 0) {
-    tmem_alloc(tmem_slot, 64);
-  }
-  // loads: Z rows (float4) and Y^T items (feature c, 4 landmarks) as four
-  // scalars, all issued before any is used
-  constexpr int kZ4 = M * M / 4;
-  constexpr int kZPer = (kZ4 + NT - 1) / NT;
-  constexpr int kYT = 16 * M;                 // Y^T items
-  constexpr int kYPer = (kYT + NT - 1) / NT;
-  const float4 *z4 = (const float4 *)(prm.z + (size_t)bh * M * M);
-  const float *yg = prm.y + (size_t)bh * M * 64;
-  float4 zv[kZPer];
-  float yv[kYPer][4];
-  if (!z_ready) {
+  constexpr int kZ4 = M * M / 4, kPer = (kZ4 + kThreads - 1) / kThreads;
+  float *zs = (float *)(smem + C::zs);
+  const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
+  float4 v[kPer];
 #pragma unroll
-    for (int u = 0; u < kZPer; ++u)
-      if (t + u * NT < kZ4) zv[u] = __ldcg(z4 + t + u * NT);
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * kThreads;
+    if (i < kZ4) v[u] = __ldcg(zg + i);
   }
 #pragma unroll
-  for (int u = 0; u < kYPer; ++u) {
-    const int it = t + u * NT;
-    if (it < kYT) {
-      const int c = it & 63, j0 = (it >> 6) * 4;
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * kThreads;
+    if (i < kZ4) *(float4 *)(zs + (i * 4 / M) * C::kZs + (i * 4) % M) = v[u];
+  }
+}
+
+// Y of head bh from global memory into shared memory (MergeCfg::ys).
+template <int M>
+__device__ __forceinline__ void load_y(const Params &prm, uint8_t *smem, int bh) {
+  using C = MergeCfg<M>;
+  constexpr int kY4 = M * 16, kPer = (kY4 + kThreads - 1) / kThreads;
+  float *ys = (float *)(smem + C::ys);
+  const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
+  float4 v[kPer];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        yv[u][e] = ysm ? ysm[(j0 + e) * 68 + c] : __ldcg(yg + (size_t)(j0 + e) * 64 + c);
-    }
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * kThreads;
+    if (i < kY4) v[u] = __ldcg(yg + i);
   }
 #pragma unroll
-  for (int u = 0; u < kZPer; ++u) {
-    const int i = t + u * NT;
-    if (!z_ready && i < kZ4) {
-      const int row = (i * 4) / M, k = (i * 4) % M;
-      const float x[4] = {zv[u].x, zv[u].y, zv[u].z, zv[u].w};
-      uint32_t hi[4], lo[4];
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * kThreads;
+    if (i < kY4) *(float4 *)(ys + (i >> 4) * C::kYs + (i & 15) * 4) = v[u];
+  }
+}
+
+// W = Z Y in fp32 (k in order) from Z and Y in shared memory, stored as fp32
+// rows and as the bf16 operand of P W (row = landmark, 16-byte chunk c at
+// c ^ (row & 7): the 128-byte swizzle of a 1 KB-aligned tile).  Threads
+// 0..255, each 4 columns of M / 16 rows; Z and Y must be visible to them.
+template <int M>
+__device__ __forceinline__ void w_product(const Params &prm, const uint8_t *smem, int bh) {
+  using C = MergeCfg<M>;
+  constexpr int R = M / 16;
+  const int t = threadIdx.x;
+  if (t >= 256) return;
+  const float *zs = (const float *)(smem + C::zs), *ys = (const float *)(smem + C::ys);
+  const int c4 = t & 15, i0 = (t >> 4) * R;
+  float acc[R][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < M; k += 4) {
+    float4 y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = *(const float4 *)(ys + (k + e) * C::kYs + 4 * c4);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 z = *(const float4 *)(zs + (i0 + r) * C::kZs + k);
+      const float zk[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float h = tf32_hi(x[e]);
-        hi[e] = __float_as_uint(h);
-        lo[e] = __float_as_uint(tf32_hi(x[e] - h));
+        acc[r][0] = fmaf(zk[e], y[e].x, acc[r][0]);
+        acc[r][1] = fmaf(zk[e], y[e].y, acc[r][1]);
+        acc[r][2] = fmaf(zk[e], y[e].z, acc[r][2]);
+        acc[r][3] = fmaf(zk[e], y[e].w, acc[r][3]);
       }
-      const uint32_t off = kmaj_f32(C::kSlabA, row, k);
-      st_shared_v4(zh + off, hi[0], hi[1], hi[2], hi[3]);
-      st_shared_v4(zl + off, lo[0], lo[1], lo[2], lo[3]);
     }
   }
-  // Y^T into the hi / lo B operands: element (k = landmark, n = feature) at
-  // row c, one 16-byte store per operand
 #pragma unroll
-  for (int u = 0; u < kYPer; ++u) {
-    const int it = t + u * NT;
-    if (it < kYT) {
-      const int c = it & 63, j0 = (it >> 6) * 4;
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float h = tf32_hi(yv[u][e]);
-        hi[e] = __float_as_uint(h);
-        lo[e] = __float_as_uint(tf32_hi(yv[u][e] - h));
-      }
-      const uint32_t off = kmaj_f32(C::kSlabB, c, j0);
-      st_shared_v4(yh + off, hi[0], hi[1], hi[2], hi[3]);
-      st_shared_v4(yl + off, lo[0], lo[1], lo[2], lo[3]);
-    }
-  }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  if (t == 0) {
-    const uint32_t idesc = make_idesc(kFmtTF32, 128, 64, 0, 0);
-    // descriptors advance by 32 bytes (2 address units) per K step of 8 and by
-    // a slab per 4 steps
-    auto prod = [&](uint32_t A, uint32_t B, bool first) {
-      const uint64_t da = make_sdesc(A, 16, 1024), db = make_sdesc(B, 16, 1024);
-#pragma unroll
-      for (int k = 0; k < M / 8; ++k)
-        mma_tf32(tmem, da + (k >> 2) * (C::kSlabA >> 4) + (k & 3) * 2u,
-                 db + (k >> 2) * (C::kSlabB >> 4) + (k & 3) * 2u, idesc,
-                 (first && k == 0) ? 0u : 1u);
-    };
-    prod(zh, yh, true);
-    prod(zh, yl, false);
-    prod(zl, yh, false);
-    mma_commit(bar);
-  }
-  // W rows from TMEM: warp w reads lanes 32 (w % 4).. and columns 32 (w / 4)..
-  const int row = (warp & 3) * 32 + lane, cg = warp >> 2;
-  const bool reader = (warp & 3) * 32 < M && cg < 2;
-  if (reader && mbar_wait(bar, 0, ab)) {
-    tc_fence_after();
-    float w[32];
-    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + cg * 32, w);
-    tmem_ld_wait();
-    float4 *dst = (float4 *)(prm.w + ((size_t)bh * M + row) * 64 + cg * 32);
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      dst[q] = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-    // and as the bf16 operand of P W: row = landmark, 16-byte chunk c at
-    // c ^ (row & 7) (the 128-byte swizzle of a 1 KB-aligned tile)
+  for (int r = 0; r < R; ++r) {
+    const int row = i0 + r;
+    *(float4 *)(prm.w + ((size_t)bh * M + row) * 64 + 4 * c4) =
+        make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
     uint8_t *op = prm.w_op + ((size_t)bh * M + row) * 128;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = cg * 4 + q;
-      *(uint4 *)(op + ((c ^ (row & 7)) << 4)) =
-          make_uint4(pack_bf16(w[8 * q], w[8 * q + 1]), pack_bf16(w[8 * q + 2], w[8 * q + 3]),
-                     pack_bf16(w[8 * q + 4], w[8 * q + 5]), pack_bf16(w[8 * q + 6], w[8 * q + 7]));
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (t == 0 && !*abort_flag) mbar_inval(bar);
-  if (warp == 0 && tmem_in == ~0u) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    *(uint2 *)(op + (((c4 >> 1) ^ (row & 7)) << 4) + (c4 & 1) * 8) =
+        make_uint2(pack_bf16(acc[r][0], acc[r][1]), pack_bf16(acc[r][2], acc[r][3]));
   }
 }
 
 // Both steps in one block (used by the persistent schedule).
 template <int M>
-__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh,
-                                           uint32_t tmem_in) {
-  merge_y_body<M>(prm, smem, bh);
-  __threadfence();
+__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh) {
+  merge_y_body<M>(prm, smem, bh, (float *)(smem + MergeCfg<M>::ys));
+  load_z<M>(prm, smem, bh);
   __syncthreads();
-  w_body<M>(prm, smem, bh, tmem_in);
+  w_product<M>(prm, smem, bh);
 }
 
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
            const Params prm) {
+  using C = MergeCfg<M>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint32_t last, tmem_base;
+  const int t = threadIdx.x;
   // one TMEM allocation for every body this block runs (an allocation
   // relinquishes the block's permit to allocate again)
-  if ((threadIdx.x >> 5) == 1) tmem_alloc(&tmem_base, 512);
+  if ((t >> 5) == 1) tmem_alloc(&tmem_base, 512);
   // launched early (programmatic dependent launch): the bodies wait for the
   // previous kernel before they read the landmarks, and only then let the
   // next kernel launch.  So the next kernel starts after the segment-mean
@@ -715,17 +641,19 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  const bool is_pinv = (int)blockIdx.x < prm.BH;
+  // Z is left in shared memory by the pseudoinverse (m <= 64, at least one step)
+  const bool z_in_smem = M <= 64 && is_pinv && prm.pinv.iters > 0;
   int bh;
-  if ((int)blockIdx.x < prm.BH) {
+  if (is_pinv) {
     bh = blockIdx.x;
     griddep_wait();
     griddep_launch_dependents();
     if constexpr (M <= 64) {
-      if (threadIdx.x < pinvpow::kBarThreads)
-        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem + MergeCfg<M>::zh,
-                              smem + MergeCfg<M>::zl);
+      if (t < pinvpow::kBarThreads)
+        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, (float *)(smem + C::zs));
     } else {
-      if (threadIdx.x < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
+      if (t < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
     }
   } else {
     const int b = blockIdx.x - prm.BH;
@@ -733,36 +661,34 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem, true);
   }
   // publish this block's results.  The last B~ V block of a head merges the
-  // partials into Y (while the pseudoinverse is still running, in general);
-  // the second of {pseudoinverse, Y merge} to finish forms W = Z Y, with Z
-  // already in shared memory as the W operand when that is the
-  // pseudoinverse block (m <= 64, at least one step).  Counters: count[bh]
-  // B~ V blocks done, count[BH + bh] inputs of W ready.
+  // partials into Y; the second of {pseudoinverse, Y merge} to finish forms
+  // W = Z Y.  Counters: count[bh] B~ V blocks done, count[BH + bh] inputs of
+  // W ready.
   __threadfence();
   __syncthreads();
-  const bool is_pinv = (int)blockIdx.x < prm.BH;
-  if (threadIdx.x == 0)
+  if (t == 0)
     last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
   __syncthreads();
   if (last) {
-    // a B~ V block that merges Y keeps a copy in shared memory for W
-    float *ysm = (M <= 64 && !is_pinv) ? (float *)(smem + MergeCfg<M>::ys) : nullptr;
     if (!is_pinv) {
       __threadfence();
-      merge_y_body<M>(prm, smem, bh, ysm);
+      merge_y_body<M>(prm, smem, bh, (float *)(smem + C::ys));
       __threadfence();
       __syncthreads();
     }
-    if (threadIdx.x == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
+    if (t == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
     __syncthreads();
     if (last) {
       __threadfence();
-      w_body<M>(prm, smem, bh, tmem, M <= 64 && is_pinv && prm.pinv.iters > 0, ysm);
+      if (is_pinv) load_y<M>(prm, smem, bh);
+      if (!z_in_smem) load_z<M>(prm, smem, bh);
+      __syncthreads();
+      w_product<M>(prm, smem, bh);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if ((threadIdx.x >> 5) == 1) {
+  if ((t >> 5) == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -155,13 +155,13 @@ __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
 // scale_log2 = log2(e) / sqrt(d).
 // tmem_in: a TMEM allocation of at least Cfg<M>::kTmemCols columns owned by
 // the caller, or ~0u to allocate (and free) one here.
-// zop_hi / zop_lo (optional): after the last step the final Z is also
-// written there as the hi / lo tf32 K-major operand (128-row slabs of 32
-// columns) of a following W = Z Y product in the same block.
+// zsm (optional, at least one step): after the last step the final Z is
+// also written there, fp32 row-major with a row stride of M + 4 floats, for a
+// following W = Z Y in the same block.  It may overlap the operand buffers
+// (written after the last product has read them).
 template <int M, class Prm>
 __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
-                                          uint32_t tmem_in = ~0u, uint8_t *zop_hi = nullptr,
-                                          uint8_t *zop_lo = nullptr) {
+                                          uint32_t tmem_in = ~0u, float *zsm = nullptr) {
   using C = Cfg<M>;
   constexpr int NC = C::NC;
   const int t = threadIdx.x, warp = t >> 5;
@@ -459,26 +459,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
           *(float4 *)(zg + (size_t)row * M + c_lo + 4 * q) =
               make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
       }
-      if (zop_hi) {
+      if (zsm) {
         named_barrier(1, kBarThreads);   // every operand buffer of the steps is dead
         if (ok && aux) {
 #pragma unroll
-          for (int q = 0; q < NC / 4; ++q) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint32_t h;
-              asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(z[4 * q + e]));
-              hi[e] = h;
-              uint32_t l;
-              asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(l) : "f"(z[4 * q + e] - __uint_as_float(h)));
-              lo[e] = l;
-            }
-            const int k = c_lo + 4 * q;
-            const uint32_t off = (uint32_t)(k >> 5) * 16384u + sw128_offset(row, (k & 31) >> 2);
-            st_shared_v4(smem_u32(zop_hi) + off, hi[0], hi[1], hi[2], hi[3]);
-            st_shared_v4(smem_u32(zop_lo) + off, lo[0], lo[1], lo[2], lo[3]);
-          }
+          for (int q = 0; q < NC / 4; ++q)
+            *(float4 *)(zsm + row * (M + 4) + c_lo + 4 * q) =
+                make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
         }
       }
     }
