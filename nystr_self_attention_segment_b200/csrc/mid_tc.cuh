@@ -1,26 +1,28 @@
 // Middle stage of the bf16 path, one launch:
 //   blocks [0, BH)            the landmark kernel A and its pseudoinverse Z
-//                             (one head each, see pinv_tc.cuh),
+//                             (one head each: pinv_pow.cuh for m <= 64,
+//                             pinv_tc.cuh for m = 128),
 //   blocks [BH, BH*(1+S))     Y = B~ V streamed over the keys, S blocks per head
 //                             ("Nystromformer: A Nystrom-Based Algorithm for
 //                             Approximating Self-Attention", section 3.4,
 //                             Eq. 17 / Algorithm 1; B~ = softmax(Q~ K^T/sqrt(d))
-//                             over the n keys is never stored),
-// and the last block of a head to finish (counted with an atomic) merges the
-// head's S partial softmax states in a fixed order into Y and forms W = Z Y.
+//                             over the n keys is never stored).
+// The last B~ V block of a head (counted with an atomic) merges the head's S
+// partial softmax states in a fixed order into Y; the second of {that
+// block, the pseudoinverse block} to finish forms W = Z Y in fp32.
 //
 // B~ V block.  The 128 accumulator rows (TMEM lanes) hold G = 128 / m copies
 // of the m landmark rows; copy g handles keys g*m .. g*m + m - 1 of every
 // 128-key chunk, so every TMEM lane has work.  Per chunk:
 //   TMA  K and V chunks (128 x 64 bf16, zero past n),
 //   MMA  S = [Q~; ..; Q~] K_c^T       (M=128, N=128, K=64, operands in smem),
-//   softmax warpgroup: running max / sum per row (log2 units), P = 2^(..) as
-//        bf16 straight into TMEM (zero outside the row's key group),
-//   MMA  Y_c = P V_c                   (M=128, N=64, K=128, P read from TMEM),
-//   softmax warpgroup: acc = acc * 2^(m_old - m_new) + Y_c in registers.
+//   softmax warpgroup: P = 2^(s - m_ref) as bf16 straight into TMEM (zero
+//        outside the row's key group), row sums in fp32,
+//   MMA  Y += P V_c                    (M=128, N=64, K=128, P read from TMEM,
+//        Y accumulated in TMEM).
 // Two softmax warpgroups take alternate chunks, each with its own TMEM
-// buffers and running state; the 2G states of a landmark are merged in the
-// block at the end, giving one partial per (block, landmark).
+// buffers, reference maxima and sums; the 2G states of a landmark are merged
+// in the block at the end, giving one partial per (block, landmark).
 // Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
 // warp 1 owns TMEM), 4-7 and 8-11 softmax.
 #pragma once
@@ -94,7 +96,7 @@ struct Params {
   float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
   float *y, *w;               // [BH][m][64]
   uint8_t *w_op;              // [BH][m][128 B] W as the bf16 B operand of P W
-  uint32_t *count;            // [BH] blocks finished per head (zeroed per call)
+  uint32_t *count;            // [2 BH] per head: B~ V blocks done, inputs of W ready (zeroed per call)
   uint32_t *err;
   int BH, n, chunks_per_head, splits;
   float scale_log2;
