@@ -65,19 +65,34 @@ KERNEL_SOURCES = {
 }
 
 
-def source_digest(kernel):
+def code_tokens(text):
+    """C++ source without comments, whitespace runs collapsed: what the
+    compiler sees, so that comment edits keep a recorded profile valid."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def source_digest(kernel, read=None):
+    """Digest of the code (comments excluded) of a kernel's source files."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES.get(kernel, []):
-        with open(os.path.join(ROOT, "nystr_self_attention_segment_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        if read is None:
+            with open(os.path.join(ROOT, "nystr_self_attention_segment_b200", "csrc", f)) as fh:
+                text = fh.read()
+        else:
+            text = read(f)
+        h.update(code_tokens(text).encode())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes (read + write) per launch from the committed ncu summary
     profiles/<kernel>_<workload>.md ("traffic_bytes:" and "source_digest:"
-    lines), or None when absent or when the kernel sources have changed."""
+    lines), or None when absent or when the code of the kernel sources has
+    changed since (comments and whitespace do not count)."""
     p = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
     if not os.path.exists(p):
         return None

@@ -1,0 +1,47 @@
+"""Host logic of the benchmark that decides whether a committed ncu figure
+still describes the kernels: the code digest ignores comments and
+whitespace, follows any change of code, and the recorded DRAM traffic is
+read only while the digest matches."""
+import os
+
+import bench
+
+
+def test_code_tokens_drop_comments_and_whitespace():
+    a = "int x = 1;  // one\n/* block\n comment */ float y=2;\n"
+    b = "int x = 1;\nfloat y=2; // other words\n"
+    assert bench.code_tokens(a) == bench.code_tokens(b)
+    assert bench.code_tokens(a) == "int x = 1; float y=2;"
+
+
+def test_code_change_changes_the_digest():
+    files = bench.KERNEL_SOURCES["mid_tc"]
+    real = {}
+    for f in files:
+        with open(os.path.join(bench.ROOT, "nystr_self_attention_segment_b200", "csrc", f)) as fh:
+            real[f] = fh.read()
+    base = bench.source_digest("mid_tc")
+    assert bench.source_digest("mid_tc", real.get) == base
+    commented = dict(real)
+    commented[files[-1]] = "// a new comment line\n" + real[files[-1]] + "\n/* trailing */\n"
+    assert bench.source_digest("mid_tc", commented.get) == base
+    edited = dict(real)
+    edited[files[-1]] = real[files[-1]].replace("kStages = 6", "kStages = 5", 1)
+    assert edited[files[-1]] != real[files[-1]]
+    assert bench.source_digest("mid_tc", edited.get) != base
+
+
+def test_recorded_traffic_needs_a_matching_digest(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "mid_tc_w.md").write_text(
+        "traffic_bytes: 1234\nsource_digest: `%s`\n" % bench.source_digest("mid_tc"))
+    (prof / "mid_tc_stale.md").write_text("traffic_bytes: 1234\nsource_digest: `0000`\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the digest reads the sources under ROOT too: give it the real tree
+    real_root = os.path.dirname(os.path.abspath(bench.__file__))
+    os.symlink(os.path.join(real_root, "nystr_self_attention_segment_b200"),
+               tmp_path / "nystr_self_attention_segment_b200")
+    assert bench.recorded_traffic("mid_tc", "w") == 1234
+    assert bench.recorded_traffic("mid_tc", "stale") is None
+    assert bench.recorded_traffic("mid_tc", "absent") is None
