@@ -76,17 +76,25 @@ def segment_means(X, m):
     Eq. 16 with the page's own 1/l correction; [P1] "How do we select
     landmarks?").
 
-    X: [n, d].  Returns [m, d]: row j is the mean of rows j*l .. j*l + l - 1,
-    l = n / m.  n must be a multiple of m (the pages assume this, "can be
-    ensured by padding")."""
+    X: [n, d].  Returns [m, d]: row j is the mean of the tokens of segment j,
+    rows j*l .. min(j*l + l, n) - 1 with l = ceil(n / m).  When m divides n
+    every segment holds l = n / m tokens, as on the pages.  Otherwise the
+    sequence is read as padded to m * l tokens ("can be ensured by padding")
+    and each landmark is the mean over the real tokens of its segment, so
+    the pad value never enters.  Raises ValueError when a segment would hold
+    no real token ((m - 1) * l >= n)."""
     X = _f64(X)
     n, d = X.shape
-    if m < 1 or n % m != 0:
-        raise ValueError("segment_means needs m >= 1 dividing n (n=%d, m=%d)" % (n, m))
-    seg = n // m
+    if m < 1 or m > n:
+        raise ValueError("segment_means needs 1 <= m <= n (n=%d, m=%d)" % (n, m))
+    seg = -(-n // m)
+    if (m - 1) * seg >= n:
+        raise ValueError("segment_means: a segment of %d tokens would be empty (n=%d, m=%d)"
+                         % (seg, n, m))
     out = np.empty((m, d), dtype=np.float64)
     for j in range(m):
-        out[j] = X[j * seg:(j + 1) * seg].sum(axis=0) / seg
+        rows = X[j * seg:min((j + 1) * seg, n)]
+        out[j] = rows.sum(axis=0) / rows.shape[0]
     return out
 
 

@@ -59,9 +59,60 @@ def test_segment_means_constant_segments():
     np.testing.assert_allclose(orc.segment_means(X, 4), vals, rtol=0, atol=1e-15)
 
 
-def test_segment_means_rejects_indivisible():
+def test_segment_means_ragged_bruteforce_loops():
+    # m does not divide n: segments of ceil(n/m) tokens, the last one short,
+    # each averaged over its own tokens (n=14, m=4: 4, 4, 4 and 2 tokens).
+    rng = _rng(41)
+    n, m, d = 14, 4, 3
+    X = rng.standard_normal((n, d))
+    got = orc.segment_means(X, m)
+    bounds = [(0, 4), (4, 8), (8, 12), (12, 14)]
+    for j, (a, b) in enumerate(bounds):
+        for c in range(d):
+            acc = 0.0
+            for t in range(a, b):
+                acc += float(X[t, c])
+            assert abs(got[j, c] - acc / (b - a)) < 1e-15
+
+
+def test_segment_means_ragged_is_zero_padding_over_true_counts():
+    # The padded reading: pad with zeros to m * ceil(n/m) tokens, sum each
+    # segment of the padded sequence, divide by the number of real tokens in
+    # it.  Any pad value other than zero would show up here.
+    rng = _rng(42)
+    n, m, d = 70, 8, 5
+    seg = -(-n // m)
+    X = rng.standard_normal((n, d))
+    P = np.zeros((m * seg, d))
+    P[:n] = X
+    sums = P.reshape(m, seg, d).sum(axis=1)
+    counts = np.minimum(seg, n - np.arange(m) * seg)
+    np.testing.assert_allclose(orc.segment_means(X, m), sums / counts[:, None], rtol=0,
+                               atol=1e-14)
+
+
+def test_segment_means_ragged_weighted_mean_and_constants():
+    # sum_j count_j * landmark_j == sum of all tokens, and a segment of equal
+    # rows keeps that row, the short last one included.
+    rng = _rng(43)
+    n, m = 4090, 128                       # 127 segments of 32, the last of 26
+    X = rng.standard_normal((n, 4))
+    L = orc.segment_means(X, m)
+    counts = np.array([32] * 127 + [26], dtype=np.float64)
+    np.testing.assert_allclose((counts[:, None] * L).sum(axis=0), X.sum(axis=0), rtol=0,
+                               atol=1e-10)
+    vals = rng.standard_normal((5, 2))
+    Y = np.repeat(vals, [4, 4, 4, 4, 1], axis=0)   # n=17, m=5: segments of 4, the last of 1
+    np.testing.assert_allclose(orc.segment_means(Y, 5), vals, rtol=0, atol=1e-15)
+
+
+def test_segment_means_rejects_empty_segments():
+    # n=5, m=4: segments of 2 tokens would leave the fourth one empty.
     with pytest.raises(ValueError):
-        orc.segment_means(np.zeros((10, 2)), 3)
+        orc.segment_means(np.zeros((5, 2)), 4)
+    with pytest.raises(ValueError):
+        orc.segment_means(np.zeros((65, 2)), 64)
+    orc.segment_means(np.zeros((10, 2)), 3)        # 4, 4, 2: all non-empty
 
 
 # ---------------------------------------------------------------- softmax kernels
