@@ -9,9 +9,12 @@
  * Approximating Self-Attention", section 3.4, and of the blog post
  * "Approximating self-attention in linear time and memory via the Nystrom
  * method"):
- *   Q~, K~  segment means of Q, K over l = n/m contiguous tokens (Eq. 16,
- *           with the page's own divide-by-l correction; blog "How do we select
- *           landmarks?"),
+ *   Q~, K~  segment means of Q, K over l = ceil(n/m) contiguous tokens
+ *           (Eq. 16, with the page's own divide-by-l correction; blog "How do
+ *           we select landmarks?").  When m does not divide n the sequence
+ *           reads as padded to m*l tokens ("can be ensured by padding"): the
+ *           last segment is shorter and each landmark is the mean over the
+ *           real tokens of its segment, so no pad value enters,
  *   F~      = softmax(Q K~^T / sqrt(d)), n x m, softmax over the m landmarks,
  *   A       = softmax(Q~ K~^T / sqrt(d)), m x m, row-wise,
  *   Z       = pinv_iters steps of Lemma 1 from Z0 = A^T / (||A||_1 ||A||_inf)
@@ -38,8 +41,10 @@
  *  - batch * heads * seq_len == 0 is valid and enqueues nothing.
  *
  * Supported shapes:
- *  - NYS_F32:  1 <= head_dim <= 64, 1 <= m <= 64, m <= seq_len, m | seq_len.
- *  - NYS_BF16: head_dim == 64, m in {32, 64, 128}, m <= seq_len, m | seq_len.
+ *  - NYS_F32:  1 <= head_dim <= 64, 1 <= m <= 64, m <= seq_len.
+ *  - NYS_BF16: head_dim == 64, m in {32, 64, 128}, m <= seq_len.
+ *  - Every segment holds at least one token: (m - 1) * ceil(seq_len / m) <
+ *    seq_len (always true when m divides seq_len or seq_len >= m * m).
  *  - conv_k odd, 1 <= conv_k <= 63 (or conv_w == NULL / conv_k == 0: no skip).
  *  - 0 <= pinv_iters <= 64.
  */
@@ -59,7 +64,7 @@ typedef enum {
   NYS_OK = 0,
   NYS_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum value      */
   NYS_ERR_UNSUPPORTED = 2,   /* valid request without a kernel (d, m, dtype, k)  */
-  NYS_ERR_NOT_DIVISIBLE = 3, /* seq_len is not a multiple of num_landmarks       */
+  NYS_ERR_NOT_DIVISIBLE = 3, /* a segment of ceil(seq_len/m) tokens would be empty */
   NYS_ERR_ALIAS = 4,         /* out overlaps Q, K, V or the workspace            */
   NYS_ERR_WORKSPACE = 5,     /* workspace smaller than nys_attn_workspace_size   */
   NYS_ERR_CUDA = 6,          /* a CUDA runtime call or kernel launch failed      */

@@ -21,6 +21,14 @@ using namespace nys;
 
 namespace {
 
+// The persistent single-launch schedule (fused.cuh) is built but not the
+// default: its task bodies still run slower there than in the three-kernel
+// pipeline.  Compile with -DNYS_FUSED=1 to use it for m <= 64.
+#ifndef NYS_FUSED
+#define NYS_FUSED 0
+#endif
+constexpr bool kUseFused = NYS_FUSED != 0;
+
 size_t elem_size(int dtype) { return dtype == NYS_BF16 ? 2 : 4; }
 
 nys_status validate_shape(const nys_desc *desc, int m) {
@@ -31,12 +39,17 @@ nys_status validate_shape(const nys_desc *desc, int m) {
   if (m < 1) return NYS_ERR_INVALID_ARG;
   if ((long)desc->batch * desc->heads * desc->seq_len == 0) return NYS_OK;   // empty
   if (m > desc->seq_len) return NYS_ERR_INVALID_ARG;
-  if (desc->seq_len % m != 0) return NYS_ERR_NOT_DIVISIBLE;
+  {   // segments of ceil(n / m) tokens, the last one possibly shorter: none empty
+    const long seg = ((long)desc->seq_len + m - 1) / m;
+    if ((long)(m - 1) * seg >= desc->seq_len) return NYS_ERR_NOT_DIVISIBLE;
+  }
   if (desc->dtype == NYS_F32) {
     if (desc->head_dim > 64 || m > 64) return NYS_ERR_UNSUPPORTED;
   } else {
     if (desc->head_dim != 64) return NYS_ERR_UNSUPPORTED;
     if (m != 32 && m != 64 && m != 128) return NYS_ERR_UNSUPPORTED;
+    // the persistent schedule sums equal segments only
+    if (kUseFused && m <= 64 && desc->seq_len % m != 0) return NYS_ERR_UNSUPPORTED;
   }
   if ((long)desc->batch * desc->heads > (1L << 24) || desc->seq_len > (1 << 24))
     return NYS_ERR_UNSUPPORTED;
@@ -47,13 +60,6 @@ bool is_empty(const nys_desc *desc) {
   return (long)desc->batch * desc->heads * desc->seq_len == 0;
 }
 
-// The persistent single-launch schedule (fused.cuh) is built but not the
-// default: its task bodies still run slower there than in the three-kernel
-// pipeline.  Compile with -DNYS_FUSED=1 to use it for m <= 64.
-#ifndef NYS_FUSED
-#define NYS_FUSED 0
-#endif
-constexpr bool kUseFused = NYS_FUSED != 0;
 
 Layout make_layout(const nys_desc *desc, int m) {
   Layout L;
@@ -372,7 +378,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     return NYS_ERR_CUDA;
 
   {   // segment means of Q and K (Eq. 16)
-    const int seg = n / M;
+    const int seg = (n + M - 1) / M;   // tokens of a full segment
     const int groups = seg < 32 ? seg : 32;
     seg_means_bf16<<<dim3(M, BH, 2), 8 * groups, 0, stream>>>(Q, K, qt, kt, n, M);
     mk.after(stream);
@@ -447,7 +453,7 @@ NYS_ATTN_API const char *nys_status_string(nys_status s) {
     case NYS_OK: return "NYS_OK";
     case NYS_ERR_INVALID_ARG: return "NYS_ERR_INVALID_ARG: null pointer, negative size or bad enum";
     case NYS_ERR_UNSUPPORTED: return "NYS_ERR_UNSUPPORTED: no kernel for this head_dim / landmarks / dtype / conv_k";
-    case NYS_ERR_NOT_DIVISIBLE: return "NYS_ERR_NOT_DIVISIBLE: seq_len is not a multiple of num_landmarks";
+    case NYS_ERR_NOT_DIVISIBLE: return "NYS_ERR_NOT_DIVISIBLE: a segment of ceil(seq_len / num_landmarks) tokens would be empty";
     case NYS_ERR_ALIAS: return "NYS_ERR_ALIAS: output overlaps an input or the workspace";
     case NYS_ERR_WORKSPACE: return "NYS_ERR_WORKSPACE: workspace too small";
     case NYS_ERR_CUDA: return "NYS_ERR_CUDA: CUDA runtime or launch failure";

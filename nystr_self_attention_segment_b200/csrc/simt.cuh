@@ -29,8 +29,9 @@ __global__ void seg_means_scalar(const T *__restrict__ Q, const T *__restrict__ 
   long jb = idx / d;            // bh * m + j
   int j = (int)(jb % m);
   long bh = jb / m;
-  int seg = n / m;
-  const T *src = X + ((size_t)bh * n + (size_t)j * seg) * d + c;
+  const int len = (n + m - 1) / m;            // l = ceil(n / m)
+  const int seg = min(len, n - j * len);      // real tokens of segment j (>= 1)
+  const T *src = X + ((size_t)bh * n + (size_t)j * len) * d + c;
   float acc = 0.f;
   for (int t = 0; t < seg; ++t) acc += to_f(src[(size_t)t * d]);
   Xt[idx] = acc / (float)seg;

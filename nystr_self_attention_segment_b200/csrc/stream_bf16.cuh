@@ -1,7 +1,9 @@
 // Memory-bound helpers of the bf16 path (head_dim = 64):
 //  * seg_means_bf16: Q~, K~ segment means ("Nystromformer: A Nystrom-Based
 //    Algorithm for Approximating Self-Attention", section 3.4, Eq. 16 with the
-//    page's 1/l correction), one pass over Q and K with 16-byte loads;
+//    page's 1/l correction), one pass over Q and K with 16-byte loads.
+//    Segment j holds tokens j*l .. min(j*l + l, n) - 1, l = ceil(n / m) (the
+//    sequence read as padded to m*l tokens), averaged over its real tokens;
 #pragma once
 
 #include "sm100.cuh"
@@ -19,10 +21,11 @@ seg_means_bf16(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restr
   const int j = blockIdx.x, bh = blockIdx.y;
   const __nv_bfloat16 *X = blockIdx.z == 0 ? Q : K;
   float *Xt = blockIdx.z == 0 ? Qt : Kt;
-  const int seg = n / m;
+  const int len = (n + m - 1) / m;                 // l
+  const int seg = min(len, n - j * len);           // real tokens of segment j (>= 1)
   const int groups = blockDim.x >> 3;          // row groups (<= 32)
   const int g = threadIdx.x >> 3, ch = threadIdx.x & 7;
-  const uint4 *src = (const uint4 *)(X + ((size_t)bh * n + (size_t)j * seg) * 64) + ch;
+  const uint4 *src = (const uint4 *)(X + ((size_t)bh * n + (size_t)j * len) * 64) + ch;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int r = g;
   // four rows in flight per thread

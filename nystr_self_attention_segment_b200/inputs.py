@@ -75,6 +75,8 @@ WORKLOADS = {
                                    values="lowrank16"),
     "headline_n8192_m32": Workload("headline_n8192_m32", 4, 2, 12, 8192, 64, 32, BF16, 33,
                                    values="lowrank16"),
+    # m does not divide n: segments of ceil(n/m) tokens, the last one shorter
+    "ragged_n8100_m64": Workload("ragged_n8100_m64", 6, 1, 2, 8100, 64, 64, BF16, 33),
 }
 for _n in (1024, 2048, 4096, 8192, 16384, 32768, 65536):
     WORKLOADS["sweep_n%d_m128" % _n] = _sweep(_n)

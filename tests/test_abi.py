@@ -73,7 +73,7 @@ S = _lib.STATUS
 
 
 def test_rejects_invalid_calls_without_launching():
-    assert forward_status(desc(n=8100), m=64) == S["NYS_ERR_NOT_DIVISIBLE"]
+    assert forward_status(desc(n=100), m=64) == S["NYS_ERR_NOT_DIVISIBLE"]   # 64 segments of 2
     assert forward_status(desc(d=32)) == S["NYS_ERR_UNSUPPORTED"]
     assert forward_status(desc(n=6144), m=48) == S["NYS_ERR_UNSUPPORTED"]
     assert forward_status(desc(nys.NYS_F32, n=8192), m=128) == S["NYS_ERR_UNSUPPORTED"]
@@ -107,6 +107,16 @@ def test_empty_problems_are_no_ops():
         assert forward_status(ds, q=None, k=None, v=None, out=None) == S["NYS_OK"]
         assert nys.nys_attn_workspace_size(ds, 64) == 0
         assert nys.nys_attn_launch_count(ds, 64, 33) == 0
+
+
+def test_ragged_segments_validate_when_none_is_empty():
+    # segments of ceil(n/m) tokens: valid while (m - 1) * ceil(n/m) < n
+    for n, m in ((8100, 64), (4090, 128), (1000, 32), (127, 64), (8192 + 1, 64)):
+        assert nys.nys_attn_workspace_size(desc(n=n), m) > 0, (n, m)
+    for n, m in ((126, 64), (100, 64), (65, 64), (4000, 128)):
+        with pytest.raises(nys.NysError) as e:
+            nys.nys_attn_workspace_size(desc(n=n), m)
+        assert e.value.name == "NYS_ERR_NOT_DIVISIBLE", (n, m)
 
 
 def test_size_queries_validate_too():

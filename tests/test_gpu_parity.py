@@ -75,7 +75,8 @@ def test_bf16_workload_against_oracle(name):
     assert max(errs) <= TOL["bf16"], errs
 
 
-@pytest.mark.parametrize("name", ["bert_n512_m64", "headline_n8192_m64", "sweep_n1024_m128"])
+@pytest.mark.parametrize("name", ["bert_n512_m64", "headline_n8192_m64", "sweep_n1024_m128",
+                                  "ragged_n8100_m64"])
 def test_bf16_intermediates(name):
     # Landmarks are fp32 sums of the same bf16 inputs; Z, Y and W are checked
     # against the oracle's steps applied to the device's own fp32 landmarks,
@@ -138,6 +139,13 @@ EDGE = [
     (1, 1, 24, 8, 3, F32, 3, 6),          # fp32, odd sizes
     (2, 2, 60, 17, 12, F32, 0, 6),
     (1, 1, 64, 64, 64, F32, 7, 2),
+    # m does not divide n: segments of ceil(n/m) tokens, the last one short
+    (1, 2, 8100, 64, 64, BF16, 33, 6),    # last segment 99 of 127 tokens
+    (1, 2, 4090, 64, 128, BF16, 33, 6),   # last segment 26 of 32
+    (2, 1, 1000, 64, 32, BF16, 33, 6),    # last segment 8 of 32
+    (1, 1, 127, 64, 64, BF16, 33, 6),     # last segment 1 of 2
+    (1, 1, 70, 32, 8, F32, 5, 6),         # last segment 7 of 9
+    (1, 1, 17, 8, 5, F32, 3, 6),          # last segment 1 of 4
 ]
 
 
