@@ -27,6 +27,14 @@ Readings where the pages are silent or inconsistent (each also listed in the
 design notes):
   * Eq. 16 prints a divide-by-m; the page itself calls that a typo.  Landmark j
     is the mean of the l = n/m contiguous tokens [j*l, (j+1)*l).
+  * When m does not divide n ("can be ensured by padding", no pad value given)
+    the sequence is read as padded to m*ceil(n/m) tokens and each landmark is
+    the mean over the real tokens of its segment of l = ceil(n/m); a shape
+    with an empty segment is rejected.
+  * Masks are not on the pages (every token attends to every token).  For
+    right-padded ragged batches (nystrom_forward_lens) an element with L real
+    tokens is the method on those L tokens alone, and its padding rows of
+    the output are zero.
   * The 1/sqrt(d) scale is applied inside all three softmaxes (P1 definitions,
     P5 Algorithm 1); the library excerpt omits it for brevity.
   * B~ is a softmax over the n keys for every landmark row (P1 definitions,
@@ -60,6 +68,7 @@ __all__ = [
     "depthwise_conv",
     "nystrom_head",
     "nystrom_forward",
+    "nystrom_forward_lens",
     "exact_attention_head",
     "exact_attention",
     "algorithmic_flops",
@@ -222,6 +231,31 @@ def nystrom_forward(Q, K, V, m, iters=6, conv_w=None, keep=()):
                 kept[name].append(r[name])
     extra = {name: np.stack(v).reshape((Bn, H) + v[0].shape) for name, v in kept.items()}
     return (out, extra) if keep else out
+
+
+def nystrom_forward_lens(Q, K, V, m, lens, iters=6, conv_w=None):
+    """Forward over right-padded ragged batches: element b holds lens[b] real
+    tokens followed by padding.  Each element is the method on its first
+    lens[b] tokens alone (landmarks, the softmax over keys, the queries and
+    the conv's zero padding all end at lens[b]); the padding rows of the
+    output are zero.  Q, K, V: [B, H, n, d]; lens: B ints, m <= lens[b] <= n.
+    Masks are not on the pages: this is the plainest reading for a caller
+    with ragged batches."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    Bn, H, n, d = Q.shape
+    lens = [int(x) for x in lens]
+    if len(lens) != Bn or any(L < m or L > n for L in lens):
+        raise ValueError("lens must hold B values in [m, n]")
+    out = np.zeros((Bn, H, n, d), dtype=np.float64)
+    for b in range(Bn):
+        L = lens[b]
+        for h in range(H):
+            w = None if conv_w is None else _f64(conv_w)[h]
+            r = nystrom_head(Q[b, h, :L], K[b, h, :L], V[b, h, :L], m, iters, w)
+            out[b, h, :L] = r["out"]
+    return out
 
 
 def exact_attention_head(Q, K, V, scale=None):

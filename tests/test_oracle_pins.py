@@ -324,3 +324,65 @@ def test_flop_and_byte_counts():
     # 8nmd + 4m^2 d + 48 m^3 per head at six iterations; 4 n d e bytes
     assert orc.algorithmic_flops(1, 1, 8192, 64, 64) == 8 * 8192 * 64 * 64 + 4 * 64 * 64 * 64 + 48 * 64 ** 3
     assert orc.algorithmic_bytes(2, 12, 8192, 64, 2) == 2 * 12 * 8192 * 64 * 2 * 4
+
+
+# ---------------------------------------------------------------- ragged batches
+
+def _ragged_inputs(seed, Bn=3, H=2, n=40, d=8):
+    rng = _rng(seed)
+    return (rng.standard_normal((Bn, H, n, d)), rng.standard_normal((Bn, H, n, d)),
+            rng.standard_normal((Bn, H, n, d)), 0.2 * rng.standard_normal((H, 5)))
+
+
+def test_lens_padding_content_never_enters():
+    # Garbage in the padding changes nothing, and padding rows come out zero.
+    Q, K, V, w = _ragged_inputs(51)
+    lens = [40, 29, 16]                     # 29: segments of 4, the last of 1
+    ref = orc.nystrom_forward_lens(Q, K, V, 8, lens, 6, w)
+    rng = _rng(52)
+    Q2, K2, V2 = Q.copy(), K.copy(), V.copy()
+    for b, L in enumerate(lens):
+        for X in (Q2, K2, V2):
+            X[b, :, L:] = 1e3 * rng.standard_normal(X[b, :, L:].shape)
+    got = orc.nystrom_forward_lens(Q2, K2, V2, 8, lens, 6, w)
+    np.testing.assert_array_equal(got, ref)
+    for b, L in enumerate(lens):
+        assert not got[b, :, L:].any()
+
+
+def test_lens_equal_to_n_is_the_plain_forward():
+    Q, K, V, w = _ragged_inputs(53)
+    np.testing.assert_array_equal(orc.nystrom_forward_lens(Q, K, V, 8, [40] * 3, 6, w),
+                                  orc.nystrom_forward(Q, K, V, 8, 6, w))
+
+
+def test_lens_lemma2_exact_attention_over_real_tokens():
+    # m = L real tokens with a converged pseudoinverse: exact softmax
+    # attention over those L tokens only (brute force on the truncated
+    # sequence); a softmax that let the padding in would miss this.
+    Q, K, V, _ = _ragged_inputs(54, Bn=2, H=1, n=24, d=6)
+    Q *= 0.3
+    K *= 0.3
+    lens = [20, 10]
+    got = orc.nystrom_forward_lens(Q, K, V, 10, lens, 60, None)
+    for b, L in enumerate(lens):
+        if L != 10:
+            continue
+        want = orc.exact_attention_head(Q[b, 0, :L], K[b, 0, :L], V[b, 0, :L])
+        np.testing.assert_allclose(got[b, 0, :L], want, rtol=0, atol=1e-9)
+
+
+def test_lens_uniform_queries_closed_form_with_boundary_conv():
+    # Q = 0: every softmax is uniform and Z0 = J/m is a fixed point, so each
+    # real row is the mean of the real V rows, plus the conv of the real rows
+    # with zeros past L (numpy.correlate).
+    Q, K, V, w = _ragged_inputs(55, Bn=2, H=2, n=30, d=4)
+    Q[:] = 0.0
+    lens = [30, 21]                         # 21: segments of 4, the last of 1
+    got = orc.nystrom_forward_lens(Q, K, V, 6, lens, 6, w)
+    for b, L in enumerate(lens):
+        for h in range(2):
+            mean = V[b, h, :L].mean(axis=0)
+            for c in range(4):
+                conv = np.correlate(np.pad(V[b, h, :L, c], 2), w[h], mode="valid")
+                np.testing.assert_allclose(got[b, h, :L, c], mean[c] + conv, rtol=0, atol=1e-12)
