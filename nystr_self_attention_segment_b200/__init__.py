@@ -44,6 +44,38 @@ def desc_of(Q):
     return make_desc(_dtype_code(Q), b, h, n, d)
 
 
+def _check_operands(Q, K, V, out, conv_w, on_cuda=True):
+    """Q, K, V and out: contiguous tensors of one shape and dtype on one
+    device (CUDA, or CPU for the host-buffer entry point); conv_w: None or a
+    contiguous float32 [heads, k] tensor on that device.  The kernels size
+    every access from Q's descriptor, so a mismatch caught here would
+    otherwise be an out-of-bounds access on the device."""
+    torch = _torch()
+    where = "CUDA" if on_cuda else "CPU"
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("out", out)):
+        if bool(t.is_cuda) != on_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous %s tensor" % (name, where))
+        if tuple(t.shape) != tuple(Q.shape) or t.dtype != Q.dtype or t.device != Q.device:
+            raise ValueError("%s must match Q in shape, dtype and device" % name)
+    if conv_w is not None:
+        if (conv_w.dtype != torch.float32 or bool(conv_w.is_cuda) != on_cuda
+                or not conv_w.is_contiguous() or conv_w.device != Q.device):
+            raise ValueError("conv_w must be a contiguous float32 %s tensor [heads, k] on "
+                             "the device of Q" % where)
+        if conv_w.dim() != 2 or conv_w.shape[0] != Q.shape[1]:
+            raise ValueError("conv_w must be [heads, k]")
+
+
+def _on_device(dev):
+    """The current-device context for a CUDA device (nothing to do when it
+    is already current, which keeps graph capture untouched)."""
+    import contextlib
+    torch = _torch()
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
+
+
 def _stream_ptr(stream):
     torch = _torch()
     s = torch.cuda.current_stream() if stream is None else stream
@@ -82,27 +114,20 @@ def nys_attn_forward(Q, K, V, num_landmarks, pinv_iters=6, conv_w=None, out=None
     or None.  workspace: a Workspace for this shape, or None (the library then
     allocates one stream-ordered per call).  Asynchronous on `stream`."""
     torch = _torch()
-    for name, t in (("Q", Q), ("K", K), ("V", V)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("%s must be a contiguous CUDA tensor" % name)
-        if t.shape != Q.shape or t.dtype != Q.dtype:
-            raise ValueError("Q, K, V must share shape and dtype")
-    desc = desc_of(Q)
-    if out is None:
+    if out is None and getattr(Q, "is_cuda", False):
         out = torch.empty_like(Q)
+    _check_operands(Q, K, V, Q if out is None else out, conv_w)
+    desc = desc_of(Q)
     conv_ptr, conv_k = None, 0
     if conv_w is not None:
-        if conv_w.dtype != torch.float32 or not conv_w.is_cuda or not conv_w.is_contiguous():
-            raise ValueError("conv_w must be a contiguous float32 CUDA tensor [heads, k]")
-        if conv_w.dim() != 2 or conv_w.shape[0] != Q.shape[1]:
-            raise ValueError("conv_w must be [heads, k]")
         conv_ptr, conv_k = conv_w.data_ptr(), conv_w.shape[1]
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = workspace.ptr, workspace.nbytes
-    st = _lib.raw_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
-                          pinv_iters, conv_ptr, conv_k, out.data_ptr(), ws_ptr, ws_bytes,
-                          _stream_ptr(stream))
+    with _on_device(Q.device):
+        st = _lib.raw_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
+                              pinv_iters, conv_ptr, conv_k, out.data_ptr(), ws_ptr, ws_bytes,
+                              _stream_ptr(stream))
     _lib.check(st, "nys_attn_forward")
     return out
 
@@ -111,15 +136,17 @@ def nys_attn_forward_timed(Q, K, V, num_landmarks, pinv_iters, conv_w, out, work
                            stream=None):
     """nys_attn_forward recording events[0] before the first kernel and
     events[i + 1] after kernel i (torch.cuda.Event objects with timing)."""
+    _check_operands(Q, K, V, out, conv_w)
     desc = desc_of(Q)
     conv_ptr, conv_k = (None, 0) if conv_w is None else (conv_w.data_ptr(), conv_w.shape[1])
     for e in events:
         if not e.cuda_event:          # torch creates the CUDA event on first record
             e.record()
-    st = _lib.raw_forward_timed(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
-                                pinv_iters, conv_ptr, conv_k, out.data_ptr(), workspace.ptr,
-                                workspace.nbytes, _stream_ptr(stream),
-                                [e.cuda_event for e in events])
+    with _on_device(Q.device):
+        st = _lib.raw_forward_timed(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc,
+                                    num_landmarks, pinv_iters, conv_ptr, conv_k, out.data_ptr(),
+                                    workspace.ptr, workspace.nbytes, _stream_ptr(stream),
+                                    [e.cuda_event for e in events])
     _lib.check(st, "nys_attn_forward_timed")
     return out
 
@@ -138,13 +165,18 @@ def nys_attn_forward_host(Qh, Kh, Vh, num_landmarks, pinv_iters, conv_w_host, ou
     all enqueued on `stream`.  device_buf: a CUDA uint8 tensor of at least
     nys_attn_host_buffer_size bytes (256-byte aligned).  Returns out_host;
     synchronise the stream before reading it."""
+    _check_operands(Qh, Kh, Vh, out_host, conv_w_host, on_cuda=False)
+    if not device_buf.is_cuda or not device_buf.is_contiguous():
+        raise ValueError("device_buf must be a contiguous CUDA tensor")
     desc = desc_of(Qh)
     conv_ptr, conv_k = None, 0
     if conv_w_host is not None:
         conv_ptr, conv_k = conv_w_host.data_ptr(), conv_w_host.shape[1]
-    st = _lib.raw_forward_host(Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), desc,
-                               num_landmarks, pinv_iters, conv_ptr, conv_k,
-                               out_host.data_ptr(), device_buf.data_ptr(), device_buf.numel(),
-                               _stream_ptr(stream))
+    with _on_device(device_buf.device):
+        st = _lib.raw_forward_host(Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), desc,
+                                   num_landmarks, pinv_iters, conv_ptr, conv_k,
+                                   out_host.data_ptr(), device_buf.data_ptr(),
+                                   device_buf.numel() * device_buf.element_size(),
+                                   _stream_ptr(stream))
     _lib.check(st, "nys_attn_forward_host")
     return out_host
