@@ -99,14 +99,15 @@ NYS_ATTN_API nys_status nys_attn_workspace_size(const nys_desc *desc, int num_la
 
 /* The forward pass (Eq. 17 / Algorithm 1 with the Figure 4 DConv skip of the
  * paper summary).
- *   Q_dev, K_dev, V_dev  inputs, layout above.
- *   num_landmarks        m; seq_len must be a multiple of m (the pages pad to
- *                        ensure this; padding is not done here).
+ *   Q_dev, K_dev, V_dev  inputs, layout above; 16-byte aligned for NYS_BF16,
+ *                        4-byte aligned for NYS_F32 (else NYS_ERR_INVALID_ARG).
+ *   num_landmarks        m; segments of ceil(seq_len / m) tokens, the last one
+ *                        possibly shorter, none empty (see Supported shapes).
  *   pinv_iters           steps of Lemma 1 (the paper uses 6).
- *   conv_w_dev           [heads][conv_k] fp32 kernel of the DConv skip, or NULL
- *                        for no skip (then conv_k is ignored).
- *   out_dev              output, same dtype and layout as Q; must not overlap
- *                        any input or the workspace.
+ *   conv_w_dev           [heads][conv_k] fp32 kernel of the DConv skip, 4-byte
+ *                        aligned, or NULL for no skip (then conv_k is ignored).
+ *   out_dev              output, same dtype, layout and alignment as Q; must
+ *                        not overlap any input or the workspace.
  *   workspace_dev        device scratch of at least nys_attn_workspace_size
  *                        bytes, 256-byte aligned, or NULL: then the call
  *                        allocates and frees it stream-ordered

@@ -506,9 +506,11 @@ static nys_status validate_call(const void *Q, const void *K, const void *V,
   }
   if (is_empty(desc)) return NYS_OK;
   if (!Q || !K || !V || !out) return NYS_ERR_INVALID_ARG;
-  if (desc->dtype == NYS_BF16 &&
-      (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)out) & 15) != 0)
+  // tensor-memory-access maps and 16-byte loads (bf16), 4-byte loads (fp32)
+  const uintptr_t align = desc->dtype == NYS_BF16 ? 15 : 3;
+  if ((((uintptr_t)Q | (uintptr_t)K | (uintptr_t)V | (uintptr_t)out) & align) != 0)
     return NYS_ERR_INVALID_ARG;
+  if (conv_w && ((uintptr_t)conv_w & 3) != 0) return NYS_ERR_INVALID_ARG;
   return NYS_OK;
 }
 

@@ -92,6 +92,12 @@ def test_rejects_invalid_calls_without_launching():
     # output aliasing an input, or partly overlapping one
     assert forward_status(desc(), out=FAKE) == S["NYS_ERR_ALIAS"]
     assert forward_status(desc(), out=FAKE + (2 << 32) + 4096) == S["NYS_ERR_ALIAS"]
+    # misaligned operands: 16 bytes for bf16, 4 for fp32 and the conv weights
+    assert forward_status(desc(), q=FAKE + 8) == S["NYS_ERR_INVALID_ARG"]
+    assert forward_status(desc(), out=FAKE + (3 << 32) + 2) == S["NYS_ERR_INVALID_ARG"]
+    f32 = desc(nys.NYS_F32, b=1, h=1, n=64, d=32)
+    assert forward_status(f32, m=8, k=FAKE + (1 << 32) + 2) == S["NYS_ERR_INVALID_ARG"]
+    assert forward_status(desc(), conv=FAKE + (5 << 32) + 2, conv_k=33) == S["NYS_ERR_INVALID_ARG"]
     # workspace too small or misaligned
     ds = desc()
     need = nys.nys_attn_workspace_size(ds, 64)
