@@ -135,3 +135,59 @@ def test_size_queries_validate_too():
     assert lib.nys_attn_workspace_size(ctypes.byref(desc()), 64, None) == S["NYS_ERR_INVALID_ARG"]
     assert lib.nys_attn_workspace_size(None, 64, ctypes.byref(ctypes.c_size_t())) == \
         S["NYS_ERR_INVALID_ARG"]
+
+
+# ------------------------------------------------------------------ layout property
+
+from hypothesis import given, settings, strategies as st   # noqa: E402
+
+
+def _valid_n(n, m):
+    seg = -(-n // m)
+    return (m - 1) * seg < n
+
+
+@settings(max_examples=300, deadline=None)
+@given(b=st.integers(1, 8), h=st.integers(1, 24), m=st.sampled_from([32, 64, 128]),
+       n=st.integers(32, 70000))
+def test_bf16_layout_holds_every_region(b, h, m, n):
+    # Every region the kernels write, for any valid shape: the five exported
+    # intermediates 256-byte aligned and disjoint inside the total, and room
+    # in the total for the split partial states (S splits of m x (64 + 2)
+    # floats per head) and the bf16 W operand the merge and the output
+    # kernel use.
+    if n < m or not _valid_n(n, m):
+        with pytest.raises(nys.NysError):
+            nys.nys_attn_workspace_size(desc(b=b, h=h, n=n), m)
+        return
+    ds = desc(b=b, h=h, n=n)
+    ws = nys.nys_attn_workspace_size(ds, m)
+    lay = nys.nys_attn_intermediates(ds, m)
+    bh = b * h
+    regions = [(lay["q_landmarks"], bh * m * 64 * 4), (lay["k_landmarks"], bh * m * 64 * 4),
+               (lay["z"], bh * m * m * 4), (lay["y"], bh * m * 64 * 4),
+               (lay["w"], bh * m * 64 * 4), (lay["error_word"], 256 + bh * 12)]
+    for off, size in regions:
+        assert off % 256 == 0 and off + size <= ws
+    regions.sort()
+    for (a, sa), (c, _) in zip(regions, regions[1:]):
+        assert a + sa <= c
+    chunks = -(-n // 128)
+    splits = max(1, min((148 - bh) // bh, chunks, 16))
+    partials = bh * splits * m * (64 + 2) * 4
+    assert ws >= sum(sz for _, sz in regions) + partials + bh * m * 128
+
+
+@settings(max_examples=200, deadline=None)
+@given(m=st.integers(1, 64), d=st.integers(1, 64), n=st.integers(1, 3000))
+def test_f32_shapes_validate_by_the_segment_rule(m, d, n):
+    ds = desc(nys.NYS_F32, b=1, h=2, n=n, d=d)
+    if m > n:
+        with pytest.raises(nys.NysError):
+            nys.nys_attn_workspace_size(ds, m)
+    elif not _valid_n(n, m):
+        with pytest.raises(nys.NysError) as e:
+            nys.nys_attn_workspace_size(ds, m)
+        assert e.value.name == "NYS_ERR_NOT_DIVISIBLE"
+    else:
+        assert nys.nys_attn_workspace_size(ds, m) > 0
