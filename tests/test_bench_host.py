@@ -1,7 +1,10 @@
-"""Host logic of the benchmark that decides whether a committed ncu figure
-still describes the kernels: the code digest ignores comments and
-whitespace, follows any change of code, and the recorded DRAM traffic is
-read only while the digest matches."""
+"""Host logic of the benchmark.
+
+- Whether a committed ncu figure still describes the kernels: the code
+  digest ignores comments and whitespace, follows any change of code, and
+  the recorded DRAM traffic is read only while the digest matches.
+- The reference arm (the fp64 oracle on the host cores): its JSON line,
+  and that only rank 0 prints it."""
 import os
 
 import bench
@@ -45,3 +48,36 @@ def test_recorded_traffic_needs_a_matching_digest(tmp_path, monkeypatch):
     assert bench.recorded_traffic("mid_tc", "w") == 1234
     assert bench.recorded_traffic("mid_tc", "stale") is None
     assert bench.recorded_traffic("mid_tc", "absent") is None
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py")] + args,
+                       capture_output=True, text=True, timeout=300, env=env, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    return lines
+
+
+def test_reference_arm_line_on_the_host():
+    # The reference arm times the fp64 oracle on the host cores and prints
+    # the contract's line with impl, cpu_baseline and a zero-copy e2e.
+    (line,) = _run_bench(["--impl", "reference", "--workload", "tiny_f32_m8",
+                          "--steps", "2", "--warmup", "1"])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 2 and line["warmup"] == 1
+    assert line["config"]["workload"] == "tiny_f32_m8"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_prints_on_rank_zero_only():
+    assert _run_bench(["--impl", "reference", "--workload", "tiny_f32_m8", "--steps", "1",
+                       "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
