@@ -65,6 +65,8 @@ WORKLOADS = {
     # tiny fp32 correctness case, and the same inputs with m = n
     "tiny_f32_m8": Workload("tiny_f32_m8", 1, 1, 1, 64, 32, 8, F32, 0),
     "tiny_f32_m64": Workload("tiny_f32_m64", 1, 1, 1, 64, 32, 64, F32, 0),
+    # tiny fp32 with m not dividing n: segments of 9 tokens, the last of 7
+    "tiny_f32_n70_m8": Workload("tiny_f32_n70_m8", 7, 1, 1, 70, 32, 8, F32, 0),
     # BERT-base shape, inputs scaled by 1/sqrt(d)
     "bert_n512_m64": Workload("bert_n512_m64", 2, 8, 12, 512, 64, 64, BF16, 33,
                               values="iid_scaled"),

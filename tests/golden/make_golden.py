@@ -9,6 +9,12 @@ steps, no conv skip) with m = 8 and m = n = 64 landmarks.  Method: Eq. 17 /
 Algorithm 1 of "Nystromformer: A Nystrom-Based Algorithm for Approximating
 Self-Attention" (section 3.4) with the Lemma 1 pseudoinverse and segment-mean
 landmarks (Eq. 16, mean over l = n/m tokens).
+
+tiny_f32_n70_m8.txt: the same method with m = 8 not dividing n = 70 (batch 1,
+heads 1, d = 32, its own seeds): segments of ceil(70 / 8) = 9 tokens, the
+last one of 7, each landmark the mean over its segment's real tokens (the
+"Landmark Selection: Segment-Means" section's padding, read with true
+counts).
 """
 import os
 import sys
@@ -67,6 +73,6 @@ def read(name):
 
 
 if __name__ == "__main__":
-    for nm in ("tiny_f32_m8", "tiny_f32_m64"):
+    for nm in ("tiny_f32_m8", "tiny_f32_m64", "tiny_f32_n70_m8"):
         write(nm)
         print("wrote", nm)

@@ -8,7 +8,7 @@ from nystr_self_attention_segment_b200.inputs import WORKLOADS, make_inputs
 from tests.golden.make_golden import read
 
 
-@pytest.mark.parametrize("name", ["tiny_f32_m8", "tiny_f32_m64"])
+@pytest.mark.parametrize("name", ["tiny_f32_m8", "tiny_f32_m64", "tiny_f32_n70_m8"])
 def test_golden_fixture_matches_oracle(name):
     wl = WORKLOADS[name]
     x = make_inputs(wl)
