@@ -106,6 +106,18 @@ def recorded_traffic(kernel, workload):
     return int(float(vals["traffic_bytes"]))
 
 
+# ----------------------------------------------------------------- config
+
+def workload_config(wl, world):
+    """The `config` object of the JSON line: the workload alone, identical for
+    both arms."""
+    return {"workload": wl.name, "batch": wl.batch, "heads": wl.heads,
+            "seq_len": wl.seq_len, "head_dim": wl.head_dim, "landmarks": wl.landmarks,
+            "pinv_iters": wl.pinv_iters, "conv_k": wl.conv_k, "values": wl.values,
+            "dtype": wl.dtype,
+            "parallelism": "dp%d (independent batches per GPU)" % world}
+
+
 # ----------------------------------------------------------------- ranks
 
 def max_over_ranks(x, world, device):
@@ -159,52 +171,70 @@ def cpu_baseline(wl, seconds):
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls the SM clock, its maximum, the power draw and the active clock
+    event reasons through NVML (read-only queries) from a host thread, about
+    once per millisecond, with host timestamps, so that samples can be
+    assigned to the timed region.  Records nothing when NVML is unavailable.
+    Changes no setting of the GPU."""
 
-    def __init__(self, uuid):
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
+
+    def __init__(self, uuid, index, period_s=0.001):
         self.uuid = uuid
-        self.proc = None
-        self.path = os.path.join("/tmp", "nys_clocks_%d.csv" % os.getpid())
+        self.index = index
+        self.period = period_s
+        self.samples = []          # (t, sm_mhz, max_mhz, reasons bitmask, power W)
+        self.thread = None
+        self.stop_flag = False
+        self.source = None
 
     def start(self):
+        import threading
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.source = "nvml"
         except Exception:
-            self.proc = None
+            return
+
+        def poll():
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self.stop_flag:
+                t = time.perf_counter()
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                except Exception:
+                    break
+                self.samples.append((t, sm, smax, rs, pw))
+                time.sleep(self.period)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
+            return
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+
+    def summary(self, windows):
+        """Clock record over the samples that fall inside the given host-time
+        windows [(t0, t1), ...]."""
+        sel = [x for x in self.samples if any(a <= x[0] <= b for a, b in windows)]
+        if not sel:
             return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [c.strip() for c in line.split(",")]
-            if len(f) < 10 or (self.uuid and f[1] != self.uuid):
-                continue
-            try:
-                sm.append(float(f[2]))
-                smax.append(float(f[3]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[6:10]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "samples": len(sm), "reasons": sorted(reasons)}
+        reasons = sorted({nm for x in sel for nm, bit in self.REASONS.items() if x[3] & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in sel),
+                "sm_min_mhz": min(x[1] for x in sel), "sm_max_mhz": max(x[2] for x in sel),
+                "power_w_median": round(statistics.median(x[4] for x in sel), 1),
+                "samples": len(sel), "reasons": reasons, "source": self.source}
 
 
 # ----------------------------------------------------------------- our arm
@@ -252,32 +282,44 @@ def run_ours(args, rank, world):
     nys.nys_attn_check_error(ws)
 
     K = args.steps
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(K)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(rot)]
     for evs in kev:                     # create the CUDA events before capture
         for e in evs:
             e.record()
     torch.cuda.synchronize()
-    # One CUDA graph per timed step (the forward's launches, with its own
-    # timing events as graph nodes), input sets rotating as above.  Replaying
-    # graphs takes the host launch cost out of the device timeline.
-    # The timed graphs hold plain forwards (an event between two kernels
-    # would serialise their programmatic overlap); a second set with
-    # per-kernel events gives the kernel breakdown, outside the timed region.
-    graphs, tgraphs = [], []
+    # CUDA graphs of the forward's launches (replays take the host launch cost
+    # out of the device timeline): one graph of `rot` forwards, one per input
+    # set in turn, and one single-forward graph per input set.  The timed
+    # region replays the rot-forward graph K // rot times and then the first
+    # K % rot single graphs: exactly K forwards, inputs rotating.  A second
+    # set of single graphs with an event after each kernel gives the kernel
+    # breakdown, outside the timed region (an event between two kernels
+    # would serialise their programmatic overlap).
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
-    for i in range(K):
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=cap):
+        for i in range(rot):
+            step(i)
+    singles, tgraphs = [], []
+    for i in range(rot):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            step(args.warmup + i)
-        graphs.append(g)
+            step(i)
+        singles.append(g)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            step(args.warmup + i, kev[i])
+            step(i, kev[i])
         tgraphs.append(g)
     torch.cuda.synchronize()
-    for i in range(min(args.warmup, K)):
-        graphs[i].replay()
+
+    def replay(k):
+        for _ in range(k // rot):
+            g_all.replay()
+        for i in range(k % rot):
+            singles[i].replay()
+
+    replay(max(args.warmup, rot))
     torch.cuda.synchronize()
     nys.nys_attn_check_error(ws)
     t_start = torch.cuda.Event(enable_timing=True)
@@ -287,28 +329,47 @@ def run_ours(args, rank, world):
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
-    clocks = ClockSampler(uuid)
+    clocks = ClockSampler(uuid, dev.index if dev.index is not None else 0)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    h0 = time.perf_counter()
     t_start.record(stream)
-    for i in range(K):
-        graphs[i].replay()
+    replay(K)
     t_end.record(stream)
     torch.cuda.synchronize()
+    h1 = time.perf_counter()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
-    nys.nys_attn_check_error(ws)
     total_ms = t_start.elapsed_time(t_end)
-    for i in range(K):            # per-kernel breakdown (not timed above)
-        tgraphs[i].replay()
+    # the same replays, untimed, for about 0.3 s: the clock record under
+    # sustained load (the timed region itself is short at the default K)
+    sus_steps = max(rot, int(0.3 / max(total_ms / K / 1e3, 1e-6)))
+    h2 = time.perf_counter()
+    replay(sus_steps)
     torch.cuda.synchronize()
+    h3 = time.perf_counter()
+    clocks.stop()
     nys.nys_attn_check_error(ws)
-    per_kernel = [sum(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(K)) / K
-                  for j in range(nl)]
+    clk = clocks.summary([(h0, h1), (h2, h3)])
+    in_timed = clocks.summary([(h0, h1)])
+    if clk is not None:
+        clk["samples_in_timed_region"] = in_timed["samples"] if in_timed else 0
+        clk["window"] = ("NVML samples at about 1 kHz during the timed region (%.1f ms) and "
+                         "during %d more untimed replays of the same graphs right after it "
+                         "(%.0f ms)" % ((h1 - h0) * 1e3, sus_steps, (h3 - h2) * 1e3))
+    # per-kernel breakdown (not timed above): the evented single graphs
+    reps = 3
+    per_kernel = [0.0] * nl
+    for _ in range(reps):
+        for i in range(rot):
+            tgraphs[i].replay()
+            torch.cuda.synchronize()
+            for j in range(nl):
+                per_kernel[j] += kev[i][j].elapsed_time(kev[i][j + 1]) / (reps * rot)
+    nys.nys_attn_check_error(ws)
     total_ms = max_over_ranks(total_ms, world, dev)
 
     # end to end through the host-buffer entry point (copies in the timed region)
@@ -359,15 +420,13 @@ def run_ours(args, rank, world):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads,
-                   "seq_len": wl.seq_len, "head_dim": wl.head_dim, "landmarks": m,
-                   "pinv_iters": iters, "conv_k": wl.conv_k, "values": wl.values,
-                   "parallelism": "dp%d (independent batches per GPU)" % world,
-                   "launch": "one CUDA graph per step (the library's launches, chained by "
-                             "programmatic dependent launch), replayed; kernel times from a "
-                             "separate replay with an event after each kernel",
-                   "l2": "inputs rotate over %d copies (%.0f MB per step set); no L2 flush"
-                         % (rot, step_bytes / 1e6)},
+        "config": workload_config(wl, world),
+        "timing": {"launch": "CUDA graphs of the library's launches (chained by programmatic "
+                             "dependent launch), replayed: K forwards in the timed region; "
+                             "kernel times from separate replays with an event after each "
+                             "kernel",
+                   "l2": "inputs rotate over %d copies (%.0f MB per step set, above 2x L2); "
+                         "no L2 flush" % (rot, step_bytes / 1e6)},
         "roofline": roof,
         "roofline_step": {"bound": "hbm", "achieved": round(step_ach, 1),
                           "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -386,7 +445,7 @@ def run_ours(args, rank, world):
     return line
 
 
-def run_reference(args, rank):
+def run_reference(args, rank, world):
     """The reference arm: the fp64 oracle on the host cores (rank 0 only),
     each step a bounded sample (one head) of the workload."""
     if rank != 0:
@@ -420,21 +479,38 @@ def run_reference(args, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads,
-                       "seq_len": wl.seq_len, "head_dim": wl.head_dim,
-                       "landmarks": wl.landmarks},
+            "config": workload_config(wl, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
+def launch_ranks(args):
+    """`--gpus N` without a launcher: start N ranks on this node with
+    torch.distributed.run (127.0.0.1 rendezvous) and return their status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node=%d" % args.gpus, "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.gpus != world:
+        if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+            sys.exit(launch_ranks(args))
+        sys.exit("bench.py: --gpus %d but WORLD_SIZE is %d; launch one process per GPU "
+                 "(torch.distributed.run --nproc-per-node %d) or drop --gpus"
+                 % (args.gpus, world, args.gpus))
     if args.impl == "reference":
-        line = run_reference(args, rank)
+        line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return

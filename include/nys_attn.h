@@ -35,7 +35,9 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and never synchronise the device.  Arguments are validated on the
  *    host before anything is enqueued: an invalid call returns a status and
- *    launches nothing.  Launch failures return NYS_ERR_CUDA.
+ *    launches nothing.  Each launch is checked as it is made: a launch that
+ *    the runtime refuses returns NYS_ERR_CUDA at once and no later kernel of
+ *    the call is enqueued (kernels enqueued before it stay enqueued).
  *  - Results are bitwise reproducible run to run (fixed-order reductions, no
  *    floating-point atomics).
  *  - batch * heads * seq_len == 0 is valid and enqueues nothing.
@@ -47,6 +49,7 @@
  *    seq_len (always true when m divides seq_len or seq_len >= m * m).
  *  - conv_k odd, 1 <= conv_k <= 63 (or conv_w == NULL / conv_k == 0: no skip).
  *  - 0 <= pinv_iters <= 64.
+ *  - batch * heads <= 65535, seq_len <= 2^24 (else NYS_ERR_UNSUPPORTED).
  */
 #ifndef NYS_ATTN_H
 #define NYS_ATTN_H
@@ -200,20 +203,32 @@ NYS_ATTN_API nys_status nys_attn_forward_timed(const void *Q_dev, const void *K_
  *  - A problem whose workspace (nys_attn_workspace_size) exceeds
  *    NYS_STATIC_SCRATCH_BYTES is rejected with NYS_ERR_WORKSPACE before
  *    anything is enqueued.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - The array's device address is looked up (cudaGetSymbolAddress) with
+ *    the device current on every call made outside stream capture, and
+ *    remembered per CUDA context; a call made while `stream` is capturing
+ *    uses the address remembered for the current context, so the first call
+ *    in a context must come before any stream capture (else NYS_ERR_CUDA).
  *  - Every call on a device shares the one array, which keeps the last
  *    call's contents (the intermediates of nys_attn_intermediates, at the
  *    same offsets); what must start at zero is cleared by each call.  Calls
  *    that overlap on the GPU (different streams, or host threads without
  *    ordering) race on the array: order them.
+ *  - A status a kernel records on the device (NYS_ERR_TIMEOUT) is read with
+ *    nys_attn_check_error_static, before the next call clears it.
  *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
 NYS_ATTN_API nys_status nys_attn_forward_static(const void *Q_dev, const void *K_dev,
                                                 const void *V_dev, const nys_desc *desc,
                                                 int num_landmarks, int pinv_iters,
                                                 const float *conv_w_dev, int conv_k,
                                                 void *out_dev, nys_stream_t stream);
+
+/* nys_attn_check_error for the scratch array of nys_attn_forward_static:
+ * synchronises `stream`, reads the error word the last static call left for
+ * this shape and clears it.  Returns NYS_OK or the recorded status;
+ * NYS_ERR_WORKSPACE for a shape the array cannot hold.  Allocates nothing.
+ * (No counterpart in the paper; it belongs to the deployment variant above.) */
+NYS_ATTN_API nys_status nys_attn_check_error_static(const nys_desc *desc, int num_landmarks,
+                                                    nys_stream_t stream);
 
 /* Number of kernel launches one nys_attn_forward call enqueues for this
  * shape (0 for an empty problem), and a short name for each launch in

@@ -39,6 +39,7 @@ EXPORTS = (
     "nys_attn_forward_timed",
     "nys_attn_launch_names",
     "nys_attn_forward_static",
+    "nys_attn_check_error_static",
 )
 
 # Size of the fixed scratch array of nys_attn_forward_static (see the header).
@@ -103,6 +104,8 @@ def load():
     lib.nys_attn_launch_names.argtypes = [D, I, ctypes.c_char_p, S]
     lib.nys_attn_forward_static.restype = I
     lib.nys_attn_forward_static.argtypes = [P, P, P, D, I, I, P, I, P, P]
+    lib.nys_attn_check_error_static.restype = I
+    lib.nys_attn_check_error_static.argtypes = [D, I, P]
     _LIB = lib
     return lib
 
@@ -191,6 +194,10 @@ def raw_forward_static(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, con
     return load().nys_attn_forward_static(q_ptr, k_ptr, v_ptr, ctypes.byref(desc),
                                           int(num_landmarks), int(pinv_iters), conv_ptr,
                                           int(conv_k), out_ptr, stream_ptr)
+
+
+def raw_check_error_static(desc, num_landmarks, stream_ptr):
+    return load().nys_attn_check_error_static(ctypes.byref(desc), int(num_landmarks), stream_ptr)
 
 
 def raw_check_error(ws_ptr, desc, num_landmarks, stream_ptr):

@@ -29,6 +29,7 @@
 
 #include "pinv_pow.cuh"
 #include "pinv_tc.cuh"
+#include "trace.cuh"
 
 namespace nys {
 namespace midtc {
@@ -174,6 +175,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   if (wait_prev) {
     griddep_wait();
     griddep_launch_dependents();
+    NYS_MARK(kTrMid, 1);
   }
   // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
   if (threadIdx.x < 256) {
@@ -272,6 +274,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
     int u = 0;
     for (int i = wg; i < nch; i += 2, ++u) {
       if (!(ok = mbar_wait(&s_full[wg], u & 1, ab))) break;
+      if (threadIdx.x == 128 && blockIdx.x == (unsigned)prm.BH && u < 32) NYS_MARK_T(kTrMid, 32 + u);
       tc_fence_after();
       float v[M];
 #pragma unroll
@@ -357,6 +360,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[wg]);
+      if (threadIdx.x == 128 && blockIdx.x == (unsigned)prm.BH && u < 32) NYS_MARK_T(kTrMid, 96 + u);
     }
     if (!ok) {
       // let the other warpgroup leave a turn it may be waiting for
@@ -631,6 +635,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint32_t last, tmem_base;
   const int t = threadIdx.x;
+  NYS_MARK(kTrMid, 0);
   // one TMEM allocation for every body this block runs (an allocation
   // relinquishes the block's permit to allocate again)
   if ((t >> 5) == 1) tmem_alloc(&tmem_base, 512);
@@ -651,6 +656,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     bh = blockIdx.x;
     griddep_wait();
     griddep_launch_dependents();
+    NYS_MARK(kTrMid, 1);
     if constexpr (M <= 64) {
       if (t < pinvpow::kBarThreads)
         pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, (float *)(smem + C::zs));
@@ -666,6 +672,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   // partials into Y; the second of {pseudoinverse, Y merge} to finish forms
   // W = Z Y.  Counters: count[bh] B~ V blocks done, count[BH + bh] inputs of
   // W ready.
+  NYS_MARK(kTrMid, 2);
   __threadfence();
   __syncthreads();
   if (t == 0)
@@ -674,18 +681,22 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   if (last) {
     if (!is_pinv) {
       __threadfence();
+      NYS_MARK(kTrMid, 3);
       merge_y_body<M>(prm, smem, bh, (float *)(smem + C::ys));
       __threadfence();
       __syncthreads();
+      NYS_MARK(kTrMid, 4);
     }
     if (t == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
     __syncthreads();
     if (last) {
       __threadfence();
+      NYS_MARK(kTrMid, 5);
       if (is_pinv) load_y<M>(prm, smem, bh);
       if (!z_in_smem) load_z<M>(prm, smem, bh);
       __syncthreads();
       w_product<M>(prm, smem, bh);
+      NYS_MARK(kTrMid, 6);
     }
   }
   tc_fence_before();
@@ -694,6 +705,7 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  NYS_MARK(kTrMid, 7);
 }
 
 }  // namespace midtc

@@ -12,7 +12,6 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
-#include "fused.cuh"
 #include "mid_tc.cuh"
 #include "out_tc.cuh"
 #include "stream_bf16.cuh"
@@ -20,14 +19,6 @@
 using namespace nys;
 
 namespace {
-
-// The persistent single-launch schedule (fused.cuh) is built but not the
-// default: its task bodies still run slower there than in the three-kernel
-// pipeline.  Compile with -DNYS_FUSED=1 to use it for m <= 64.
-#ifndef NYS_FUSED
-#define NYS_FUSED 0
-#endif
-constexpr bool kUseFused = NYS_FUSED != 0;
 
 size_t elem_size(int dtype) { return dtype == NYS_BF16 ? 2 : 4; }
 
@@ -48,10 +39,10 @@ nys_status validate_shape(const nys_desc *desc, int m) {
   } else {
     if (desc->head_dim != 64) return NYS_ERR_UNSUPPORTED;
     if (m != 32 && m != 64 && m != 128) return NYS_ERR_UNSUPPORTED;
-    // the persistent schedule sums equal segments only
-    if (kUseFused && m <= 64 && desc->seq_len % m != 0) return NYS_ERR_UNSUPPORTED;
   }
-  if ((long)desc->batch * desc->heads > (1L << 24) || desc->seq_len > (1 << 24))
+  // batch * heads indexes gridDim.y of the segment-mean and SIMT launches
+  // (at most 65535); seq_len indexes TMA coordinates and int offsets
+  if ((long)desc->batch * desc->heads > 65535L || desc->seq_len > (1 << 24))
     return NYS_ERR_UNSUPPORTED;
   return NYS_OK;
 }
@@ -73,10 +64,7 @@ Layout make_layout(const nys_desc *desc, int m) {
     // one pseudoinverse block per head plus `splits` B~ V blocks per head in
     // one wave of 148 blocks; each B~ V block leaves one merged partial
     const int chunks = (int)((n + midtc::kChunk - 1) / midtc::kChunk);
-    // m <= 64 (fused kernel): B~ V tasks of about 8 chunks; m = 128: one
-    // wave of 148 blocks with one pseudoinverse block per head
-    int per_head = kUseFused && m <= 64 ? chunks / 8
-                                         : (BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1);
+    int per_head = BH ? (int)((kNumSms - (int)BH) / (int)BH) : 1;
     if (per_head < 1) per_head = 1;
     if (per_head > chunks) per_head = chunks;
     if (per_head > midtc::kMaxSplits) per_head = midtc::kMaxSplits;
@@ -133,6 +121,7 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 struct Marks {
   cudaEvent_t const *ev = nullptr;
   int n = 0, next = 1;
+  int launched = 0;   // kernels enqueued so far by this call
   static void record(cudaEvent_t e, cudaStream_t s) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
@@ -144,9 +133,78 @@ struct Marks {
     if (ev) record(ev[0], s);
   }
   void after(cudaStream_t s) {
+    ++launched;
     if (ev && next < n) record(ev[next++], s);
   }
 };
+
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+// Test builds only (a separate library the tests load): the launch with this
+// index in the next forward call asks for more dynamic shared memory than a
+// block may have, so that the launch is refused and nothing of it runs.
+int g_fail_launch = -1;
+#endif
+
+// Dynamic shared memory of launch `idx` of a call (a test build may make one
+// launch impossible, see above).
+size_t launch_smem(int idx, size_t smem) {
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+  if (idx == g_fail_launch) {
+    g_fail_launch = -1;
+    return (size_t)1 << 20;
+  }
+#endif
+  (void)idx;
+  return smem;
+}
+
+// Launches one kernel and reports the launch's own status (the return value
+// of cudaLaunchKernelEx, so an unrelated earlier error cannot be mistaken
+// for it).  pdl: programmatic stream serialisation, i.e. the kernel may start
+// while the previous kernel of the stream drains and must wait
+// (griddepcontrol.wait) before it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t stream, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+// Test build only: a bounded wait that runs out (see nys_test_timeout_probe).
+__global__ void timeout_probe(uint32_t *err, long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const sm100::Abort ab{&flag, err};
+    if (!sm100::mbar_wait_for(&bar, 0, ab, limit_cycles)) sm100::mbar_inval(&bar);
+  }
+}
+#endif
+
+// Opts a kernel in to `smem` bytes of dynamic shared memory when it needs
+// more than the default 48 KB.
+template <typename... KArgs>
+bool allow_smem(void (*kern)(KArgs...), size_t smem) {
+  return smem <= 48 * 1024 ||
+         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+             cudaSuccess;
+}
 
 constexpr int kSimtLaunches = 5;
 const char *kSimtNames = "seg_means,pinv,bv_partial,merge_w,out";
@@ -164,61 +222,55 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   const float scale = 1.0f / sqrtf((float)d);
   const float scale_log2 = scale * kLog2e;
 
+  // every launch is checked at once: a refused launch returns before the
+  // next one is enqueued
   {
     long total = (long)BH * m * d;
     dim3 grid((unsigned)((total + 255) / 256), 2);
-    seg_means_scalar<T><<<grid, 256, 0, stream>>>(Q, K, qt, kt, BH, n, d, m);
+    if (launch(seg_means_scalar<T>, grid, dim3(256), launch_smem(mk.launched, 0), stream, false,
+               Q, K, qt, kt, BH, n, d, m) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {
     const int use_smem = m <= 64;
     size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
-    if (sm > 48 * 1024)
-      cudaFuncSetAttribute(pinv_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    pinv_simt<<<BH, 256, sm, stream>>>(qt, kt, z, scratch, m, d, scale, iters, use_smem);
+    if (!allow_smem(pinv_simt, sm) ||
+        launch(pinv_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
+               kt, z, scratch, m, d, scale, iters, use_smem) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {
     size_t sm = ((size_t)m * d + kSimtKeyTile * (d + 1) + kSimtKeyTile * d) * 4;
     dim3 grid(L.splits, BH);
-    if (m <= 64) {
-      auto kern = bv_partial_simt<T, 8>;
-      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      kern<<<grid, 256, sm, stream>>>(qt, K, V, pmax, psum, py, n, d, m, L.splits,
-                                      L.keys_per_split, scale_log2);
-    } else {
-      auto kern = bv_partial_simt<T, 16>;
-      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      kern<<<grid, 256, sm, stream>>>(qt, K, V, pmax, psum, py, n, d, m, L.splits,
-                                      L.keys_per_split, scale_log2);
-    }
+    auto kern = m <= 64 ? bv_partial_simt<T, 8> : bv_partial_simt<T, 16>;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, qt, K, V,
+               pmax, psum, py, n, d, m, L.splits, L.keys_per_split, scale_log2) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {
     size_t sm = (size_t)m * d * 4;
-    if (sm > 48 * 1024)
-      cudaFuncSetAttribute(merge_w_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    merge_w_simt<<<BH, 256, sm, stream>>>(pmax, psum, py, z, y, w, m, d, L.splits);
+    if (!allow_smem(merge_w_simt, sm) ||
+        launch(merge_w_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false,
+               pmax, psum, py, z, y, w, m, d, L.splits) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {
     size_t sm = ((size_t)m * (d + 1) + (size_t)m * d + 8 * d + (conv_w ? conv_k : 0)) * 4;
     dim3 grid((n + kSimtOutRowsPerBlock - 1) / kSimtOutRowsPerBlock, BH);
     const int ck = conv_w ? conv_k : 0;
-    if (m <= 64) {
-      auto kern = out_simt<T, 2>;
-      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      kern<<<grid, 256, sm, stream>>>(Q, V, kt, w, conv_w, out, n, d, m, desc->heads, ck,
-                                      scale_log2);
-    } else {
-      auto kern = out_simt<T, 4>;
-      if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      kern<<<grid, 256, sm, stream>>>(Q, V, kt, w, conv_w, out, n, d, m, desc->heads, ck,
-                                      scale_log2);
-    }
+    auto kern = m <= 64 ? out_simt<T, 2> : out_simt<T, 4>;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, Q, V, kt, w,
+               conv_w, out, n, d, m, desc->heads, ck, scale_log2) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
-  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+  return NYS_OK;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -256,103 +308,9 @@ bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
          CUDA_SUCCESS;
 }
 
-// Launch with programmatic stream serialisation: the kernel may start while
-// the previous kernel of the stream drains (it waits in griddep_wait before
-// reading that kernel's results).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args &&...args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
-// launches of the bf16 path: one fused kernel, or three
-int tc_launches(int m) { return kUseFused && m <= 64 ? 1 : 3; }
-const char *tc_names(int m) {
-  return kUseFused && m <= 64 ? "fused" : "seg_means,mid_tc,out_tc";
-}
-
-// The fused persistent kernel (m <= 64).
-template <int M>
-nys_status launch_fused(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
-                        const nys_desc *desc, int iters, const float *conv_w, int conv_k,
-                        __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
-                        Marks &mk) {
-  const int BH = desc->batch * desc->heads;
-  const int n = desc->seq_len;
-  float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
-  uint32_t *err = (uint32_t *)(ws + L.err);
-  const float scale_log2 = 0.125f * kLog2e;   // log2(e) / sqrt(64)
-  const bool conv = conv_w != nullptr;
-  const int kconv = conv ? ((128 + conv_k - 1 + 15) / 16) * 16 : 0;
-  CUtensorMap mq, mkk, mv, mvh, mo;
-  if (!make_map(&mq, Q, BH, n, 128) || !make_map(&mkk, K, BH, n, 128) ||
-      !make_map(&mv, V, BH, n, 128) || !make_map(&mvh, V, BH, n, conv ? kconv : 128) ||
-      !make_map(&mo, out, BH, n, 128))
-    return NYS_ERR_CUDA;
-  fused::Params p;
-  memset(&p, 0, sizeof(p));
-  const int chunks = (n + midtc::kChunk - 1) / midtc::kChunk;
-  const int tph = (n + outtc::kTileRows - 1) / outtc::kTileRows;
-  p.mid.pinv = pinvtc::Params{qt, kt, (float *)(ws + L.z), err, iters, scale_log2};
-  p.mid.q_land = qt;
-  p.mid.z = (float *)(ws + L.z);
-  p.mid.pmax = (float *)(ws + L.pmax);
-  p.mid.psum = (float *)(ws + L.psum);
-  p.mid.py = (float *)(ws + L.py);
-  p.mid.y = (float *)(ws + L.y);
-  p.mid.w = (float *)(ws + L.w);
-  p.mid.w_op = (uint8_t *)(ws + L.w_bf);
-  p.mid.count = nullptr;
-  p.mid.err = err;
-  p.mid.BH = BH;
-  p.mid.n = n;
-  p.mid.chunks_per_head = chunks;
-  p.mid.splits = L.splits;
-  p.mid.scale_log2 = scale_log2;
-  p.out = outtc::Params{kt, (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads,
-                        conv ? conv_k : 1, kconv, tph, 1, scale_log2};
-  p.q_land = qt;
-  p.k_land = kt;
-  p.err = err;
-  p.queue = err + 1;
-  p.seg_cnt = (uint32_t *)(ws + L.count);
-  p.head_cnt = p.seg_cnt + BH;
-  p.w_ready = p.seg_cnt + 2 * BH;
-  p.BH = BH;
-  p.seg_len = n / M;
-  // about 1024 rows (128 KB) per segment-sum task
-  p.seg_per_task = 1024 / p.seg_len;
-  if (p.seg_per_task < 1) p.seg_per_task = 1;
-  if (p.seg_per_task > M) p.seg_per_task = M;
-  p.seg_tasks = (M + p.seg_per_task - 1) / p.seg_per_task;
-  p.splits = L.splits;
-  p.tiles_per_task = 8;
-  p.out_tasks = (tph + p.tiles_per_task - 1) / p.tiles_per_task;
-  p.lag_p = 1;
-  p.lag_b = 2;
-  p.lag_o = BH < 2 ? 2 : (BH / 2 + 4 < BH ? BH / 2 + 4 : BH);
-  if (p.lag_o < p.lag_b) p.lag_o = p.lag_b;
-  p.steps = BH + p.lag_o;
-  p.total = BH * (2 * p.seg_tasks + 1 + p.splits + p.out_tasks);
-  p.inv_len = 1.f / (float)p.seg_len;
-  auto kern = fused::fused_kernel<M>;
-  const uint32_t sm = fused::smem_bytes<M>(conv ? kconv : 0);
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  const int grid = p.total < kNumSms ? p.total : kNumSms;
-  kern<<<grid, fused::kThreads, sm, stream>>>(mq, mkk, mv, mvh, mo, p);
-  mk.after(stream);
-  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
-}
+// launches of the bf16 path
+constexpr int kTcLaunches = 3;
+const char *kTcNames = "seg_means,mid_tc,out_tc";
 
 template <int M>
 nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
@@ -380,7 +338,9 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
   {   // segment means of Q and K (Eq. 16)
     const int seg = (n + M - 1) / M;   // tokens of a full segment
     const int groups = seg < 32 ? seg : 32;
-    seg_means_bf16<<<dim3(M, BH, 2), 8 * groups, 0, stream>>>(Q, K, qt, kt, n, M);
+    if (launch(seg_means_bf16, dim3(M, BH, 2), dim3(8 * groups), launch_smem(mk.launched, 0),
+               stream, false, Q, K, qt, kt, n, M) != cudaSuccess)
+      return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {   // pseudoinverse || B~ V, then merge + W = Z Y
@@ -403,9 +363,9 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     p.scale_log2 = scale_log2;
     auto kern = midtc::mid_kernel<M>;
     const uint32_t sm = midtc::smem_bytes<M>();
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (launch_pdl(kern, dim3(BH * (1 + L.splits)), dim3(midtc::kThreads), sm, stream, mkk, mv,
-                   p) != cudaSuccess)
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH * (1 + L.splits)), dim3(midtc::kThreads),
+               launch_smem(mk.launched, sm), stream, true, mkk, mv, p) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -418,23 +378,19 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
                     scale_log2};
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (launch_pdl(kern, dim3(BH * cpb), dim3(outtc::kThreads), sm, stream, mq, mvh, mo, p) !=
-        cudaSuccess)
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH * cpb), dim3(outtc::kThreads), launch_smem(mk.launched, sm), stream,
+               true, mq, mvh, mo, p) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
-  return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+  return NYS_OK;
 }
 
 nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                      const nys_desc *desc, int m, int iters, const float *conv_w, int conv_k,
                      __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
                      Marks &mk) {
-  if (kUseFused) {
-    if (m == 32) return launch_fused<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
-    if (m == 64) return launch_fused<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
-  }
   switch (m) {
     case 32: return launch_tc_m<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
     case 64: return launch_tc_m<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
@@ -520,7 +476,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
                                nys_stream_t stream_, void *const *events, int n_events) {
   nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
   if (st != NYS_OK) return st;
-  if (events && n_events < (desc->dtype == NYS_BF16 ? tc_launches(m) : kSimtLaunches) + 1)
+  if (events && n_events < (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches) + 1)
     return NYS_ERR_INVALID_ARG;
   if (is_empty(desc)) return NYS_OK;
   Marks mk;
@@ -577,26 +533,81 @@ NYS_ATTN_API nys_status nys_attn_forward(const void *Q, const void *K, const voi
 // this library's module: every device that loads the library holds it until
 // the process exits.  Host code cannot pass the array's name to a kernel (on
 // the host it is only a stand-in for the symbol), so its device address is
-// looked up with cudaGetSymbolAddress once per device, on that device's first
-// call, with that device current.
+// looked up with cudaGetSymbolAddress, with the device current (below).
 static __device__ __align__(256) unsigned char g_static_scratch[NYS_STATIC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-void *g_static_addr[kMaxDevices];            // device address per device, once resolved
+// The array's device address belongs to the module as loaded in one CUDA
+// context: a context that is destroyed and created again (cudaDeviceReset,
+// for instance) may load the module at another address.  So the address is
+// looked up again on every call outside stream capture, and the lookup is
+// remembered per context (by its unique id) for calls made while a stream is
+// capturing, when no lookup should run.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+constexpr int kMaxContexts = 64;
+struct StaticAddr {
+  unsigned long long ctx_id;
+  void *addr;
+};
+StaticAddr g_static_addr[kMaxContexts];
+int g_static_n = 0;
 std::mutex g_static_mu;
 
-nys_status static_scratch(void **addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return NYS_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return NYS_ERR_UNSUPPORTED;
+// The id of the calling thread's current context; if the thread has none
+// yet, the current device's primary context is made current first
+// (cudaSetDevice initialises it).
+nys_status current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_ctx = nullptr;
+  static CtxGetIdFn get_id = nullptr;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_addr[dev]) {
+  if (!get_ctx || !get_id) {
+    void *p = nullptr, *q = nullptr;
+    cudaDriverEntryPointQueryResult r1, r2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) != cudaSuccess ||
+        r1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) != cudaSuccess ||
+        r2 != cudaDriverEntryPointSuccess)
+      return NYS_ERR_CUDA;
+    get_ctx = (CtxGetCurrentFn)p;
+    get_id = (CtxGetIdFn)q;
+  }
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return NYS_ERR_CUDA;
+  if (!ctx) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+        get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+      return NYS_ERR_CUDA;
+  }
+  if (get_id(ctx, id) != CUDA_SUCCESS) return NYS_ERR_CUDA;
+  return NYS_OK;
+}
+
+// Device address of g_static_scratch in the current context.
+nys_status static_scratch(cudaStream_t stream, void **addr) {
+  unsigned long long id = 0;
+  nys_status st = current_context_id(&id);
+  if (st != NYS_OK) return st;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return NYS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  int slot = -1;
+  for (int i = 0; i < g_static_n; ++i)
+    if (g_static_addr[i].ctx_id == id) slot = i;
+  if (cs == cudaStreamCaptureStatusNone || slot < 0) {
+    if (cs != cudaStreamCaptureStatusNone) return NYS_ERR_CUDA;   // first call inside a capture
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return NYS_ERR_CUDA;
-    g_static_addr[dev] = p;
+    if (slot < 0) {
+      if (g_static_n == kMaxContexts) return NYS_ERR_UNSUPPORTED;
+      slot = g_static_n++;
+      g_static_addr[slot].ctx_id = id;
+    }
+    g_static_addr[slot].addr = p;
   }
-  *addr = g_static_addr[dev];
+  *addr = g_static_addr[slot].addr;
   return NYS_OK;
 }
 }  // namespace
@@ -611,7 +622,7 @@ NYS_ATTN_API nys_status nys_attn_forward_static(const void *Q, const void *K, co
   if (make_layout(desc, m).total > (size_t)NYS_STATIC_SCRATCH_BYTES)
     return NYS_ERR_WORKSPACE;   // the problem needs more scratch than the fixed array holds
   void *ws = nullptr;
-  st = static_scratch(&ws);
+  st = static_scratch((cudaStream_t)stream, &ws);
   if (st != NYS_OK) return st;
   // the error word and the per-head counters are cleared by forward_impl
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, ws,
@@ -650,6 +661,19 @@ NYS_ATTN_API nys_status nys_attn_check_error(void *workspace, const nys_desc *de
     return (nys_status)word;
   }
   return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_check_error_static(const nys_desc *desc, int m,
+                                                    nys_stream_t stream_) {
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) return NYS_OK;
+  if (make_layout(desc, m).total > (size_t)NYS_STATIC_SCRATCH_BYTES) return NYS_ERR_WORKSPACE;
+  cudaStream_t stream = (cudaStream_t)stream_;
+  void *ws = nullptr;
+  st = static_scratch(stream, &ws);
+  if (st != NYS_OK) return st;
+  return nys_attn_check_error(ws, desc, m, stream_);
 }
 
 struct HostBufLayout {
@@ -726,7 +750,7 @@ NYS_ATTN_API nys_status nys_attn_launch_count(const nys_desc *desc, int m, int c
   if (!launches) return NYS_ERR_INVALID_ARG;
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  *launches = is_empty(desc) ? 0 : (desc->dtype == NYS_BF16 ? tc_launches(m) : kSimtLaunches);
+  *launches = is_empty(desc) ? 0 : (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches);
   return NYS_OK;
 }
 
@@ -734,12 +758,60 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
                                               size_t names_bytes) {
   nys_status st = validate_shape(desc, m);
   if (st != NYS_OK) return st;
-  const char *src = is_empty(desc) ? "" : (desc->dtype == NYS_BF16 ? tc_names(m) : kSimtNames);
+  const char *src = is_empty(desc) ? "" : (desc->dtype == NYS_BF16 ? kTcNames : kSimtNames);
   if (names) {
     if (names_bytes < strlen(src) + 1) return NYS_ERR_INVALID_ARG;
     strcpy(names, src);
   }
   return NYS_OK;
 }
+
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+// ---------------------------------------------------------------------------
+// Entry points of the test build only (not part of the product ABI):
+//  nys_test_fail_launch(idx)   the launch with index idx of the next forward
+//                              call is refused (see launch_smem);
+//  nys_test_timeout_probe(...) one block waits on an mbarrier that nothing
+//                              completes, with a limit of limit_cycles SM
+//                              cycles; the bounded wait gives up, records
+//                              NYS_ERR_TIMEOUT in the workspace error word and
+//                              the block returns.  No copy or MMA is in flight
+//                              when it gives up.
+NYS_ATTN_API void nys_test_fail_launch(int idx) { g_fail_launch = idx; }
+
+NYS_ATTN_API nys_status nys_test_timeout_probe(void *workspace, const nys_desc *desc, int m,
+                                               long long limit_cycles, nys_stream_t stream) {
+  if (!workspace || limit_cycles < 0 || limit_cycles > (1ll << 32)) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (is_empty(desc)) return NYS_ERR_INVALID_ARG;
+  uint32_t *err = (uint32_t *)((char *)workspace + make_layout(desc, m).err);
+  return launch(timeout_probe, dim3(1), dim3(32), 0, (cudaStream_t)stream, false, err,
+                limit_cycles) == cudaSuccess
+             ? NYS_OK
+             : NYS_ERR_CUDA;
+}
+#endif
+
+#if defined(NYS_TIMELINE) && NYS_TIMELINE
+// Diagnostic build only: copies up to `cap` timeline records (see trace.cuh)
+// to host memory, writes how many were recorded, and clears the count when
+// `reset` is set.  Synchronises the device.
+NYS_ATTN_API nys_status nys_debug_timeline(void *host, size_t cap, uint32_t *count, int reset) {
+  if (!count) return NYS_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(count, g_trace_n, sizeof(uint32_t)) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  size_t n = *count < (uint32_t)kTraceCap ? *count : (size_t)kTraceCap;
+  if (n > cap) n = cap;
+  if (host && n && cudaMemcpyFromSymbol(host, g_trace, n * sizeof(TraceRec)) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  if (reset) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_trace_n, &zero, sizeof(zero)) != cudaSuccess) return NYS_ERR_CUDA;
+  }
+  return NYS_OK;
+}
+#endif
 
 }  // extern "C"

@@ -25,6 +25,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace nys {
 namespace outtc {
@@ -106,6 +107,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
   float *cw = (float *)(smem + L.cw);
+  NYS_MARK(kTrOut, 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -184,8 +186,10 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  NYS_MARK(kTrOut, 1);
   if (warp == 3 && lane == 0) {
     if (wait_prev) griddep_wait();
+    NYS_MARK_T(kTrOut, 2);
     mbar_expect_tx(w_ready, M * 128u);
     bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
   }
@@ -301,6 +305,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&tm_free[wg]);
+      if (threadIdx.x == 128 && u < 4) NYS_MARK_T(kTrOut, 8 + u);
       // this warpgroup's staging buffer was last used two of its tiles ago
       if (r == 0) bulk_wait_read0();
       named_barrier(2 + wg, 128);
@@ -327,6 +332,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  NYS_MARK(kTrOut, 4);
 }
 
 template <int M>

@@ -42,6 +42,7 @@
 #include <type_traits>
 
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace nys {
 namespace pinvpow {
@@ -312,6 +313,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     put_row<M>(pf0, r, 0, v);
   }
   if (!sync_ops()) ok = false;
+  NYS_MARK(kTrMid, 8);
   // ---- A A^T on the tensor cores; meanwhile the Z rows take the columns of
   //      A (their Z0 rows up to c0) and their partial column sums
   if (ok && issuer) {
@@ -358,6 +360,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     put_row<NC>(pf0, row, c_lo, p);
   }
   if (!sync_ops()) ok = false;
+  NYS_MARK(kTrMid, 9);
 
   // ---- Lemma 1 steps.  Z pipeline: the update Z_j = Z_{j-1} r_{j-1} is
   //      issued in stage 2 of step j (behind the chain's MMA) and read back
@@ -418,6 +421,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       put_split<NC, true>(ph, pl, row, c_lo, d, split_next);
       put_row<NC>(pf0 + ((j + 1) & 1) * 4096, row, c_lo, d);
     }
+    if (j < 8) NYS_MARK(kTrMid, 16 + j);
     if (ok && aux) {   // r_j = 1/4 (13I - 15 P + 7 P^2 - P^3)
       float d[NC], a[NC];
       ld_cols<NC>(t_d + c_lo, d);

@@ -81,19 +81,23 @@ struct Abort {
 // another thread of the block has already aborted.
 // The limit is counted in SM clock cycles (cheap to read, unlike the global
 // timer); kWaitLimitCycles is about 0.2 s at the B200's clocks.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Abort &ab) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, const Abort &ab,
+                                              long long limit_cycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test(a, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_test(a, parity)) return true;
     if (*ab.flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       *ab.flag = 1u;
       set_error(ab.err, NYS_ERR_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Abort &ab) {
+  return mbar_wait_for(bar, parity, ab, kWaitLimitCycles);
 }
 
 // ------------------------------------------------------------------ launch overlap

@@ -7,6 +7,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace nys {
 
@@ -17,6 +18,7 @@ __global__ void __launch_bounds__(256)
 seg_means_bf16(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                float *__restrict__ Qt, float *__restrict__ Kt, int n, int m) {
   __shared__ float part[32][64];
+  NYS_MARK(kTrSeg, 0);
   sm100::griddep_launch_dependents();   // the next kernel waits for this grid anyway
   const int j = blockIdx.x, bh = blockIdx.y;
   const __nv_bfloat16 *X = blockIdx.z == 0 ? Q : K;
@@ -62,6 +64,7 @@ seg_means_bf16(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restr
     for (int q = 0; q < groups; ++q) s += part[q][c];
     Xt[((size_t)bh * m + j) * 64 + c] = s / (float)seg;
   }
+  NYS_MARK(kTrSeg, 1);
 }
 
 }  // namespace nys

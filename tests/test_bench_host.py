@@ -4,7 +4,8 @@
   digest ignores comments and whitespace, follows any change of code, and
   the recorded DRAM traffic is read only while the digest matches.
 - The reference arm (the fp64 oracle on the host cores): its JSON line,
-  and that only rank 0 prints it."""
+  the same config object as the device arm, and that only rank 0 prints it.
+- --gpus N must match the launcher's world size."""
 import os
 
 import bench
@@ -50,7 +51,7 @@ def test_recorded_traffic_needs_a_matching_digest(tmp_path, monkeypatch):
     assert bench.recorded_traffic("mid_tc", "absent") is None
 
 
-def _run_bench(args, env_extra=None):
+def _run_bench(args, env_extra=None, rc=0):
     import json
     import subprocess
     import sys
@@ -58,6 +59,9 @@ def _run_bench(args, env_extra=None):
     env.update(env_extra or {})
     r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py")] + args,
                        capture_output=True, text=True, timeout=300, env=env, cwd=bench.ROOT)
+    if rc != 0:
+        assert r.returncode != 0
+        return r.stderr
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
     return lines
@@ -72,6 +76,8 @@ def test_reference_arm_line_on_the_host():
     assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
     assert line["value"] > 0 and line["steps"] == 2 and line["warmup"] == 1
     assert line["config"]["workload"] == "tiny_f32_m8"
+    from nystr_self_attention_segment_b200.inputs import WORKLOADS
+    assert line["config"] == bench.workload_config(WORKLOADS["tiny_f32_m8"], 1)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
@@ -80,4 +86,13 @@ def test_reference_arm_line_on_the_host():
 
 def test_reference_arm_prints_on_rank_zero_only():
     assert _run_bench(["--impl", "reference", "--workload", "tiny_f32_m8", "--steps", "1",
-                       "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
+                       "--warmup", "0", "--gpus", "2"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_gpus_must_match_the_world_size():
+    err = _run_bench(["--impl", "reference", "--workload", "tiny_f32_m8", "--steps", "1",
+                      "--warmup", "0", "--gpus", "2"], {"RANK": "0", "WORLD_SIZE": "1"}, rc=1)
+    assert "WORLD_SIZE" in err
+    err = _run_bench(["--impl", "reference", "--workload", "tiny_f32_m8", "--steps", "1",
+                      "--warmup", "0"], {"RANK": "0", "WORLD_SIZE": "4"}, rc=1)
+    assert "--gpus 1" in err

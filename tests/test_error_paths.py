@@ -1,0 +1,125 @@
+"""Error paths of the C ABI on the GPU, through the test build of the library
+(libnys_attn_test.so: the same sources with two test-only entry points).
+
+- A launch that the runtime refuses (one launch of the call asks for more
+  dynamic shared memory than a block may have) returns NYS_ERR_CUDA at once:
+  no later kernel of the call runs, so the output is left untouched, and the
+  next call works.
+- A bounded device wait that runs out (an mbarrier nothing completes, with a
+  short limit, no copy or MMA in flight) records NYS_ERR_TIMEOUT in the
+  workspace error word; nys_attn_check_error reports it once and clears it.
+
+Nothing here faults or hangs the GPU: the refused launch never starts, and
+the wait gives up after about a millisecond."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import nystr_self_attention_segment_b200 as nys
+from nystr_self_attention_segment_b200 import _lib
+from nystr_self_attention_segment_b200 import build as nys_build
+from nystr_self_attention_segment_b200.inputs import BF16, F32, make_custom
+from tests.gpu_util import TOL, normwise, run, torch
+
+TEST_LIB = nys_build.VARIANTS["test"][0]
+
+
+def _test_lib():
+    nys_build.build(variant="test")
+    lib = ctypes.CDLL(TEST_LIB)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    D = ctypes.POINTER(_lib.nys_desc)
+    lib.nys_attn_forward.restype = I
+    lib.nys_attn_forward.argtypes = [P, P, P, D, I, I, P, I, P, P, S, P]
+    lib.nys_attn_workspace_size.restype = I
+    lib.nys_attn_workspace_size.argtypes = [D, I, ctypes.POINTER(S)]
+    lib.nys_attn_check_error.restype = I
+    lib.nys_attn_check_error.argtypes = [P, D, I, P]
+    lib.nys_attn_launch_count.restype = I
+    lib.nys_attn_launch_count.argtypes = [D, I, I, ctypes.POINTER(I)]
+    lib.nys_test_fail_launch.restype = None
+    lib.nys_test_fail_launch.argtypes = [I]
+    lib.nys_test_timeout_probe.restype = I
+    lib.nys_test_timeout_probe.argtypes = [P, D, I, ctypes.c_longlong, P]
+    return lib
+
+
+def test_hooks_exist_only_in_the_test_build():
+    lib = _test_lib()
+    prod = nys.load()
+    for name in ("nys_test_fail_launch", "nys_test_timeout_probe"):
+        assert hasattr(lib, name)
+        assert not hasattr(prod, name)
+
+
+def _stream():
+    t = torch()
+    return ctypes.c_void_p(t.cuda.current_stream().cuda_stream)
+
+
+def _forward(lib, Q, K, V, m, cw, out, ws, ws_bytes):
+    t = torch()
+    dt = _lib.NYS_BF16 if Q.dtype == t.bfloat16 else _lib.NYS_F32
+    desc = _lib.make_desc(dt, *Q.shape)
+    return lib.nys_attn_forward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(desc), m,
+                                6, cw.data_ptr() if cw is not None else None,
+                                cw.shape[1] if cw is not None else 0, out.data_ptr(),
+                                ctypes.c_void_p(ws), ctypes.c_size_t(ws_bytes), _stream())
+
+
+CASES = [((1, 2, 1000, 64), 32, BF16, 33), ((1, 1, 70, 32), 8, F32, 5)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("shape,m,dtype,conv_k", CASES)
+def test_refused_launch_returns_cuda_error_and_runs_nothing_after_it(shape, m, dtype, conv_k):
+    t = torch()
+    lib = _test_lib()
+    x = make_custom(shape, dtype, seed=11, conv_k=conv_k)
+    want, _, (Q, K, V, cw) = run(x, dtype, m)
+    desc = _lib.make_desc(_lib.NYS_BF16 if dtype == BF16 else _lib.NYS_F32, *shape)
+    nl = ctypes.c_int(0)
+    assert lib.nys_attn_launch_count(ctypes.byref(desc), m, conv_k, ctypes.byref(nl)) == 0
+    wsb = ctypes.c_size_t(0)
+    assert lib.nys_attn_workspace_size(ctypes.byref(desc), m, ctypes.byref(wsb)) == 0
+    buf = t.zeros(wsb.value + 256, dtype=t.uint8, device="cuda")
+    ws = buf.data_ptr() + (-buf.data_ptr()) % 256
+    for idx in range(nl.value):
+        out = t.full_like(Q, 7.0)
+        lib.nys_test_fail_launch(idx)
+        st = _forward(lib, Q, K, V, m, cw, out, ws, wsb.value)
+        assert _lib.STATUS_NAMES[st] == "NYS_ERR_CUDA", idx
+        t.cuda.synchronize()
+        # the output kernel is the last launch: it never ran
+        assert bool((out == 7.0).all()), idx
+        # the next call is unaffected and matches the product library
+        st = _forward(lib, Q, K, V, m, cw, out, ws, wsb.value)
+        assert st == 0
+        assert lib.nys_attn_check_error(ctypes.c_void_p(ws), ctypes.byref(desc), m, _stream()) == 0
+        got = out.float().cpu().numpy().astype(np.float64)
+        assert normwise(got, want) <= TOL[dtype]
+
+
+@pytest.mark.gpu
+def test_bounded_wait_that_runs_out_reports_timeout_once():
+    t = torch()
+    lib = _test_lib()
+    shape, m = (1, 2, 512, 64), 64
+    desc = _lib.make_desc(_lib.NYS_BF16, *shape)
+    wsb = ctypes.c_size_t(0)
+    assert lib.nys_attn_workspace_size(ctypes.byref(desc), m, ctypes.byref(wsb)) == 0
+    buf = t.zeros(wsb.value + 256, dtype=t.uint8, device="cuda")
+    ws = ctypes.c_void_p(buf.data_ptr() + (-buf.data_ptr()) % 256)
+    # about a millisecond of SM cycles, then the wait gives up
+    assert lib.nys_test_timeout_probe(ws, ctypes.byref(desc), m, 2_000_000, _stream()) == 0
+    st = lib.nys_attn_check_error(ws, ctypes.byref(desc), m, _stream())
+    assert _lib.STATUS_NAMES[st] == "NYS_ERR_TIMEOUT"
+    assert lib.nys_attn_check_error(ws, ctypes.byref(desc), m, _stream()) == 0   # cleared
+    # and the same workspace serves a normal forward afterwards
+    x = make_custom(shape, BF16, seed=3, conv_k=33)
+    want, _, (Q, K, V, cw) = run(x, BF16, m)
+    out = t.empty_like(Q)
+    assert _forward(lib, Q, K, V, m, cw, out, ws.value, wsb.value) == 0
+    assert lib.nys_attn_check_error(ws, ctypes.byref(desc), m, _stream()) == 0
+    assert normwise(out.float().cpu().numpy().astype(np.float64), want) <= TOL[BF16]
