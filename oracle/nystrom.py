@@ -69,6 +69,8 @@ __all__ = [
     "nystrom_head",
     "nystrom_forward",
     "nystrom_forward_lens",
+    "nystrom_head_backward",
+    "nystrom_backward",
     "exact_attention_head",
     "exact_attention",
     "algorithmic_flops",
@@ -256,6 +258,161 @@ def nystrom_forward_lens(Q, K, V, m, lens, iters=6, conv_w=None):
             r = nystrom_head(Q[b, h, :L], K[b, h, :L], V[b, h, :L], m, iters, w)
             out[b, h, :L] = r["out"]
     return out
+
+
+# ----------------------------------------------------------------- backward
+#
+# Gradients of one head's output with respect to Q, K, V and the conv kernel
+# ([P5] "Moore-Penrose Pseudoinverse Computation", gradient computation:
+# backpropagation runs through the iteration's matrix products like any other
+# layer).  Each step below is the chain rule of one forward step, taken in
+# reverse order.  Readings (not on the pages):
+#   * softmax rows: dS = P * (dP - rowsum(dP * P)) (P the softmax, dP its
+#     upstream gradient), times the 1/sqrt(d) scale for the logits' inputs;
+#   * the two norms of Z0 are maxima of absolute sums: the gradient flows to
+#     the maximising column / row (numpy.argmax order at ties), d|a|/da =
+#     sign(a).  A row-softmax has every row sum 1, so the infinity-norm term
+#     vanishes after the softmax backward whichever row is chosen.
+
+
+def _softmax_rows_backward(P, dP):
+    return P * (dP - (dP * P).sum(axis=1, keepdims=True))
+
+
+def _segment_means_backward(dXt, n, m):
+    """Gradient of segment_means: every token of segment j receives
+    dXt[j] / (tokens of segment j)."""
+    seg = -(-n // m)
+    dX = np.zeros((n, dXt.shape[1]), dtype=np.float64)
+    for j in range(m):
+        lo, hi = j * seg, min((j + 1) * seg, n)
+        dX[lo:hi] = dXt[j] / (hi - lo)
+    return dX
+
+
+def _pinv_backward(A, Zs, dZ):
+    """Gradient with respect to A of Z = iterative_pinv(A, len(Zs) - 1), given
+    the iterates Zs = [Z0, .., ZT] and dZ = dL/dZT."""
+    A = _f64(A)
+    m = A.shape[0]
+    I = np.eye(m)
+    dA = np.zeros_like(A)
+    for j in range(len(Zs) - 2, -1, -1):
+        Z = Zs[j]
+        P = A @ Z
+        T1 = 7.0 * I - P
+        T2 = 15.0 * I - P @ T1
+        T3 = 13.0 * I - P @ T2
+        # Z' = 1/4 Z T3
+        dT3 = 0.25 * Z.T @ dZ
+        dZ_prev = 0.25 * dZ @ T3.T
+        # T3 = 13 I - P T2
+        dP = -dT3 @ T2.T
+        dT2 = -P.T @ dT3
+        # T2 = 15 I - P T1
+        dP += -dT2 @ T1.T
+        dT1 = -P.T @ dT2
+        # T1 = 7 I - P
+        dP += -dT1
+        # P = A Z
+        dA += dP @ Z.T
+        dZ_prev += A.T @ dP
+        dZ = dZ_prev
+    # Z0 = A^T c, c = 1 / (||A||_1 ||A||_inf)
+    col = np.abs(A).sum(axis=0)
+    row = np.abs(A).sum(axis=1)
+    n1, ninf = col.max(), row.max()
+    c = 1.0 / (n1 * ninf)
+    dA += c * dZ.T
+    dc = float((dZ * A.T).sum())
+    jc, ir = int(np.argmax(col)), int(np.argmax(row))
+    dA[:, jc] += (-dc * c / n1) * np.sign(A[:, jc])
+    dA[ir, :] += (-dc * c / ninf) * np.sign(A[ir, :])
+    return dA
+
+
+def nystrom_head_backward(Q, K, V, m, dout, iters=6, w=None, scale=None):
+    """Gradients of sum(dout * nystrom_head(Q, K, V, m, iters, w)["out"])
+    with respect to Q, K, V and w.  Returns a dict dQ, dK, dV ([n, d]) and
+    dw ([k], or None without the conv skip)."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    G = _f64(dout)
+    n, d = Q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    # forward, keeping every intermediate the chain rule needs
+    Qt = segment_means(Q, m)
+    Kt = segment_means(K, m)
+    F = kernel_F(Q, Kt, scale)
+    A = kernel_A(Qt, Kt, scale)
+    Zs = iterative_pinv(A, iters, return_all=True)
+    Z = Zs[-1]
+    B = kernel_B(Qt, K, scale)
+    Y = B @ V
+    W = Z @ Y
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dw = None
+    # out = O + C, C = DConv(V): C[i] = sum_t w[t] V[i + t - half]
+    if w is not None:
+        w = _f64(w).reshape(-1)
+        k = w.shape[0]
+        half = (k - 1) // 2
+        dw = np.zeros(k, dtype=np.float64)
+        for t in range(k):
+            off = t - half
+            lo, hi = max(0, -off), min(n, n - off)
+            if hi > lo:
+                dV[lo + off:hi + off] += w[t] * G[lo:hi]
+                dw[t] = float((G[lo:hi] * V[lo + off:hi + off]).sum())
+    # O = F W
+    dF = G @ W.T
+    dW = F.T @ G
+    # W = Z Y
+    dZ = dW @ Y.T
+    dY = Z.T @ dW
+    # Y = B V
+    dB = dY @ V.T
+    dV += B.T @ dY
+    # B = softmax(s Qt K^T)
+    dSB = _softmax_rows_backward(B, dB)
+    dQt = scale * dSB @ K
+    dK += scale * dSB.T @ Qt
+    # F = softmax(s Q Kt^T)
+    dSF = _softmax_rows_backward(F, dF)
+    dQ += scale * dSF @ Kt
+    dKt = scale * dSF.T @ Q
+    # Z = iterative_pinv(A), A = softmax(s Qt Kt^T)
+    dA = _pinv_backward(A, Zs, dZ)
+    dSA = _softmax_rows_backward(A, dA)
+    dQt += scale * dSA @ Kt
+    dKt += scale * dSA.T @ Qt
+    # Qt, Kt = segment means
+    dQ += _segment_means_backward(dQt, n, m)
+    dK += _segment_means_backward(dKt, n, m)
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dw": dw}
+
+
+def nystrom_backward(Q, K, V, m, dout, iters=6, conv_w=None):
+    """Batched backward over [B, H, n, d]: dQ, dK, dV [B, H, n, d] and dconv
+    [H, k] (summed over the batch) or None."""
+    Q = _f64(Q)
+    Bn, H, n, d = Q.shape
+    dQ = np.empty_like(Q)
+    dK = np.empty_like(Q)
+    dV = np.empty_like(Q)
+    dconv = None if conv_w is None else np.zeros(_f64(conv_w).shape, dtype=np.float64)
+    for b in range(Bn):
+        for h in range(H):
+            w = None if conv_w is None else _f64(conv_w)[h]
+            g = nystrom_head_backward(Q[b, h], K[b, h], V[b, h], m, dout[b, h], iters, w)
+            dQ[b, h], dK[b, h], dV[b, h] = g["dQ"], g["dK"], g["dV"]
+            if dconv is not None:
+                dconv[h] += g["dw"]
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dconv": dconv}
 
 
 def exact_attention_head(Q, K, V, scale=None):
