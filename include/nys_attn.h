@@ -126,6 +126,34 @@ NYS_ATTN_API nys_status nys_attn_forward(const void *Q_dev, const void *K_dev, c
                                          void *workspace_dev, size_t workspace_bytes,
                                          nys_stream_t stream);
 
+/* nys_attn_forward on right-padded ragged batches: element b holds
+ * lens_dev[b] real tokens followed by padding, and is computed as the method
+ * on its first lens_dev[b] tokens alone.  The pages describe no mask (every
+ * token attends to every token) and make divisibility a matter of padding
+ * ("Landmark Selection: Segment-Means"); this is that reading for a caller
+ * with ragged batches:
+ *   - landmarks are the segment means over the element's L = lens_dev[b]
+ *     tokens (segments of ceil(L / m) tokens, the last one possibly shorter),
+ *   - B~'s softmax runs over its L keys and F~ over its L queries,
+ *   - the DConv skip pads with zeros from row L on,
+ *   - output rows L .. seq_len - 1 are zero.
+ *   lens_dev   device array of `batch` int32, 4-byte aligned; each
+ *              m <= L <= seq_len with no empty segment ((m - 1) * ceil(L/m) <
+ *              L).  A length that breaks this records NYS_ERR_INVALID_ARG in
+ *              the workspace error word (nys_attn_check_error) and its
+ *              element's output is all zero; the other elements are computed.
+ * Every other argument, the workspace size and the error behaviour are those
+ * of nys_attn_forward; lens_dev == NULL (with a non-empty problem) is
+ * NYS_ERR_INVALID_ARG.  With every L = seq_len the result equals
+ * nys_attn_forward's. */
+NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q_dev, const void *K_dev,
+                                              const void *V_dev, const nys_desc *desc,
+                                              int num_landmarks, int pinv_iters,
+                                              const float *conv_w_dev, int conv_k,
+                                              const int *lens_dev, void *out_dev,
+                                              void *workspace_dev, size_t workspace_bytes,
+                                              nys_stream_t stream);
+
 /* Offsets (in bytes from the start of the workspace) of the fp32
  * intermediates a forward leaves there, for parity checks:
  *   q_landmarks, k_landmarks  [batch*heads][m][head_dim]   Q~, K~

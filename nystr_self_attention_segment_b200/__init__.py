@@ -18,7 +18,7 @@ __all__ = [
     "nys_attn_forward_host", "nys_attn_workspace_size", "nys_attn_intermediates",
     "nys_attn_host_buffer_size", "nys_attn_check_error", "nys_attn_launch_count",
     "nys_status_string", "nys_version", "Workspace", "nys_attn_launch_names",
-    "nys_attn_forward_timed",
+    "nys_attn_forward_timed", "nys_attn_forward_lens",
 ]
 
 
@@ -129,6 +129,29 @@ def nys_attn_forward(Q, K, V, num_landmarks, pinv_iters=6, conv_w=None, out=None
                               pinv_iters, conv_ptr, conv_k, out.data_ptr(), ws_ptr, ws_bytes,
                               _stream_ptr(stream))
     _lib.check(st, "nys_attn_forward")
+    return out
+
+
+def nys_attn_forward_lens(Q, K, V, num_landmarks, lens, pinv_iters=6, conv_w=None, out=None,
+                          workspace=None, stream=None):
+    """nys_attn_forward on right-padded ragged batches: element b holds
+    lens[b] real tokens (lens: int32 CUDA tensor [batch]); its output rows
+    from lens[b] on are zero.  See nys_attn_forward_lens in the header."""
+    torch = _torch()
+    if out is None and getattr(Q, "is_cuda", False):
+        out = torch.empty_like(Q)
+    _check_operands(Q, K, V, Q if out is None else out, conv_w)
+    if (not lens.is_cuda or lens.dtype != torch.int32 or not lens.is_contiguous()
+            or lens.dim() != 1 or lens.shape[0] != Q.shape[0] or lens.device != Q.device):
+        raise ValueError("lens must be a contiguous int32 CUDA tensor [batch] on Q's device")
+    desc = desc_of(Q)
+    conv_ptr, conv_k = (None, 0) if conv_w is None else (conv_w.data_ptr(), conv_w.shape[1])
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.ptr, workspace.nbytes)
+    with _on_device(Q.device):
+        st = _lib.raw_forward_lens(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc,
+                                   num_landmarks, pinv_iters, conv_ptr, conv_k, lens.data_ptr(),
+                                   out.data_ptr(), ws_ptr, ws_bytes, _stream_ptr(stream))
+    _lib.check(st, "nys_attn_forward_lens")
     return out
 
 

@@ -40,6 +40,7 @@ EXPORTS = (
     "nys_attn_launch_names",
     "nys_attn_forward_static",
     "nys_attn_check_error_static",
+    "nys_attn_forward_lens",
 )
 
 # Size of the fixed scratch array of nys_attn_forward_static (see the header).
@@ -106,6 +107,8 @@ def load():
     lib.nys_attn_forward_static.argtypes = [P, P, P, D, I, I, P, I, P, P]
     lib.nys_attn_check_error_static.restype = I
     lib.nys_attn_check_error_static.argtypes = [D, I, P]
+    lib.nys_attn_forward_lens.restype = I
+    lib.nys_attn_forward_lens.argtypes = [P, P, P, D, I, I, P, I, P, P, P, S, P]
     _LIB = lib
     return lib
 
@@ -194,6 +197,15 @@ def raw_forward_static(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, con
     return load().nys_attn_forward_static(q_ptr, k_ptr, v_ptr, ctypes.byref(desc),
                                           int(num_landmarks), int(pinv_iters), conv_ptr,
                                           int(conv_k), out_ptr, stream_ptr)
+
+
+def raw_forward_lens(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_ptr, conv_k,
+                     lens_ptr, out_ptr, ws_ptr, ws_bytes, stream_ptr):
+    """nys_attn_forward_lens on raw addresses (lens_ptr: device int32 [batch])."""
+    return load().nys_attn_forward_lens(q_ptr, k_ptr, v_ptr, ctypes.byref(desc),
+                                        int(num_landmarks), int(pinv_iters), conv_ptr,
+                                        int(conv_k), lens_ptr, out_ptr, ws_ptr,
+                                        ctypes.c_size_t(ws_bytes), stream_ptr)
 
 
 def raw_check_error_static(desc, num_landmarks, stream_ptr):

@@ -7,9 +7,9 @@
 //                             Approximating Self-Attention", section 3.4,
 //                             Eq. 17 / Algorithm 1; B~ = softmax(Q~ K^T/sqrt(d))
 //                             over the n keys is never stored).
-// The last B~ V block of a head (counted with an atomic) merges the head's S
-// partial softmax states in a fixed order into Y; the second of {that
-// block, the pseudoinverse block} to finish forms W = Z Y in fp32.
+// Each B~ V block leaves one partial softmax state per landmark (running
+// maximum, sum, unnormalised Y); the next kernel (wmerge.cuh) merges them and
+// forms W = Z Y.
 //
 // B~ V block.  The 128 accumulator rows (TMEM lanes) hold G = 128 / m copies
 // of the m landmark rows; copy g handles keys g*m .. g*m + m - 1 of every
@@ -63,17 +63,6 @@ __host__ __device__ inline BvSmem bv_smem() {
 }
 
 template <int M>
-struct MergeCfg {
-  static constexpr int kZs = M + 4, kYs = 68;                // row strides (floats)
-  static constexpr uint32_t zs = 0;                          // Z [M][M + 4] fp32
-  static constexpr uint32_t ys = zs + M * kZs * 4u;          // Y [M][68] fp32
-  static constexpr uint32_t wgt = ys + M * kYs * 4u;         // [kMaxSplits][M] weights
-  static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
-  static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
-  static constexpr uint32_t total = den + M * 4u;
-};
-
-template <int M>
 __host__ __device__ constexpr uint32_t pinv_smem() {
   if constexpr (M <= 64) {
     return pinvpow::Cfg<M>::total;
@@ -84,21 +73,18 @@ __host__ __device__ constexpr uint32_t pinv_smem() {
 
 template <int M>
 __host__ __device__ constexpr uint32_t smem_bytes() {
-  // pinv operands, B~ V buffers, and the merge scratch (Z, Y, weights)
+  // pinv operands or B~ V buffers
   constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
-  constexpr uint32_t a = pinv_smem<M>() > bv ? pinv_smem<M>() : bv;
-  return 1024u + (a > MergeCfg<M>::total ? a : MergeCfg<M>::total);
+  return 1024u + (pinv_smem<M>() > bv ? pinv_smem<M>() : bv);
 }
 
 struct Params {
   pinvtc::Params pinv;
   const float *q_land;        // [BH][m][64]
-  const float *z;             // [BH][m][m]  (pinv output)
   float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
-  float *y, *w;               // [BH][m][64]
-  uint8_t *w_op;              // [BH][m][128 B] W as the bf16 B operand of P W
-  uint32_t *count;            // [2 BH] per head: B~ V blocks done, inputs of W ready (zeroed per call)
   uint32_t *err;
+  const int *lens;            // [batch] tokens per element (ragged batches) or null
+  int heads;
   int BH, n, chunks_per_head, splits;
   float scale_log2;
 };
@@ -125,9 +111,17 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   constexpr int G = 128 / M;
   const BvSmem L = bv_smem();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // keys [0, L): L = n, or the element's own length (an invalid one reads as
+  // 0 and leaves the split empty; the segment-mean kernel reports it)
+  int seq = prm.n;
+  if (prm.lens) {
+    seq = prm.lens[bh / prm.heads];
+    if (seq < M || seq > prm.n || (long)(M - 1) * ((seq + M - 1) / M) >= seq) seq = 0;
+  }
   const int c_begin = (int)((long)split * prm.chunks_per_head / prm.splits);
-  const int c_end = (int)((long)(split + 1) * prm.chunks_per_head / prm.splits);
-  const int nch = c_end - c_begin;
+  const int c_end = min((int)((long)(split + 1) * prm.chunks_per_head / prm.splits),
+                        (seq + kChunk - 1) / kChunk);
+  const int nch = c_end > c_begin ? c_end - c_begin : 0;
 
   uint64_t *bars = (uint64_t *)(smem + L.bars);
   uint64_t *full = bars;                  // [kStages]
@@ -283,7 +277,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       tc_fence_before();
       mbar_arrive(&s_free[wg]);
       const int key0 = (c_begin + i) * kChunk + g * M;
-      const int valid = min(M, prm.n - key0);     // keys of this group inside [0, n)
+      const int valid = min(M, seq - key0);       // keys of this group inside [0, L)
       named_barrier(2 + wg, 256);                  // this warpgroup's turn
       float mx[8];
 #pragma unroll
@@ -425,215 +419,13 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   }
 }
 
-// ------------------------------------------------------------------ merge + W
-// Y = sum_s f_s py_s / sum_s f_s psum_s, f_s = 2^(pmax_s - max), over the S
-// key splits of the head in split order (merge_y_body, run by the last B~ V
-// block of the head), then W = Z Y in fp32 (w_product), run by the second of
-// {pseudoinverse block, that B~ V block} to finish.
-
-// All 384 threads, three phases: the S x M maxima and sums into shared
-// memory; the weights f_s and 1 / sum_s f_s psum_s of each row; then the
-// partials, a batch of up to kBatch splits of every item of a thread loaded
-// at once.  (Partials in flight during the weights phase would queue its
-// shared-memory reads behind their data.)
-// ysm: optional [M][68] fp32 copy of Y in shared memory (the W operand).
-template <int M>
-__device__ __forceinline__ void merge_y_body(const Params &prm, uint8_t *smem, int bh,
-                                             float *ysm = nullptr) {
-  using C = MergeCfg<M>;
-  constexpr int NT = kThreads;
-  const int t = threadIdx.x;
-  const int S = prm.splits;
-  float *wgt = (float *)(smem + C::wgt);
-  float *psm = (float *)(smem + C::psm);
-  float *den = (float *)(smem + C::den);
-  const size_t pb = (size_t)bh * S * M;
-  {
-    constexpr int kPer = (kMaxSplits * M + NT - 1) / NT;
-    float a[kPer], b[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = t + u * NT;
-      if (i < S * M) {
-        a[u] = __ldcg(prm.pmax + pb + i);
-        b[u] = __ldcg(prm.psum + pb + i);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = t + u * NT;
-      if (i < S * M) {
-        wgt[i] = a[u];
-        psm[i] = b[u];
-      }
-    }
-  }
-  __syncthreads();
-  if (t < M) {
-    const int j = t;
-    float mx = -INFINITY;
-    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + j]);
-    float d = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + j] - mx);
-      wgt[s * M + j] = f;
-      d = fmaf(psm[s * M + j], f, d);
-    }
-    den[j] = 1.f / d;
-  }
-  __syncthreads();
-  constexpr int kItems = M * 16;   // float4 items of Y
-  constexpr int kIpt = 3;          // items per thread per round
-  constexpr int kBatch = 8;        // splits per load batch
-  for (int base = 0; base < kItems; base += NT * kIpt) {
-    float4 a[kIpt];
-#pragma unroll
-    for (int q = 0; q < kIpt; ++q) a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < S; s0 += kBatch) {
-      float4 v[kIpt][kBatch];
-#pragma unroll
-      for (int q = 0; q < kIpt; ++q) {
-        const int idx = base + q * NT + t;
-        if (idx < kItems) {
-          const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u)
-            if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < kIpt; ++q) {
-        const int idx = base + q * NT + t;
-        if (idx < kItems) {
-          const int j = idx >> 4;
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u)
-            if (s0 + u < S) {
-              const float f = wgt[(s0 + u) * M + j];
-              a[q].x = fmaf(f, v[q][u].x, a[q].x);
-              a[q].y = fmaf(f, v[q][u].y, a[q].y);
-              a[q].z = fmaf(f, v[q][u].z, a[q].z);
-              a[q].w = fmaf(f, v[q][u].w, a[q].w);
-            }
-        }
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < kIpt; ++q) {
-      const int idx = base + q * NT + t;
-      if (idx < kItems) {
-        const float inv = den[idx >> 4];
-        const float4 y = make_float4(a[q].x * inv, a[q].y * inv, a[q].z * inv, a[q].w * inv);
-        ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] = y;
-        if (ysm) *(float4 *)(ysm + (idx >> 4) * C::kYs + (idx & 15) * 4) = y;
-      }
-    }
-  }
-  __syncthreads();
-}
-
-// Z of head bh from global memory into shared memory (MergeCfg::zs); all
-// threads, every load issued before the first store.
-template <int M>
-__device__ __forceinline__ void load_z(const Params &prm, uint8_t *smem, int bh) {
-  using C = MergeCfg<M>;
-  constexpr int kZ4 = M * M / 4, kPer = (kZ4 + kThreads - 1) / kThreads;
-  float *zs = (float *)(smem + C::zs);
-  const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
-  float4 v[kPer];
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = threadIdx.x + u * kThreads;
-    if (i < kZ4) v[u] = __ldcg(zg + i);
-  }
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = threadIdx.x + u * kThreads;
-    if (i < kZ4) *(float4 *)(zs + (i * 4 / M) * C::kZs + (i * 4) % M) = v[u];
-  }
-}
-
-// Y of head bh from global memory into shared memory (MergeCfg::ys).
-template <int M>
-__device__ __forceinline__ void load_y(const Params &prm, uint8_t *smem, int bh) {
-  using C = MergeCfg<M>;
-  constexpr int kY4 = M * 16, kPer = (kY4 + kThreads - 1) / kThreads;
-  float *ys = (float *)(smem + C::ys);
-  const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
-  float4 v[kPer];
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = threadIdx.x + u * kThreads;
-    if (i < kY4) v[u] = __ldcg(yg + i);
-  }
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = threadIdx.x + u * kThreads;
-    if (i < kY4) *(float4 *)(ys + (i >> 4) * C::kYs + (i & 15) * 4) = v[u];
-  }
-}
-
-// W = Z Y in fp32 (k in order) from Z and Y in shared memory, stored as fp32
-// rows and as the bf16 operand of P W (row = landmark, 16-byte chunk c at
-// c ^ (row & 7): the 128-byte swizzle of a 1 KB-aligned tile).  Threads
-// 0..255, each 4 columns of M / 16 rows; Z and Y must be visible to them.
-template <int M>
-__device__ __forceinline__ void w_product(const Params &prm, const uint8_t *smem, int bh) {
-  using C = MergeCfg<M>;
-  constexpr int R = M / 16;
-  const int t = threadIdx.x;
-  if (t >= 256) return;
-  const float *zs = (const float *)(smem + C::zs), *ys = (const float *)(smem + C::ys);
-  const int c4 = t & 15, i0 = (t >> 4) * R;
-  float acc[R][4];
-#pragma unroll
-  for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-#pragma unroll 2
-  for (int k = 0; k < M; k += 4) {
-    float4 y[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = *(const float4 *)(ys + (k + e) * C::kYs + 4 * c4);
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const float4 z = *(const float4 *)(zs + (i0 + r) * C::kZs + k);
-      const float zk[4] = {z.x, z.y, z.z, z.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[r][0] = fmaf(zk[e], y[e].x, acc[r][0]);
-        acc[r][1] = fmaf(zk[e], y[e].y, acc[r][1]);
-        acc[r][2] = fmaf(zk[e], y[e].z, acc[r][2]);
-        acc[r][3] = fmaf(zk[e], y[e].w, acc[r][3]);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int row = i0 + r;
-    *(float4 *)(prm.w + ((size_t)bh * M + row) * 64 + 4 * c4) =
-        make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-    uint8_t *op = prm.w_op + ((size_t)bh * M + row) * 128;
-    *(uint2 *)(op + (((c4 >> 1) ^ (row & 7)) << 4) + (c4 & 1) * 8) =
-        make_uint2(pack_bf16(acc[r][0], acc[r][1]), pack_bf16(acc[r][2], acc[r][3]));
-  }
-}
-
-// Both steps in one block (used by the persistent schedule).
-template <int M>
-__device__ __forceinline__ void merge_body(const Params &prm, uint8_t *smem, int bh) {
-  merge_y_body<M>(prm, smem, bh, (float *)(smem + MergeCfg<M>::ys));
-  load_z<M>(prm, smem, bh);
-  __syncthreads();
-  w_product<M>(prm, smem, bh);
-}
-
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
            const Params prm) {
-  using C = MergeCfg<M>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint32_t last, tmem_base;
+  __shared__ uint32_t tmem_base;
   const int t = threadIdx.x;
   NYS_MARK(kTrMid, 0);
   // one TMEM allocation for every body this block runs (an allocation
@@ -649,56 +441,22 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = tmem_base;
   const bool is_pinv = (int)blockIdx.x < prm.BH;
-  // Z is left in shared memory by the pseudoinverse (m <= 64, at least one step)
-  const bool z_in_smem = M <= 64 && is_pinv && prm.pinv.iters > 0;
-  int bh;
   if (is_pinv) {
-    bh = blockIdx.x;
+    const int bh = blockIdx.x;
     griddep_wait();
     griddep_launch_dependents();
     NYS_MARK(kTrMid, 1);
     if constexpr (M <= 64) {
       if (t < pinvpow::kBarThreads)
-        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, (float *)(smem + C::zs));
+        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
     } else {
       if (t < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
     }
   } else {
     const int b = blockIdx.x - prm.BH;
-    bh = b / prm.splits;
-    bv_body<M>(&map_k, &map_v, prm, smem, bh, b % prm.splits, tmem, true);
+    bv_body<M>(&map_k, &map_v, prm, smem, b / prm.splits, b % prm.splits, tmem, true);
   }
-  // publish this block's results.  The last B~ V block of a head merges the
-  // partials into Y; the second of {pseudoinverse, Y merge} to finish forms
-  // W = Z Y.  Counters: count[bh] B~ V blocks done, count[BH + bh] inputs of
-  // W ready.
   NYS_MARK(kTrMid, 2);
-  __threadfence();
-  __syncthreads();
-  if (t == 0)
-    last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
-  __syncthreads();
-  if (last) {
-    if (!is_pinv) {
-      __threadfence();
-      NYS_MARK(kTrMid, 3);
-      merge_y_body<M>(prm, smem, bh, (float *)(smem + C::ys));
-      __threadfence();
-      __syncthreads();
-      NYS_MARK(kTrMid, 4);
-    }
-    if (t == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
-    __syncthreads();
-    if (last) {
-      __threadfence();
-      NYS_MARK(kTrMid, 5);
-      if (is_pinv) load_y<M>(prm, smem, bh);
-      if (!z_in_smem) load_z<M>(prm, smem, bh);
-      __syncthreads();
-      w_product<M>(prm, smem, bh);
-      NYS_MARK(kTrMid, 6);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if ((t >> 5) == 1) {

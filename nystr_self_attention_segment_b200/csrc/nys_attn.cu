@@ -14,6 +14,7 @@
 #include "sm100.cuh"
 #include "mid_tc.cuh"
 #include "out_tc.cuh"
+#include "wmerge.cuh"
 #include "stream_bf16.cuh"
 
 using namespace nys;
@@ -95,10 +96,7 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.z = take(BH * m * m * 4);
   L.y = take(BH * m * d * 4);
   L.w = take(BH * m * d * 4);
-  // error word and task queue, then three counters per head (segment sums,
-  // pseudoinverse + B~ V tasks, W ready); all zeroed by every call
-  L.err = take(256 + BH * 12);
-  L.count = L.err + 256;
+  L.err = take(256);   // the error word, zeroed by every call
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
   L.py = take(BH * splits * m * d * 4);
@@ -211,14 +209,16 @@ const char *kSimtNames = "seg_means,pinv,bv_partial,merge_w,out";
 
 template <typename T>
 nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc, int m,
-                       int iters, const float *conv_w, int conv_k, T *out, char *ws,
-                       const Layout &L, cudaStream_t stream, Marks &mk) {
+                       int iters, const float *conv_w, int conv_k, const int *lens, T *out,
+                       char *ws, const Layout &L, cudaStream_t stream, Marks &mk) {
   const int BH = desc->batch * desc->heads;
   const int n = desc->seq_len, d = desc->head_dim;
   float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
   float *z = (float *)(ws + L.z), *y = (float *)(ws + L.y), *w = (float *)(ws + L.w);
   float *pmax = (float *)(ws + L.pmax), *psum = (float *)(ws + L.psum);
   float *py = (float *)(ws + L.py), *scratch = (float *)(ws + L.scratch);
+  uint32_t *err = (uint32_t *)(ws + L.err);
+  const int heads = desc->heads;
   const float scale = 1.0f / sqrtf((float)d);
   const float scale_log2 = scale * kLog2e;
 
@@ -228,7 +228,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     long total = (long)BH * m * d;
     dim3 grid((unsigned)((total + 255) / 256), 2);
     if (launch(seg_means_scalar<T>, grid, dim3(256), launch_smem(mk.launched, 0), stream, false,
-               Q, K, qt, kt, BH, n, d, m) != cudaSuccess)
+               Q, K, qt, kt, BH, n, d, m, lens, heads, err) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -247,7 +247,8 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     auto kern = m <= 64 ? bv_partial_simt<T, 8> : bv_partial_simt<T, 16>;
     if (!allow_smem(kern, sm) ||
         launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, qt, K, V,
-               pmax, psum, py, n, d, m, L.splits, L.keys_per_split, scale_log2) != cudaSuccess)
+               pmax, psum, py, n, d, m, L.splits, L.keys_per_split, scale_log2, lens,
+               heads) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -266,7 +267,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     auto kern = m <= 64 ? out_simt<T, 2> : out_simt<T, 4>;
     if (!allow_smem(kern, sm) ||
         launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, Q, V, kt, w,
-               conv_w, out, n, d, m, desc->heads, ck, scale_log2) != cudaSuccess)
+               conv_w, out, n, d, m, desc->heads, ck, scale_log2, lens) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -309,14 +310,14 @@ bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
 }
 
 // launches of the bf16 path
-constexpr int kTcLaunches = 3;
-const char *kTcNames = "seg_means,mid_tc,out_tc";
+constexpr int kTcLaunches = 4;
+const char *kTcNames = "seg_means,mid_tc,w_merge,out_tc";
 
 template <int M>
 nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                        const nys_desc *desc, int iters, const float *conv_w, int conv_k,
-                       __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
-                       Marks &mk) {
+                       const int *lens, __nv_bfloat16 *out, char *ws, const Layout &L,
+                       cudaStream_t stream, Marks &mk) {
   const int BH = desc->batch * desc->heads;
   const int n = desc->seq_len;
   float *qt = (float *)(ws + L.q_land), *kt = (float *)(ws + L.k_land);
@@ -324,7 +325,6 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
   float *pmax = (float *)(ws + L.pmax), *psum = (float *)(ws + L.psum);
   float *py = (float *)(ws + L.py);
   uint32_t *err = (uint32_t *)(ws + L.err);
-  uint32_t *count = (uint32_t *)(ws + L.count);
   const float scale_log2 = 0.125f * kLog2e;   // log2(e) / sqrt(64)
   const bool conv = conv_w != nullptr;
   const int kconv = conv ? ((128 + conv_k - 1 + 15) / 16) * 16 : 0;
@@ -336,26 +336,25 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     return NYS_ERR_CUDA;
 
   {   // segment means of Q and K (Eq. 16)
-    const int seg = (n + M - 1) / M;   // tokens of a full segment
-    const int groups = seg < 32 ? seg : 32;
-    if (launch(seg_means_bf16, dim3(M, BH, 2), dim3(8 * groups), launch_smem(mk.launched, 0),
-               stream, false, Q, K, qt, kt, n, M) != cudaSuccess)
+    const segm::Shape sh{n, M, desc->heads, lens};
+    const dim3 grid(segm::groups_for(BH, M), BH, 2);
+    if (!allow_smem(segm::seg_means_bf16, segm::kSmem) ||
+        launch(segm::seg_means_bf16, grid, dim3(segm::kThreads),
+               launch_smem(mk.launched, segm::kSmem), stream, false, Q, K, qt, kt, sh,
+               err) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
-  {   // pseudoinverse || B~ V, then merge + W = Z Y
+  {   // pseudoinverse || B~ V
     midtc::Params p;
     p.pinv = pinvtc::Params{qt, kt, z, err, iters, scale_log2};
     p.q_land = qt;
-    p.z = z;
     p.pmax = pmax;
     p.psum = psum;
     p.py = py;
-    p.y = y;
-    p.w = w;
-    p.w_op = (uint8_t *)(ws + L.w_bf);
-    p.count = count;
     p.err = err;
+    p.lens = lens;
+    p.heads = desc->heads;
     p.BH = BH;
     p.n = n;
     p.chunks_per_head = (n + midtc::kChunk - 1) / midtc::kChunk;
@@ -369,13 +368,23 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
+  {   // merge of the B~ V partials, W = Z Y
+    const wmerge::Params p{pmax, psum, py, z, y, w, (uint8_t *)(ws + L.w_bf), L.splits};
+    auto kern = wmerge::wmerge_kernel<M>;
+    const uint32_t sm = wmerge::Smem<M>::total;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH * (M / wmerge::kRows)), dim3(wmerge::kThreads),
+               launch_smem(mk.launched, sm), stream, true, p) != cudaSuccess)
+      return NYS_ERR_CUDA;
+    mk.after(stream);
+  }
   {   // F~ W + DConv(V)
     const int tph = (n + outtc::kTileRows - 1) / outtc::kTileRows;
     int cpb = kNumSms / BH;
     if (cpb < 1) cpb = 1;
     if (cpb > tph) cpb = tph;
-    outtc::Params p{kt, (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads, conv ? conv_k : 1, kconv, tph, cpb,
-                    scale_log2};
+    outtc::Params p{kt,  (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads,
+                    conv ? conv_k : 1, kconv, tph, cpb, scale_log2, lens, M};
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
     if (!allow_smem(kern, sm) ||
@@ -389,13 +398,13 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
 
 nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                      const nys_desc *desc, int m, int iters, const float *conv_w, int conv_k,
-                     __nv_bfloat16 *out, char *ws, const Layout &L, cudaStream_t stream,
-                     Marks &mk) {
+                     const int *lens, __nv_bfloat16 *out, char *ws, const Layout &L,
+                     cudaStream_t stream, Marks &mk) {
   switch (m) {
-    case 32: return launch_tc_m<32>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
-    case 64: return launch_tc_m<64>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+    case 32: return launch_tc_m<32>(Q, K, V, desc, iters, conv_w, conv_k, lens, out, ws, L, stream, mk);
+    case 64: return launch_tc_m<64>(Q, K, V, desc, iters, conv_w, conv_k, lens, out, ws, L, stream, mk);
     case 128:
-      return launch_tc_m<128>(Q, K, V, desc, iters, conv_w, conv_k, out, ws, L, stream, mk);
+      return launch_tc_m<128>(Q, K, V, desc, iters, conv_w, conv_k, lens, out, ws, L, stream, mk);
   }
   return NYS_ERR_UNSUPPORTED;
 }
@@ -473,7 +482,8 @@ static nys_status validate_call(const void *Q, const void *K, const void *V,
 static nys_status forward_impl(const void *Q, const void *K, const void *V,
                                const nys_desc *desc, int m, int iters, const float *conv_w,
                                int conv_k, void *out, void *workspace, size_t workspace_bytes,
-                               nys_stream_t stream_, void *const *events, int n_events) {
+                               nys_stream_t stream_, void *const *events, int n_events,
+                               const int *lens = nullptr) {
   nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
   if (st != NYS_OK) return st;
   if (events && n_events < (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches) + 1)
@@ -500,17 +510,15 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (cudaMemsetAsync(ws + L.err, 0, 256 + (size_t)desc->batch * desc->heads * 12, stream) !=
-      cudaSuccess)
-    st = NYS_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
   mk.first(stream);
   if (st == NYS_OK) {
     if (desc->dtype == NYS_F32)
       st = launch_simt<float>((const float *)Q, (const float *)K, (const float *)V, desc, m,
-                              iters, conv_w, conv_k, (float *)out, ws, L, stream, mk);
+                              iters, conv_w, conv_k, lens, (float *)out, ws, L, stream, mk);
     else
       st = launch_tc((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
-                     (const __nv_bfloat16 *)V, desc, m, iters, conv_w, conv_k,
+                     (const __nv_bfloat16 *)V, desc, m, iters, conv_w, conv_k, lens,
                      (__nv_bfloat16 *)out, ws, L, stream, mk);
   }
   if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && st == NYS_OK) st = NYS_ERR_CUDA;
@@ -524,6 +532,18 @@ NYS_ATTN_API nys_status nys_attn_forward(const void *Q, const void *K, const voi
                                          nys_stream_t stream) {
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
                       stream, nullptr, 0);
+}
+
+NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q, const void *K, const void *V,
+                                              const nys_desc *desc, int m, int iters,
+                                              const float *conv_w, int conv_k,
+                                              const int *lens_dev, void *out, void *workspace,
+                                              size_t workspace_bytes, nys_stream_t stream) {
+  const nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if ((!lens_dev && !is_empty(desc)) || ((uintptr_t)lens_dev & 3) != 0) return NYS_ERR_INVALID_ARG;
+  return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
+                      stream, nullptr, 0, lens_dev);
 }
 
 // ---------------------------------------------------------------------------

@@ -72,6 +72,8 @@ struct Params {
   int n, heads, conv_k, kconv;
   int tiles_per_head, ctas_per_head;
   float scale_log2;
+  const int *lens;         // [batch] tokens per element (ragged batches) or null
+  int m;
 };
 
 // One run of 128-row tiles [t_begin, t_end) of (batch, head) bh.  tmem_in: a
@@ -92,6 +94,17 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   const int ntiles = t_end - t_begin;
   const bool conv = prm.conv_w != nullptr;
   const int half = (prm.conv_k - 1) / 2;
+  // rows [0, L) of the element are real (L = n, or its own length for ragged
+  // batches; an invalid length reads as 0).  Output rows from L on are zero,
+  // and V rows from L on read as zero in the conv: a warp (3) clears them in
+  // the staged V tile before the conv MMA may read it.
+  int seq = prm.n;
+  if (prm.lens) {
+    seq = prm.lens[bh / prm.heads];
+    if (seq < prm.m || seq > prm.n || (long)(prm.m - 1) * ((seq + prm.m - 1) / prm.m) >= seq)
+      seq = 0;
+  }
+  const bool mask_v = conv && prm.lens != nullptr;
   constexpr uint32_t kStride = M + 64;        // TMEM columns per softmax warpgroup
   constexpr uint32_t kT = 2 * kStride;        // Toeplitz operand columns
 
@@ -103,7 +116,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   uint64_t *o_full = p_ready + 2;
   uint64_t *tm_free = o_full + 2;
   uint64_t *w_ready = tm_free + 2;         // W operand in shared memory
-  uint32_t *tmem_slot = (uint32_t *)(w_ready + 1);
+  uint64_t *v_ready = w_ready + 1;         // [kStages] V tile masked past L
+  uint32_t *tmem_slot = (uint32_t *)(v_ready + kStages);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
   float *cw = (float *)(smem + L.cw);
@@ -121,6 +135,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       mbar_init(&tm_free[b], 128);
     }
     mbar_init(w_ready, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&v_ready[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(map_q);
@@ -193,6 +208,24 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     mbar_expect_tx(w_ready, M * 128u);
     bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
   }
+  if (warp == 3 && mask_v) {
+    // ragged batches: halo rows at or past L of every staged V tile become
+    // zero before its conv MMA (v_ready); tiles are taken in order, each
+    // after its load, so the barrier phases cannot run ahead
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % kStages;
+      if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) break;
+      const int first = seq - ((t_begin + i) * kTileRows - half);   // first halo row past L
+      if (first < prm.kconv) {
+        const uint32_t base = smem_u32(smem + L.v[s]);
+        for (int q = (first > 0 ? first : 0) * 8 + lane; q < prm.kconv * 8; q += 32)
+          st_shared_v4(base + (uint32_t)q * 16u, 0u, 0u, 0u, 0u);
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_ready[s]);
+    }
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -240,6 +273,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
         if (!mbar_wait(&tm_free[w], (u & 1) ^ 1, ab)) break;
         tc_fence_after();
         if (conv) {
+          if (mask_v && !mbar_wait(&v_ready[s], (i / kStages) & 1, ab)) break;
+          tc_fence_after();
           const uint32_t v_a = smem_u32(smem + L.v[s]);
           for (int k = 0; k < prm.kconv / 16; ++k)
             mma_bf16_ts(tmem + w * kStride + M, tmem + kT + 8 * k,
@@ -309,6 +344,10 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       // this warpgroup's staging buffer was last used two of its tiles ago
       if (r == 0) bulk_wait_read0();
       named_barrier(2 + wg, 128);
+      if ((t_begin + i) * kTileRows + r >= seq) {   // padding rows of a ragged element
+#pragma unroll
+        for (int c = 0; c < 64; ++c) o[c] = 0.f;
+      }
       const uint32_t o_row = smem_u32(smem + L.o[wg]);
 #pragma unroll
       for (int c = 0; c < 8; ++c)
@@ -327,7 +366,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && !*abort_flag)
-    for (int b = 0; b < 2 * kStages + 9; ++b) mbar_inval(bars + b);
+    for (int b = 0; b < 3 * kStages + 9; ++b) mbar_inval(bars + b);
   if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

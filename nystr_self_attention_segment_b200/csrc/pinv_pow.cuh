@@ -156,13 +156,9 @@ __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
 // scale_log2 = log2(e) / sqrt(d).
 // tmem_in: a TMEM allocation of at least Cfg<M>::kTmemCols columns owned by
 // the caller, or ~0u to allocate (and free) one here.
-// zsm (optional, at least one step): after the last step the final Z is
-// also written there, fp32 row-major with a row stride of M + 4 floats, for a
-// following W = Z Y in the same block.  It may overlap the operand buffers
-// (written after the last product has read them).
 template <int M, class Prm>
 __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
-                                          uint32_t tmem_in = ~0u, float *zsm = nullptr) {
+                                          uint32_t tmem_in = ~0u) {
   using C = Cfg<M>;
   constexpr int NC = C::NC;
   const int t = threadIdx.x, warp = t >> 5;
@@ -462,15 +458,6 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
         for (int q = 0; q < NC / 4; ++q)
           *(float4 *)(zg + (size_t)row * M + c_lo + 4 * q) =
               make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-      }
-      if (zsm) {
-        named_barrier(1, kBarThreads);   // every operand buffer of the steps is dead
-        if (ok && aux) {
-#pragma unroll
-          for (int q = 0; q < NC / 4; ++q)
-            *(float4 *)(zsm + row * (M + 4) + c_lo + 4 * q) =
-                make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-        }
       }
     }
   }

@@ -12,14 +12,30 @@
 
 namespace nys {
 
+// Tokens of element bh / heads: its own length for ragged batches (lens, one
+// per batch element, on the device), else n.  A length outside [m, n] or with
+// an empty segment reads as 0 (the element's output is all zero) and records
+// NYS_ERR_INVALID_ARG.
+__device__ __forceinline__ int seq_len_of(const int *lens, int bh, int heads, int n, int m,
+                                          uint32_t *err) {
+  if (!lens) return n;
+  const int L = lens[bh / heads];
+  if (L < m || L > n || (long)(m - 1) * ((L + m - 1) / m) >= L) {
+    set_error(err, NYS_ERR_INVALID_ARG);
+    return 0;
+  }
+  return L;
+}
+
 // ---------------------------------------------------------------------------
-// Segment means (Eq. 16, mean over l = n/m contiguous tokens).  One thread per
-// (head, landmark, feature); blockIdx.y selects Q (0) or K (1).  Sums in fp32
-// in token order, then divides by l.
+// Segment means (Eq. 16, mean over l = ceil(L/m) contiguous tokens, L the
+// element's length).  One thread per (head, landmark, feature); blockIdx.y
+// selects Q (0) or K (1).  Sums in fp32 in token order, then divides by the
+// segment's real tokens.
 template <typename T>
 __global__ void seg_means_scalar(const T *__restrict__ Q, const T *__restrict__ K,
                                  float *__restrict__ Qt, float *__restrict__ Kt, int BH, int n,
-                                 int d, int m) {
+                                 int d, int m, const int *lens, int heads, uint32_t *err) {
   const T *X = blockIdx.y == 0 ? Q : K;
   float *Xt = blockIdx.y == 0 ? Qt : Kt;
   long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -29,8 +45,10 @@ __global__ void seg_means_scalar(const T *__restrict__ Q, const T *__restrict__ 
   long jb = idx / d;            // bh * m + j
   int j = (int)(jb % m);
   long bh = jb / m;
-  const int len = (n + m - 1) / m;            // l = ceil(n / m)
-  const int seg = min(len, n - j * len);      // real tokens of segment j (>= 1)
+  const int L = seq_len_of(lens, (int)bh, heads, n, m, err);
+  if (L == 0) return;
+  const int len = (L + m - 1) / m;            // l = ceil(L / m)
+  const int seg = min(len, L - j * len);      // real tokens of segment j (>= 1)
   const T *src = X + ((size_t)bh * n + (size_t)j * len) * d + c;
   float acc = 0.f;
   for (int t = 0; t < seg; ++t) acc += to_f(src[(size_t)t * d]);
@@ -142,7 +160,8 @@ template <typename T, int kSimtMaxRowsPerWarp>   // m <= 8 * kSimtMaxRowsPerWarp
 __global__ void __launch_bounds__(256)
 bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *__restrict__ V,
                 float *__restrict__ pmax, float *__restrict__ psum, float *__restrict__ py,
-                int n, int d, int m, int splits, int keys_per_split, float scale_log2) {
+                int n, int d, int m, int splits, int keys_per_split, float scale_log2,
+                const int *lens, int heads) {
   extern __shared__ float smem[];
   const int split = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -160,8 +179,10 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
     y0[r] = 0.f;
     y1[r] = 0.f;
   }
+  // keys of the element: [0, L) (an invalid length reads as 0: no keys)
+  const int L = seq_len_of(lens, bh, heads, n, m, nullptr);
   const int k0 = split * keys_per_split;
-  const int k1 = min(n, k0 + keys_per_split);
+  const int k1 = min(L, k0 + keys_per_split);
   const T *Kh = K + (size_t)bh * n * d;
   const T *Vh = V + (size_t)bh * n * d;
   for (int t0 = k0; t0 < k1; t0 += kSimtKeyTile) {
@@ -259,7 +280,7 @@ template <typename T, int LPL>   // landmarks per lane: m <= 32 * LPL
 __global__ void __launch_bounds__(256)
 out_simt(const T *__restrict__ Q, const T *__restrict__ V, const float *__restrict__ Kt,
          const float *__restrict__ Wg, const float *__restrict__ convw, T *__restrict__ out,
-         int n, int d, int m, int heads, int convk, float scale_log2) {
+         int n, int d, int m, int heads, int convk, float scale_log2, const int *lens) {
   extern __shared__ float smem[];
   const int bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,9 +301,17 @@ out_simt(const T *__restrict__ Q, const T *__restrict__ V, const float *__restri
   const T *Vh = V + (size_t)bh * n * d;
   T *Oh = out + (size_t)bh * n * d;
   const int half = (convk - 1) / 2;
+  // rows of the element: [0, L); padding rows (and every row of an element
+  // with an invalid length) are zero, and the conv pads with zeros from L on
+  const int L = seq_len_of(lens, bh, heads, n, m, nullptr);
   for (int rr = warp; rr < kSimtOutRowsPerBlock; rr += 8) {
     const int i = blockIdx.x * kSimtOutRowsPerBlock + rr;
     if (i >= n) break;
+    if (i >= L) {
+      if (lane < d) Oh[(size_t)i * d + lane] = from_f<T>(0.f);
+      if (lane + 32 < d) Oh[(size_t)i * d + lane + 32] = from_f<T>(0.f);
+      continue;
+    }
     if (lane < d) qrow[warp * d + lane] = to_f(Qh[(size_t)i * d + lane]);
     if (lane + 32 < d) qrow[warp * d + lane + 32] = to_f(Qh[(size_t)i * d + lane + 32]);
     __syncwarp();
@@ -321,7 +350,7 @@ out_simt(const T *__restrict__ Q, const T *__restrict__ V, const float *__restri
       float c0 = 0.f, c1 = 0.f;
       for (int t = 0; t < convk; ++t) {
         int src = i + t - half;
-        if (src < 0 || src >= n) continue;
+        if (src < 0 || src >= L) continue;
         if (lane < d) c0 = fmaf(wc[t], to_f(Vh[(size_t)src * d + lane]), c0);
         if (lane + 32 < d) c1 = fmaf(wc[t], to_f(Vh[(size_t)src * d + lane + 32]), c1);
       }

@@ -166,7 +166,7 @@ def test_bf16_layout_holds_every_region(b, h, m, n):
     bh = b * h
     regions = [(lay["q_landmarks"], bh * m * 64 * 4), (lay["k_landmarks"], bh * m * 64 * 4),
                (lay["z"], bh * m * m * 4), (lay["y"], bh * m * 64 * 4),
-               (lay["w"], bh * m * 64 * 4), (lay["error_word"], 256 + bh * 12)]
+               (lay["w"], bh * m * 64 * 4), (lay["error_word"], 256)]
     for off, size in regions:
         assert off % 256 == 0 and off + size <= ws
     regions.sort()
