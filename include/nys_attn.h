@@ -154,6 +154,38 @@ NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q_dev, const void *K_d
                                               void *workspace_dev, size_t workspace_bytes,
                                               nys_stream_t stream);
 
+/* Backward pass ("Moore-Penrose Pseudoinverse Computation": gradients flow
+ * through the iteration's matrix products like through any other layer):
+ * given dO = dL/dout of the forward with the same arguments, writes
+ *   dQ_dev, dK_dev, dV_dev   dL/dQ, dL/dK, dL/dV, same dtype, layout and
+ *                            alignment as Q; must not overlap each other, the
+ *                            inputs, dO or the workspace,
+ *   dconv_w_dev              dL/dconv_w, [heads][conv_k] fp32 (summed over
+ *                            the batch), non-NULL exactly when conv_w_dev is.
+ * The forward's landmark steps are recomputed (A, every iterate of Lemma 1
+ * and B~'s normaliser are kept in the workspace); the chain rule then runs
+ * through the conv, F~ W, Z Y, B~ V, the three softmaxes (row-softmax
+ * backward), each Lemma 1 step's products in reverse, Z0's norms (the
+ * gradient goes to the maximising column and row) and the segment means.
+ * Arithmetic is fp32 on the CUDA cores; for NYS_BF16 the gradients are
+ * rounded to bf16 (dQ twice: its F~ part, then the landmark part added).
+ *   workspace_dev            at least nys_attn_backward_workspace_size
+ *                            bytes, 256-byte aligned, or NULL (allocated and
+ *                            freed stream-ordered).
+ * Shapes, validation, errors and determinism as for nys_attn_forward.
+ * Ragged batches (nys_attn_forward_lens) have no backward here. */
+NYS_ATTN_API nys_status nys_attn_backward_workspace_size(const nys_desc *desc, int num_landmarks,
+                                                         int pinv_iters, int conv_k,
+                                                         size_t *bytes);
+NYS_ATTN_API nys_status nys_attn_backward(const void *Q_dev, const void *K_dev,
+                                          const void *V_dev, const nys_desc *desc,
+                                          int num_landmarks, int pinv_iters,
+                                          const float *conv_w_dev, int conv_k,
+                                          const void *dO_dev, void *dQ_dev, void *dK_dev,
+                                          void *dV_dev, float *dconv_w_dev,
+                                          void *workspace_dev, size_t workspace_bytes,
+                                          nys_stream_t stream);
+
 /* Offsets (in bytes from the start of the workspace) of the fp32
  * intermediates a forward leaves there, for parity checks:
  *   q_landmarks, k_landmarks  [batch*heads][m][head_dim]   Q~, K~

@@ -18,7 +18,7 @@ __all__ = [
     "nys_attn_forward_host", "nys_attn_workspace_size", "nys_attn_intermediates",
     "nys_attn_host_buffer_size", "nys_attn_check_error", "nys_attn_launch_count",
     "nys_status_string", "nys_version", "Workspace", "nys_attn_launch_names",
-    "nys_attn_forward_timed", "nys_attn_forward_lens",
+    "nys_attn_forward_timed", "nys_attn_forward_lens", "nys_attn_backward",
 ]
 
 
@@ -130,6 +130,37 @@ def nys_attn_forward(Q, K, V, num_landmarks, pinv_iters=6, conv_w=None, out=None
                               _stream_ptr(stream))
     _lib.check(st, "nys_attn_forward")
     return out
+
+
+def nys_attn_backward(Q, K, V, num_landmarks, dO, pinv_iters=6, conv_w=None, workspace=None,
+                      stream=None):
+    """Gradients of the forward with respect to Q, K, V (and conv_w) given
+    dO = dL/dout: returns (dQ, dK, dV, dconv) with dconv None without the
+    conv skip.  workspace: a CUDA uint8 tensor of at least
+    nys_attn_backward_workspace_size bytes, or None (the library allocates
+    one stream-ordered per call)."""
+    torch = _torch()
+    _check_operands(Q, K, V, dO, conv_w)
+    desc = desc_of(Q)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(Q), torch.empty_like(Q)
+    conv_ptr, conv_k, dconv = None, 0, None
+    if conv_w is not None:
+        conv_ptr, conv_k = conv_w.data_ptr(), conv_w.shape[1]
+        dconv = torch.empty_like(conv_w)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        if not workspace.is_cuda or workspace.device != Q.device:
+            raise ValueError("workspace must be a CUDA tensor on Q's device")
+        ws_ptr = workspace.data_ptr() + (-workspace.data_ptr()) % 256
+        ws_bytes = workspace.numel() * workspace.element_size() - (ws_ptr - workspace.data_ptr())
+    with _on_device(Q.device):
+        st = _lib.raw_backward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), desc, num_landmarks,
+                               pinv_iters, conv_ptr, conv_k, dO.data_ptr(), dQ.data_ptr(),
+                               dK.data_ptr(), dV.data_ptr(),
+                               dconv.data_ptr() if dconv is not None else None, ws_ptr,
+                               ws_bytes, _stream_ptr(stream))
+    _lib.check(st, "nys_attn_backward")
+    return dQ, dK, dV, dconv
 
 
 def nys_attn_forward_lens(Q, K, V, num_landmarks, lens, pinv_iters=6, conv_w=None, out=None,

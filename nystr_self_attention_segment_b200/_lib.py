@@ -41,6 +41,8 @@ EXPORTS = (
     "nys_attn_forward_static",
     "nys_attn_check_error_static",
     "nys_attn_forward_lens",
+    "nys_attn_backward_workspace_size",
+    "nys_attn_backward",
 )
 
 # Size of the fixed scratch array of nys_attn_forward_static (see the header).
@@ -107,6 +109,10 @@ def load():
     lib.nys_attn_forward_static.argtypes = [P, P, P, D, I, I, P, I, P, P]
     lib.nys_attn_check_error_static.restype = I
     lib.nys_attn_check_error_static.argtypes = [D, I, P]
+    lib.nys_attn_backward_workspace_size.restype = I
+    lib.nys_attn_backward_workspace_size.argtypes = [D, I, I, I, ctypes.POINTER(S)]
+    lib.nys_attn_backward.restype = I
+    lib.nys_attn_backward.argtypes = [P, P, P, D, I, I, P, I, P, P, P, P, P, P, S, P]
     lib.nys_attn_forward_lens.restype = I
     lib.nys_attn_forward_lens.argtypes = [P, P, P, D, I, I, P, I, P, P, P, S, P]
     _LIB = lib
@@ -206,6 +212,24 @@ def raw_forward_lens(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_
                                         int(num_landmarks), int(pinv_iters), conv_ptr,
                                         int(conv_k), lens_ptr, out_ptr, ws_ptr,
                                         ctypes.c_size_t(ws_bytes), stream_ptr)
+
+
+def nys_attn_backward_workspace_size(desc, num_landmarks, pinv_iters, conv_k):
+    out = ctypes.c_size_t(0)
+    check(load().nys_attn_backward_workspace_size(ctypes.byref(desc), int(num_landmarks),
+                                                  int(pinv_iters), int(conv_k),
+                                                  ctypes.byref(out)),
+          "nys_attn_backward_workspace_size")
+    return out.value
+
+
+def raw_backward(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_ptr, conv_k, do_ptr,
+                 dq_ptr, dk_ptr, dv_ptr, dconv_ptr, ws_ptr, ws_bytes, stream_ptr):
+    """nys_attn_backward on raw addresses; returns the status code."""
+    return load().nys_attn_backward(q_ptr, k_ptr, v_ptr, ctypes.byref(desc), int(num_landmarks),
+                                    int(pinv_iters), conv_ptr, int(conv_k), do_ptr, dq_ptr,
+                                    dk_ptr, dv_ptr, dconv_ptr, ws_ptr, ctypes.c_size_t(ws_bytes),
+                                    stream_ptr)
 
 
 def raw_check_error_static(desc, num_landmarks, stream_ptr):

@@ -1,0 +1,604 @@
+// Backward pass of the Nystrom attention: gradients of the loss with respect
+// to Q, K, V and the DConv kernel, given dO ("Nystromformer: A Nystrom-Based
+// Algorithm for Approximating Self-Attention", section 3.4: "Moore-Penrose
+// Pseudoinverse Computation" -- the gradient flows through the iteration's
+// matrix products like through any other layer; Eq. 17 / Algorithm 1 and
+// Figure 4 for the forward it differentiates).
+//
+// The chain rule of every forward step, in reverse (s = 1/sqrt(d)):
+//   DConv:  dV += conv^T(dO),  dw[t] = sum_i dO_i . V_{i+t-half}
+//   O = F W:  dF = dO W^T,  dW = F^T dO
+//   W = Z Y:  dZ = dW Y^T,  dY = Z^T dW
+//   Y = B V:  dB = dY V^T,  dV += B^T dY
+//   softmax rows (F, B, A):  dS = P * (dP - rowsum(dP * P))
+//   B = softmax(s Q~ K^T):  dQ~ += s dS_B K,  dK += s dS_B^T Q~
+//   F = softmax(s Q K~^T):  dQ += s dS_F K~,  dK~ += s dS_F^T Q
+//   Z = Lemma 1 steps from Z0:  each step back through its four products
+//   Z0 = A^T / (||A||_1 ||A||_inf):  the norms' maximising column / row
+//   A = softmax(s Q~ K~^T):  dQ~ += s dS_A K~,  dK~ += s dS_A^T Q~
+//   Q~, K~ = segment means:  each token of segment j gets dX~_j / count_j
+// with rowsum(dB * B)_j = dY_j . Y_j (Y = B V), so B is never stored.
+//
+// Kernels (fp32 arithmetic on the CUDA cores; inputs and gradients in the
+// forward's dtype, the conv gradient fp32), after the forward's own segment
+// means, pseudoinverse (all iterates kept), B~ V partials and merge:
+//   bwd_rows   per 64-row tile: F, dF, dS_F; dQ (the F part); block partials
+//              of dW, dK~ and dw
+//   bwd_head   per head: dW, dY, dZ, the Lemma 1 steps backwards, dA, dQ~_A,
+//              dK~ (total), D = rowsum(dY * Y)
+//   bwd_keys   per 64-key tile: B, dB, dS_B; dK, dV (with the conv part);
+//              block partials of dQ~
+//   bwd_dq     dQ += dQ~_{seg(i)} / count
+//   bwd_dconv  dw summed over the batch and the row blocks, in order
+// Every sum runs in a fixed order: results are bitwise reproducible.
+#pragma once
+
+#include "common.cuh"
+
+namespace nys {
+namespace bwd {
+
+constexpr int kThreads = 256;
+constexpr int kTile = 64;   // rows / keys per tile
+
+// acc[r][c] += sum_k A(i, k) B(k, j) for the outputs this thread owns:
+// i = ty + 16 r, j = tx + 16 c (ty = t / 16, tx = t % 16), i < M, j < N.
+// A(i, k) = A[i * sai + k * sak], B(k, j) = B[k * sbk + j * sbj].
+template <int RM, int RN>
+__device__ __forceinline__ void mm_acc(float (&acc)[RM][RN], const float *A, int sai, int sak,
+                                       const float *B, int sbk, int sbj, int K, int M, int N) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  for (int k = 0; k < K; ++k) {
+    float a[RM], b[RN];
+#pragma unroll
+    for (int r = 0; r < RM; ++r) {
+      const int i = ty + 16 * r;
+      a[r] = i < M ? A[i * sai + k * sak] : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < RN; ++c) {
+      const int j = tx + 16 * c;
+      b[c] = j < N ? B[k * sbk + j * sbj] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+  }
+}
+
+template <int RM, int RN>
+__device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < RN; ++c) acc[r][c] = 0.f;
+}
+
+// C(i, j) = alpha * acc for the owned outputs (C row stride ldc).
+template <int RM, int RN>
+__device__ __forceinline__ void store(const float (&acc)[RM][RN], float *C, int ldc, int M, int N,
+                                      float alpha = 1.f) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < RN; ++c) {
+      const int i = ty + 16 * r, j = tx + 16 * c;
+      if (i < M && j < N) C[i * ldc + j] = alpha * acc[r][c];
+    }
+}
+
+// segment of token i, and its token count, for l = ceil(L / m)
+__device__ __forceinline__ int seg_of(int i, int l) { return i / l; }
+__device__ __forceinline__ int seg_count(int j, int l, int L) { return min(l, L - j * l); }
+
+// ---------------------------------------------------------------------------
+struct RowsParams {
+  const void *Q, *V, *G;        // [BH][n][d] (T)
+  const float *kt, *w;          // [BH][m][d] K~, W
+  const float *conv_w;          // [H][k] or null
+  void *dQ;                     // [BH][n][d] (T): the F part of dQ
+  float *dw_part, *dkt_part;    // [BH][R][m][d] partials of dW, dK~ (F part)
+  float *dconv_part;            // [BH][R][k]
+  int n, d, m, heads, conv_k, R;
+  float scale;
+};
+
+template <int M>
+struct RowsSmem {
+  // padded fp32 tiles
+  static constexpr int LD = 65, LM = M + 1;
+  static constexpr uint32_t kt = 0;                            // [M][LD]
+  static constexpr uint32_t w = kt + M * LD * 4;               // [M][LD]
+  static constexpr uint32_t q = w + M * LD * 4;                // [64][LD]
+  static constexpr uint32_t g = q + kTile * LD * 4;            // [64][LD]
+  static constexpr uint32_t f = g + kTile * LD * 4;            // [64][LM]
+  static constexpr uint32_t ds = f + kTile * LM * 4;           // [64][LM]
+  static constexpr uint32_t vh = ds + kTile * LM * 4;          // [64 + 62][LD] V halo
+  static constexpr uint32_t cw = vh + (kTile + 62) * LD * 4;   // [64]
+  static constexpr uint32_t dwc = cw + 64 * 4;                 // [64] conv partial
+  static constexpr uint32_t total = dwc + 64 * 4;
+};
+
+template <typename T, int M>
+__global__ void __launch_bounds__(kThreads) bwd_rows(const RowsParams p) {
+  using S = RowsSmem<M>;
+  constexpr int LD = S::LD, LM = S::LM;
+  constexpr int RM = M / 16;   // dW / dK~ rows per thread (m x 64 outputs)
+  extern __shared__ __align__(16) uint8_t smem[];
+  float *kt = (float *)(smem + S::kt), *w = (float *)(smem + S::w);
+  float *qs = (float *)(smem + S::q), *gs = (float *)(smem + S::g);
+  float *fs = (float *)(smem + S::f), *ds = (float *)(smem + S::ds);
+  float *vh = (float *)(smem + S::vh), *cw = (float *)(smem + S::cw);
+  float *dwc = (float *)(smem + S::dwc);
+  const int blk = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int n = p.n, d = p.d, m = p.m, head = bh % p.heads;
+  const int k = p.conv_w ? p.conv_k : 0, half = (k - 1) / 2;
+  const T *Q = (const T *)p.Q + (size_t)bh * n * d;
+  const T *V = (const T *)p.V + (size_t)bh * n * d;
+  const T *G = (const T *)p.G + (size_t)bh * n * d;
+  T *dQ = (T *)p.dQ + (size_t)bh * n * d;
+  for (int i = t; i < M * LD; i += kThreads) {
+    const int j = i / LD, c = i % LD;
+    const bool in = j < m && c < d;
+    kt[i] = in ? p.kt[((size_t)bh * m + j) * d + c] : 0.f;
+    w[i] = in ? p.w[((size_t)bh * m + j) * d + c] : 0.f;
+  }
+  if (t < 64) {
+    cw[t] = t < k ? p.conv_w[head * k + t] : 0.f;
+    dwc[t] = 0.f;
+  }
+  const int tiles = (n + kTile - 1) / kTile;
+  const int tb = (int)((long)blk * tiles / p.R), te = (int)((long)(blk + 1) * tiles / p.R);
+  float dW[RM][4], dK[RM][4];
+  zero(dW);
+  zero(dK);
+  for (int tile = tb; tile < te; ++tile) {
+    const int r0 = tile * kTile;
+    __syncthreads();
+    for (int i = t; i < kTile * LD; i += kThreads) {
+      const int r = i / LD, c = i % LD, row = r0 + r;
+      const bool in = row < n && c < d;
+      qs[i] = in ? to_f(Q[(size_t)row * d + c]) : 0.f;
+      gs[i] = in ? to_f(G[(size_t)row * d + c]) : 0.f;
+    }
+    if (k > 0)
+      for (int i = t; i < (kTile + k - 1) * LD; i += kThreads) {
+        const int r = i / LD, c = i % LD, row = r0 - half + r;
+        vh[i] = (row >= 0 && row < n && c < d) ? to_f(V[(size_t)row * d + c]) : 0.f;
+      }
+    __syncthreads();
+    {   // logits S = Q K~^T (64 x m) into fs, dF = dO W^T into ds
+      float a[4][RM], b[4][RM];
+      zero(a);
+      zero(b);
+      mm_acc(a, qs, LD, 1, kt, 1, LD, d, kTile, M);
+      mm_acc(b, gs, LD, 1, w, 1, LD, d, kTile, M);
+      store(a, fs, LM, kTile, m, p.scale);
+      store(b, ds, LM, kTile, m);
+    }
+    __syncthreads();
+    // row softmax of F and dS_F = F (dF - rowsum(dF F)): a warp per row
+    {
+      const int warp = t >> 5, lane = t & 31;
+      for (int r = warp; r < kTile; r += 8) {
+        const bool in = r0 + r < n;
+        float mx = -INFINITY;
+        for (int j = lane; j < m; j += 32) mx = fmaxf(mx, fs[r * LM + j]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int j = lane; j < m; j += 32) {
+          const float e = expf(fs[r * LM + j] - mx);
+          fs[r * LM + j] = e;
+          sum += e;
+        }
+        const float inv = 1.f / warp_sum(sum);
+        float dot = 0.f;
+        for (int j = lane; j < m; j += 32) {
+          const float f = fs[r * LM + j] * inv;
+          fs[r * LM + j] = in ? f : 0.f;
+          dot = fmaf(f, ds[r * LM + j], dot);
+        }
+        dot = warp_sum(dot);
+        for (int j = lane; j < m; j += 32) {
+          const float f = fs[r * LM + j];
+          ds[r * LM + j] = in ? f * (ds[r * LM + j] - dot) : 0.f;
+        }
+      }
+    }
+    __syncthreads();
+    {   // dQ (F part) = s dS_F K~ (64 x d)
+      float a[4][4];
+      zero(a);
+      mm_acc(a, ds, LM, 1, kt, LD, 1, m, kTile, d);
+      const int ty = t >> 4, tx = t & 15;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int row = r0 + ty + 16 * r, col = tx + 16 * c;
+          if (row < n && col < d) dQ[(size_t)row * d + col] = from_f<T>(p.scale * a[r][c]);
+        }
+    }
+    // dW += F^T dO, dK~ += dS_F^T Q (m x d, over the tile's rows)
+    mm_acc(dW, fs, 1, LM, gs, LD, 1, kTile, m, d);
+    mm_acc(dK, ds, 1, LM, qs, LD, 1, kTile, m, d);
+    // conv kernel gradient: tap j gets sum_i sum_c dO_i,c V_{i+j-half},c
+    if (k > 0) {
+      const int warp = t >> 5, lane = t & 31;
+      for (int j = warp; j < k; j += 8) {
+        float acc = 0.f;
+        for (int e = lane; e < kTile * d; e += 32) {
+          const int r = e / d, c = e % d;
+          acc = fmaf(gs[r * LD + c], vh[(r + j) * LD + c], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) dwc[j] += acc;
+      }
+    }
+  }
+  // block partials
+  const size_t pb = ((size_t)bh * p.R + blk) * m * d;
+  store(dW, p.dw_part + pb, d, m, d);
+  store(dK, p.dkt_part + pb, d, m, d, p.scale);
+  __syncthreads();
+  if (t < k) p.dconv_part[((size_t)bh * p.R + blk) * k + t] = dwc[t];
+}
+
+// ---------------------------------------------------------------------------
+struct HeadParams {
+  const float *dw_part, *dkt_part;   // [BH][R][m][d]
+  const float *qt, *kt, *y;          // [BH][m][d]
+  const float *a, *zs;               // [BH][m][m], [BH][iters + 1][m][m]
+  float *dy, *dqt_a, *dkt;           // [BH][m][d]
+  float *dd;                         // [BH][m]: rowsum(dY * Y)
+  float *scratch;                    // [BH][head_bytes] when the matrices do not fit smem
+  int d, m, iters, R, use_smem;
+  float scale;
+};
+
+// C = alpha op(A) op(B) (+ beta C) over m x m (or m x d) matrices with row
+// stride ld, all in one block; the product runs with every thread.
+template <int RM, int RN>
+__device__ __forceinline__ void mm_block(float *C, int ldc, const float *A, int sai, int sak,
+                                         const float *B, int sbk, int sbj, int K, int M, int N,
+                                         float alpha, float beta) {
+  float acc[RM][RN];
+  zero(acc);
+  mm_acc(acc, A, sai, sak, B, sbk, sbj, K, M, N);
+  __syncthreads();   // C may alias an operand's previous contents
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < RN; ++c) {
+      const int i = ty + 16 * r, j = tx + 16 * c;
+      if (i < M && j < N) {
+        float *o = C + i * ldc + j;
+        *o = alpha * acc[r][c] + (beta != 0.f ? beta * *o : 0.f);
+      }
+    }
+  __syncthreads();
+}
+
+// Bytes of the twelve matrices of bwd_head<M>.
+template <int M>
+__host__ __device__ constexpr size_t head_bytes() {
+  return (size_t)12 * M * (M > 64 ? M : 64) * 4;
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
+  constexpr int RM = M / 16;
+  extern __shared__ __align__(16) float smem_f[];
+  const int bh = blockIdx.x, t = threadIdx.x;
+  // twelve M x LDH matrices (m <= M rows; row stride LDH holds m columns and
+  // the d <= 64 columns of the m x d ones)
+  constexpr int ld = M > 64 ? M : 64, kMat = M * ld;
+  const int m = p.m, d = p.d;
+  float *base = p.use_smem ? smem_f : p.scratch + (size_t)bh * (head_bytes<M>() / 4);
+  float *A = base, *Zj = A + kMat, *P = Zj + kMat, *T1 = P + kMat, *T2 = T1 + kMat,
+        *T3 = T2 + kMat, *dZ = T3 + kMat, *dP = dZ + kMat, *dT = dP + kMat,
+        *dA = dT + kMat, *X = dA + kMat, *Y2 = X + kMat;
+  // X: dW (m x d) then scratch; Y2: Y (m x d)
+  const size_t hd = (size_t)bh * m * d;
+  for (int e = t; e < m * d; e += kThreads) {
+    const int i = e / d, c = e % d;
+    float sw = 0.f;
+    for (int r = 0; r < p.R; ++r) sw += p.dw_part[((size_t)bh * p.R + r) * m * d + e];
+    X[i * ld + c] = sw;
+    Y2[i * ld + c] = p.y[hd + e];
+  }
+  for (int e = t; e < m * m; e += kThreads) {
+    const int i = e / m, j = e % m;
+    A[i * ld + j] = p.a[(size_t)bh * m * m + e];
+    Zj[i * ld + j] = p.zs[((size_t)bh * (p.iters + 1) + p.iters) * m * m + e];
+    dA[i * ld + j] = 0.f;
+  }
+  __syncthreads();
+  // dZ = dW Y^T (m x m), dY = Z^T dW (m x d)
+  mm_block<RM, RM>(dZ, ld, X, ld, 1, Y2, 1, ld, d, m, m, 1.f, 0.f);
+  mm_block<RM, 4>(T1, ld, Zj, 1, ld, X, ld, 1, m, m, d, 1.f, 0.f);
+  for (int e = t; e < m * d; e += kThreads) {
+    const int i = e / d, c = e % d;
+    p.dy[hd + e] = T1[i * ld + c];
+  }
+  if (t < m) {   // D_j = dY_j . Y_j
+    float s = 0.f;
+    for (int c = 0; c < d; ++c) s = fmaf(T1[t * ld + c], Y2[t * ld + c], s);
+    p.dd[(size_t)bh * m + t] = s;
+  }
+  __syncthreads();
+  // Lemma 1 steps backwards: Z' = 1/4 Z T3, T3 = 13I - P T2, T2 = 15I - P T1,
+  // T1 = 7I - P, P = A Z
+  for (int j = p.iters - 1; j >= 0; --j) {
+    for (int e = t; e < m * m; e += kThreads)
+      Zj[(e / m) * ld + e % m] = p.zs[((size_t)bh * (p.iters + 1) + j) * m * m + e];
+    __syncthreads();
+    mm_block<RM, RM>(P, ld, A, ld, 1, Zj, ld, 1, m, m, m, 1.f, 0.f);            // P = A Z
+    for (int e = t; e < m * m; e += kThreads) {
+      const int i = e / m, c = e % m;
+      T1[i * ld + c] = (i == c ? 7.f : 0.f) - P[i * ld + c];
+    }
+    __syncthreads();
+    mm_block<RM, RM>(T2, ld, P, ld, 1, T1, ld, 1, m, m, m, -1.f, 0.f);          // -P T1
+    for (int e = t; e < m * m; e += kThreads) {
+      const int i = e / m, c = e % m;
+      T2[i * ld + c] += (i == c ? 15.f : 0.f);
+    }
+    __syncthreads();
+    mm_block<RM, RM>(T3, ld, P, ld, 1, T2, ld, 1, m, m, m, -1.f, 0.f);          // -P T2
+    for (int e = t; e < m * m; e += kThreads) {
+      const int i = e / m, c = e % m;
+      T3[i * ld + c] += (i == c ? 13.f : 0.f);
+    }
+    __syncthreads();
+    mm_block<RM, RM>(dT, ld, Zj, 1, ld, dZ, ld, 1, m, m, m, 0.25f, 0.f);       // dT3 = 1/4 Z^T dZ
+    mm_block<RM, RM>(X, ld, dZ, ld, 1, T3, 1, ld, m, m, m, 0.25f, 0.f);        // dZ_prev = 1/4 dZ T3^T
+    mm_block<RM, RM>(dP, ld, dT, ld, 1, T2, 1, ld, m, m, m, -1.f, 0.f);        // dP = -dT3 T2^T
+    mm_block<RM, RM>(T3, ld, P, 1, ld, dT, ld, 1, m, m, m, -1.f, 0.f);         // dT2 = -P^T dT3
+    mm_block<RM, RM>(dP, ld, T3, ld, 1, T1, 1, ld, m, m, m, -1.f, 1.f);        // dP -= dT2 T1^T
+    mm_block<RM, RM>(dT, ld, P, 1, ld, T3, ld, 1, m, m, m, -1.f, 0.f);         // dT1 = -P^T dT2
+    for (int e = t; e < m * m; e += kThreads) {
+      const int i = e / m, c = e % m;
+      dP[i * ld + c] -= dT[i * ld + c];                                          // dP -= dT1
+    }
+    __syncthreads();
+    mm_block<RM, RM>(dA, ld, dP, ld, 1, Zj, 1, ld, m, m, m, 1.f, 1.f);         // dA += dP Z^T
+    mm_block<RM, RM>(X, ld, A, 1, ld, dP, ld, 1, m, m, m, 1.f, 1.f);           // dZ_prev += A^T dP
+    for (int e = t; e < m * m; e += kThreads) dZ[(e / m) * ld + e % m] = X[(e / m) * ld + e % m];
+    __syncthreads();
+  }
+  // Z0 = A^T c, c = 1 / (||A||_1 ||A||_inf): gradients through c and the
+  // maximising column / row (first index at ties)
+  __shared__ float red[4];
+  __shared__ int arg[2];
+  if (t == 0) {
+    float n1 = -1.f, ninf = -1.f, dc = 0.f;
+    int jc = 0, ir = 0;
+    for (int j = 0; j < m; ++j) {
+      float cs = 0.f;
+      for (int i = 0; i < m; ++i) cs += fabsf(A[i * ld + j]);
+      if (cs > n1) { n1 = cs; jc = j; }
+    }
+    for (int i = 0; i < m; ++i) {
+      float rs = 0.f;
+      for (int j = 0; j < m; ++j) rs += fabsf(A[i * ld + j]);
+      if (rs > ninf) { ninf = rs; ir = i; }
+    }
+    for (int i = 0; i < m; ++i)
+      for (int j = 0; j < m; ++j) dc = fmaf(dZ[i * ld + j], A[j * ld + i], dc);
+    red[0] = 1.f / (n1 * ninf);
+    red[1] = dc;
+    red[2] = n1;
+    red[3] = ninf;
+    arg[0] = jc;
+    arg[1] = ir;
+  }
+  __syncthreads();
+  {
+    const float c = red[0], dc = red[1], n1 = red[2], ninf = red[3];
+    for (int e = t; e < m * m; e += kThreads) {
+      const int i = e / m, j = e % m;
+      float g = dA[i * ld + j] + c * dZ[j * ld + i];
+      if (j == arg[0]) g += -dc * c / n1 * (A[i * ld + j] > 0.f ? 1.f : (A[i * ld + j] < 0.f ? -1.f : 0.f));
+      if (i == arg[1]) g += -dc * c / ninf * (A[i * ld + j] > 0.f ? 1.f : (A[i * ld + j] < 0.f ? -1.f : 0.f));
+      dA[i * ld + j] = g;
+    }
+  }
+  __syncthreads();
+  // softmax backward of A: dS_A = A (dA - rowsum(dA A)), into dP
+  if (t < m) {
+    float dot = 0.f;
+    for (int j = 0; j < m; ++j) dot = fmaf(dA[t * ld + j], A[t * ld + j], dot);
+    for (int j = 0; j < m; ++j) dP[t * ld + j] = A[t * ld + j] * (dA[t * ld + j] - dot);
+  }
+  // Q~, K~ into T1, T2 (m x d)
+  for (int e = t; e < m * d; e += kThreads) {
+    const int i = e / d, c = e % d;
+    T1[i * ld + c] = p.qt[hd + e];
+    T2[i * ld + c] = p.kt[hd + e];
+  }
+  __syncthreads();
+  // dQ~_A = s dS_A K~ ; dK~ = (F part) + s dS_A^T Q~
+  mm_block<RM, 4>(T3, ld, dP, ld, 1, T2, ld, 1, m, m, d, p.scale, 0.f);
+  for (int e = t; e < m * d; e += kThreads) p.dqt_a[hd + e] = T3[(e / d) * ld + e % d];
+  mm_block<RM, 4>(X, ld, dP, 1, ld, T1, ld, 1, m, m, d, p.scale, 0.f);
+  for (int e = t; e < m * d; e += kThreads) {
+    const int i = e / d, c = e % d;
+    float s = 0.f;
+    for (int r = 0; r < p.R; ++r) s += p.dkt_part[((size_t)bh * p.R + r) * m * d + e];
+    p.dkt[hd + e] = s + X[i * ld + c];
+  }
+}
+
+// ---------------------------------------------------------------------------
+struct KeysParams {
+  const void *K, *V, *G;        // [BH][n][d] (T)
+  const float *qt, *dy, *dkt;   // [BH][m][d]
+  const float *lse2, *dd;       // [BH][m]: log2-sum-exp of B~'s scaled logits, rowsum(dY Y)
+  const float *conv_w;          // [H][k] or null
+  void *dK, *dV;                // [BH][n][d] (T)
+  float *dqt_part;              // [BH][S2][m][d]
+  int n, d, m, heads, conv_k, S2;
+  float scale, scale_log2;
+};
+
+template <int M>
+struct KeysSmem {
+  static constexpr int LD = 65, LK = kTile + 1;
+  static constexpr uint32_t qt = 0;                              // [M][LD]
+  static constexpr uint32_t dy = qt + M * LD * 4;                // [M][LD]
+  static constexpr uint32_t ks = dy + M * LD * 4;                // [64][LD]
+  static constexpr uint32_t vs = ks + kTile * LD * 4;            // [64][LD]
+  static constexpr uint32_t b = vs + kTile * LD * 4;             // [M][LK]
+  static constexpr uint32_t db = b + M * LK * 4;                 // [M][LK]
+  static constexpr uint32_t gh = db + M * LK * 4;                // [64 + 62][LD] dO halo
+  static constexpr uint32_t cw = gh + (kTile + 62) * LD * 4;     // [64]
+  static constexpr uint32_t lse = cw + 64 * 4;                   // [M]
+  static constexpr uint32_t dd = lse + M * 4;                    // [M]
+  static constexpr uint32_t total = dd + M * 4;
+};
+
+template <typename T, int M>
+__global__ void __launch_bounds__(kThreads) bwd_keys(const KeysParams p) {
+  using S = KeysSmem<M>;
+  constexpr int LD = S::LD, LK = S::LK, RM = M / 16;
+  extern __shared__ __align__(16) uint8_t smem[];
+  float *qt = (float *)(smem + S::qt), *dy = (float *)(smem + S::dy);
+  float *ks = (float *)(smem + S::ks), *vs = (float *)(smem + S::vs);
+  float *bs = (float *)(smem + S::b), *dbs = (float *)(smem + S::db);
+  float *gh = (float *)(smem + S::gh);
+  float *cw = (float *)(smem + S::cw), *lse = (float *)(smem + S::lse);
+  float *ddv = (float *)(smem + S::dd);
+  const int blk = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int n = p.n, d = p.d, m = p.m, head = bh % p.heads;
+  const int k = p.conv_w ? p.conv_k : 0, half = (k - 1) / 2;
+  const int l = (n + m - 1) / m;
+  const T *K = (const T *)p.K + (size_t)bh * n * d;
+  const T *V = (const T *)p.V + (size_t)bh * n * d;
+  const T *G = (const T *)p.G + (size_t)bh * n * d;
+  T *dK = (T *)p.dK + (size_t)bh * n * d;
+  T *dV = (T *)p.dV + (size_t)bh * n * d;
+  const size_t hd = (size_t)bh * m * d;
+  for (int i = t; i < M * LD; i += kThreads) {
+    const int j = i / LD, c = i % LD;
+    const bool in = j < m && c < d;
+    qt[i] = in ? p.qt[hd + j * d + c] : 0.f;
+    dy[i] = in ? p.dy[hd + j * d + c] : 0.f;
+  }
+  if (t < 64) cw[t] = t < k ? p.conv_w[head * k + t] : 0.f;
+  for (int j = t; j < M; j += kThreads) {
+    lse[j] = j < m ? p.lse2[(size_t)bh * m + j] : 0.f;
+    ddv[j] = j < m ? p.dd[(size_t)bh * m + j] : 0.f;
+  }
+  const int tiles = (n + kTile - 1) / kTile;
+  const int tb = (int)((long)blk * tiles / p.S2), te = (int)((long)(blk + 1) * tiles / p.S2);
+  float dq[RM][4];
+  zero(dq);
+  for (int tile = tb; tile < te; ++tile) {
+    const int k0 = tile * kTile;
+    __syncthreads();
+    for (int i = t; i < kTile * LD; i += kThreads) {
+      const int r = i / LD, c = i % LD, row = k0 + r;
+      const bool in = row < n && c < d;
+      ks[i] = in ? to_f(K[(size_t)row * d + c]) : 0.f;
+      vs[i] = in ? to_f(V[(size_t)row * d + c]) : 0.f;
+    }
+    if (k > 0)   // dO rows k0 + half - (k - 1) .. k0 + 63 + half: conv^T
+      for (int i = t; i < (kTile + k - 1) * LD; i += kThreads) {
+        const int r = i / LD, c = i % LD, row = k0 + half - (k - 1) + r;
+        gh[i] = (row >= 0 && row < n && c < d) ? to_f(G[(size_t)row * d + c]) : 0.f;
+      }
+    __syncthreads();
+    {   // B = 2^(s log2e Q~ K^T - lse) (m x 64), dB = dY V^T
+      float a[RM][4], b[RM][4];
+      zero(a);
+      zero(b);
+      mm_acc(a, qt, LD, 1, ks, 1, LD, d, m, kTile);
+      mm_acc(b, dy, LD, 1, vs, 1, LD, d, m, kTile);
+      const int ty = t >> 4, tx = t & 15;
+#pragma unroll
+      for (int r = 0; r < RM; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int j = ty + 16 * r, key = tx + 16 * c;
+          if (j < m) {
+            const float bv = (k0 + key < n) ? exp2f(a[r][c] * p.scale_log2 - lse[j]) : 0.f;
+            bs[j * LK + key] = bv;
+            dbs[j * LK + key] = bv * (b[r][c] - ddv[j]);   // dS_B
+          }
+        }
+    }
+    __syncthreads();
+    {   // dK = s dS_B^T Q~ + dK~_seg / count ; dV = B^T dY + conv^T(dO)
+      float a[4][4], b[4][4];
+      zero(a);
+      zero(b);
+      mm_acc(a, dbs, 1, LK, qt, LD, 1, m, kTile, d);
+      mm_acc(b, bs, 1, LK, dy, LD, 1, m, kTile, d);
+      const int ty = t >> 4, tx = t & 15;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int key = ty + 16 * r, col = tx + 16 * c, row = k0 + key;
+          if (row < n && col < d) {
+            const int j = seg_of(row, l);
+            const float gk =
+                p.scale * a[r][c] + __ldg(p.dkt + hd + j * d + col) / (float)seg_count(j, l, n);
+            float gv = b[r][c];
+            for (int tp = 0; tp < k; ++tp)   // dV_row += w[tp] dO[row - tp + half]
+              gv = fmaf(cw[tp], gh[(key + (k - 1) - tp) * LD + col], gv);
+            dK[(size_t)row * d + col] = from_f<T>(gk);
+            dV[(size_t)row * d + col] = from_f<T>(gv);
+          }
+        }
+    }
+    // dQ~ += s dS_B K (m x d, over the tile's keys)
+    mm_acc(dq, dbs, LK, 1, ks, LD, 1, kTile, m, d);
+  }
+  store(dq, p.dqt_part + ((size_t)bh * p.S2 + blk) * m * d, d, m, d, p.scale);
+}
+
+// ---------------------------------------------------------------------------
+// dQ += dQ~_{seg(i)} / count: dQ~ = dQ~_A + the key blocks' partials in
+// order, recomputed by every block of the head.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+bwd_dq(void *dQv, const float *dqt_a, const float *dqt_part, int n, int d, int m, int S2,
+       int rows_per_block) {
+  extern __shared__ float dq[];   // [m][d]
+  const int bh = blockIdx.y, t = threadIdx.x;
+  const size_t hd = (size_t)bh * m * d;
+  for (int e = t; e < m * d; e += kThreads) {
+    float s = dqt_a[hd + e];
+    for (int r = 0; r < S2; ++r) s += dqt_part[((size_t)bh * S2 + r) * m * d + e];
+    dq[e] = s;
+  }
+  __syncthreads();
+  T *dQ = (T *)dQv + (size_t)bh * n * d;
+  const int l = (n + m - 1) / m;
+  const int r0 = blockIdx.x * rows_per_block, r1 = min(n, r0 + rows_per_block);
+  for (int e = t; e < (r1 - r0) * d; e += kThreads) {
+    const int row = r0 + e / d, c = e % d;
+    const int j = seg_of(row, l);
+    const size_t o = (size_t)row * d + c;
+    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[j * d + c] / (float)seg_count(j, l, n));
+  }
+}
+
+// dconv[h][t] = sum over batch elements b (in order) of the row blocks'
+// partials (in order).
+__global__ void bwd_dconv(float *dconv, const float *part, int batch, int heads, int R, int k) {
+  const int h = blockIdx.x, t = threadIdx.x;
+  if (t >= k) return;
+  float s = 0.f;
+  for (int b = 0; b < batch; ++b)
+    for (int r = 0; r < R; ++r) s += part[(((size_t)b * heads + h) * R + r) * k + t];
+  dconv[h * k + t] = s;
+}
+
+}  // namespace bwd
+}  // namespace nys

@@ -97,6 +97,11 @@ struct Params {
 // warpgroups take turns through their exponential-heavy section (named
 // barriers 2 and 3), so one computes while the other waits on its MMAs.
 constexpr float kTau = 8.f;
+// Turn-taking of the two softmax warpgroups through their exponential
+// sections (1), or both at once (0).
+#ifndef NYS_BV_TURNS
+#define NYS_BV_TURNS 1
+#endif
 
 // tmem_in: a 512-column TMEM allocation owned by the caller, or ~0u to
 // allocate (and free) one here.
@@ -158,11 +163,14 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   }
   __syncthreads();   // barriers initialised
   const int pre = nch < kStages ? nch : kStages;   // chunk loads issued up front
+  // K is read here for the last time in the pass (V again by the output
+  // kernel): its lines leave L2 first
+  const uint64_t last_use = policy_evict_first();
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < pre; ++i) {
       const int k0 = (c_begin + i) * kChunk;
       mbar_expect_tx(&full[i], 32768u);
-      tma_load_3d(smem + L.k[i], map_k, &full[i], 0, k0, bh);
+      tma_load_3d_hint(smem + L.k[i], map_k, &full[i], 0, k0, bh, last_use);
       tma_load_3d(smem + L.v[i], map_v, &full[i], 0, k0, bh);
     }
   }
@@ -200,7 +208,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
         const int k0 = (c_begin + i) * kChunk;
         mbar_expect_tx(&full[s], 32768u);
-        tma_load_3d(smem + L.k[s], map_k, &full[s], 0, k0, bh);
+        tma_load_3d_hint(smem + L.k[s], map_k, &full[s], 0, k0, bh, last_use);
         tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
       }
       // consume the stage releases nobody else waits for, so that no
@@ -263,7 +271,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       tmem_st32(t_s + 160, z);
       tmem_st_wait();
     }
-    if (wg == 1 && nch > 0) named_barrier_arrive(2, 256);   // warpgroup 0 goes first
+    if (NYS_BV_TURNS && wg == 1 && nch > 0) named_barrier_arrive(2, 256);   // warpgroup 0 first
     bool ok = true;
     int u = 0;
     for (int i = wg; i < nch; i += 2, ++u) {
@@ -278,7 +286,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       mbar_arrive(&s_free[wg]);
       const int key0 = (c_begin + i) * kChunk + g * M;
       const int valid = min(M, seq - key0);       // keys of this group inside [0, L)
-      named_barrier(2 + wg, 256);                  // this warpgroup's turn
+      if (NYS_BV_TURNS) named_barrier(2 + wg, 256);   // this warpgroup's turn
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
@@ -343,7 +351,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         }
       }
       run_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      if (i + 1 < nch) named_barrier_arrive(2 + (wg ^ 1), 256);   // the other's turn
+      if (NYS_BV_TURNS && i + 1 < nch) named_barrier_arrive(2 + (wg ^ 1), 256);   // the other's turn
       // P is read by the previous P V of this warpgroup: wait for it
       if (u > 0 && !y_done) {
         if (!(ok = mbar_wait(&y_full[wg], (u - 1) & 1, ab))) break;
@@ -356,7 +364,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
       mbar_arrive(&p_ready[wg]);
       if (threadIdx.x == 128 && blockIdx.x == (unsigned)prm.BH && u < 32) NYS_MARK_T(kTrMid, 96 + u);
     }
-    if (!ok) {
+    if (NYS_BV_TURNS && !ok) {
       // let the other warpgroup leave a turn it may be waiting for
       named_barrier_arrive(2 + (wg ^ 1), 256);
     }

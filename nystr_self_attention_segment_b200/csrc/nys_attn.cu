@@ -15,6 +15,7 @@
 #include "mid_tc.cuh"
 #include "out_tc.cuh"
 #include "wmerge.cuh"
+#include "bwd_simt.cuh"
 #include "stream_bf16.cuh"
 
 using namespace nys;
@@ -237,7 +238,8 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
     if (!allow_smem(pinv_simt, sm) ||
         launch(pinv_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
-               kt, z, scratch, m, d, scale, iters, use_smem) != cudaSuccess)
+               kt, z, scratch, m, d, scale, iters, use_smem, (float *)nullptr,
+               (float *)nullptr) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -256,7 +258,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     size_t sm = (size_t)m * d * 4;
     if (!allow_smem(merge_w_simt, sm) ||
         launch(merge_w_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false,
-               pmax, psum, py, z, y, w, m, d, L.splits) != cudaSuccess)
+               pmax, psum, py, z, y, w, m, d, L.splits, (float *)nullptr) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -409,6 +411,166 @@ nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_
   return NYS_ERR_UNSUPPORTED;
 }
 
+// ---------------------------------------------------------------------------
+// Backward pass: workspace layout and launch sequence (bwd_simt.cuh).
+struct BwdLayout {
+  size_t qt, kt, z, a, zall, pscr, pmax, psum, py, y, w, lse, dwp, dktp, dcp, dy, dqta, dkt,
+      dd, hscr, dqtp, err, total;
+  int S, keys_per_split, R, S2, mb;
+};
+
+int bwd_mbucket(int m) { return m <= 32 ? 32 : (m <= 64 ? 64 : 128); }
+
+BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
+  BwdLayout L;
+  memset(&L, 0, sizeof(L));
+  const size_t BH = (size_t)desc->batch * desc->heads;
+  const size_t n = desc->seq_len, d = desc->head_dim;
+  const int tile = kSimtKeyTile;
+  const int ntiles = (int)((n + tile - 1) / tile);
+  int splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
+  if (splits > ntiles) splits = ntiles;
+  if (splits < 1) splits = 1;
+  const int tps = (ntiles + splits - 1) / splits;
+  L.S = (ntiles + tps - 1) / tps;
+  L.keys_per_split = tps * tile;
+  const int t64 = (int)((n + bwd::kTile - 1) / bwd::kTile);
+  int r = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
+  if (r > t64) r = t64;
+  if (r < 1) r = 1;
+  L.R = L.S2 = r;
+  L.mb = bwd_mbucket(m);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t md = BH * m * d * 4, mm = BH * m * m * 4;
+  L.qt = take(md);
+  L.kt = take(md);
+  L.z = take(mm);
+  L.a = take(mm);
+  L.zall = take(mm * (iters + 1));
+  L.pscr = take(m > 64 ? 5 * mm : 0);
+  L.pmax = take(BH * L.S * m * 4);
+  L.psum = take(BH * L.S * m * 4);
+  L.py = take(BH * L.S * m * d * 4);
+  L.y = take(md);
+  L.w = take(md);
+  L.lse = take(BH * m * 4);
+  L.dwp = take(md * L.R);
+  L.dktp = take(md * L.R);
+  L.dcp = take(BH * L.R * (conv_k > 0 ? conv_k : 0) * 4);
+  L.dy = take(md);
+  L.dqta = take(md);
+  L.dkt = take(md);
+  L.dd = take(BH * m * 4);
+  L.hscr = take(L.mb > 64 ? BH * bwd::head_bytes<128>() : 0);
+  L.dqtp = take(md * L.S2);
+  L.err = take(256);
+  L.total = off;
+  return L;
+}
+
+template <typename T, int MB>
+nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, int m, int iters,
+                      const float *conv_w, int conv_k, const T *dO, T *dQ, T *dK, T *dV,
+                      float *dconv, char *ws, const BwdLayout &L, cudaStream_t stream) {
+  const int BH = desc->batch * desc->heads, H = desc->heads;
+  const int n = desc->seq_len, d = desc->head_dim;
+  const float scale = 1.0f / sqrtf((float)d), scale_log2 = scale * kLog2e;
+  float *qt = (float *)(ws + L.qt), *kt = (float *)(ws + L.kt), *z = (float *)(ws + L.z);
+  float *a = (float *)(ws + L.a), *zall = (float *)(ws + L.zall);
+  float *pmax = (float *)(ws + L.pmax), *psum = (float *)(ws + L.psum);
+  float *py = (float *)(ws + L.py), *y = (float *)(ws + L.y), *w = (float *)(ws + L.w);
+  float *lse = (float *)(ws + L.lse);
+  uint32_t *err = (uint32_t *)(ws + L.err);
+  const int ck = conv_w ? conv_k : 0;
+  // the forward's landmark steps, keeping A, every Z iterate and B~'s
+  // log-sum-exp
+  {
+    long total = (long)BH * m * d;
+    if (launch(seg_means_scalar<T>, dim3((unsigned)((total + 255) / 256), 2), dim3(256), 0,
+               stream, false, Q, K, qt, kt, BH, n, d, m, (const int *)nullptr, H,
+               err) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const int use_smem = m <= 64;
+    const size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
+    if (!allow_smem(pinv_simt, sm) ||
+        launch(pinv_simt, dim3(BH), dim3(256), sm, stream, false, (const float *)qt,
+               (const float *)kt, z, (float *)(ws + L.pscr), m, d, scale, iters, use_smem, a,
+               zall) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const size_t sm = ((size_t)m * d + kSimtKeyTile * (d + 1) + kSimtKeyTile * d) * 4;
+    auto kern = m <= 64 ? bv_partial_simt<T, 8> : bv_partial_simt<T, 16>;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(L.S, BH), dim3(256), sm, stream, false, (const float *)qt, K, V, pmax,
+               psum, py, n, d, m, L.S, L.keys_per_split, scale_log2, (const int *)nullptr,
+               H) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const size_t sm = (size_t)m * d * 4;
+    if (!allow_smem(merge_w_simt, sm) ||
+        launch(merge_w_simt, dim3(BH), dim3(256), sm, stream, false, (const float *)pmax,
+               (const float *)psum, (const float *)py, (const float *)z, y, w, m, d, L.S,
+               lse) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  // the backward proper
+  {
+    const bwd::RowsParams p{Q,  V,  dO, kt,  w,    conv_w, dQ,     (float *)(ws + L.dwp),
+                            (float *)(ws + L.dktp), (float *)(ws + L.dcp), n, d, m, H, ck,
+                            L.R, scale};
+    auto kern = bwd::bwd_rows<T, MB>;
+    const size_t sm = bwd::RowsSmem<MB>::total;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(L.R, BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const bwd::HeadParams p{(const float *)(ws + L.dwp), (const float *)(ws + L.dktp), qt, kt, y,
+                            a, zall, (float *)(ws + L.dy), (float *)(ws + L.dqta),
+                            (float *)(ws + L.dkt), (float *)(ws + L.dd),
+                            (float *)(ws + L.hscr), d, m, iters, L.R, MB <= 64 ? 1 : 0, scale};
+    auto kern = bwd::bwd_head<MB>;
+    const size_t sm = MB <= 64 ? bwd::head_bytes<MB>() : 0;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const bwd::KeysParams p{K, V, dO, qt, (const float *)(ws + L.dy), (const float *)(ws + L.dkt),
+                            lse, (const float *)(ws + L.dd), conv_w, dK, dV,
+                            (float *)(ws + L.dqtp), n, d, m, H, ck, L.S2, scale, scale_log2};
+    auto kern = bwd::bwd_keys<T, MB>;
+    const size_t sm = bwd::KeysSmem<MB>::total;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(L.S2, BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  {
+    const int rpb = 256;
+    const size_t sm = (size_t)m * d * 4;
+    auto kern = bwd::bwd_dq<T>;
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3((n + rpb - 1) / rpb, BH), dim3(bwd::kThreads), sm, stream, false,
+               (void *)dQ, (const float *)(ws + L.dqta), (const float *)(ws + L.dqtp), n, d, m,
+               L.S2, rpb) != cudaSuccess)
+      return NYS_ERR_CUDA;
+  }
+  if (ck > 0 &&
+      launch(bwd::bwd_dconv, dim3(H), dim3(64), 0, stream, false, dconv,
+             (const float *)(ws + L.dcp), desc->batch, H, L.R, ck) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  return NYS_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -544,6 +706,91 @@ NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q, const void *K, cons
   if ((!lens_dev && !is_empty(desc)) || ((uintptr_t)lens_dev & 3) != 0) return NYS_ERR_INVALID_ARG;
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
                       stream, nullptr, 0, lens_dev);
+}
+
+NYS_ATTN_API nys_status nys_attn_backward_workspace_size(const nys_desc *desc, int m,
+                                                         int pinv_iters, int conv_k,
+                                                         size_t *bytes) {
+  if (!bytes) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (pinv_iters < 0 || conv_k < 0) return NYS_ERR_INVALID_ARG;
+  if (pinv_iters > kMaxIters || conv_k > kMaxConvK) return NYS_ERR_UNSUPPORTED;
+  *bytes = is_empty(desc) ? 0 : make_bwd_layout(desc, m, pinv_iters, conv_k).total;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_backward(const void *Q, const void *K, const void *V,
+                                          const nys_desc *desc, int m, int iters,
+                                          const float *conv_w, int conv_k, const void *dO,
+                                          void *dQ, void *dK, void *dV, float *dconv_w,
+                                          void *workspace, size_t workspace_bytes,
+                                          nys_stream_t stream_) {
+  nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, dQ);
+  if (st != NYS_OK) return st;
+  if ((conv_w == nullptr) != (dconv_w == nullptr)) return NYS_ERR_INVALID_ARG;
+  if (conv_w && ((uintptr_t)dconv_w & 3) != 0) return NYS_ERR_INVALID_ARG;
+  if (is_empty(desc)) {
+    if (conv_w && desc->heads > 0)   // no tokens: the conv gradient is zero
+      return cudaMemsetAsync(dconv_w, 0, (size_t)desc->heads * conv_k * 4,
+                             (cudaStream_t)stream_) == cudaSuccess
+                 ? NYS_OK
+                 : NYS_ERR_CUDA;
+    return NYS_OK;
+  }
+  if (!dO || !dK || !dV) return NYS_ERR_INVALID_ARG;
+  const uintptr_t align = desc->dtype == NYS_BF16 ? 15 : 3;
+  if ((((uintptr_t)dO | (uintptr_t)dK | (uintptr_t)dV) & align) != 0) return NYS_ERR_INVALID_ARG;
+  const size_t tbytes = (size_t)desc->batch * desc->heads * desc->seq_len * desc->head_dim *
+                        elem_size(desc->dtype);
+  // gradients overlap neither each other nor any input
+  const void *ins[4] = {Q, K, V, dO};
+  void *outs[3] = {dQ, dK, dV};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 4; ++j)
+      if (overlaps(outs[i], tbytes, ins[j], tbytes)) return NYS_ERR_ALIAS;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], tbytes, outs[j], tbytes)) return NYS_ERR_ALIAS;
+  }
+  const BwdLayout L = make_bwd_layout(desc, m, iters, conv_w ? conv_k : 0);
+  cudaStream_t stream = (cudaStream_t)stream_;
+  if (workspace) {
+    if (workspace_bytes < L.total) return NYS_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255) != 0) return NYS_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+      if (overlaps(outs[i], tbytes, workspace, L.total)) return NYS_ERR_ALIAS;
+  }
+  char *ws = (char *)workspace;
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
+    owned = true;
+  }
+  if (cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  if (st == NYS_OK) {
+    const int mb = L.mb;
+    if (desc->dtype == NYS_F32) {
+      const float *q = (const float *)Q, *k = (const float *)K, *v = (const float *)V,
+                  *g = (const float *)dO;
+      float *dq = (float *)dQ, *dk = (float *)dK, *dv = (float *)dV;
+      st = mb == 32 ? launch_bwd<float, 32>(q, k, v, desc, m, iters, conv_w, conv_k, g, dq, dk,
+                                            dv, dconv_w, ws, L, stream)
+                    : launch_bwd<float, 64>(q, k, v, desc, m, iters, conv_w, conv_k, g, dq, dk,
+                                            dv, dconv_w, ws, L, stream);
+    } else {
+      typedef __nv_bfloat16 B;
+      const B *q = (const B *)Q, *k = (const B *)K, *v = (const B *)V, *g = (const B *)dO;
+      B *dq = (B *)dQ, *dk = (B *)dK, *dv = (B *)dV;
+      st = mb == 32   ? launch_bwd<B, 32>(q, k, v, desc, m, iters, conv_w, conv_k, g, dq, dk, dv,
+                                          dconv_w, ws, L, stream)
+           : mb == 64 ? launch_bwd<B, 64>(q, k, v, desc, m, iters, conv_w, conv_k, g, dq, dk, dv,
+                                          dconv_w, ws, L, stream)
+                      : launch_bwd<B, 128>(q, k, v, desc, m, iters, conv_w, conv_k, g, dq, dk,
+                                           dv, dconv_w, ws, L, stream);
+    }
+  }
+  if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && st == NYS_OK) st = NYS_ERR_CUDA;
+  return st;
 }
 
 // ---------------------------------------------------------------------------

@@ -105,6 +105,9 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       seq = 0;
   }
   const bool mask_v = conv && prm.lens != nullptr;
+  // Q and V are read here for the last time in the pass and out is not read
+  // again: their lines leave L2 first
+  const uint64_t last_use = policy_evict_first();
   constexpr uint32_t kStride = M + 64;        // TMEM columns per softmax warpgroup
   constexpr uint32_t kT = 2 * kStride;        // Toeplitz operand columns
 
@@ -160,8 +163,15 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     for (int i = 0; i < pre; ++i) {
       const int r0 = (t_begin + i) * kTileRows;
       mbar_expect_tx(&full[i], bytes);
-      tma_load_3d(smem + L.q[i], map_q, &full[i], 0, r0, bh);
-      if (conv) tma_load_3d(smem + L.v[i], map_v, &full[i], 0, r0 - half, bh);
+      tma_load_3d_hint(smem + L.q[i], map_q, &full[i], 0, r0, bh, last_use);
+      if (conv) tma_load_3d_hint(smem + L.v[i], map_v, &full[i], 0, r0 - half, bh, last_use);
+    }
+    // the block's other tiles into L2 while it waits for W: HBM is mostly
+    // idle between the end of B~ V and W
+    for (int i = pre; i < ntiles; ++i) {
+      const int r0 = (t_begin + i) * kTileRows;
+      tma_prefetch_l2_3d(map_q, 0, r0, bh);
+      if (conv) tma_prefetch_l2_3d(map_v, 0, r0 - half, bh);
     }
   }
   // Toeplitz operand into TMEM: row r (lane r), columns j = halo rows
@@ -235,8 +245,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
         if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
         const int r0 = (t_begin + i) * kTileRows;
         mbar_expect_tx(&full[s], bytes);
-        tma_load_3d(smem + L.q[s], map_q, &full[s], 0, r0, bh);
-        if (conv) tma_load_3d(smem + L.v[s], map_v, &full[s], 0, r0 - half, bh);
+        tma_load_3d_hint(smem + L.q[s], map_q, &full[s], 0, r0, bh, last_use);
+        if (conv) tma_load_3d_hint(smem + L.v[s], map_v, &full[s], 0, r0 - half, bh, last_use);
       }
       // consume the stage releases nobody else waits for (no tensor-core
       // arrival may be pending when the barriers are invalidated)
@@ -357,7 +367,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       fence_async_smem();
       named_barrier(2 + wg, 128);
       if (r == 0) {
-        tma_store_3d(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh);
+        tma_store_3d_hint(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh, last_use);
         bulk_commit();
       }
     }

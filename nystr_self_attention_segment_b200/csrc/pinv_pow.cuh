@@ -382,6 +382,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       }
     }
     wait_main(crit);
+    if (j < 8) NYS_MARK(kTrMid, 40 + j);
     if (ok && crit) {
       float p2[NC], uu[NC];
       ld_cols<NC>(t_d + c_lo, p2);
@@ -407,6 +408,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       }
     }
     wait_main(crit || aux);
+    if (j < 8) NYS_MARK(kTrMid, 48 + j);
     if (ok && crit) {   // P_{j+1} = 1/4 (13 P - 15 P2 + 7 P^3 - P^4)
       float d[NC], a[NC], b[NC];
       ld_cols<NC>(t_d + c_lo, d);

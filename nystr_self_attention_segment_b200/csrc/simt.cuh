@@ -79,9 +79,12 @@ __device__ __forceinline__ void block_diag_minus(float *dst, const float *src, f
   __syncthreads();
 }
 
+// a_out, z_all (optional, for the backward pass): A [BH][m][m] and every
+// iterate Z0 .. Z_iters [BH][iters + 1][m][m].
 __global__ void pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt,
                           float *__restrict__ Zout, float *__restrict__ scratch, int m, int d,
-                          float scale, int iters, int use_smem) {
+                          float scale, int iters, int use_smem, float *__restrict__ a_out = nullptr,
+                          float *__restrict__ z_all = nullptr) {
   extern __shared__ float smem[];
   const int bh = blockIdx.x;
   float *mats = use_smem ? smem : scratch + (size_t)bh * 5 * m * m;
@@ -131,6 +134,8 @@ __global__ void pinv_simt(const float *__restrict__ Qt, const float *__restrict_
   for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
     int i = idx / m, j = idx % m;
     Z[idx] = A[j * m + i] * c0;
+    if (a_out) a_out[(size_t)bh * m * m + idx] = A[idx];
+    if (z_all) z_all[(size_t)bh * (iters + 1) * m * m + idx] = A[j * m + i] * c0;
   }
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
@@ -141,7 +146,10 @@ __global__ void pinv_simt(const float *__restrict__ Qt, const float *__restrict_
     block_gemm(T2, P, T1, m);             // AZ (15I - ...)
     block_diag_minus(T1, T2, 13.f, m);    // 13I - ...
     block_gemm(T2, Z, T1, m);             // Z (13I - ...)
-    for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) Z[idx] = 0.25f * T2[idx];
+    for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
+      Z[idx] = 0.25f * T2[idx];
+      if (z_all) z_all[((size_t)bh * (iters + 1) + it + 1) * m * m + idx] = 0.25f * T2[idx];
+    }
     __syncthreads();
   }
   float *zo = Zout + (size_t)bh * m * m;
@@ -242,7 +250,7 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
 __global__ void merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
                              const float *__restrict__ py, const float *__restrict__ Zg,
                              float *__restrict__ Yg, float *__restrict__ Wg, int m, int d,
-                             int splits) {
+                             int splits, float *__restrict__ lse2 = nullptr) {
   extern __shared__ float ys[];   // [m][d]
   const int bh = blockIdx.x;
   const size_t pb = (size_t)bh * splits * m;
@@ -257,6 +265,7 @@ __global__ void merge_w_simt(const float *__restrict__ pmax, const float *__rest
       acc = fmaf(py[(pb + (size_t)s * m + j) * d + c], f, acc);
     }
     float y = acc / sum;
+    if (lse2 && c == 0) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
     ys[idx] = y;
     Yg[(size_t)bh * m * d + idx] = y;
   }
