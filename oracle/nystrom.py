@@ -71,6 +71,7 @@ __all__ = [
     "nystrom_forward_lens",
     "nystrom_head_backward",
     "nystrom_backward",
+    "nystrom_layer_forward",
     "exact_attention_head",
     "exact_attention",
     "algorithmic_flops",
@@ -413,6 +414,30 @@ def nystrom_backward(Q, K, V, m, dout, iters=6, conv_w=None):
             if dconv is not None:
                 dconv[h] += g["dw"]
     return {"dQ": dQ, "dK": dK, "dV": dV, "dconv": dconv}
+
+
+def nystrom_layer_forward(X, Wqkv, Wo, heads, m, iters=6, conv_w=None):
+    """The attention layer around the method ([P5] "Standard Self-Attention:
+    The Mathematical Baseline": Q = X W_Q, K = X W_K, V = X W_V; Figure 4
+    takes the layer input X): per-head Nystrom attention of the projections,
+    heads concatenated, then an output projection.
+    X: [B, n, D]; Wqkv: [3D, D] (rows 0..D-1 give Q, D..2D-1 K, 2D..3D-1 V,
+    head h the features h*d .. h*d + d - 1 of each, d = D / heads); Wo:
+    [D, D] (nn.Linear layout: Y = concat(O) Wo^T).  Returns Y [B, n, D]."""
+    X = _f64(X)
+    Wqkv = _f64(Wqkv)
+    Wo = _f64(Wo)
+    Bn, n, D = X.shape
+    d = D // heads
+
+    def split(M):   # [B, n, D] -> [B, H, n, d]
+        return M.reshape(Bn, n, heads, d).transpose(0, 2, 1, 3)
+
+    Q = split(X @ Wqkv[:D].T)
+    K = split(X @ Wqkv[D:2 * D].T)
+    V = split(X @ Wqkv[2 * D:].T)
+    O = nystrom_forward(Q, K, V, m, iters, conv_w)
+    return O.transpose(0, 2, 1, 3).reshape(Bn, n, D) @ Wo.T
 
 
 def exact_attention_head(Q, K, V, scale=None):

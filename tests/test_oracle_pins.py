@@ -386,3 +386,44 @@ def test_lens_uniform_queries_closed_form_with_boundary_conv():
             for c in range(4):
                 conv = np.correlate(np.pad(V[b, h, :L, c], 2), w[h], mode="valid")
                 np.testing.assert_allclose(got[b, h, :L, c], mean[c] + conv, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ layer
+
+def test_layer_with_identity_projections_is_the_attention():
+    # one head, D = d, W_Q = W_K = W_V = W_O = I: the layer is the method on
+    # Q = K = V = X
+    rng = np.random.default_rng(31)
+    B, n, d, m = 2, 24, 8, 4
+    X = rng.standard_normal((B, n, d))
+    I = np.eye(d)
+    Y = orc.nystrom_layer_forward(X, np.vstack([I, I, I]), I, 1, m)
+    want = orc.nystrom_forward(X[:, None], X[:, None], X[:, None], m)[:, 0]
+    assert np.allclose(Y, want, rtol=0, atol=1e-13)
+
+
+def test_layer_head_split_and_concat_follow_the_features():
+    # the layer equals the per-head attention of the head's feature slices,
+    # placed at the head's columns before Wo; swapping two heads' slices in
+    # W_Q, W_K, W_V and the matching columns of Wo leaves Y unchanged
+    rng = np.random.default_rng(32)
+    B, n, H, d, m = 1, 16, 2, 4, 4
+    D = H * d
+    X = rng.standard_normal((B, n, D))
+    W = rng.standard_normal((3 * D, D)) / np.sqrt(D)
+    Wo = rng.standard_normal((D, D)) / np.sqrt(D)
+    cw = 0.1 * rng.standard_normal((H, 3))
+    Y = orc.nystrom_layer_forward(X, W, Wo, H, m, 6, cw)
+    O = np.zeros((B, n, D))
+    for h in range(H):
+        sl = slice(h * d, (h + 1) * d)
+        q = X @ W[:D][sl].T
+        k = X @ W[D:2 * D][sl].T
+        v = X @ W[2 * D:][sl].T
+        O[:, :, sl] = orc.nystrom_forward(q[:, None], k[:, None], v[:, None], m, 6,
+                                          cw[h:h + 1])[:, 0]
+    assert np.allclose(Y, O @ Wo.T, rtol=0, atol=1e-12)
+    perm = np.r_[np.arange(d, 2 * d), np.arange(0, d)]
+    Wp = np.vstack([W[:D][perm], W[D:2 * D][perm], W[2 * D:][perm]])
+    Yp = orc.nystrom_layer_forward(X, Wp, Wo[:, perm], H, m, 6, cw[::-1])
+    assert np.allclose(Y, Yp, rtol=0, atol=1e-12)
