@@ -154,6 +154,37 @@ NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q_dev, const void *K_d
                                               void *workspace_dev, size_t workspace_bytes,
                                               nys_stream_t stream);
 
+/* The attention layer around the forward: the projections of "Standard
+ * Self-Attention: The Mathematical Baseline" (Q = X W_Q, K = X W_K,
+ * V = X W_V) and an output projection, with the forward in between
+ * (Figure 4 takes the layer input X):
+ *   Y = concat_h( forward(Q_h, K_h, V_h) ) Wo^T
+ * NYS_BF16 and head_dim 64 only; D = heads * 64.
+ *   X_dev     [batch][seq_len][D] bf16, the layer input;
+ *   Wqkv_dev  [3 D][D] bf16: rows 0 .. D-1 give Q, D .. 2D-1 K, 2D .. 3D-1 V
+ *             (nn.Linear weight layout: output feature, input feature), head
+ *             h takes features h*64 .. h*64 + 63 of each;
+ *   Wo_dev    [D][D] bf16; Y_dev [batch][seq_len][D] bf16 (must not overlap
+ *             X, the weights or the workspace);
+ *   workspace_dev  nys_attn_layer_workspace_size bytes, 256-byte aligned
+ *             (required): Q, K, V and the attention output in bf16, then the
+ *             forward's workspace;
+ * all pointers 16-byte aligned.  The projections are tensor-core GEMMs (fp32
+ * accumulation, bf16 results); Q, K, V and the attention output are rounded
+ * to bf16 between the steps.  A status a kernel records on the device is read
+ * with nys_attn_layer_check_error.  (The pages' layer wraps the attention in
+ * these projections; the library measures the attention itself.) */
+NYS_ATTN_API nys_status nys_attn_layer_workspace_size(const nys_desc *desc, int num_landmarks,
+                                                      size_t *bytes);
+NYS_ATTN_API nys_status nys_attn_layer_forward(const void *X_dev, const void *Wqkv_dev,
+                                               const void *Wo_dev, const nys_desc *desc,
+                                               int num_landmarks, int pinv_iters,
+                                               const float *conv_w_dev, int conv_k, void *Y_dev,
+                                               void *workspace_dev, size_t workspace_bytes,
+                                               nys_stream_t stream);
+NYS_ATTN_API nys_status nys_attn_layer_check_error(void *workspace_dev, const nys_desc *desc,
+                                                   int num_landmarks, nys_stream_t stream);
+
 /* Backward pass ("Moore-Penrose Pseudoinverse Computation": gradients flow
  * through the iteration's matrix products like through any other layer):
  * given dO = dL/dout of the forward with the same arguments, writes

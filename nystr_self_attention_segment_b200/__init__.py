@@ -19,6 +19,7 @@ __all__ = [
     "nys_attn_host_buffer_size", "nys_attn_check_error", "nys_attn_launch_count",
     "nys_status_string", "nys_version", "Workspace", "nys_attn_launch_names",
     "nys_attn_forward_timed", "nys_attn_forward_lens", "nys_attn_backward",
+    "nys_attn_layer_forward",
 ]
 
 
@@ -130,6 +131,55 @@ def nys_attn_forward(Q, K, V, num_landmarks, pinv_iters=6, conv_w=None, out=None
                               _stream_ptr(stream))
     _lib.check(st, "nys_attn_forward")
     return out
+
+
+def nys_attn_layer_forward(X, Wqkv, Wo, heads, num_landmarks, pinv_iters=6, conv_w=None,
+                           workspace=None, stream=None):
+    """The attention layer: Y = concat_h(forward(X Wq_h^T, X Wk_h^T, X Wv_h^T)) Wo^T for
+    X [batch, n, D] bf16 (D = heads * 64), Wqkv [3D, D], Wo [D, D] bf16 CUDA tensors.
+    workspace: a CUDA uint8 tensor of at least nys_attn_layer_workspace_size bytes
+    (+256 for alignment), or None (allocated here).  Returns (Y, workspace_view): the
+    view holds Q, K, V and the attention output (bf16, [batch, heads, n, 64] each) at
+    its start."""
+    torch = _torch()
+    if X.dim() != 3 or X.dtype != torch.bfloat16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous bfloat16 CUDA tensor [batch, n, D]")
+    B, n, D = X.shape
+    if D != heads * 64:
+        raise ValueError("D must be heads * 64")
+    for name, w, shape in (("Wqkv", Wqkv, (3 * D, D)), ("Wo", Wo, (D, D))):
+        if (tuple(w.shape) != shape or w.dtype != torch.bfloat16 or w.device != X.device
+                or not w.is_contiguous()):
+            raise ValueError("%s must be a contiguous bfloat16 tensor %s on X's device"
+                             % (name, shape))
+    if conv_w is not None:
+        if (conv_w.dtype != torch.float32 or conv_w.device != X.device or conv_w.dim() != 2
+                or conv_w.shape[0] != heads or not conv_w.is_contiguous()):
+            raise ValueError("conv_w must be a contiguous float32 [heads, k] tensor on X's device")
+    desc = make_desc(NYS_BF16, B, heads, n, 64)
+    nb = _lib.nys_attn_layer_workspace_size(desc, num_landmarks)
+    if workspace is None:
+        workspace = torch.empty(nb + 256, dtype=torch.uint8, device=X.device)
+    base = workspace.data_ptr()
+    off = (-base) % 256
+    if workspace.numel() - off < nb or workspace.device != X.device:
+        raise ValueError("workspace too small or on another device")
+    Y = torch.empty_like(X)
+    conv_ptr, conv_k = (None, 0) if conv_w is None else (conv_w.data_ptr(), conv_w.shape[1])
+    with _on_device(X.device):
+        st = _lib.raw_layer_forward(X.data_ptr(), Wqkv.data_ptr(), Wo.data_ptr(), desc,
+                                    num_landmarks, pinv_iters, conv_ptr, conv_k, Y.data_ptr(),
+                                    base + off, nb, _stream_ptr(stream))
+    _lib.check(st, "nys_attn_layer_forward")
+    return Y, workspace[off:off + nb]
+
+
+def nys_attn_layer_check_error(workspace_view, heads, batch, n, num_landmarks, stream=None):
+    """Synchronises and raises if a layer kernel recorded an error."""
+    desc = make_desc(NYS_BF16, batch, heads, n, 64)
+    st = _lib.raw_layer_check_error(workspace_view.data_ptr(), desc, num_landmarks,
+                                    _stream_ptr(stream))
+    _lib.check(st, "nys_attn_layer_check_error")
 
 
 def nys_attn_backward(Q, K, V, num_landmarks, dO, pinv_iters=6, conv_w=None, workspace=None,

@@ -43,6 +43,9 @@ EXPORTS = (
     "nys_attn_forward_lens",
     "nys_attn_backward_workspace_size",
     "nys_attn_backward",
+    "nys_attn_layer_workspace_size",
+    "nys_attn_layer_forward",
+    "nys_attn_layer_check_error",
 )
 
 # Size of the fixed scratch array of nys_attn_forward_static (see the header).
@@ -113,6 +116,12 @@ def load():
     lib.nys_attn_backward_workspace_size.argtypes = [D, I, I, I, ctypes.POINTER(S)]
     lib.nys_attn_backward.restype = I
     lib.nys_attn_backward.argtypes = [P, P, P, D, I, I, P, I, P, P, P, P, P, P, S, P]
+    lib.nys_attn_layer_workspace_size.restype = I
+    lib.nys_attn_layer_workspace_size.argtypes = [D, I, ctypes.POINTER(S)]
+    lib.nys_attn_layer_forward.restype = I
+    lib.nys_attn_layer_forward.argtypes = [P, P, P, D, I, I, P, I, P, P, S, P]
+    lib.nys_attn_layer_check_error.restype = I
+    lib.nys_attn_layer_check_error.argtypes = [P, D, I, P]
     lib.nys_attn_forward_lens.restype = I
     lib.nys_attn_forward_lens.argtypes = [P, P, P, D, I, I, P, I, P, P, P, S, P]
     _LIB = lib
@@ -230,6 +239,26 @@ def raw_backward(q_ptr, k_ptr, v_ptr, desc, num_landmarks, pinv_iters, conv_ptr,
                                     int(pinv_iters), conv_ptr, int(conv_k), do_ptr, dq_ptr,
                                     dk_ptr, dv_ptr, dconv_ptr, ws_ptr, ctypes.c_size_t(ws_bytes),
                                     stream_ptr)
+
+
+def nys_attn_layer_workspace_size(desc, num_landmarks):
+    out = ctypes.c_size_t(0)
+    check(load().nys_attn_layer_workspace_size(ctypes.byref(desc), int(num_landmarks),
+                                               ctypes.byref(out)), "nys_attn_layer_workspace_size")
+    return out.value
+
+
+def raw_layer_forward(x_ptr, wqkv_ptr, wo_ptr, desc, num_landmarks, pinv_iters, conv_ptr, conv_k,
+                      y_ptr, ws_ptr, ws_bytes, stream_ptr):
+    return load().nys_attn_layer_forward(x_ptr, wqkv_ptr, wo_ptr, ctypes.byref(desc),
+                                         int(num_landmarks), int(pinv_iters), conv_ptr,
+                                         int(conv_k), y_ptr, ws_ptr, ctypes.c_size_t(ws_bytes),
+                                         stream_ptr)
+
+
+def raw_layer_check_error(ws_ptr, desc, num_landmarks, stream_ptr):
+    return load().nys_attn_layer_check_error(ws_ptr, ctypes.byref(desc), int(num_landmarks),
+                                             stream_ptr)
 
 
 def raw_check_error_static(desc, num_landmarks, stream_ptr):

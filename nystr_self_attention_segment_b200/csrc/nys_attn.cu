@@ -16,6 +16,7 @@
 #include "out_tc.cuh"
 #include "wmerge.cuh"
 #include "bwd_simt.cuh"
+#include "gemm_tc.cuh"
 #include "stream_bf16.cuh"
 
 using namespace nys;
@@ -311,6 +312,22 @@ bool make_map(CUtensorMap *map, const void *base, int BH, int n, int rows) {
          CUDA_SUCCESS;
 }
 
+// A bf16 tensor [d2][d1][d0] (d0 contiguous) as a 3-D map with a box of
+// 64 x rows x 1 and the 128-byte swizzle; reads outside the tensor are zero.
+bool make_map3(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+               int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // launches of the bf16 path
 constexpr int kTcLaunches = 4;
 const char *kTcNames = "seg_means,mid_tc,w_merge,out_tc";
@@ -409,6 +426,42 @@ nys_status launch_tc(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_
       return launch_tc_m<128>(Q, K, V, desc, iters, conv_w, conv_k, lens, out, ws, L, stream, mk);
   }
   return NYS_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------
+// The attention layer: QKV projection, the forward, output projection.
+struct LayerLayout {
+  size_t q, k, v, o, ws, total;
+};
+
+LayerLayout make_layer_layout(const nys_desc *desc, int m) {
+  LayerLayout L;
+  const size_t t = (size_t)desc->batch * desc->heads * desc->seq_len * 64 * 2;
+  size_t off = 0;
+  auto take = [&](size_t b) {
+    size_t at = off;
+    off = align256(off + b);
+    return at;
+  };
+  L.q = take(t);
+  L.k = take(t);
+  L.v = take(t);
+  L.o = take(t);
+  L.ws = take(make_layout(desc, m).total);
+  L.total = off;
+  return L;
+}
+
+template <int MODE>
+nys_status launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const gemm::Params &p,
+                       cudaStream_t stream) {
+  auto kern = gemm::gemm_kernel<MODE>;
+  const int grid = p.batch * p.mtiles * p.ntiles;
+  if (!allow_smem(kern, gemm::kSmem) ||
+      launch(kern, dim3(grid), dim3(gemm::kThreads), gemm::kSmem, stream, false, ma, mb, p) !=
+          cudaSuccess)
+    return NYS_ERR_CUDA;
+  return NYS_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -645,7 +698,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
                                const nys_desc *desc, int m, int iters, const float *conv_w,
                                int conv_k, void *out, void *workspace, size_t workspace_bytes,
                                nys_stream_t stream_, void *const *events, int n_events,
-                               const int *lens = nullptr) {
+                               const int *lens = nullptr, bool clear_err = true) {
   nys_status st = validate_call(Q, K, V, desc, m, iters, conv_w, conv_k, out);
   if (st != NYS_OK) return st;
   if (events && n_events < (desc->dtype == NYS_BF16 ? kTcLaunches : kSimtLaunches) + 1)
@@ -672,7 +725,7 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  if (clear_err && cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
   mk.first(stream);
   if (st == NYS_OK) {
     if (desc->dtype == NYS_F32)
@@ -706,6 +759,89 @@ NYS_ATTN_API nys_status nys_attn_forward_lens(const void *Q, const void *K, cons
   if ((!lens_dev && !is_empty(desc)) || ((uintptr_t)lens_dev & 3) != 0) return NYS_ERR_INVALID_ARG;
   return forward_impl(Q, K, V, desc, m, iters, conv_w, conv_k, out, workspace, workspace_bytes,
                       stream, nullptr, 0, lens_dev);
+}
+
+NYS_ATTN_API nys_status nys_attn_layer_workspace_size(const nys_desc *desc, int m,
+                                                      size_t *bytes) {
+  if (!bytes) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (desc->dtype != NYS_BF16) return NYS_ERR_UNSUPPORTED;
+  *bytes = is_empty(desc) ? 0 : make_layer_layout(desc, m).total;
+  return NYS_OK;
+}
+
+NYS_ATTN_API nys_status nys_attn_layer_forward(const void *X, const void *Wqkv, const void *Wo,
+                                               const nys_desc *desc, int m, int iters,
+                                               const float *conv_w, int conv_k, void *Y,
+                                               void *workspace, size_t workspace_bytes,
+                                               nys_stream_t stream_) {
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (desc->dtype != NYS_BF16) return NYS_ERR_UNSUPPORTED;
+  if (iters < 0) return NYS_ERR_INVALID_ARG;
+  if (iters > kMaxIters) return NYS_ERR_UNSUPPORTED;
+  if (conv_w && (conv_k < 1 || conv_k % 2 == 0 || ((uintptr_t)conv_w & 3) != 0))
+    return NYS_ERR_INVALID_ARG;
+  if (conv_w && conv_k > kMaxConvK) return NYS_ERR_UNSUPPORTED;
+  if (is_empty(desc)) return NYS_OK;
+  if (!X || !Wqkv || !Wo || !Y || !workspace) return NYS_ERR_INVALID_ARG;
+  if ((((uintptr_t)X | (uintptr_t)Wqkv | (uintptr_t)Wo | (uintptr_t)Y) & 15) != 0 ||
+      ((uintptr_t)workspace & 255) != 0)
+    return NYS_ERR_INVALID_ARG;
+  const LayerLayout LL = make_layer_layout(desc, m);
+  if (workspace_bytes < LL.total) return NYS_ERR_WORKSPACE;
+  const int B = desc->batch, H = desc->heads, n = desc->seq_len, D = H * 64;
+  const size_t xbytes = (size_t)B * n * D * 2;
+  if (overlaps(Y, xbytes, X, xbytes) || overlaps(Y, xbytes, workspace, LL.total) ||
+      overlaps(Y, xbytes, Wqkv, (size_t)3 * D * D * 2) || overlaps(Y, xbytes, Wo, (size_t)D * D * 2))
+    return NYS_ERR_ALIAS;
+  cudaStream_t stream = (cudaStream_t)stream_;
+  char *ws = (char *)workspace;
+  __nv_bfloat16 *q = (__nv_bfloat16 *)(ws + LL.q), *k = (__nv_bfloat16 *)(ws + LL.k),
+                *v = (__nv_bfloat16 *)(ws + LL.v), *o = (__nv_bfloat16 *)(ws + LL.o);
+  CUtensorMap mx, mwq, mo, mwo;
+  if (!make_map3(&mx, X, D, n, B, gemm::kBM) || !make_map3(&mwq, Wqkv, D, 3 * D, 1, gemm::kBN) ||
+      !make_map3(&mo, o, 64, n, (uint64_t)B * H, gemm::kBM) ||
+      !make_map3(&mwo, Wo, D, D, 1, gemm::kBN))
+    return NYS_ERR_CUDA;
+  if (cudaMemsetAsync(ws + LL.ws + make_layout(desc, m).err, 0, 256, stream) != cudaSuccess)
+    return NYS_ERR_CUDA;
+  gemm::Params gp{};
+  gp.n = n;
+  gp.batch = B;
+  gp.heads = H;
+  gp.mtiles = (n + gemm::kBM - 1) / gemm::kBM;
+  gp.err = (uint32_t *)(ws + LL.ws + make_layout(desc, m).err);
+  // Q, K, V = X W^T, written per head
+  gp.N = 3 * D;
+  gp.K = D;
+  gp.ntiles = (3 * D + gemm::kBN - 1) / gemm::kBN;
+  gp.q = q;
+  gp.k = k;
+  gp.v = v;
+  st = launch_gemm<gemm::kQkv>(mx, mwq, gp, stream);
+  if (st != NYS_OK) return st;
+  // the attention proper, with its workspace after Q, K, V, O
+  st = forward_impl(q, k, v, desc, m, iters, conv_w, conv_k, o, ws + LL.ws, LL.total - LL.ws,
+                    stream_, nullptr, 0, nullptr, false);
+  if (st != NYS_OK) return st;
+  // Y = concat_h(O_h) Wo^T
+  gp.N = D;
+  gp.K = D;
+  gp.ntiles = (D + gemm::kBN - 1) / gemm::kBN;
+  gp.y = (__nv_bfloat16 *)Y;
+  return launch_gemm<gemm::kOut>(mo, mwo, gp, stream);
+}
+
+NYS_ATTN_API nys_status nys_attn_layer_check_error(void *workspace, const nys_desc *desc, int m,
+                                                   nys_stream_t stream) {
+  if (!workspace) return NYS_ERR_INVALID_ARG;
+  nys_status st = validate_shape(desc, m);
+  if (st != NYS_OK) return st;
+  if (desc->dtype != NYS_BF16) return NYS_ERR_UNSUPPORTED;
+  if (is_empty(desc)) return NYS_OK;
+  return nys_attn_check_error((char *)workspace + make_layer_layout(desc, m).ws, desc, m, stream);
 }
 
 NYS_ATTN_API nys_status nys_attn_backward_workspace_size(const nys_desc *desc, int m,

@@ -97,11 +97,12 @@ def test_bf16_intermediates(name):
         Q, K, V = (x[t][b, h].astype(np.float64) for t in ("Q", "K", "V"))
         assert normwise(qt[i], orc.segment_means(Q, m)) <= 1e-5
         assert normwise(kt[i], orc.segment_means(K, m)) <= 1e-5
-        # The device runs the iteration in tf32 (fp32 accumulation); Z of a
-        # nearly uniform, ill-conditioned A differs visibly from fp64 even
-        # though the output stays within 2e-2 (checked above).
+        # Z against the oracle's iteration on the device's own landmarks.
+        # m <= 64 runs the power form with split fp16 / bf16 products
+        # (measured <= 1.9e-3 on every workload, held to 5e-3); m = 128 the
+        # Horner form with tf32 operands (measured <= 2.9e-2, held to 6e-2).
         Z = orc.iterative_pinv(orc.kernel_A(qt[i], kt[i], s), wl.pinv_iters)
-        assert normwise(Zg[i], Z) <= 0.25
+        assert normwise(Zg[i], Z) <= (5e-3 if m <= 64 else 6e-2)
         Y = orc.kernel_B(qt[i], K, s) @ V
         assert normwise(Yg[i], Y) <= 2e-2
         assert normwise(Wg[i], Zg[i] @ Yg[i]) <= 1e-4
