@@ -102,6 +102,11 @@ constexpr float kTau = 8.f;
 #ifndef NYS_BV_TURNS
 #define NYS_BV_TURNS 1
 #endif
+// V's loads with the evict-first policy (1) or not (0: the output kernel
+// reads V again).
+#ifndef NYS_V_EVICT_FIRST
+#define NYS_V_EVICT_FIRST 0
+#endif
 
 // tmem_in: a 512-column TMEM allocation owned by the caller, or ~0u to
 // allocate (and free) one here.
@@ -166,12 +171,18 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   // K is read here for the last time in the pass (V again by the output
   // kernel): its lines leave L2 first
   const uint64_t last_use = policy_evict_first();
+  auto load_v = [&](int s, int k0) {
+    if (NYS_V_EVICT_FIRST)
+      tma_load_3d_hint(smem + L.v[s], map_v, &full[s], 0, k0, bh, last_use);
+    else
+      tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
+  };
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < pre; ++i) {
       const int k0 = (c_begin + i) * kChunk;
       mbar_expect_tx(&full[i], 32768u);
       tma_load_3d_hint(smem + L.k[i], map_k, &full[i], 0, k0, bh, last_use);
-      tma_load_3d(smem + L.v[i], map_v, &full[i], 0, k0, bh);
+      load_v(i, k0);
     }
   }
   if (wait_prev) {
@@ -209,7 +220,7 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
         const int k0 = (c_begin + i) * kChunk;
         mbar_expect_tx(&full[s], 32768u);
         tma_load_3d_hint(smem + L.k[s], map_k, &full[s], 0, k0, bh, last_use);
-        tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
+        load_v(s, k0);
       }
       // consume the stage releases nobody else waits for, so that no
       // tensor-core arrival is pending when the barriers are invalidated

@@ -356,11 +356,8 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
 
   {   // segment means of Q and K (Eq. 16)
     const segm::Shape sh{n, M, desc->heads, lens};
-    const dim3 grid(segm::groups_for(BH, M), BH, 2);
-    if (!allow_smem(segm::seg_means_bf16, segm::kSmem) ||
-        launch(segm::seg_means_bf16, grid, dim3(segm::kThreads),
-               launch_smem(mk.launched, segm::kSmem), stream, false, Q, K, qt, kt, sh,
-               err) != cudaSuccess)
+    if (launch(segm::seg_means_bf16, dim3(M, BH, 2), dim3(segm::threads_for(n, M)),
+               launch_smem(mk.launched, 0), stream, false, Q, K, qt, kt, sh, err) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }

@@ -13,12 +13,13 @@
 // every P_j is a polynomial in P_0 = A Z_0 = A A^T / (||A||_1 ||A||_inf), so
 // the P_j are symmetric and commute.  One step is two dependent products,
 //   stage 1:  P2 = P P                       (U = 7P - P2 formed from it)
-//   stage 2:  [P2; P] U = [7P^3 - P^4; 7P^2 - P^3]   (one 128-row MMA)
-// after which P_{j+1} and r_j are elementwise.  Z_{j+1} = Z_j r_j is a
-// third product off the dependent chain (issued in two K halves beside the
-// chain's MMAs).  Equal to the printed recurrence in exact arithmetic; only
-// rounding differs.  Because the P_j are symmetric, a matrix's rows serve as
-// its columns: every operand is written once, K-major, and used as A and B.
+//   stage 2:  U [P2 | P] = [7P^3 - P^4 | 7P^2 - P^3]   (one N = 128 MMA)
+// after which P_{j+1} and r_j are elementwise in the thread that holds the
+// row (P_j and P_j^2 stay in its registers).  Z_{j+1} = Z_j r_j is a third
+// product off the dependent chain (issued beside the chain's MMAs).  Equal
+// to the printed recurrence in exact arithmetic; only rounding differs.
+// Because the P_j are symmetric, a matrix's rows serve as its columns: every
+// operand is written once, K-major, and used as A and B.
 //
 // Precision.  Every product is formed from split operands, x = hi + lo with
 // hi the rounding of x and lo the rounding of x - hi, as hi*hi + hi*lo +
@@ -32,8 +33,8 @@
 // amplify to several 1e-2 in the output.
 //
 // Threads 0..255: thread t owns TMEM lane r = t % 128 and column half
-// h = t / 128.  Lanes 0..m-1 carry the P chain, lanes 64..64+m-1 the Z
-// update and r_j (their MMA rows are stacked at row 64), so the two run on
+// h = t / 128.  Lanes 0..m-1 carry the P chain and r_j, lanes 64..64+m-1
+// the Z update (its MMA rows are stacked at row 64), so the two run on
 // different warps.  Thread 256 (warp 8) issues the MMAs: an MMA issue
 // blocks the issuing thread until the tensor pipe takes it, which must not
 // hold up a row thread.
@@ -84,7 +85,7 @@ struct Cfg {
   static constexpr uint32_t red = kl + 64u * 128u;      // [3][M]
   static constexpr uint32_t bars = (red + 3u * M * 4u + 1023u) & ~1023u;
   static constexpr uint32_t total = bars + 1024u;
-  static constexpr uint32_t kTmemCols = 128;        // D at column 0, Z update at 64
+  static constexpr uint32_t kTmemCols = 256;        // D at column 0 (128 wide), Z update at 128
 };
 
 // N (a multiple of 8) values of row `row`, columns c0.. (c0 a multiple of 8),
@@ -228,7 +229,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t t_d = tmem + lane_base, t_z = tmem + lane_base + 64;
+  const uint32_t t_d = tmem + lane_base, t_z = tmem + lane_base + 128;
   const uint32_t id_bf = make_idesc(kFmtBF16, 128, M, 0, 0);
   const uint32_t id_f16 = make_idesc(kFmtF16, 128, M, 0, 0);
   uint32_t pm = 0, pz = 0;   // mbarrier phases
@@ -347,13 +348,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
   }
   wait_main(crit);
+  // P_j of this thread's row and columns stays in registers through the steps
+  float preg[NC];
   if (ok && crit) {   // P0 = c0 A A^T
-    float p[NC];
-    ld_cols<NC>(t_d + c_lo, p);
+    ld_cols<NC>(t_d + c_lo, preg);
 #pragma unroll
-    for (int k = 0; k < NC; ++k) p[k] *= c0;
-    put_split<NC, true>(ph, pl, row, c_lo, p);
-    put_row<NC>(pf0, row, c_lo, p);
+    for (int k = 0; k < NC; ++k) preg[k] *= c0;
+    put_split<NC, true>(ph, pl, row, c_lo, preg);
   }
   if (!sync_ops()) ok = false;
   NYS_MARK(kTrMid, 9);
@@ -366,6 +367,12 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   bool good = ok;   // block-uniform: no stage failed
   const uint32_t id_z = make_idesc(kFmtBF16, 128, M, 0, 0);
   constexpr uint32_t kBr = 64u * 128u;            // one r buffer
+  // stage 2 multiplies U (A, 128 rows of which the first m are U) by the
+  // 128 rows of [P2; P] (B, N = 128): columns 0.. give U P2 = 7P^3 - P^4 and
+  // columns 64.. give U P = 7P^2 - P^3, in the same TMEM lane (the P_j
+  // commute), so the thread that holds P_j and P_j^2 of a row forms both
+  // P_{j+1} and r_j of it
+  const uint32_t id_s2 = make_idesc(kFmtF16, 128, 128, 0, 0);
   for (int j = 0; j < iters; ++j) {
     const bool split = j < kSplitIters, split_next = j + 1 < kSplitIters;
     // stage 1: P2 = P P
@@ -383,53 +390,50 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     }
     wait_main(crit);
     if (j < 8) NYS_MARK(kTrMid, 40 + j);
+    float p2[NC];
     if (ok && crit) {
-      float p2[NC], uu[NC];
+      float uu[NC];
       ld_cols<NC>(t_d + c_lo, p2);
-      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, uu);     // P_j
 #pragma unroll
-      for (int k = 0; k < NC; ++k) uu[k] = fmaf(7.f, uu[k], -p2[k]);
+      for (int k = 0; k < NC; ++k) uu[k] = fmaf(7.f, preg[k], -p2[k]);
       put_split<NC, true>(a2h, a2l, row, c_lo, p2, split);
       put_split<NC, true>(uh, ul, row, c_lo, uu, split);
-      put_row<NC>(p2f, row, c_lo, p2);
     }
     if (!sync_ops()) {
       good = false;
       break;
     }
-    // stage 2: [P2; P] U, then Z_j = Z_{j-1} r_{j-1}
+    // stage 2: U [P2; P], then Z_j = Z_{j-1} r_{j-1}
     if (issuer) {
-      mma3(tmem, sd(a2h), sd(a2l), sd(uh), sd(ul), id_f16, KM{}, split);
+      mma3(tmem, sd(uh), sd(ul), sd(a2h), sd(a2l), id_s2, KM{}, split);
       mma_commit(bar_main);
       if (j > 0) {
         const uint32_t rb = ((j - 1) & 1) * (kBr >> 4);
-        mma3(tmem + 64, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
+        mma3(tmem + 128, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
         mma_commit(bar_z);
       }
     }
-    wait_main(crit || aux);
+    wait_main(crit);
     if (j < 8) NYS_MARK(kTrMid, 48 + j);
-    if (ok && crit) {   // P_{j+1} = 1/4 (13 P - 15 P2 + 7 P^3 - P^4)
-      float d[NC], a[NC], b[NC];
-      ld_cols<NC>(t_d + c_lo, d);
-      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, a);       // P_j
-      get_row<NC>(p2f, row, c_lo, b);                        // P_j^2
+    if (ok && crit) {
+      // P_{j+1} = 1/4 (13 P - 15 P2 + 7 P^3 - P^4), r_j = 1/4 (13I - 15 P + 7 P^2 - P^3)
+      float x[NC], y[NC];
+      tmem_ld16(t_d + c_lo, x);
+      if constexpr (NC == 32) tmem_ld16(t_d + c_lo + 16, x + 16);
+      tmem_ld16(t_d + 64 + c_lo, y);
+      if constexpr (NC == 32) tmem_ld16(t_d + 64 + c_lo + 16, y + 16);
+      tmem_ld_wait();
 #pragma unroll
-      for (int k = 0; k < NC; ++k) d[k] = 0.25f * fmaf(13.f, a[k], fmaf(-15.f, b[k], d[k]));
-      put_split<NC, true>(ph, pl, row, c_lo, d, split_next);
-      put_row<NC>(pf0 + ((j + 1) & 1) * 4096, row, c_lo, d);
+      for (int k = 0; k < NC; ++k) {
+        const float pj = preg[k];
+        preg[k] = 0.25f * fmaf(13.f, pj, fmaf(-15.f, p2[k], x[k]));
+        y[k] = 0.25f * ((c_lo + k == row ? 13.f : 0.f) + fmaf(-15.f, pj, y[k]));
+      }
+      put_split<NC, true>(ph, pl, row, c_lo, preg, split_next);
+      const uint32_t rb = (j & 1) * kBr;
+      put_split<NC, false>(brh + rb, brl + rb, row, c_lo, y);
     }
     if (j < 8) NYS_MARK(kTrMid, 16 + j);
-    if (ok && aux) {   // r_j = 1/4 (13I - 15 P + 7 P^2 - P^3)
-      float d[NC], a[NC];
-      ld_cols<NC>(t_d + c_lo, d);
-      get_row<NC>(pf0 + (j & 1) * 4096, row, c_lo, a);       // P_j
-#pragma unroll
-      for (int k = 0; k < NC; ++k)
-        d[k] = 0.25f * ((c_lo + k == row ? 13.f : 0.f) + fmaf(-15.f, a[k], d[k]));
-      const uint32_t rb = (j & 1) * kBr;
-      put_split<NC, false>(brh + rb, brl + rb, row, c_lo, d);
-    }
     if (!sync_ops()) {
       good = false;
       break;
@@ -449,7 +453,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     if (good) {
       if (issuer) {
         const uint32_t rb = ((iters - 1) & 1) * (kBr >> 4);
-        mma3(tmem + 64, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
+        mma3(tmem + 128, sd(azh), sd(azl), sd(brh) + rb, sd(brl) + rb, id_z, KM{}, true);
         mma_commit(bar_z);
       }
       wait_z(aux);

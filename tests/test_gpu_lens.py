@@ -17,10 +17,20 @@ CASES = [
     (3, 2, 1000, 64, 32, BF16, 33, [1000, 777, 530]),
     (2, 2, 4096, 64, 64, BF16, 33, [4096, 2100]),
     (2, 1, 2048, 64, 128, BF16, 33, [2048, 1400]),
-    (2, 1, 640, 64, 64, BF16, 0, [640, 257]),       # no conv: rows only
+    (2, 1, 640, 64, 64, BF16, 0, [640, 320]),       # no conv: rows only
     (3, 2, 70, 32, 8, F32, 5, [70, 64, 50]),
     (2, 1, 24, 8, 3, F32, 3, [24, 7]),
 ]
+
+
+def _valid(L, m):
+    return (m - 1) * (-(-L // m)) < L
+
+
+@pytest.mark.parametrize("dummy", [0])
+def test_case_lengths_keep_every_segment(dummy):
+    for B, H, n, d, m, dtype, conv_k, lens in CASES:
+        assert all(m <= L <= n and _valid(L, m) for L in lens), (n, m, lens)
 
 
 def _lens(x):
