@@ -46,6 +46,7 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t code) {
 // a machine without a GPU.  All regions are 256-byte aligned.
 struct Layout {
   size_t q_land, k_land, z, y, w, err;     // parity-visible fp32 intermediates
+  size_t count;                            // per-head hand-off counters (bf16 path)
   size_t pmax, psum, py;                   // split-n partials of B~ V
   size_t scratch;                          // per-head pinv scratch (m > 64)
   size_t w_bf;                             // W as the bf16 operand of P W

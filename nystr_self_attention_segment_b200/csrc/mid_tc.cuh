@@ -8,8 +8,9 @@
 //                             Eq. 17 / Algorithm 1; B~ = softmax(Q~ K^T/sqrt(d))
 //                             over the n keys is never stored).
 // Each B~ V block leaves one partial softmax state per landmark (running
-// maximum, sum, unnormalised Y); the next kernel (wmerge.cuh) merges them and
-// forms W = Z Y.
+// maximum, sum, unnormalised Y); the last B~ V block of a head merges them
+// into Y, and the second of {that block, the pseudoinverse block} to finish
+// forms W = Z Y on the tensor cores (merge_y, form_w below).
 //
 // B~ V block.  The 128 accumulator rows (TMEM lanes) hold G = 128 / m copies
 // of the m landmark rows; copy g handles keys g*m .. g*m + m - 1 of every
@@ -71,17 +72,15 @@ __host__ __device__ constexpr uint32_t pinv_smem() {
   }
 }
 
-template <int M>
-__host__ __device__ constexpr uint32_t smem_bytes() {
-  // pinv operands or B~ V buffers
-  constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
-  return 1024u + (pinv_smem<M>() > bv ? pinv_smem<M>() : bv);
-}
 
 struct Params {
   pinvtc::Params pinv;
   const float *q_land;        // [BH][m][64]
   float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
+  const float *z;             // [BH][m][m] (the pseudoinverse blocks' result)
+  float *y, *w;               // [BH][m][64]
+  uint8_t *w_op;              // [BH][m][128 B]: W as the bf16 B operand of P W
+  uint32_t *count;            // [2 BH], zeroed per call: B~V blocks done, W inputs ready
   uint32_t *err;
   const int *lens;            // [batch] tokens per element (ragged batches) or null
   int heads;
@@ -438,10 +437,250 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   }
 }
 
+// ------------------------------------------------------------------ merge + W
+// The last B~ V block of a head (counted with an atomic) merges the head's S
+// partial states into Y in split order:
+//   Y_j = sum_s f_s Y_s,j / sum_s f_s l_s,j,  f_s = 2^(m_s - max_s m_s).
+// The second of {that block, the head's pseudoinverse block} to finish forms
+// W = Z Y (form_w): the same function on the same global Z and Y whichever
+// block runs it, so the result does not depend on which finishes first.
+
+template <int M>
+struct MergeSmem {
+  static constexpr uint32_t wgt = 0;                       // f [kMaxSplits][M]
+  static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
+  static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
+  static constexpr uint32_t total = den + M * 4u;
+};
+
+// All kThreads threads: the S x M maxima and sums into shared memory, the
+// weights, then the partials (a batch of splits of every item of a thread
+// loaded at once); Y in fp32 to global memory.
+template <int M>
+__device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh) {
+  using C = MergeSmem<M>;
+  const int t = threadIdx.x, S = prm.splits;
+  float *wgt = (float *)(smem + C::wgt), *psm = (float *)(smem + C::psm);
+  float *den = (float *)(smem + C::den);
+  const size_t pb = (size_t)bh * S * M;
+  {
+    constexpr int kPer = (kMaxSplits * M + kThreads - 1) / kThreads;
+    float a[kPer], b[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = t + u * kThreads;
+      if (i < S * M) {
+        a[u] = __ldcg(prm.pmax + pb + i);
+        b[u] = __ldcg(prm.psum + pb + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = t + u * kThreads;
+      if (i < S * M) {
+        wgt[i] = a[u];
+        psm[i] = b[u];
+      }
+    }
+  }
+  __syncthreads();
+  if (t < M) {
+    float mx = -INFINITY;
+    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
+    float d = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + t] - mx);
+      wgt[s * M + t] = f;
+      d = fmaf(psm[s * M + t], f, d);
+    }
+    den[t] = 1.f / d;
+  }
+  __syncthreads();
+  constexpr int kItems = M * 16;   // float4 items of Y
+  constexpr int kIpt = (kItems + kThreads - 1) / kThreads;
+  constexpr int kBatch = 16 / kIpt > 0 ? 16 / kIpt : 1;
+  float4 acc[kIpt];
+#pragma unroll
+  for (int q = 0; q < kIpt; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += kBatch) {
+    float4 v[kIpt][kBatch];
+#pragma unroll
+    for (int q = 0; q < kIpt; ++q) {
+      const int idx = q * kThreads + t;
+      if (idx < kItems) {
+        const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kIpt; ++q) {
+      const int idx = q * kThreads + t;
+      if (idx < kItems) {
+        const int j = idx >> 4;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (s0 + u < S) {
+            const float f = wgt[(s0 + u) * M + j];
+            acc[q].x = fmaf(f, v[q][u].x, acc[q].x);
+            acc[q].y = fmaf(f, v[q][u].y, acc[q].y);
+            acc[q].z = fmaf(f, v[q][u].z, acc[q].z);
+            acc[q].w = fmaf(f, v[q][u].w, acc[q].w);
+          }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kIpt; ++q) {
+    const int idx = q * kThreads + t;
+    if (idx < kItems) {
+      const float inv = den[idx >> 4];
+      ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] =
+          make_float4(acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
+    }
+  }
+}
+
+// W = Z Y on the tensor cores from split bf16 operands (hi = rounding of x,
+// lo = rounding of x - hi; Z_h Y_h + Z_h Y_l + Z_l Y_h, fp32 accumulation,
+// about 16 bits), Z K-major (A, m rows), Y MN-major (B, row k = landmark, 64
+// features); W stored in fp32 and as the bf16 operand of P W (128 bytes per
+// landmark row, 16-byte chunk c at c ^ (row & 7)).  All kThreads threads;
+// TMEM columns 0..63 of the block's allocation.
+template <int M>
+struct WSmem {
+  static constexpr int kAtoms = M > 64 ? M / 64 : 1;     // 128-byte K atoms of Z
+  static constexpr uint32_t ah = 0, al = ah + kAtoms * 16384u;
+  static constexpr uint32_t bh = al + kAtoms * 16384u, bl = bh + M * 128u;
+  static constexpr uint32_t bar = bl + M * 128u;
+  static constexpr uint32_t total = bar + 64u;
+};
+
+__device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+    l[e] = pack_bf16(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <int M>
+__device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh, uint32_t tmem,
+                                       const Abort &ab) {
+  using C = WSmem<M>;
+  const int t = threadIdx.x, warp = t >> 5;
+  uint64_t *bar = (uint64_t *)(smem + C::bar);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  const uint32_t s_ah = smem_u32(smem + C::ah), s_al = smem_u32(smem + C::al);
+  const uint32_t s_bh = smem_u32(smem + C::bh), s_bl = smem_u32(smem + C::bl);
+  {   // operands: 16-byte chunks of 8 values, split on the way in
+    constexpr int kZc = M * M / 8, kYc = M * 64 / 8;
+    const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
+    const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
+    for (int c = t; c < kZc + kYc; c += kThreads) {
+      float x[8];
+      const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
+      const float4 a = __ldcg(src), b = __ldcg(src + 1);
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      uint4 hi, lo;
+      split8(x, hi, lo);
+      if (c < kZc) {   // Z row i, K chunk kc (8 columns): atom kc / 8
+        const int i = c / (M / 8), kc = c % (M / 8);
+        const uint32_t off = (uint32_t)(kc >> 3) * 16384u + sw128_offset(i, kc & 7);
+        st_shared_v4(s_ah + off, hi.x, hi.y, hi.z, hi.w);
+        st_shared_v4(s_al + off, lo.x, lo.y, lo.z, lo.w);
+      } else {         // Y row k (landmark), feature chunk fc
+        const int k = (c - kZc) >> 3, fc = (c - kZc) & 7;
+        const uint32_t off = sw128_offset(k, fc);
+        st_shared_v4(s_bh + off, hi.x, hi.y, hi.z, hi.w);
+        st_shared_v4(s_bl + off, lo.x, lo.y, lo.z, lo.w);
+      }
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (t == 0) {
+    const uint32_t idesc = make_idesc(kFmtBF16, 128, 64, 0, 1);
+    auto da = [&](uint32_t base, int k) {
+      return make_sdesc(base + (uint32_t)(k >> 2) * 16384u + 32u * (k & 3), 16, 1024);
+    };
+    auto db = [&](uint32_t base, int k) { return make_sdesc(base + 2048u * k, 16, 1024); };
+#pragma unroll
+    for (int k = 0; k < M / 16; ++k) mma_bf16(tmem, da(s_ah, k), db(s_bh, k), idesc, k > 0);
+#pragma unroll
+    for (int k = 0; k < M / 16; ++k) mma_bf16(tmem, da(s_ah, k), db(s_bl, k), idesc, 1u);
+#pragma unroll
+    for (int k = 0; k < M / 16; ++k) mma_bf16(tmem, da(s_al, k), db(s_bh, k), idesc, 1u);
+    mma_commit(bar);
+  }
+  if (warp < 4) {
+    const int r = t;   // W row == TMEM lane
+    const bool done = mbar_wait(bar, 0, ab);
+    tc_fence_after();
+    float v[64];
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32, v + 32);
+    tmem_ld_wait();
+    if (done && r < M) {
+      float4 *wr = (float4 *)(prm.w + ((size_t)bh * M + r) * 64);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) wr[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      uint4 *op = (uint4 *)(prm.w_op + ((size_t)bh * M + r) * 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        op[c ^ (r & 7)] = make_uint4(pack_bf16(v[8 * c], v[8 * c + 1]),
+                                     pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                                     pack_bf16(v[8 * c + 4], v[8 * c + 5]),
+                                     pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0 && !*ab.flag) mbar_inval(bar);
+}
+
+template <int M>
+__host__ __device__ constexpr uint32_t smem_bytes() {
+  // pinv operands or B~ V buffers, then the merge / W scratch
+  constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
+  constexpr uint32_t body = pinv_smem<M>() > bv ? pinv_smem<M>() : bv;
+  constexpr uint32_t tail = MergeSmem<M>::total > WSmem<M>::total ? MergeSmem<M>::total
+                                                                  : WSmem<M>::total;
+  return 1024u + (body > tail ? body : tail);
+}
+
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+// Test builds only: a busy delay (bounded by the SM clock, waiting on
+// nothing) before a block reports its W input, so that the tests can make
+// either block the second to finish: 1 delays the pseudoinverse blocks, 2 the
+// Y-merging blocks.
+__device__ int g_test_w_order;
+__device__ __forceinline__ void test_delay(int side) {
+  if (g_test_w_order != side) return;
+  const long long t0 = clock64();
+  while (clock64() - t0 < 200000ll) {
+  }
+}
+#else
+__device__ __forceinline__ void test_delay(int) {}
+#endif
+
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-           const Params prm) {
+           const __grid_constant__ CUtensorMap map_q, const Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint32_t tmem_base;
@@ -473,9 +712,53 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     }
   } else {
     const int b = blockIdx.x - prm.BH;
-    bv_body<M>(&map_k, &map_v, prm, smem, b / prm.splits, b % prm.splits, tmem, true);
+    const int bh = b / prm.splits, split = b % prm.splits;
+    bv_body<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
+    // HBM is mostly idle from here until W is ready: bring this split's
+    // share of the head's Q rows into L2 for the output kernel (V's rows
+    // were just read and stay)
+    if (t == 0) {
+      const int tiles = (prm.n + 127) / 128;
+      const int t0 = (int)((long)split * tiles / prm.splits);
+      const int t1 = (int)((long)(split + 1) * tiles / prm.splits);
+      for (int i = t0; i < t1; ++i) tma_prefetch_l2_3d(&map_q, 0, i * 128, bh);
+    }
   }
   NYS_MARK(kTrMid, 2);
+  // hand-off: the last B~ V block of a head merges Y; the second of {that
+  // block, the pseudoinverse block} forms W.  Counters: count[bh] B~ V
+  // blocks done, count[BH + bh] W inputs (Z, Y) in global memory.
+  __shared__ uint32_t last;
+  __shared__ volatile uint32_t w_abort;
+  if (t == 0) w_abort = 0;
+  const int bh = is_pinv ? (int)blockIdx.x : (int)(blockIdx.x - prm.BH) / prm.splits;
+  __threadfence();
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0) {
+    test_delay(is_pinv ? 1 : 2);
+    last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
+  }
+  __syncthreads();
+  if (last) {
+    if (!is_pinv) {
+      __threadfence();
+      NYS_MARK(kTrMid, 3);
+      merge_y<M>(prm, smem, bh);
+      __threadfence();
+      __syncthreads();
+      NYS_MARK(kTrMid, 4);
+    }
+    if (t == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      NYS_MARK(kTrMid, 5);
+      tc_fence_after();
+      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err});
+      NYS_MARK(kTrMid, 6);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if ((t >> 5) == 1) {

@@ -14,7 +14,6 @@
 #include "sm100.cuh"
 #include "mid_tc.cuh"
 #include "out_tc.cuh"
-#include "wmerge.cuh"
 #include "bwd_simt.cuh"
 #include "gemm_tc.cuh"
 #include "stream_bf16.cuh"
@@ -98,7 +97,10 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.z = take(BH * m * m * 4);
   L.y = take(BH * m * d * 4);
   L.w = take(BH * m * d * 4);
-  L.err = take(256);   // the error word, zeroed by every call
+  // the error word, then two counters per head (B~ V blocks done, W inputs
+  // ready); all zeroed by every call
+  L.err = take(256 + BH * 8);
+  L.count = L.err + 256;
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
   L.py = take(BH * splits * m * d * 4);
@@ -329,8 +331,8 @@ bool make_map3(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uin
 }
 
 // launches of the bf16 path
-constexpr int kTcLaunches = 4;
-const char *kTcNames = "seg_means,mid_tc,w_merge,out_tc";
+constexpr int kTcLaunches = 3;
+const char *kTcNames = "seg_means,mid_tc,out_tc";
 
 template <int M>
 nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
@@ -361,13 +363,18 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
-  {   // pseudoinverse || B~ V
+  {   // pseudoinverse || B~ V, then the merge of Y and W = Z Y
     midtc::Params p;
     p.pinv = pinvtc::Params{qt, kt, z, err, iters, scale_log2};
     p.q_land = qt;
     p.pmax = pmax;
     p.psum = psum;
     p.py = py;
+    p.z = z;
+    p.y = y;
+    p.w = w;
+    p.w_op = (uint8_t *)(ws + L.w_bf);
+    p.count = (uint32_t *)(ws + L.count);
     p.err = err;
     p.lens = lens;
     p.heads = desc->heads;
@@ -380,17 +387,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     const uint32_t sm = midtc::smem_bytes<M>();
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH * (1 + L.splits)), dim3(midtc::kThreads),
-               launch_smem(mk.launched, sm), stream, true, mkk, mv, p) != cudaSuccess)
-      return NYS_ERR_CUDA;
-    mk.after(stream);
-  }
-  {   // merge of the B~ V partials, W = Z Y
-    const wmerge::Params p{pmax, psum, py, z, y, w, (uint8_t *)(ws + L.w_bf), L.splits};
-    auto kern = wmerge::wmerge_kernel<M>;
-    const uint32_t sm = wmerge::Smem<M>::total;
-    if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(BH * (M / wmerge::kRows)), dim3(wmerge::kThreads),
-               launch_smem(mk.launched, sm), stream, true, p) != cudaSuccess)
+               launch_smem(mk.launched, sm), stream, true, mkk, mv, mq, p) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -722,7 +719,13 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (clear_err && cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  const size_t nclear = clear_err ? 256 + (size_t)desc->batch * desc->heads * 8 : 0;
+  if (nclear && cudaMemsetAsync(ws + L.err, 0, nclear, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  // the layer clears the error word itself; the counters still start at zero
+  if (!clear_err &&
+      cudaMemsetAsync(ws + L.count, 0, (size_t)desc->batch * desc->heads * 8, stream) !=
+          cudaSuccess)
+    st = NYS_ERR_CUDA;
   mk.first(stream);
   if (st == NYS_OK) {
     if (desc->dtype == NYS_F32)
@@ -1171,6 +1174,7 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
 // Entry points of the test build only (not part of the product ABI):
 //  nys_test_fail_launch(idx)   the launch with index idx of the next forward
 //                              call is refused (see launch_smem);
+//  nys_test_w_order(mode)      which block of a head forms W (see below);
 //  nys_test_timeout_probe(...) one block waits on an mbarrier that nothing
 //                              completes, with a limit of limit_cycles SM
 //                              cycles; the bounded wait gives up, records
@@ -1178,6 +1182,15 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
 //                              the block returns.  No copy or MMA is in flight
 //                              when it gives up.
 NYS_ATTN_API void nys_test_fail_launch(int idx) { g_fail_launch = idx; }
+
+// nys_test_w_order(mode): 1 delays every pseudoinverse block, 2 every
+// Y-merging block, before it reports its W input (0: no delay), so that the
+// other one forms W.
+NYS_ATTN_API nys_status nys_test_w_order(int mode) {
+  return cudaMemcpyToSymbol(midtc::g_test_w_order, &mode, sizeof(int)) == cudaSuccess
+             ? NYS_OK
+             : NYS_ERR_CUDA;
+}
 
 NYS_ATTN_API nys_status nys_test_timeout_probe(void *workspace, const nys_desc *desc, int m,
                                                long long limit_cycles, nys_stream_t stream) {

@@ -42,6 +42,6 @@ __device__ __forceinline__ void trace_mark(uint32_t kernel, uint32_t event) {
 #endif
 
 // kernel ids of the marks
-enum : uint32_t { kTrSeg = 1, kTrMid = 2, kTrOut = 3, kTrW = 4 };
+enum : uint32_t { kTrSeg = 1, kTrMid = 2, kTrOut = 3 };
 
 }  // namespace nys

@@ -123,3 +123,38 @@ def test_bounded_wait_that_runs_out_reports_timeout_once():
     assert _forward(lib, Q, K, V, m, cw, out, ws.value, wsb.value) == 0
     assert lib.nys_attn_check_error(ws, ctypes.byref(desc), m, _stream()) == 0
     assert normwise(out.float().cpu().numpy().astype(np.float64), want) <= TOL[BF16]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["bert_n512_m64", "headline_n8192_m32", "sweep_n1024_m128"])
+def test_w_is_the_same_whichever_block_forms_it(name):
+    # W = Z Y is formed by the second of {the pseudoinverse block, the block
+    # that merges Y} to finish.  The test build delays one side or the other
+    # (a bounded busy delay), so each hand-off runs; both run the same
+    # function on the same inputs and must give the same bits.
+    from nystr_self_attention_segment_b200.inputs import WORKLOADS, make_inputs
+    t = torch()
+    lib = _test_lib()
+    lib.nys_test_w_order.restype = ctypes.c_int
+    lib.nys_test_w_order.argtypes = [ctypes.c_int]
+    wl = WORKLOADS[name]
+    x = make_inputs(wl, batch=1, heads=min(wl.heads, 4))
+    want, _, (Q, K, V, cw) = run(x, BF16, wl.landmarks)
+    desc = _lib.make_desc(_lib.NYS_BF16, *Q.shape)
+    wsb = ctypes.c_size_t(0)
+    assert lib.nys_attn_workspace_size(ctypes.byref(desc), wl.landmarks, ctypes.byref(wsb)) == 0
+    buf = t.zeros(wsb.value + 256, dtype=t.uint8, device="cuda")
+    ws = buf.data_ptr() + (-buf.data_ptr()) % 256
+    outs = []
+    try:
+        for mode in (1, 2, 0):
+            assert lib.nys_test_w_order(mode) == 0
+            out = t.empty_like(Q)
+            assert _forward(lib, Q, K, V, wl.landmarks, cw, out, ws, wsb.value) == 0
+            assert lib.nys_attn_check_error(ctypes.c_void_p(ws), ctypes.byref(desc),
+                                            wl.landmarks, _stream()) == 0
+            outs.append(out.float().cpu().numpy().astype(np.float64))
+    finally:
+        lib.nys_test_w_order(0)
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
+    assert np.array_equal(outs[2], want)
