@@ -582,16 +582,27 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
   }
   const uint32_t s_ah = smem_u32(smem + C::ah), s_al = smem_u32(smem + C::al);
   const uint32_t s_bh = smem_u32(smem + C::bh), s_bl = smem_u32(smem + C::bl);
-  {   // operands: 16-byte chunks of 8 values, split on the way in
+  {   // operands: 16-byte chunks of 8 values, every load issued before the
+      // first is used, split on the way in
     constexpr int kZc = M * M / 8, kYc = M * 64 / 8;
+    constexpr int kPer = (kZc + kYc + kThreads - 1) / kThreads;
     const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
     const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
-    for (int c = t; c < kZc + kYc; c += kThreads) {
-      float x[8];
-      const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
-      const float4 a = __ldcg(src), b = __ldcg(src + 1);
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-      x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    float4 va[kPer], vb[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int c = t + u * kThreads;
+      if (c < kZc + kYc) {
+        const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
+        va[u] = __ldcg(src);
+        vb[u] = __ldcg(src + 1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int c = t + u * kThreads;
+      if (c >= kZc + kYc) break;
+      const float x[8] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
       uint4 hi, lo;
       split8(x, hi, lo);
       if (c < kZc) {   // Z row i, K chunk kc (8 columns): atom kc / 8

@@ -311,6 +311,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     for (int i = wg; i < ntiles; i += 2) {
       const int u = i >> 1;
       if (!mbar_wait(&s_full[wg], u & 1, ab)) break;
+      if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 16 + u);
       tc_fence_after();
       float v[M];
 #pragma unroll
@@ -342,7 +343,9 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[wg]);
+      if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 24 + u);
       if (!mbar_wait(&o_full[wg], u & 1, ab)) break;
+      if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 32 + u);
       tc_fence_after();
       float o[64];
       tmem_ld32(t_s + M, o);
@@ -369,6 +372,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       if (r == 0) {
         tma_store_3d_hint(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh, last_use);
         bulk_commit();
+        if (blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 40 + u);
       }
     }
     if (r == 0) bulk_wait0();

@@ -61,14 +61,15 @@ struct Cfg {
   static constexpr int NC = M / 2;                  // columns per thread
   // 16-bit operands, K-major, one 128-byte swizzle row per matrix row (K = M
   // <= 64), each as a hi and a lo copy:
-  //   a2  [P2 ; P] fp16: rows 0..M-1 = P2, rows 64..64+M-1 = P; 64 rows of
-  //       slack after it because stage 1 reads 128 rows from row 64
-  //   u   U = 7P - P2 fp16: M rows
+  //   a2  [P2 ; P ; P] fp16: rows 0..M-1 = P2, rows 64..64+M-1 = P and rows
+  //       128..128+M-1 = P again (stage 1 reads 128 rows from row 64, so that
+  //       lanes 64.. of its result repeat lanes 0..)
+  //   u   U = 7P - P2 fp16: rows 0..M-1 and again 64..64+M-1
   //   az  Z bf16 at rows 64..64+M-1 (128 rows)
   //   br  r bf16: M rows, two buffers (by step parity: the Z update of a step
   //       reads r of the step before while the new r is written)
   //   q, k  landmark logits operands (bf16, 64 features)
-  static constexpr uint32_t kA2 = 192u * 128u, kU = 64u * 128u;
+  static constexpr uint32_t kA2 = 192u * 128u, kU = 128u * 128u;
   static constexpr uint32_t a2h = 0, a2l = a2h + kA2;
   static constexpr uint32_t uh = a2l + kA2, ul = uh + kU;
   static constexpr uint32_t azh = ul + kU, azl = azh + 128u * 128u;
@@ -94,27 +95,35 @@ struct Cfg {
 template <int N, bool F16>
 __device__ __forceinline__ void put_split(uint32_t hi_base, uint32_t lo_base, int row, int c0,
                                           const float *v, bool with_lo = true) {
+  // with_lo is uniform over the block: the lo halves are formed only when
+  // they are stored
 #pragma unroll
   for (int q = 0; q < N / 8; ++q) {
-    uint32_t h[4], l[4];
+    uint32_t h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = v[8 * q + 2 * e], x1 = v[8 * q + 2 * e + 1];
+      h[e] = F16 ? pack_f16(x0, x1) : pack_bf16(x0, x1);
+    }
+    const uint32_t off = sw128_offset(row, (c0 >> 3) + q);
+    st_shared_v4(hi_base + off, h[0], h[1], h[2], h[3]);
+  }
+  if (!with_lo) return;
+#pragma unroll
+  for (int q = 0; q < N / 8; ++q) {
+    uint32_t l[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float x0 = v[8 * q + 2 * e], x1 = v[8 * q + 2 * e + 1];
       if constexpr (F16) {
-        const __half2 hh = __floats2half2_rn(x0, x1);
-        const float2 hf = __half22float2(hh);
-        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+        const float2 hf = __half22float2(__floats2half2_rn(x0, x1));
         l[e] = pack_f16(x0 - hf.x, x1 - hf.y);
       } else {
-        const __nv_bfloat162 hh = __floats2bfloat162_rn(x0, x1);
-        const float2 hf = __bfloat1622float2(hh);
-        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+        const float2 hf = __bfloat1622float2(__floats2bfloat162_rn(x0, x1));
         l[e] = pack_bf16(x0 - hf.x, x1 - hf.y);
       }
     }
-    const uint32_t off = sw128_offset(row, (c0 >> 3) + q);
-    st_shared_v4(hi_base + off, h[0], h[1], h[2], h[3]);
-    if (with_lo) st_shared_v4(lo_base + off, l[0], l[1], l[2], l[3]);
+    st_shared_v4(lo_base + sw128_offset(row, (c0 >> 3) + q), l[0], l[1], l[2], l[3]);
   }
 }
 
@@ -145,8 +154,10 @@ template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
   if constexpr (N == 32) {
     tmem_ld32(taddr, v);
-  } else {
+  } else if constexpr (N == 16) {
     tmem_ld16(taddr, v);
+  } else {
+    tmem_ld8(taddr, v);
   }
   tmem_ld_wait();
 }
@@ -170,6 +181,13 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
   const bool aux = rows && r >= 64 && r < 64 + M;   // Z update rows
   const int row = crit ? r : r - 64;             // matrix row of this thread
   const int c_lo = h * NC;
+  // the P chain's elementwise work: the results of stages 1 and 2 repeat in
+  // lanes 64.. (their A operands hold every row twice), so four threads share
+  // each row, a quarter of its columns each
+  constexpr int NQ = M / 4;
+  const bool pc = rows && (r & 63) < M;
+  const int prow = r & 63;
+  const int cq = ((r >> 6) * 2 + h) * NQ;
   uint64_t *bar_main = (uint64_t *)(smem + C::bars);
   uint64_t *bar_z = bar_main + 1;
   uint32_t *tmem_slot = (uint32_t *)(bar_main + 2);
@@ -220,6 +238,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       const float k[8] = {kv[i][0].x, kv[i][0].y, kv[i][0].z, kv[i][0].w,
                           kv[i][1].x, kv[i][1].y, kv[i][1].z, kv[i][1].w};
       put_split<8, false>(qh, ql, rr, ch * 8, q);
+      put_split<8, false>(qh, ql, 64 + rr, ch * 8, q);   // logits repeat in lanes 64..
       put_split<8, false>(kh, kl, rr, ch * 8, k);
     }
   }
@@ -280,34 +299,48 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     mma3(tmem, sd(qh), sd(ql), sd(kh), sd(kl), id_bf, K64{}, true);
     mma_commit(bar_main);
   }
-  wait_main(crit && h == 0);
-  // ---- row softmax (one thread per row): A rows -> split fp16 operand at
-  //      row 64 (the P position, for A A^T) and an fp32 copy; row sums of |A|
-  if (ok && crit && h == 0) {
-    float v[M];
+  wait_main(pc);
+  // ---- row softmax, four threads per row (a quarter of the columns each;
+  //      the row's maximum and sum combine the quarters in order through
+  //      shared memory): A into the split fp16 operand at rows 64.. and
+  //      128.. of a2 (the P position, twice, for A A^T) and an fp32 copy;
+  //      quarter row sums of |A|
+  float* red4 = p2f;   // [3][4][64]: maxima, sums, |A| sums (logits operands are dead)
+  const int qi = cq / NQ;
+  float av[NQ];
+  if (ok && pc) {
+    ld_cols<NQ>(t_d + cq, av);
+    float mx = av[0];
 #pragma unroll
-    for (int c = 0; c < M; c += 32) tmem_ld32(t_d + c, v + c);
-    tmem_ld_wait();
-    float mx[4] = {v[0], v[1], v[2], v[3]};
+    for (int k = 1; k < NQ; ++k) mx = fmaxf(mx, av[k]);
+    red4[qi * 64 + prow] = mx;
+  }
+  named_barrier(1, kBarThreads);
+  if (ok && pc) {
+    const float moff = fmaxf(fmaxf(red4[prow], red4[64 + prow]),
+                             fmaxf(red4[128 + prow], red4[192 + prow])) * prm.scale_log2;
+    float sm = 0.f;
 #pragma unroll
-    for (int j = 4; j < M; ++j) mx[j & 3] = fmaxf(mx[j & 3], v[j]);
-    const float moff = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * prm.scale_log2;
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < M; ++j) {
-      v[j] = fast_exp2(fmaf(v[j], prm.scale_log2, -moff));
-      s[j & 3] += v[j];
+    for (int k = 0; k < NQ; ++k) {
+      av[k] = fast_exp2(fmaf(av[k], prm.scale_log2, -moff));
+      sm += av[k];
     }
-    const float inv = 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
-    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+    red4[256 + qi * 64 + prow] = sm;
+  }
+  named_barrier(1, kBarThreads);
+  if (ok && pc) {
+    const float inv = 1.f / (((red4[256 + prow] + red4[320 + prow]) + red4[384 + prow]) +
+                             red4[448 + prow]);
+    float rs = 0.f;
 #pragma unroll
-    for (int j = 0; j < M; ++j) {
-      v[j] *= inv;
-      rs[j & 3] += fabsf(v[j]);
+    for (int k = 0; k < NQ; ++k) {
+      av[k] *= inv;
+      rs += fabsf(av[k]);
     }
-    red[r] = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-    put_split<M, true>(ph, pl, r, 0, v);
-    put_row<M>(pf0, r, 0, v);
+    red4[512 + qi * 64 + prow] = rs;
+    put_split<NQ, true>(ph, pl, prow, cq, av);
+    put_split<NQ, true>(ph, pl, 64 + prow, cq, av);
+    put_row<NQ>(pf0, prow, cq, av);
   }
   if (!sync_ops()) ok = false;
   NYS_MARK(kTrMid, 8);
@@ -332,7 +365,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
 #pragma unroll 8
   for (int i = 0; i < M; ++i) {
     n1 = fmaxf(n1, red[M + i] + red[2 * M + i]);
-    ninf = fmaxf(ninf, red[i]);
+    ninf = fmaxf(ninf, ((red4[512 + i] + red4[576 + i]) + red4[640 + i]) + red4[704 + i]);
   }
   const float c0 = 1.f / (n1 * ninf);
   if (ok && aux) {   // Z0 = c0 A^T, rows 64.. of the Z operand
@@ -347,14 +380,15 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       put_split<NC, false>(azh, azl, 64 + row, c_lo, acol);
     }
   }
-  wait_main(crit);
-  // P_j of this thread's row and columns stays in registers through the steps
-  float preg[NC];
-  if (ok && crit) {   // P0 = c0 A A^T
-    ld_cols<NC>(t_d + c_lo, preg);
+  wait_main(pc);
+  // P_j of this thread's row quarter stays in registers through the steps
+  float preg[NQ];
+  if (ok && pc) {   // P0 = c0 A A^T
+    ld_cols<NQ>(t_d + cq, preg);
 #pragma unroll
-    for (int k = 0; k < NC; ++k) preg[k] *= c0;
-    put_split<NC, true>(ph, pl, row, c_lo, preg);
+    for (int k = 0; k < NQ; ++k) preg[k] *= c0;
+    put_split<NQ, true>(ph, pl, prow, cq, preg);
+    put_split<NQ, true>(ph, pl, 64 + prow, cq, preg);
   }
   if (!sync_ops()) ok = false;
   NYS_MARK(kTrMid, 9);
@@ -388,16 +422,17 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
         put_split<NC, false>(azh, azl, 64 + row, c_lo, z);
       }
     }
-    wait_main(crit);
+    wait_main(pc);
     if (j < 8) NYS_MARK(kTrMid, 40 + j);
-    float p2[NC];
-    if (ok && crit) {
-      float uu[NC];
-      ld_cols<NC>(t_d + c_lo, p2);
+    float p2[NQ];
+    if (ok && pc) {
+      float uu[NQ];
+      ld_cols<NQ>(t_d + cq, p2);
 #pragma unroll
-      for (int k = 0; k < NC; ++k) uu[k] = fmaf(7.f, preg[k], -p2[k]);
-      put_split<NC, true>(a2h, a2l, row, c_lo, p2, split);
-      put_split<NC, true>(uh, ul, row, c_lo, uu, split);
+      for (int k = 0; k < NQ; ++k) uu[k] = fmaf(7.f, preg[k], -p2[k]);
+      put_split<NQ, true>(a2h, a2l, prow, cq, p2, split);
+      put_split<NQ, true>(uh, ul, prow, cq, uu, split);
+      put_split<NQ, true>(uh, ul, 64 + prow, cq, uu, split);
     }
     if (!sync_ops()) {
       good = false;
@@ -413,25 +448,23 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
         mma_commit(bar_z);
       }
     }
-    wait_main(crit);
+    wait_main(pc);
     if (j < 8) NYS_MARK(kTrMid, 48 + j);
-    if (ok && crit) {
+    if (ok && pc) {
       // P_{j+1} = 1/4 (13 P - 15 P2 + 7 P^3 - P^4), r_j = 1/4 (13I - 15 P + 7 P^2 - P^3)
-      float x[NC], y[NC];
-      tmem_ld16(t_d + c_lo, x);
-      if constexpr (NC == 32) tmem_ld16(t_d + c_lo + 16, x + 16);
-      tmem_ld16(t_d + 64 + c_lo, y);
-      if constexpr (NC == 32) tmem_ld16(t_d + 64 + c_lo + 16, y + 16);
-      tmem_ld_wait();
+      float x[NQ], y[NQ];
+      ld_cols<NQ>(t_d + cq, x);
+      ld_cols<NQ>(t_d + 64 + cq, y);
 #pragma unroll
-      for (int k = 0; k < NC; ++k) {
+      for (int k = 0; k < NQ; ++k) {
         const float pj = preg[k];
         preg[k] = 0.25f * fmaf(13.f, pj, fmaf(-15.f, p2[k], x[k]));
-        y[k] = 0.25f * ((c_lo + k == row ? 13.f : 0.f) + fmaf(-15.f, pj, y[k]));
+        y[k] = 0.25f * ((cq + k == prow ? 13.f : 0.f) + fmaf(-15.f, pj, y[k]));
       }
-      put_split<NC, true>(ph, pl, row, c_lo, preg, split_next);
+      put_split<NQ, true>(ph, pl, prow, cq, preg, split_next);
+      put_split<NQ, true>(ph, pl, 64 + prow, cq, preg, split_next);
       const uint32_t rb = (j & 1) * kBr;
-      put_split<NC, false>(brh + rb, brl + rb, row, c_lo, y);
+      put_split<NQ, false>(brh + rb, brl + rb, prow, cq, y);
     }
     if (j < 8) NYS_MARK(kTrMid, 16 + j);
     if (!sync_ops()) {
