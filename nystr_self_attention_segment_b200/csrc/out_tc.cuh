@@ -108,7 +108,14 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   // Q and V are read here for the last time in the pass and out is not read
   // again: their lines leave L2 first
   const uint64_t last_use = policy_evict_first();
-  constexpr uint32_t kStride = M + 64;        // TMEM columns per softmax warpgroup
+  // TMEM per softmax warpgroup: S (M columns), P (M / 2 columns of bf16
+  // pairs; m <= 64 only, else P is written over S) and O (64 columns).  With
+  // P in its own columns the next tile's S can go out as soon as this tile's
+  // S has been read.
+  constexpr bool kSepP = M <= 64;
+  constexpr uint32_t kPcol = kSepP ? M : 0;
+  constexpr uint32_t kOcol = kSepP ? M + M / 2 : M;
+  constexpr uint32_t kStride = kOcol + 64;    // TMEM columns per softmax warpgroup
   constexpr uint32_t kT = 2 * kStride;        // Toeplitz operand columns
 
   uint64_t *bars = (uint64_t *)(smem + L.bars);
@@ -120,7 +127,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   uint64_t *tm_free = o_full + 2;
   uint64_t *w_ready = tm_free + 2;         // W operand in shared memory
   uint64_t *v_ready = w_ready + 1;         // [kStages] V tile masked past L
-  uint32_t *tmem_slot = (uint32_t *)(v_ready + kStages);
+  uint64_t *s_free = v_ready + kStages;    // [2] S of the tile read (P in its own columns)
+  uint32_t *tmem_slot = (uint32_t *)(s_free + 2);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
   float *cw = (float *)(smem + L.cw);
@@ -139,6 +147,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     }
     mbar_init(w_ready, 1);
     for (int s = 0; s < kStages; ++s) mbar_init(&v_ready[s], 1);
+    mbar_init(&s_free[0], 128);
+    mbar_init(&s_free[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(map_q);
@@ -287,19 +297,23 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
           tc_fence_after();
           const uint32_t v_a = smem_u32(smem + L.v[s]);
           for (int k = 0; k < prm.kconv / 16; ++k)
-            mma_bf16_ts(tmem + w * kStride + M, tmem + kT + 8 * k,
+            mma_bf16_ts(tmem + w * kStride + kOcol, tmem + kT + 8 * k,
                         make_sdesc(v_a + k * 2048u, 16, 1024), id_o, k > 0);
         }
         mma_commit(&empty[s]);
+        if (kSepP && i + 2 < ntiles) {   // the next S once this S has been read
+          if (!mbar_wait(&s_free[w], u & 1, ab)) break;
+          if (!(ok = issue_s(i + 2))) break;
+        }
         if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
         if (u == 0 && !mbar_wait(w_ready, 0, ab)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < M / 16; ++k)
-          mma_bf16_ts(tmem + w * kStride + M, tmem + w * kStride + 8 * k,
+          mma_bf16_ts(tmem + w * kStride + kOcol, tmem + w * kStride + kPcol + 8 * k,
                       make_sdesc(w_a + k * 2048u, 16, 1024), id_o, (conv || k > 0) ? 1u : 0u);
         mma_commit(&o_full[w]);
-        if (i + 2 < ntiles) ok = issue_s(i + 2);
+        if (!kSepP && i + 2 < ntiles) ok = issue_s(i + 2);
       }
     }
   } else if (warp >= 4) {
@@ -317,6 +331,10 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 #pragma unroll
       for (int c = 0; c < M; c += 32) tmem_ld32(t_s + c, v + c);
       tmem_ld_wait();
+      if (kSepP) {   // S may be overwritten by the next tile's S from here on
+        tc_fence_before();
+        mbar_arrive(&s_free[wg]);
+      }
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = v[q];
@@ -339,7 +357,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 #pragma unroll
       for (int c = 0; c < M; c += 2) pk[c >> 1] = pack_bf16(v[c] * inv, v[c + 1] * inv);
 #pragma unroll
-      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + c, pk + c);
+      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + kPcol + c, pk + c);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[wg]);
@@ -348,8 +366,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 32 + u);
       tc_fence_after();
       float o[64];
-      tmem_ld32(t_s + M, o);
-      tmem_ld32(t_s + M + 32, o + 32);
+      tmem_ld32(t_s + kOcol, o);
+      tmem_ld32(t_s + kOcol + 32, o + 32);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&tm_free[wg]);
@@ -380,7 +398,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && !*abort_flag)
-    for (int b = 0; b < 3 * kStages + 9; ++b) mbar_inval(bars + b);
+    for (int b = 0; b < 3 * kStages + 11; ++b) mbar_inval(bars + b);
   if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
