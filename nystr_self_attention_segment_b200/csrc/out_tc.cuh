@@ -17,7 +17,8 @@
 //   softmax warpgroup: row softmax of S (one TMEM lane = one row); P (the F~
 //        tile, bf16) written into TMEM over S,
 //   MMA  O += P W                   (M=128, N=64, K=m; P read from TMEM),
-//   softmax warpgroup: O -> bf16 -> shared memory -> TMA store (clipped at n).
+//   softmax warpgroup: O -> bf16 -> global memory, one 128-byte row per thread
+//        (rows past n are not stored).
 // Two softmax warpgroups take alternate tiles.
 // Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
 // warp 1 owns TMEM), 4-7 and 8-11 softmax + epilogue.  TMEM: warpgroup w has
@@ -38,7 +39,7 @@ constexpr int kTileRows = 128;
 constexpr int kMaxKconv = 192;
 
 struct SmemLayout {
-  uint32_t kt, w, q[kStages], v[kStages], o[2], cw, bars, total;
+  uint32_t kt, w, q[kStages], v[kStages], cw, bars, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
@@ -55,8 +56,6 @@ __host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
     L.q[s] = take(16384u);
     L.v[s] = take(kconv * 128u);
   }
-  L.o[0] = take(16384u);
-  L.o[1] = take(16384u);
   L.cw = take(256u);
   L.bars = take(256u);
   L.total = off + 1024u;   // slack for aligning the dynamic smem base to 1 KB
@@ -68,6 +67,7 @@ struct Params {
   const uint8_t *w_op;     // [BH][m][128 B]: W as the bf16 B operand of P W
                            // (row j = landmark, 64 features, 128-byte swizzle)
   const float *conv_w;     // [H][k] or null
+  __nv_bfloat16 *out;      // [BH][n][64]
   uint32_t *err;
   int n, heads, conv_k, kconv;
   int tiles_per_head, ctas_per_head;
@@ -85,7 +85,7 @@ template <int M>
 // kStages tile loads) runs before the wait for the previous kernel, the K~ /
 // W operand loads after it.
 __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtensorMap *map_v,
-                                         const CUtensorMap *map_o, const Params &prm,
+                                         const Params &prm,
                                          uint8_t *smem, int bh, int t_begin, int t_end,
                                          uint32_t tmem_in, bool wait_prev = false) {
   const SmemLayout L = smem_layout(M, prm.kconv);
@@ -152,7 +152,6 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(map_q);
-    tma_prefetch_desc(map_o);
     if (conv) tma_prefetch_desc(map_v);
   }
   if (tmem_in != ~0u) {
@@ -372,28 +371,23 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       tc_fence_before();
       mbar_arrive(&tm_free[wg]);
       if (threadIdx.x == 128 && u < 4) NYS_MARK_T(kTrOut, 8 + u);
-      // this warpgroup's staging buffer was last used two of its tiles ago
-      if (r == 0) bulk_wait_read0();
-      named_barrier(2 + wg, 128);
-      if ((t_begin + i) * kTileRows + r >= seq) {   // padding rows of a ragged element
+      // the row straight from registers to global memory: 128 bytes per
+      // thread, rows past n are not stored, padding rows of a ragged element
+      // are zero
+      const int grow = (t_begin + i) * kTileRows + r;
+      if (grow < prm.n) {
+        const bool pad = grow >= seq;
+        uint8_t *dst = (uint8_t *)(prm.out + ((size_t)bh * prm.n + grow) * 64);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = 0.f;
+        for (int c = 0; c < 8; ++c)
+          st_global_v4_hint(dst + 16 * c, pad ? 0u : pack_bf16(o[8 * c], o[8 * c + 1]),
+                            pad ? 0u : pack_bf16(o[8 * c + 2], o[8 * c + 3]),
+                            pad ? 0u : pack_bf16(o[8 * c + 4], o[8 * c + 5]),
+                            pad ? 0u : pack_bf16(o[8 * c + 6], o[8 * c + 7]), last_use);
       }
-      const uint32_t o_row = smem_u32(smem + L.o[wg]);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(o_row + sw128_offset(r, c), pack_bf16(o[8 * c], o[8 * c + 1]),
-                     pack_bf16(o[8 * c + 2], o[8 * c + 3]), pack_bf16(o[8 * c + 4], o[8 * c + 5]),
-                     pack_bf16(o[8 * c + 6], o[8 * c + 7]));
-      fence_async_smem();
-      named_barrier(2 + wg, 128);
-      if (r == 0) {
-        tma_store_3d_hint(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh, last_use);
-        bulk_commit();
-        if (blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 40 + u);
-      }
+      if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 40 + u);
     }
-    if (r == 0) bulk_wait0();
+
   }
   tc_fence_before();
   __syncthreads();
@@ -409,7 +403,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
-              const __grid_constant__ CUtensorMap map_o, const Params prm) {
+              const Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int bh = blockIdx.x / prm.ctas_per_head;
@@ -418,7 +412,7 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
   // launched early (programmatic dependent launch): out_body waits for the
   // previous kernels before it reads K~ and W
-  out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u, true);
+  out_body<M>(&map_q, &map_v, prm, smem, bh, t_begin, t_end, ~0u, true);
 }
 
 }  // namespace outtc

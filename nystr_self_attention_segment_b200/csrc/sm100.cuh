@@ -149,6 +149,14 @@ __device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap *m, const vo
       "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
+// 16-byte global store with an L2 policy (e.g. evict-first for output that
+// is not read again in the pass).
+__device__ __forceinline__ void st_global_v4_hint(void *p, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(a),
+               "r"(b), "r"(c), "r"(d), "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *src, int x, int y,
                                              int z) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::
