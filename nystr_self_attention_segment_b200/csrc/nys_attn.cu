@@ -350,9 +350,10 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
   const bool conv = conv_w != nullptr;
   const int kconv = conv ? ((128 + conv_k - 1 + 15) / 16) * 16 : 0;
 
-  CUtensorMap mq, mkk, mv, mvh;
+  CUtensorMap mq, mkk, mv, mvh, mo;
   if (!make_map(&mq, Q, BH, n, 128) || !make_map(&mkk, K, BH, n, 128) ||
-      !make_map(&mv, V, BH, n, 128) || !make_map(&mvh, V, BH, n, conv ? kconv : 128))
+      !make_map(&mv, V, BH, n, 128) || !make_map(&mvh, V, BH, n, conv ? kconv : 128) ||
+      !make_map(&mo, out, BH, n, 128))
     return NYS_ERR_CUDA;
 
   {   // segment means of Q and K (Eq. 16)
@@ -395,13 +396,14 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     int cpb = kNumSms / BH;
     if (cpb < 1) cpb = 1;
     if (cpb > tph) cpb = tph;
-    outtc::Params p{kt,  (const uint8_t *)(ws + L.w_bf), conv_w, out, err, n, desc->heads,
+    outtc::Params p{kt,  (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads,
                     conv ? conv_k : 1, kconv, tph, cpb, scale_log2, lens, M};
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(BH * cpb), dim3(outtc::kThreads), launch_smem(mk.launched, sm), stream,
-               true, mq, mvh, p) != cudaSuccess)
+        launch(kern, dim3(BH * cpb), dim3(outtc::Warps<M>::kThreads), launch_smem(mk.launched, sm),
+               stream,
+               true, mq, mvh, mo, p) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }

@@ -17,8 +17,7 @@
 //   softmax warpgroup: row softmax of S (one TMEM lane = one row); P (the F~
 //        tile, bf16) written into TMEM over S,
 //   MMA  O += P W                   (M=128, N=64, K=m; P read from TMEM),
-//   softmax warpgroup: O -> bf16 -> global memory, one 128-byte row per thread
-//        (rows past n are not stored).
+//   softmax warpgroup: O -> bf16 -> shared memory -> TMA store (clipped at n).
 // Two softmax warpgroups take alternate tiles.
 // Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
 // warp 1 owns TMEM), 4-7 and 8-11 softmax + epilogue.  TMEM: warpgroup w has
@@ -33,13 +32,24 @@ namespace outtc {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
 constexpr int kStages = 4;
+
+// Softmax warpgroups per block (tiles in flight): three for m <= 64, two for
+// m = 128 (TMEM holds S and O of each, plus the Toeplitz operand).  Warps: 0
+// TMA producer, 1..NW MMA issuers (one per softmax warpgroup; warp 1 owns
+// TMEM), 4.. the softmax warpgroups, kLoader the W operand copy and the
+// ragged-batch masking.
+template <int M>
+struct Warps {
+  static constexpr int NW = M <= 64 ? 3 : 2;
+  static constexpr int kLoader = NW == 3 ? 4 + 4 * NW : 3;
+  static constexpr int kThreads = NW == 3 ? 32 * (kLoader + 1) : 384;
+};
 constexpr int kTileRows = 128;
 constexpr int kMaxKconv = 192;
 
 struct SmemLayout {
-  uint32_t kt, w, q[kStages], v[kStages], cw, bars, total;
+  uint32_t kt, w, q[kStages], v[kStages], o[3], cw, bars, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
@@ -56,6 +66,8 @@ __host__ __device__ inline SmemLayout smem_layout(int m, int kconv) {
     L.q[s] = take(16384u);
     L.v[s] = take(kconv * 128u);
   }
+  // an output staging tile per softmax warpgroup (three for m <= 64)
+  for (int w = 0; w < 3; ++w) L.o[w] = w < (m <= 64 ? 3 : 2) ? take(16384u) : 0u;
   L.cw = take(256u);
   L.bars = take(256u);
   L.total = off + 1024u;   // slack for aligning the dynamic smem base to 1 KB
@@ -67,7 +79,6 @@ struct Params {
   const uint8_t *w_op;     // [BH][m][128 B]: W as the bf16 B operand of P W
                            // (row j = landmark, 64 features, 128-byte swizzle)
   const float *conv_w;     // [H][k] or null
-  __nv_bfloat16 *out;      // [BH][n][64]
   uint32_t *err;
   int n, heads, conv_k, kconv;
   int tiles_per_head, ctas_per_head;
@@ -85,7 +96,7 @@ template <int M>
 // kStages tile loads) runs before the wait for the previous kernel, the K~ /
 // W operand loads after it.
 __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtensorMap *map_v,
-                                         const Params &prm,
+                                         const CUtensorMap *map_o, const Params &prm,
                                          uint8_t *smem, int bh, int t_begin, int t_end,
                                          uint32_t tmem_in, bool wait_prev = false) {
   const SmemLayout L = smem_layout(M, prm.kconv);
@@ -108,27 +119,24 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   // Q and V are read here for the last time in the pass and out is not read
   // again: their lines leave L2 first
   const uint64_t last_use = policy_evict_first();
-  // TMEM per softmax warpgroup: S (M columns), P (M / 2 columns of bf16
-  // pairs; m <= 64 only, else P is written over S) and O (64 columns).  With
-  // P in its own columns the next tile's S can go out as soon as this tile's
-  // S has been read.
-  constexpr bool kSepP = M <= 64;
-  constexpr uint32_t kPcol = kSepP ? M : 0;
-  constexpr uint32_t kOcol = kSepP ? M + M / 2 : M;
+  // TMEM per softmax warpgroup: S (M columns, P written over it as bf16
+  // pairs) and O (64 columns); the Toeplitz operand after them.
+  constexpr int NW = Warps<M>::NW, kThreads = Warps<M>::kThreads;
+  constexpr uint32_t kOcol = M;
   constexpr uint32_t kStride = kOcol + 64;    // TMEM columns per softmax warpgroup
-  constexpr uint32_t kT = 2 * kStride;        // Toeplitz operand columns
+  constexpr uint32_t kT = NW * kStride;       // Toeplitz operand columns
+  static_assert(kT + kMaxKconv / 2 <= 512, "TMEM");
 
   uint64_t *bars = (uint64_t *)(smem + L.bars);
   uint64_t *full = bars;                   // [kStages]
   uint64_t *empty = bars + kStages;        // [kStages]
-  uint64_t *s_full = bars + 2 * kStages;   // [2] per softmax warpgroup
-  uint64_t *p_ready = s_full + 2;
-  uint64_t *o_full = p_ready + 2;
-  uint64_t *tm_free = o_full + 2;
-  uint64_t *w_ready = tm_free + 2;         // W operand in shared memory
+  uint64_t *s_full = bars + 2 * kStages;   // [NW] per softmax warpgroup
+  uint64_t *p_ready = s_full + NW;
+  uint64_t *o_full = p_ready + NW;
+  uint64_t *tm_free = o_full + NW;
+  uint64_t *w_ready = tm_free + NW;        // W operand in shared memory
   uint64_t *v_ready = w_ready + 1;         // [kStages] V tile masked past L
-  uint64_t *s_free = v_ready + kStages;    // [2] S of the tile read (P in its own columns)
-  uint32_t *tmem_slot = (uint32_t *)(s_free + 2);
+  uint32_t *tmem_slot = (uint32_t *)(v_ready + kStages);
   volatile uint32_t *abort_flag = tmem_slot + 1;
   const Abort ab{abort_flag, prm.err};
   float *cw = (float *)(smem + L.cw);
@@ -139,7 +147,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NW; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_ready[b], 128);
       mbar_init(&o_full[b], 1);
@@ -147,11 +155,10 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     }
     mbar_init(w_ready, 1);
     for (int s = 0; s < kStages; ++s) mbar_init(&v_ready[s], 1);
-    mbar_init(&s_free[0], 128);
-    mbar_init(&s_free[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(map_q);
+    tma_prefetch_desc(map_o);
     if (conv) tma_prefetch_desc(map_v);
   }
   if (tmem_in != ~0u) {
@@ -221,13 +228,13 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   __syncthreads();
   tc_fence_after();
   NYS_MARK(kTrOut, 1);
-  if (warp == 3 && lane == 0) {
+  if (warp == Warps<M>::kLoader && lane == 0) {
     if (wait_prev) griddep_wait();
     NYS_MARK_T(kTrOut, 2);
     mbar_expect_tx(w_ready, M * 128u);
     bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
   }
-  if (warp == 3 && mask_v) {
+  if (warp == Warps<M>::kLoader && mask_v) {
     // ragged batches: halo rows at or past L of every staged V tile become
     // zero before its conv MMA (v_ready); tiles are taken in order, each
     // after its load, so the barrier phases cannot run ahead
@@ -262,7 +269,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       for (int i = ntiles > kStages ? ntiles - kStages : 0; i < ntiles; ++i)
         if (!mbar_wait(&empty[i % kStages], (i / kStages) & 1, ab)) break;
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp >= 1 && warp <= NW) {
     // ------------------------------------------------------------ MMA issuers
     // one per softmax warpgroup, so that neither waits behind the other
     if (lane == 0) {
@@ -287,8 +294,8 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
         return true;
       };
       bool ok = w < ntiles ? issue_s(w) : true;
-      for (int i = w; i < ntiles && ok; i += 2) {
-        const int s = i % kStages, u = i >> 1;
+      for (int i = w; i < ntiles && ok; i += NW) {
+        const int s = i % kStages, u = i / NW;
         if (!mbar_wait(&tm_free[w], (u & 1) ^ 1, ab)) break;
         tc_fence_after();
         if (conv) {
@@ -300,29 +307,25 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
                         make_sdesc(v_a + k * 2048u, 16, 1024), id_o, k > 0);
         }
         mma_commit(&empty[s]);
-        if (kSepP && i + 2 < ntiles) {   // the next S once this S has been read
-          if (!mbar_wait(&s_free[w], u & 1, ab)) break;
-          if (!(ok = issue_s(i + 2))) break;
-        }
         if (!mbar_wait(&p_ready[w], u & 1, ab)) break;
         if (u == 0 && !mbar_wait(w_ready, 0, ab)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < M / 16; ++k)
-          mma_bf16_ts(tmem + w * kStride + kOcol, tmem + w * kStride + kPcol + 8 * k,
+          mma_bf16_ts(tmem + w * kStride + kOcol, tmem + w * kStride + 8 * k,
                       make_sdesc(w_a + k * 2048u, 16, 1024), id_o, (conv || k > 0) ? 1u : 0u);
         mma_commit(&o_full[w]);
-        if (!kSepP && i + 2 < ntiles) ok = issue_s(i + 2);
+        if (i + NW < ntiles) ok = issue_s(i + NW);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + 4 * NW) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int wg = warp >= 8 ? 1 : 0;
+    const int wg = (warp - 4) >> 2;
     const int r = threadIdx.x & 127;                 // tile row == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_base + wg * kStride;
-    for (int i = wg; i < ntiles; i += 2) {
-      const int u = i >> 1;
+    for (int i = wg; i < ntiles; i += NW) {
+      const int u = i / NW;
       if (!mbar_wait(&s_full[wg], u & 1, ab)) break;
       if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 16 + u);
       tc_fence_after();
@@ -330,10 +333,6 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 #pragma unroll
       for (int c = 0; c < M; c += 32) tmem_ld32(t_s + c, v + c);
       tmem_ld_wait();
-      if (kSepP) {   // S may be overwritten by the next tile's S from here on
-        tc_fence_before();
-        mbar_arrive(&s_free[wg]);
-      }
       float mx[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) mx[q] = v[q];
@@ -356,7 +355,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 #pragma unroll
       for (int c = 0; c < M; c += 2) pk[c >> 1] = pack_bf16(v[c] * inv, v[c + 1] * inv);
 #pragma unroll
-      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + kPcol + c, pk + c);
+      for (int c = 0; c < M / 2; c += 16) tmem_st16(t_s + c, pk + c);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[wg]);
@@ -371,28 +370,34 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       tc_fence_before();
       mbar_arrive(&tm_free[wg]);
       if (threadIdx.x == 128 && u < 4) NYS_MARK_T(kTrOut, 8 + u);
-      // the row straight from registers to global memory: 128 bytes per
-      // thread, rows past n are not stored, padding rows of a ragged element
-      // are zero
-      const int grow = (t_begin + i) * kTileRows + r;
-      if (grow < prm.n) {
-        const bool pad = grow >= seq;
-        uint8_t *dst = (uint8_t *)(prm.out + ((size_t)bh * prm.n + grow) * 64);
+      // this warpgroup's staging buffer was last used NW tiles ago
+      if (r == 0) bulk_wait_read0();
+      named_barrier(2 + wg, 128);
+      if ((t_begin + i) * kTileRows + r >= seq) {   // padding rows of a ragged element
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_global_v4_hint(dst + 16 * c, pad ? 0u : pack_bf16(o[8 * c], o[8 * c + 1]),
-                            pad ? 0u : pack_bf16(o[8 * c + 2], o[8 * c + 3]),
-                            pad ? 0u : pack_bf16(o[8 * c + 4], o[8 * c + 5]),
-                            pad ? 0u : pack_bf16(o[8 * c + 6], o[8 * c + 7]), last_use);
+        for (int c = 0; c < 64; ++c) o[c] = 0.f;
+      }
+      const uint32_t o_row = smem_u32(smem + L.o[wg]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(o_row + sw128_offset(r, c), pack_bf16(o[8 * c], o[8 * c + 1]),
+                     pack_bf16(o[8 * c + 2], o[8 * c + 3]), pack_bf16(o[8 * c + 4], o[8 * c + 5]),
+                     pack_bf16(o[8 * c + 6], o[8 * c + 7]));
+      fence_async_smem();
+      named_barrier(2 + wg, 128);
+      if (r == 0) {
+        tma_store_3d_hint(map_o, smem + L.o[wg], 0, (t_begin + i) * kTileRows, bh, last_use);
+        bulk_commit();
       }
       if (threadIdx.x == 128 && blockIdx.x == 0 && u < 8) NYS_MARK_T(kTrOut, 40 + u);
     }
+    if (r == 0) bulk_wait0();
 
   }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && !*abort_flag)
-    for (int b = 0; b < 3 * kStages + 11; ++b) mbar_inval(bars + b);
+    for (int b = 0; b < 3 * kStages + 4 * NW + 1; ++b) mbar_inval(bars + b);
   if (warp == 1 && tmem_in == ~0u) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -401,9 +406,9 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
 }
 
 template <int M>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<M>::kThreads, 1)
 out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
-              const Params prm) {
+              const __grid_constant__ CUtensorMap map_o, const Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int bh = blockIdx.x / prm.ctas_per_head;
@@ -412,7 +417,7 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
   // launched early (programmatic dependent launch): out_body waits for the
   // previous kernels before it reads K~ and W
-  out_body<M>(&map_q, &map_v, prm, smem, bh, t_begin, t_end, ~0u, true);
+  out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u, true);
 }
 
 }  // namespace outtc
