@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (nys_attn_backward) instead of the forward")
     return ap.parse_args()
 
 
@@ -236,6 +238,61 @@ class ClockSampler:
                 "sm_min_mhz": min(x[1] for x in sel), "sm_max_mhz": max(x[2] for x in sel),
                 "power_w_median": round(statistics.median(x[4] for x in sel), 1),
                 "samples": len(sel), "reasons": reasons, "source": self.source}
+
+
+# ----------------------------------------------------------------- backward
+
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core fp32 FMA, max clock
+
+
+def backward_flops(wl):
+    """fp32 flops of one backward step: per head the two streaming passes
+    (rows: S, dF, dQ, dW, dK~; keys: S, dB, dK, dV, dQ~; 2 n m d each), the
+    recomputed B~ V (4 n m d), the pseudoinverse forward and backward (8 m^3
+    and about 28 m^3 per step) and the conv (4 n k d)."""
+    n, m, d, k, it = wl.seq_len, wl.landmarks, wl.head_dim, wl.conv_k, wl.pinv_iters
+    per_head = 24 * n * m * d + it * 36 * m ** 3 + 4 * n * k * d
+    return wl.bh * per_head
+
+
+def run_backward(args, rank, world):
+    import torch
+    import nystr_self_attention_segment_b200 as nys
+    from nystr_self_attention_segment_b200.inputs import WORKLOADS, make_inputs
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    x = make_inputs(wl)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x[k]).to(dev).to(tdt) for k in ("Q", "K", "V"))
+    G = torch.randn(Q.shape, device=dev).to(tdt)
+    cw = torch.from_numpy(x["conv_w"]).to(dev) if x["conv_w"] is not None else None
+    nb = nys._lib.nys_attn_backward_workspace_size(nys.desc_of(Q), wl.landmarks, wl.pinv_iters,
+                                                   wl.conv_k)
+    ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        nys.nys_attn_backward(Q, K, V, wl.landmarks, G, wl.pinv_iters, cw, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        nys.nys_attn_backward(Q, K, V, wl.landmarks, G, wl.pinv_iters, cw, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if rank != 0:
+        return None
+    fl = backward_flops(wl)
+    ach = fl / (ms / 1e3) / 1e12
+    return {"metric": "Nyström attention bwd tokens/sec (b×h×n)", "value": wl.tokens * world / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 arithmetic, %s tensors" % wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, world),
+            "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(FP32_FMA_PEAK_TFLOPS, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / FP32_FMA_PEAK_TFLOPS, 4),
+                         "traffic": None, "algorithmic_flops": fl,
+                         "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz"}}
 
 
 # ----------------------------------------------------------------- our arm
@@ -522,7 +579,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        line = run_ours(args, rank, world)
+        line = run_backward(args, rank, world) if args.backward else run_ours(args, rank, world)
     finally:
         if world > 1:
             dist.destroy_process_group()

@@ -44,9 +44,14 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t code) {
 
 // Workspace layout, a pure function of the shape so that it can be sized on
 // a machine without a GPU.  All regions are 256-byte aligned.
+// Per-head words of the bf16 path's hand-off, zeroed by every call:
+// [0, BH) B~ V blocks done, [BH, 2 BH) W inputs (Z, Y) in global memory,
+// [2 BH, 3 BH) W of the head stored (the output kernel's flag).
+constexpr int kCountsPerHead = 3;
+
 struct Layout {
   size_t q_land, k_land, z, y, w, err;     // parity-visible fp32 intermediates
-  size_t count;                            // per-head hand-off counters (bf16 path)
+  size_t count;                            // kCountsPerHead words per head (bf16 path)
   size_t pmax, psum, py;                   // split-n partials of B~ V
   size_t scratch;                          // per-head pinv scratch (m > 64)
   size_t w_bf;                             // W as the bf16 operand of P W

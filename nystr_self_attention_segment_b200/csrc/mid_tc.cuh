@@ -80,7 +80,7 @@ struct Params {
   const float *z;             // [BH][m][m] (the pseudoinverse blocks' result)
   float *y, *w;               // [BH][m][64]
   uint8_t *w_op;              // [BH][m][128 B]: W as the bf16 B operand of P W
-  uint32_t *count;            // [2 BH], zeroed per call: B~V blocks done, W inputs ready
+  uint32_t *count;            // [kCountsPerHead BH], zeroed per call
   uint32_t *err;
   const int *lens;            // [batch] tokens per element (ragged batches) or null
   int heads;
@@ -439,115 +439,17 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
 
 // ------------------------------------------------------------------ merge + W
 // The last B~ V block of a head (counted with an atomic) merges the head's S
-// partial states into Y in split order:
-//   Y_j = sum_s f_s Y_s,j / sum_s f_s l_s,j,  f_s = 2^(m_s - max_s m_s).
+// partial states (m_s, l_s, Y_s) of every landmark into Y, in split order
+// with a running maximum:
+//   M <- max(M, m_s),  a = 2^(M_old - M),  b = 2^(m_s - M),
+//   L <- a L + b l_s,  Y~ <- a Y~ + b Y_s,   and finally Y = Y~ / L.
 // The second of {that block, the head's pseudoinverse block} to finish forms
-// W = Z Y (form_w): the same function on the same global Z and Y whichever
-// block runs it, so the result does not depend on which finishes first.
+// W = Z Y (form_w).  Each of the two can leave its own result in the W
+// operands in shared memory (the same split of the same values that form_w
+// would load), so form_w loads only the other one; either way W is the same.
 
-template <int M>
-struct MergeSmem {
-  static constexpr uint32_t wgt = 0;                       // f [kMaxSplits][M]
-  static constexpr uint32_t psm = wgt + kMaxSplits * M * 4u;
-  static constexpr uint32_t den = psm + kMaxSplits * M * 4u;
-  static constexpr uint32_t total = den + M * 4u;
-};
-
-// All kThreads threads: the S x M maxima and sums into shared memory, the
-// weights, then the partials (a batch of splits of every item of a thread
-// loaded at once); Y in fp32 to global memory.
-template <int M>
-__device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh) {
-  using C = MergeSmem<M>;
-  const int t = threadIdx.x, S = prm.splits;
-  float *wgt = (float *)(smem + C::wgt), *psm = (float *)(smem + C::psm);
-  float *den = (float *)(smem + C::den);
-  const size_t pb = (size_t)bh * S * M;
-  {
-    constexpr int kPer = (kMaxSplits * M + kThreads - 1) / kThreads;
-    float a[kPer], b[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = t + u * kThreads;
-      if (i < S * M) {
-        a[u] = __ldcg(prm.pmax + pb + i);
-        b[u] = __ldcg(prm.psum + pb + i);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = t + u * kThreads;
-      if (i < S * M) {
-        wgt[i] = a[u];
-        psm[i] = b[u];
-      }
-    }
-  }
-  __syncthreads();
-  if (t < M) {
-    float mx = -INFINITY;
-    for (int s = 0; s < S; ++s) mx = fmaxf(mx, wgt[s * M + t]);
-    float d = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float f = mx == -INFINITY ? 0.f : fast_exp2(wgt[s * M + t] - mx);
-      wgt[s * M + t] = f;
-      d = fmaf(psm[s * M + t], f, d);
-    }
-    den[t] = 1.f / d;
-  }
-  __syncthreads();
-  constexpr int kItems = M * 16;   // float4 items of Y
-  constexpr int kIpt = (kItems + kThreads - 1) / kThreads;
-  constexpr int kBatch = 16 / kIpt > 0 ? 16 / kIpt : 1;
-  float4 acc[kIpt];
-#pragma unroll
-  for (int q = 0; q < kIpt; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < S; s0 += kBatch) {
-    float4 v[kIpt][kBatch];
-#pragma unroll
-    for (int q = 0; q < kIpt; ++q) {
-      const int idx = q * kThreads + t;
-      if (idx < kItems) {
-        const float4 *src = (const float4 *)(prm.py + (pb + (idx >> 4)) * 64) + (idx & 15);
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (s0 + u < S) v[q][u] = __ldcg(src + (size_t)(s0 + u) * M * 16);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < kIpt; ++q) {
-      const int idx = q * kThreads + t;
-      if (idx < kItems) {
-        const int j = idx >> 4;
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (s0 + u < S) {
-            const float f = wgt[(s0 + u) * M + j];
-            acc[q].x = fmaf(f, v[q][u].x, acc[q].x);
-            acc[q].y = fmaf(f, v[q][u].y, acc[q].y);
-            acc[q].z = fmaf(f, v[q][u].z, acc[q].z);
-            acc[q].w = fmaf(f, v[q][u].w, acc[q].w);
-          }
-      }
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < kIpt; ++q) {
-    const int idx = q * kThreads + t;
-    if (idx < kItems) {
-      const float inv = den[idx >> 4];
-      ((float4 *)(prm.y + (size_t)bh * M * 64))[idx] =
-          make_float4(acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
-    }
-  }
-}
-
-// W = Z Y on the tensor cores from split bf16 operands (hi = rounding of x,
-// lo = rounding of x - hi; Z_h Y_h + Z_h Y_l + Z_l Y_h, fp32 accumulation,
-// about 16 bits), Z K-major (A, m rows), Y MN-major (B, row k = landmark, 64
-// features); W stored in fp32 and as the bf16 operand of P W (128 bytes per
-// landmark row, 16-byte chunk c at c ^ (row & 7)).  All kThreads threads;
-// TMEM columns 0..63 of the block's allocation.
+// W operand scratch: Z (A, K-major, m rows) and Y (B, MN-major, m landmark
+// rows of 64 features), each as a split bf16 pair; the MMA barrier.
 template <int M>
 struct WSmem {
   static constexpr int kAtoms = M > 64 ? M / 64 : 1;     // 128-byte K atoms of Z
@@ -570,9 +472,83 @@ __device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Threads 0..255: 256 / M threads per landmark row, 64 M / 256 features
+// each.  The loads of a batch of splits (maxima, sums and partial rows) are
+// all issued before the first is used, so a merge of up to kSB splits is one
+// round trip to L2.  Y goes to global memory in fp32 and, when stage_y, into
+// the W operand's Y pair in shared memory.
+template <int M>
+__device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh, bool stage_y) {
+  constexpr int kTpr = 256 / M, kF = 64 / kTpr;   // threads per row, features per thread
+  constexpr int kSB = kF >= 32 ? 1 : 80 / kF;     // splits per batch of loads (registers)
+  const int t = threadIdx.x, S = prm.splits;
+  if (t >= 256) return;
+  const int j = t / kTpr, f0 = (t % kTpr) * kF;
+  const size_t pb = (size_t)bh * S * M + j;
+  float mx = -INFINITY, den = 0.f, acc[kF];
+#pragma unroll
+  for (int f = 0; f < kF; ++f) acc[f] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += kSB) {
+    float pm[kSB], pl[kSB];
+    float4 py[kSB][kF / 4];
+#pragma unroll
+    for (int u = 0; u < kSB; ++u)
+      if (s0 + u < S) {
+        const size_t i = pb + (size_t)(s0 + u) * M;
+        pm[u] = __ldcg(prm.pmax + i);
+        pl[u] = __ldcg(prm.psum + i);
+        const float4 *src = (const float4 *)(prm.py + i * 64 + f0);
+#pragma unroll
+        for (int q = 0; q < kF / 4; ++q) py[u][q] = __ldcg(src + q);
+      }
+#pragma unroll
+    for (int u = 0; u < kSB; ++u)
+      if (s0 + u < S) {
+        const float nm = fmaxf(mx, pm[u]);
+        const float a = mx == -INFINITY ? 0.f : fast_exp2(mx - nm);
+        const float b = pm[u] == -INFINITY ? 0.f : fast_exp2(pm[u] - nm);
+        den = fmaf(den, a, pl[u] * b);
+#pragma unroll
+        for (int q = 0; q < kF / 4; ++q) {
+          acc[4 * q] = fmaf(acc[4 * q], a, py[u][q].x * b);
+          acc[4 * q + 1] = fmaf(acc[4 * q + 1], a, py[u][q].y * b);
+          acc[4 * q + 2] = fmaf(acc[4 * q + 2], a, py[u][q].z * b);
+          acc[4 * q + 3] = fmaf(acc[4 * q + 3], a, py[u][q].w * b);
+        }
+        mx = nm;
+      }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int f = 0; f < kF; ++f) acc[f] *= inv;
+  float4 *dst = (float4 *)(prm.y + ((size_t)bh * M + j) * 64 + f0);
+#pragma unroll
+  for (int q = 0; q < kF / 4; ++q)
+    dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+  if (stage_y) {
+    const uint32_t s_bh = smem_u32(smem + WSmem<M>::bh), s_bl = smem_u32(smem + WSmem<M>::bl);
+#pragma unroll
+    for (int c = 0; c < kF / 8; ++c) {
+      uint4 hi, lo;
+      split8(acc + 8 * c, hi, lo);
+      const uint32_t off = sw128_offset(j, f0 / 8 + c);
+      st_shared_v4(s_bh + off, hi.x, hi.y, hi.z, hi.w);
+      st_shared_v4(s_bl + off, lo.x, lo.y, lo.z, lo.w);
+    }
+  }
+}
+
+// W = Z Y on the tensor cores from split bf16 operands (hi = rounding of x,
+// lo = rounding of x - hi; Z_h Y_h + Z_h Y_l + Z_l Y_h, fp32 accumulation,
+// about 16 bits), Z K-major (A, m rows), Y MN-major (B, row k = landmark, 64
+// features); W stored in fp32 and as the bf16 operand of P W (128 bytes per
+// landmark row, 16-byte chunk c at c ^ (row & 7)).  All kThreads threads;
+// TMEM columns 0..63 of the block's allocation.  z_staged / y_staged: that
+// operand pair is already in place (written by this block from the values it
+// stored to global memory, split the same way), so it is not loaded.
 template <int M>
 __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh, uint32_t tmem,
-                                       const Abort &ab) {
+                                       const Abort &ab, bool z_staged, bool y_staged) {
   using C = WSmem<M>;
   const int t = threadIdx.x, warp = t >> 5;
   uint64_t *bar = (uint64_t *)(smem + C::bar);
@@ -588,11 +564,12 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
     constexpr int kPer = (kZc + kYc + kThreads - 1) / kThreads;
     const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
     const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
+    const int c0 = z_staged ? kZc : 0, c1 = y_staged ? kZc : kZc + kYc;
     float4 va[kPer], vb[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int c = t + u * kThreads;
-      if (c < kZc + kYc) {
+      const int c = c0 + t + u * kThreads;
+      if (c < c1) {
         const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
         va[u] = __ldcg(src);
         vb[u] = __ldcg(src + 1);
@@ -600,8 +577,8 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
     }
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int c = t + u * kThreads;
-      if (c >= kZc + kYc) break;
+      const int c = c0 + t + u * kThreads;
+      if (c >= c1) break;
       const float x[8] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
       uint4 hi, lo;
       split8(x, hi, lo);
@@ -664,11 +641,10 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
 
 template <int M>
 __host__ __device__ constexpr uint32_t smem_bytes() {
-  // pinv operands or B~ V buffers, then the merge / W scratch
+  // pinv operands or B~ V buffers, then the W operands
   constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
   constexpr uint32_t body = pinv_smem<M>() > bv ? pinv_smem<M>() : bv;
-  constexpr uint32_t tail = MergeSmem<M>::total > WSmem<M>::total ? MergeSmem<M>::total
-                                                                  : WSmem<M>::total;
+  constexpr uint32_t tail = WSmem<M>::total;
   return 1024u + (body > tail ? body : tail);
 }
 
@@ -717,7 +693,8 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     NYS_MARK(kTrMid, 1);
     if constexpr (M <= 64) {
       if (t < pinvpow::kBarThreads)
-        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem);
+        pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem_u32(smem + WSmem<M>::ah),
+                              smem_u32(smem + WSmem<M>::al));
     } else {
       if (t < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
     }
@@ -737,36 +714,51 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   }
   NYS_MARK(kTrMid, 2);
   // hand-off: the last B~ V block of a head merges Y; the second of {that
-  // block, the pseudoinverse block} forms W.  Counters: count[bh] B~ V
-  // blocks done, count[BH + bh] W inputs (Z, Y) in global memory.
+  // block, the pseudoinverse block} forms W and raises the head's flag for
+  // the output kernel.  Counters: count[bh] B~ V blocks done, count[BH + bh]
+  // W inputs (Z, Y) in global memory, count[2 BH + bh] W stored.  Each
+  // count is taken by thread 0 between block barriers, with a fence on each
+  // side of the atomic: the barrier orders the block's stores before the
+  // first fence, the second fence orders the other block's stores (seen
+  // through the count) before the block's loads after the next barrier.
   __shared__ uint32_t last;
   __shared__ volatile uint32_t w_abort;
   if (t == 0) w_abort = 0;
   const int bh = is_pinv ? (int)blockIdx.x : (int)(blockIdx.x - prm.BH) / prm.splits;
-  __threadfence();
-  tc_fence_before();
-  __syncthreads();
-  if (t == 0) {
-    test_delay(is_pinv ? 1 : 2);
-    last = is_pinv ? 1u : (atomicAdd(prm.count + bh, 1u) == (uint32_t)prm.splits - 1u);
+  auto count_in = [&](uint32_t *c, uint32_t target) {
+    tc_fence_before();
+    __syncthreads();
+    if (t == 0) {
+      __threadfence();
+      last = atomicAdd(c, 1u) == target;
+      __threadfence();
+    }
+    __syncthreads();
+    tc_fence_after();
+  };
+  if (t == 0) test_delay(is_pinv ? 1 : 2);
+  if (is_pinv) {
+    if (t == 0) last = 1u;
+    __syncthreads();
+  } else {
+    count_in(prm.count + bh, (uint32_t)prm.splits - 1u);
   }
-  __syncthreads();
-  if (last) {
+  if (last) {   // block-uniform
     if (!is_pinv) {
-      __threadfence();
       NYS_MARK(kTrMid, 3);
-      merge_y<M>(prm, smem, bh);
-      __threadfence();
-      __syncthreads();
+      merge_y<M>(prm, smem, bh, true);
       NYS_MARK(kTrMid, 4);
     }
-    if (t == 0) last = atomicAdd(prm.count + prm.BH + bh, 1u) == 1u;
-    __syncthreads();
+    count_in(prm.count + prm.BH + bh, 1u);
     if (last) {
-      __threadfence();
       NYS_MARK(kTrMid, 5);
-      tc_fence_after();
-      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err});
+      // this block's own result is in the W operands already (Z for m <= 64)
+      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err}, is_pinv && M <= 64, !is_pinv);
+      // form_w ends with a block barrier after every thread's stores
+      if (t == 0) {
+        fence_async_global();   // the output kernel reads W with a bulk copy
+        flag_release(prm.count + 2 * prm.BH + bh, 1u);
+      }
       NYS_MARK(kTrMid, 6);
     }
   }

@@ -97,9 +97,9 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.z = take(BH * m * m * 4);
   L.y = take(BH * m * d * 4);
   L.w = take(BH * m * d * 4);
-  // the error word, then two counters per head (B~ V blocks done, W inputs
-  // ready); all zeroed by every call
-  L.err = take(256 + BH * 8);
+  // the error word, then the hand-off words of every head; all zeroed by
+  // every call
+  L.err = take(256 + BH * 4 * kCountsPerHead);
   L.count = L.err + 256;
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
@@ -393,11 +393,14 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
   }
   {   // F~ W + DConv(V)
     const int tph = (n + outtc::kTileRows - 1) / outtc::kTileRows;
-    int cpb = kNumSms / BH;
+    // blocks per head: the SMs that the pseudoinverse blocks (one per head,
+    // busy until about W) leave free, so that no block starts late
+    int cpb = (kNumSms - BH) / BH;
     if (cpb < 1) cpb = 1;
     if (cpb > tph) cpb = tph;
+    const uint32_t *w_flag = (const uint32_t *)(ws + L.count) + 2 * (size_t)BH;
     outtc::Params p{kt,  (const uint8_t *)(ws + L.w_bf), conv_w, err, n, desc->heads,
-                    conv ? conv_k : 1, kconv, tph, cpb, scale_log2, lens, M};
+                    conv ? conv_k : 1, kconv, tph, cpb, scale_log2, lens, M, w_flag};
     auto kern = outtc::out_tc_kernel<M>;
     const uint32_t sm = outtc::smem_layout(M, conv ? kconv : 0).total;
     if (!allow_smem(kern, sm) ||
@@ -720,11 +723,12 @@ static nys_status forward_impl(const void *Q, const void *K, const void *V,
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  const size_t nclear = clear_err ? 256 + (size_t)desc->batch * desc->heads * 8 : 0;
+  const size_t ncount = (size_t)desc->batch * desc->heads * 4 * kCountsPerHead;
+  const size_t nclear = clear_err ? 256 + ncount : 0;
   if (nclear && cudaMemsetAsync(ws + L.err, 0, nclear, stream) != cudaSuccess) st = NYS_ERR_CUDA;
   // the layer clears the error word itself; the counters still start at zero
   if (!clear_err &&
-      cudaMemsetAsync(ws + L.count, 0, (size_t)desc->batch * desc->heads * 8, stream) !=
+      cudaMemsetAsync(ws + L.count, 0, ncount, stream) !=
           cudaSuccess)
     st = NYS_ERR_CUDA;
   mk.first(stream);

@@ -85,16 +85,21 @@ struct Params {
   float scale_log2;
   const int *lens;         // [batch] tokens per element (ragged batches) or null
   int m;
+  const uint32_t *w_flag;  // [BH]: nonzero once the previous kernel has stored W of the head
 };
 
 // One run of 128-row tiles [t_begin, t_end) of (batch, head) bh.  tmem_in: a
 // 512-column TMEM allocation owned by the caller, or ~0u to allocate (and
 // free) one here.  smem: smem_layout(M, kconv).total bytes, 1 KB aligned.
 template <int M>
-// wait_prev: launched with programmatic dependent launch; everything that
-// reads only the inputs (barriers, TMEM, the Toeplitz operand, the first
-// kStages tile loads) runs before the wait for the previous kernel, the K~ /
-// W operand loads after it.
+// wait_prev: launched with programmatic dependent launch while the previous
+// kernel still runs.  Everything that reads only the inputs and K~ (barriers,
+// TMEM, the Toeplitz operand, the first kStages tiles' S and conv) runs at
+// once; the W operand is loaded once the head's flag (prm.w_flag) says the
+// previous kernel has stored it, so a head's P W starts as soon as its own W
+// exists, not when the whole previous grid has completed.  The block waits
+// for the previous grid before it exits, so that this grid completes after
+// it.
 __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtensorMap *map_v,
                                          const CUtensorMap *map_o, const Params &prm,
                                          uint8_t *smem, int bh, int t_begin, int t_end,
@@ -229,10 +234,16 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
   tc_fence_after();
   NYS_MARK(kTrOut, 1);
   if (warp == Warps<M>::kLoader && lane == 0) {
-    if (wait_prev) griddep_wait();
+    // the flag's acquire orders the previous kernel's W stores before this
+    // thread's generic accesses; the proxy fence then orders them before the
+    // bulk copy
+    const bool have_w = !wait_prev || flag_wait(prm.w_flag + bh, ab, kWaitLimitCycles);
     NYS_MARK_T(kTrOut, 2);
-    mbar_expect_tx(w_ready, M * 128u);
-    bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
+    if (have_w) {
+      fence_async_global();
+      mbar_expect_tx(w_ready, M * 128u);
+      bulk_load(smem + L.w, prm.w_op + (size_t)bh * M * 128, M * 128u, w_ready);
+    }
   }
   if (warp == Warps<M>::kLoader && mask_v) {
     // ragged batches: halo rows at or past L of every staged V tile become
@@ -402,6 +413,7 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (wait_prev && threadIdx.x == 0) griddep_wait();
   NYS_MARK(kTrOut, 4);
 }
 
@@ -415,8 +427,9 @@ out_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int part = blockIdx.x % prm.ctas_per_head;
   const int t_begin = (int)((long)part * prm.tiles_per_head / prm.ctas_per_head);
   const int t_end = (int)((long)(part + 1) * prm.tiles_per_head / prm.ctas_per_head);
-  // launched early (programmatic dependent launch): out_body waits for the
-  // previous kernels before it reads K~ and W
+  // launched early (programmatic dependent launch): out_body reads K~ at
+  // once (its kernel completed before the previous one could let this grid
+  // launch) and W after the head's flag
   out_body<M>(&map_q, &map_v, &map_o, prm, smem, bh, t_begin, t_end, ~0u, true);
 }
 

@@ -168,9 +168,15 @@ __device__ __forceinline__ void ld_cols(uint32_t taddr, float *v) {
 // scale_log2 = log2(e) / sqrt(d).
 // tmem_in: a TMEM allocation of at least Cfg<M>::kTmemCols columns owned by
 // the caller, or ~0u to allocate (and free) one here.
+// zs_hi, zs_lo (shared-memory addresses, or 0): the final Z is also written
+// there as a split bf16 operand pair, K-major, one 128-byte swizzle row per
+// matrix row (hi = rounding of z, lo = rounding of z - hi), for a product
+// with Z that follows in the same block.  They may lie over this function's
+// own operands: they are written after its last MMA has completed.
 template <int M, class Prm>
 __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
-                                          uint32_t tmem_in = ~0u) {
+                                          uint32_t tmem_in = ~0u, uint32_t zs_hi = 0,
+                                          uint32_t zs_lo = 0) {
   using C = Cfg<M>;
   constexpr int NC = C::NC;
   const int t = threadIdx.x, warp = t >> 5;
@@ -376,6 +382,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
       for (int q = 0; q < NC / 4; ++q)
         *(float4 *)(zg + (size_t)row * M + c_lo + 4 * q) =
             make_float4(acol[4 * q], acol[4 * q + 1], acol[4 * q + 2], acol[4 * q + 3]);
+      if (zs_hi) put_split<NC, false>(zs_hi, zs_lo, row, c_lo, acol);
     } else {
       put_split<NC, false>(azh, azl, 64 + row, c_lo, acol);
     }
@@ -497,6 +504,7 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
         for (int q = 0; q < NC / 4; ++q)
           *(float4 *)(zg + (size_t)row * M + c_lo + 4 * q) =
               make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+        if (zs_hi) put_split<NC, false>(zs_hi, zs_lo, row, c_lo, z);
       }
     }
   }

@@ -113,6 +113,43 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ flags between blocks
+// A per-item flag that a block sets once its results for the item are in
+// global memory, read by blocks of this or a later kernel: the producer
+// stores it with release semantics after a block barrier (so that it covers
+// every thread's writes), the consumer loads it with acquire semantics.
+__device__ __forceinline__ void flag_release(uint32_t *p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t flag_acquire(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Orders generic-proxy global memory accesses before the async-proxy ones
+// (bulk copies, TMA) that follow in this thread.
+__device__ __forceinline__ void fence_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Spins until *p != 0, bounded like the mbarrier waits: false (timeout
+// recorded, block abort flag raised) after limit_cycles, or at once when
+// another thread of the block has aborted.
+__device__ __forceinline__ bool flag_wait(const uint32_t *p, const Abort &ab,
+                                          long long limit_cycles) {
+  if (flag_acquire(p)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if (flag_acquire(p)) return true;
+    if (*ab.flag) return false;
+    if (clock64() - t0 > limit_cycles) {
+      *ab.flag = 1u;
+      set_error(ab.err, NYS_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
