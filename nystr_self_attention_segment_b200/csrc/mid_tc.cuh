@@ -667,7 +667,7 @@ __device__ __forceinline__ void test_delay(int) {}
 template <int M>
 __global__ void __launch_bounds__(kThreads, 1)
 mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-           const __grid_constant__ CUtensorMap map_q, const Params prm) {
+           const Params prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint32_t tmem_base;
@@ -702,15 +702,6 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     const int b = blockIdx.x - prm.BH;
     const int bh = b / prm.splits, split = b % prm.splits;
     bv_body<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
-    // HBM is mostly idle from here until W is ready: bring this split's
-    // share of the head's Q rows into L2 for the output kernel (V's rows
-    // were just read and stay)
-    if (t == 0) {
-      const int tiles = (prm.n + 127) / 128;
-      const int t0 = (int)((long)split * tiles / prm.splits);
-      const int t1 = (int)((long)(split + 1) * tiles / prm.splits);
-      for (int i = t0; i < t1; ++i) tma_prefetch_l2_3d(&map_q, 0, i * 128, bh);
-    }
   }
   NYS_MARK(kTrMid, 2);
   // hand-off: the last B~ V block of a head merges Y; the second of {that

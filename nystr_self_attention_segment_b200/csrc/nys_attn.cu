@@ -387,7 +387,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
     const uint32_t sm = midtc::smem_bytes<M>();
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH * (1 + L.splits)), dim3(midtc::kThreads),
-               launch_smem(mk.launched, sm), stream, true, mkk, mv, mq, p) != cudaSuccess)
+               launch_smem(mk.launched, sm), stream, true, mkk, mv, p) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }

@@ -187,13 +187,6 @@ __device__ __forceinline__ void out_body(const CUtensorMap *map_q, const CUtenso
       tma_load_3d_hint(smem + L.q[i], map_q, &full[i], 0, r0, bh, last_use);
       if (conv) tma_load_3d_hint(smem + L.v[i], map_v, &full[i], 0, r0 - half, bh, last_use);
     }
-    // the block's other tiles into L2 while it waits for W: HBM is mostly
-    // idle between the end of B~ V and W
-    for (int i = pre; i < ntiles; ++i) {
-      const int r0 = (t_begin + i) * kTileRows;
-      tma_prefetch_l2_3d(map_q, 0, r0, bh);
-      if (conv) tma_prefetch_l2_3d(map_v, 0, r0 - half, bh);
-    }
   }
   // Toeplitz operand into TMEM: row r (lane r), columns j = halo rows
   if (conv && warp >= 4 && warp < 8) {

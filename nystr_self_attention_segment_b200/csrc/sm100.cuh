@@ -201,13 +201,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *s
                "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
-// L2 prefetch of one tile of a tensor map (no shared-memory destination, no
-// multicast): the tile is in L2 when a later load asks for it.
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *m, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(m),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
 // 1-D bulk copy global -> shared (no multicast), completing on an mbarrier
 // with complete_tx; both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
