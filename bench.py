@@ -61,7 +61,7 @@ def peaks():
 # Sources of each kernel of the bf16 path: a DRAM traffic figure recorded
 # from an ncu capture holds only while these files are unchanged.
 KERNEL_SOURCES = {
-    "mid_tc": ["common.cuh", "sm100.cuh", "trace.cuh", "pinv_pow.cuh", "pinv_tc.cuh",
+    "mid_tc": ["common.cuh", "sm100.cuh", "trace.cuh", "pinv_pow.cuh", "pinv_pow128.cuh",
                "mid_tc.cuh"],
     "out_tc": ["common.cuh", "sm100.cuh", "trace.cuh", "out_tc.cuh"],
     "seg_means": ["common.cuh", "sm100.cuh", "trace.cuh", "stream_bf16.cuh"],

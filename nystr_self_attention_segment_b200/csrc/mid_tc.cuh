@@ -1,7 +1,7 @@
 // Middle stage of the bf16 path, one launch:
 //   blocks [0, BH)            the landmark kernel A and its pseudoinverse Z
 //                             (one head each: pinv_pow.cuh for m <= 64,
-//                             pinv_tc.cuh for m = 128),
+//                             pinv_pow128.cuh for m = 128),
 //   blocks [BH, BH*(1+S))     Y = B~ V streamed over the keys, S blocks per head
 //                             ("Nystromformer: A Nystrom-Based Algorithm for
 //                             Approximating Self-Attention", section 3.4,
@@ -29,7 +29,7 @@
 #pragma once
 
 #include "pinv_pow.cuh"
-#include "pinv_tc.cuh"
+#include "pinv_pow128.cuh"
 #include "trace.cuh"
 
 namespace nys {
@@ -68,13 +68,13 @@ __host__ __device__ constexpr uint32_t pinv_smem() {
   if constexpr (M <= 64) {
     return pinvpow::Cfg<M>::total;
   } else {
-    return pinvtc::Cfg<M>::total;
+    return pinvpow128::Cfg::total;
   }
 }
 
 
 struct Params {
-  pinvtc::Params pinv;
+  pinvpow::Params pinv;
   const float *q_land;        // [BH][m][64]
   float *pmax, *psum, *py;    // [BH][S][m], [BH][S][m], [BH][S][m][64]
   const float *z;             // [BH][m][m] (the pseudoinverse blocks' result)
@@ -472,52 +472,92 @@ __device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-// Threads 0..255: 256 / M threads per landmark row, 64 M / 256 features
-// each.  The loads of a batch of splits (maxima, sums and partial rows) are
-// all issued before the first is used, so a merge of up to kSB splits is one
-// round trip to L2.  Y goes to global memory in fp32 and, when stage_y, into
-// the W operand's Y pair in shared memory.
+// Merge scratch, after the W operands: per split of a batch its partial Y
+// rows [M][64] fp32, then the batch's maxima and sums [kMergeBatch][M]; an
+// mbarrier for the bulk copies.
 template <int M>
-__device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh, bool stage_y) {
+struct MergeSmem {
+  static constexpr uint32_t base = (WSmem<M>::total + 1023u) & ~1023u;
+  static constexpr uint32_t kPy = M * 256u;
+  static constexpr int kBatch = M <= 64 ? 8 : 3;   // splits per batch of copies
+  static constexpr uint32_t py = base;
+  static constexpr uint32_t pm = py + kBatch * kPy;
+  static constexpr uint32_t pl = pm + kBatch * M * 4u;
+  static constexpr uint32_t bar = pl + kBatch * M * 4u;
+  static constexpr uint32_t total = bar + 64u;
+};
+
+// All kThreads threads.  Thread 0 brings a batch of splits' partials (rows,
+// maxima, sums) into shared memory with bulk copies, all in flight at once
+// (the partials were stored by other blocks' generic stores, ordered before
+// this block's count by their fences and ours; the proxy fence orders them
+// before the copies); then threads 0..255, 256 / M per landmark row and
+// 64 M / 256 features each, fold the batch into their running state.  Y goes
+// to global memory in fp32 and, when stage_y, into the W operand's Y pair in
+// shared memory.
+template <int M>
+__device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh, bool stage_y,
+                                        const Abort &ab) {
+  using C = MergeSmem<M>;
   constexpr int kTpr = 256 / M, kF = 64 / kTpr;   // threads per row, features per thread
-  constexpr int kSB = kF >= 32 ? 1 : 80 / kF;     // splits per batch of loads (registers)
   const int t = threadIdx.x, S = prm.splits;
-  if (t >= 256) return;
-  const int j = t / kTpr, f0 = (t % kTpr) * kF;
-  const size_t pb = (size_t)bh * S * M + j;
+  const int j = (t & 255) / kTpr, f0 = (t % kTpr) * kF;
+  uint64_t *bar = (uint64_t *)(smem + C::bar);
+  const float *sp = (const float *)(smem + C::py);
+  const float *sm = (const float *)(smem + C::pm);
+  const float *sl = (const float *)(smem + C::pl);
+  const size_t pb = (size_t)bh * S * M;
+  if (t == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   float mx = -INFINITY, den = 0.f, acc[kF];
 #pragma unroll
   for (int f = 0; f < kF; ++f) acc[f] = 0.f;
-  for (int s0 = 0; s0 < S; s0 += kSB) {
-    float pm[kSB], pl[kSB];
-    float4 py[kSB][kF / 4];
-#pragma unroll
-    for (int u = 0; u < kSB; ++u)
-      if (s0 + u < S) {
+  bool ok = true;
+  uint32_t phase = 0;
+  for (int s0 = 0; s0 < S; s0 += C::kBatch) {
+    const int nb = min(C::kBatch, S - s0);
+    if (t == 0) {
+      fence_async_global();
+      mbar_expect_tx(bar, (uint32_t)nb * (C::kPy + 2u * M * 4u));
+      for (int u = 0; u < nb; ++u) {
         const size_t i = pb + (size_t)(s0 + u) * M;
-        pm[u] = __ldcg(prm.pmax + i);
-        pl[u] = __ldcg(prm.psum + i);
-        const float4 *src = (const float4 *)(prm.py + i * 64 + f0);
-#pragma unroll
-        for (int q = 0; q < kF / 4; ++q) py[u][q] = __ldcg(src + q);
+        bulk_load(smem + C::py + u * C::kPy, prm.py + i * 64, C::kPy, bar);
+        bulk_load(smem + C::pm + u * M * 4u, prm.pmax + i, M * 4u, bar);
+        bulk_load(smem + C::pl + u * M * 4u, prm.psum + i, M * 4u, bar);
       }
-#pragma unroll
-    for (int u = 0; u < kSB; ++u)
-      if (s0 + u < S) {
-        const float nm = fmaxf(mx, pm[u]);
+    }
+    ok = ok && mbar_wait(bar, phase, ab);
+    phase ^= 1u;
+    if (t < 256 && ok) {
+      for (int u = 0; u < nb; ++u) {
+        const float pm = sm[u * M + j], pl = sl[u * M + j];
+        const float nm = fmaxf(mx, pm);
         const float a = mx == -INFINITY ? 0.f : fast_exp2(mx - nm);
-        const float b = pm[u] == -INFINITY ? 0.f : fast_exp2(pm[u] - nm);
-        den = fmaf(den, a, pl[u] * b);
+        const float b = pm == -INFINITY ? 0.f : fast_exp2(pm - nm);
+        den = fmaf(den, a, pl * b);
+        const float4 *row = (const float4 *)(sp + u * (M * 64) + j * 64 + f0);
 #pragma unroll
         for (int q = 0; q < kF / 4; ++q) {
-          acc[4 * q] = fmaf(acc[4 * q], a, py[u][q].x * b);
-          acc[4 * q + 1] = fmaf(acc[4 * q + 1], a, py[u][q].y * b);
-          acc[4 * q + 2] = fmaf(acc[4 * q + 2], a, py[u][q].z * b);
-          acc[4 * q + 3] = fmaf(acc[4 * q + 3], a, py[u][q].w * b);
+          const float4 y = row[q];
+          acc[4 * q] = fmaf(acc[4 * q], a, y.x * b);
+          acc[4 * q + 1] = fmaf(acc[4 * q + 1], a, y.y * b);
+          acc[4 * q + 2] = fmaf(acc[4 * q + 2], a, y.z * b);
+          acc[4 * q + 3] = fmaf(acc[4 * q + 3], a, y.w * b);
         }
         mx = nm;
       }
+    }
+    // the buffers are refilled by the next batch; a failed wait ends the merge
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      break;
+    }
   }
+  if (t == 0 && ok) mbar_inval(bar);
+  if (t >= 256) return;
   const float inv = 1.f / den;
 #pragma unroll
   for (int f = 0; f < kF; ++f) acc[f] *= inv;
@@ -644,7 +684,7 @@ __host__ __device__ constexpr uint32_t smem_bytes() {
   // pinv operands or B~ V buffers, then the W operands
   constexpr uint32_t bv = 16384u + kStages * 32768u + 1024u;
   constexpr uint32_t body = pinv_smem<M>() > bv ? pinv_smem<M>() : bv;
-  constexpr uint32_t tail = WSmem<M>::total;
+  constexpr uint32_t tail = MergeSmem<M>::total;
   return 1024u + (body > tail ? body : tail);
 }
 
@@ -696,7 +736,9 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
         pinvpow::pinv_body<M>(prm.pinv, smem, bh, tmem, smem_u32(smem + WSmem<M>::ah),
                               smem_u32(smem + WSmem<M>::al));
     } else {
-      if (t < pinvtc::kThreads) pinvtc::pinv_body<M>(prm.pinv, smem, bh, tmem);
+      if (t < pinvpow128::kBarThreads)
+        pinvpow128::pinv_body(prm.pinv, smem, bh, tmem, smem_u32(smem + WSmem<M>::ah),
+                              smem_u32(smem + WSmem<M>::al));
     }
   } else {
     const int b = blockIdx.x - prm.BH;
@@ -737,14 +779,14 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   if (last) {   // block-uniform
     if (!is_pinv) {
       NYS_MARK(kTrMid, 3);
-      merge_y<M>(prm, smem, bh, true);
+      merge_y<M>(prm, smem, bh, true, Abort{&w_abort, prm.err});
       NYS_MARK(kTrMid, 4);
     }
     count_in(prm.count + prm.BH + bh, 1u);
     if (last) {
       NYS_MARK(kTrMid, 5);
-      // this block's own result is in the W operands already (Z for m <= 64)
-      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err}, is_pinv && M <= 64, !is_pinv);
+      // this block's own result is in the W operands already
+      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err}, is_pinv, !is_pinv);
       // form_w ends with a block barrier after every thread's stores
       if (t == 0) {
         fence_async_global();   // the output kernel reads W with a bulk copy

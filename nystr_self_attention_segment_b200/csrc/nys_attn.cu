@@ -365,7 +365,7 @@ nys_status launch_tc_m(const __nv_bfloat16 *Q, const __nv_bfloat16 *K, const __n
   }
   {   // pseudoinverse || B~ V, then the merge of Y and W = Z Y
     midtc::Params p;
-    p.pinv = pinvtc::Params{qt, kt, z, err, iters, scale_log2};
+    p.pinv = pinvpow::Params{qt, kt, z, err, iters, scale_log2};
     p.q_land = qt;
     p.pmax = pmax;
     p.psum = psum;

@@ -50,6 +50,15 @@ namespace pinvpow {
 
 using namespace sm100;
 
+// Arguments of the pseudoinverse bodies (this file's and pinv_pow128.cuh's).
+struct Params {
+  const float *q_land, *k_land;   // [BH][m][64]
+  float *z_out;                   // [BH][m][m]
+  uint32_t *err;
+  int iters;
+  float scale_log2;               // log2(e) / sqrt(d)
+};
+
 constexpr int kThreads = 256;       // matrix-row threads
 constexpr int kBarThreads = 288;    // plus one issuer warp (warp 8, lane 0 issues)
 
@@ -367,11 +376,21 @@ __device__ __forceinline__ void pinv_body(const Prm &prm, uint8_t *smem, int bh,
     red[M + h * M + row] = cs;
   }
   named_barrier(1, kBarThreads);
+  // ||A||_1 (largest column sum) and ||A||_inf (largest row sum): every warp
+  // reduces the m rows' partials, lane l taking rows l and l + 32
   float n1 = 0.f, ninf = 0.f;
-#pragma unroll 8
-  for (int i = 0; i < M; ++i) {
-    n1 = fmaxf(n1, red[M + i] + red[2 * M + i]);
-    ninf = fmaxf(ninf, ((red4[512 + i] + red4[576 + i]) + red4[640 + i]) + red4[704 + i]);
+  {
+    const int l = t & 31;
+#pragma unroll
+    for (int i = l; i < M; i += 32) {
+      n1 = fmaxf(n1, red[M + i] + red[2 * M + i]);
+      ninf = fmaxf(ninf, ((red4[512 + i] + red4[576 + i]) + red4[640 + i]) + red4[704 + i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      n1 = fmaxf(n1, __shfl_xor_sync(0xffffffffu, n1, o));
+      ninf = fmaxf(ninf, __shfl_xor_sync(0xffffffffu, ninf, o));
+    }
   }
   const float c0 = 1.f / (n1 * ninf);
   if (ok && aux) {   // Z0 = c0 A^T, rows 64.. of the Z operand

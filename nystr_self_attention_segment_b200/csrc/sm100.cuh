@@ -253,15 +253,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Same with tf32 inputs (fp32 storage, 10-bit mantissa used).
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // Arrives once on the mbarrier when all previously issued MMAs of this thread
 // have completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -354,16 +345,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ------------------------------------------------------------------ descriptors
-// Instruction descriptor of tcgen05.mma kind::f16 / kind::tf32 with fp32
+// Instruction descriptor of tcgen05.mma kind::f16 with fp32
 // accumulation: c_format F32 (bits 4-5 = 1), a/b format (bits 7-9 / 10-12:
-// BF16 = 1, TF32 = 2), operand majorness (bit 15 A, bit 16 B: 0 = K-major,
+// F16 = 0, BF16 = 1), operand majorness (bit 15 A, bit 16 B: 0 = K-major,
 // 1 = MN-major), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t M, uint32_t N,
                                                   uint32_t a_mn_major, uint32_t b_mn_major) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
-constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1, kFmtTF32 = 2;
+constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version
 // 1: start address, leading-dimension byte offset and stride-dimension byte

@@ -76,7 +76,7 @@ def test_bf16_workload_against_oracle(name):
 
 
 @pytest.mark.parametrize("name", ["bert_n512_m64", "headline_n8192_m64", "sweep_n1024_m128",
-                                  "ragged_n8100_m64"])
+                                  "sweep_n8192_m128", "ragged_n8100_m64"])
 def test_bf16_intermediates(name):
     # Landmarks are fp32 sums of the same bf16 inputs; Z, Y and W are checked
     # against the oracle's steps applied to the device's own fp32 landmarks,
@@ -100,9 +100,10 @@ def test_bf16_intermediates(name):
         # Z against the oracle's iteration on the device's own landmarks.
         # m <= 64 runs the power form with split fp16 / bf16 products
         # (measured <= 1.9e-3 on every workload, held to 5e-3); m = 128 the
-        # Horner form with tf32 operands (measured <= 2.9e-2, held to 6e-2).
+        # power form on fp16 operands without lo halves (measured 2.2e-3 at
+        # n = 1024 and 1.4e-2 at n = 8192, held to 3e-2).
         Z = orc.iterative_pinv(orc.kernel_A(qt[i], kt[i], s), wl.pinv_iters)
-        assert normwise(Zg[i], Z) <= (5e-3 if m <= 64 else 6e-2)
+        assert normwise(Zg[i], Z) <= (5e-3 if m <= 64 else 3e-2)
         Y = orc.kernel_B(qt[i], K, s) @ V
         assert normwise(Yg[i], Y) <= 2e-2
         assert normwise(Wg[i], Zg[i] @ Yg[i]) <= 1e-4

@@ -61,7 +61,8 @@ def _other_inputs(x):
     return y
 
 
-# m = 64 and m = 32 (power-form pseudoinverse), m = 128 (Horner form), fp32
+# m = 64 and m = 32 (power-form pseudoinverse, split products), m = 128
+# (power form at full width), fp32
 NAMES = ["tiny_f32_m8", "headline_n8192_m64", "headline_n8192_m32", "long_n4096_m64",
          "sweep_n4096_m128"]
 
