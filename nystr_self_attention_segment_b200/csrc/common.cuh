@@ -45,8 +45,8 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t code) {
 // Workspace layout, a pure function of the shape so that it can be sized on
 // a machine without a GPU.  All regions are 256-byte aligned.
 // Per-head words of the bf16 path's hand-off, zeroed by every call:
-// [0, BH) B~ V blocks done, [BH, 2 BH) W inputs (Z, Y) in global memory,
-// [2 BH, 3 BH) W of the head stored (the output kernel's flag).
+// [0, BH) key-split blocks done, [BH, 2 BH) W inputs (merged Y, Z) in global
+// memory, [2 BH, 3 BH) W of the head stored (the output kernel's flag).
 constexpr int kCountsPerHead = 3;
 
 struct Layout {

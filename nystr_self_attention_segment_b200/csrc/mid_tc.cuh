@@ -484,7 +484,11 @@ struct MergeSmem {
   static constexpr uint32_t pm = py + kBatch * kPy;
   static constexpr uint32_t pl = pm + kBatch * M * 4u;
   static constexpr uint32_t bar = pl + kBatch * M * 4u;
-  static constexpr uint32_t total = bar + 64u;
+  // Z in fp32 for W, copied with the first batch (m <= 64; at m = 128 it
+  // does not fit and form_w loads it)
+  static constexpr bool kZ = M <= 64;
+  static constexpr uint32_t zf = (bar + 64u + 1023u) & ~1023u;
+  static constexpr uint32_t total = kZ ? zf + M * M * 4u : bar + 64u;
 };
 
 // All kThreads threads.  Thread 0 brings a batch of splits' partials (rows,
@@ -497,7 +501,7 @@ struct MergeSmem {
 // shared memory.
 template <int M>
 __device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh, bool stage_y,
-                                        const Abort &ab) {
+                                        const Abort &ab, bool load_z) {
   using C = MergeSmem<M>;
   constexpr int kTpr = 256 / M, kF = 64 / kTpr;   // threads per row, features per thread
   const int t = threadIdx.x, S = prm.splits;
@@ -520,8 +524,10 @@ __device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh
   for (int s0 = 0; s0 < S; s0 += C::kBatch) {
     const int nb = min(C::kBatch, S - s0);
     if (t == 0) {
+      const bool z = C::kZ && load_z && s0 == 0;   // Z of the head with the first batch
       fence_async_global();
-      mbar_expect_tx(bar, (uint32_t)nb * (C::kPy + 2u * M * 4u));
+      mbar_expect_tx(bar, (uint32_t)nb * (C::kPy + 2u * M * 4u) + (z ? M * M * 4u : 0u));
+      if (z) bulk_load(smem + C::zf, prm.z + (size_t)bh * M * M, M * M * 4u, bar);
       for (int u = 0; u < nb; ++u) {
         const size_t i = pb + (size_t)(s0 + u) * M;
         bulk_load(smem + C::py + u * C::kPy, prm.py + i * 64, C::kPy, bar);
@@ -585,10 +591,13 @@ __device__ __forceinline__ void merge_y(const Params &prm, uint8_t *smem, int bh
 // landmark row, 16-byte chunk c at c ^ (row & 7)).  All kThreads threads;
 // TMEM columns 0..63 of the block's allocation.  z_staged / y_staged: that
 // operand pair is already in place (written by this block from the values it
-// stored to global memory, split the same way), so it is not loaded.
+// stored to global memory, split the same way), so it is not loaded.  z_smem:
+// Z in fp32 in this block's shared memory (copied there by merge_y), or null
+// to read it from global memory.
 template <int M>
 __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh, uint32_t tmem,
-                                       const Abort &ab, bool z_staged, bool y_staged) {
+                                       const Abort &ab, bool z_staged, bool y_staged,
+                                       const float *z_smem) {
   using C = WSmem<M>;
   const int t = threadIdx.x, warp = t >> 5;
   uint64_t *bar = (uint64_t *)(smem + C::bar);
@@ -602,7 +611,7 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
       // first is used, split on the way in
     constexpr int kZc = M * M / 8, kYc = M * 64 / 8;
     constexpr int kPer = (kZc + kYc + kThreads - 1) / kThreads;
-    const float4 *zg = (const float4 *)(prm.z + (size_t)bh * M * M);
+    const float4 *zg = (const float4 *)(z_smem ? z_smem : prm.z + (size_t)bh * M * M);
     const float4 *yg = (const float4 *)(prm.y + (size_t)bh * M * 64);
     const int c0 = z_staged ? kZc : 0, c1 = y_staged ? kZc : kZc + kYc;
     float4 va[kPer], vb[kPer];
@@ -610,9 +619,14 @@ __device__ __forceinline__ void form_w(const Params &prm, uint8_t *smem, int bh,
     for (int u = 0; u < kPer; ++u) {
       const int c = c0 + t + u * kThreads;
       if (c < c1) {
-        const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
-        va[u] = __ldcg(src);
-        vb[u] = __ldcg(src + 1);
+        if (c < kZc && z_smem) {
+          va[u] = zg[2 * c];
+          vb[u] = zg[2 * c + 1];
+        } else {
+          const float4 *src = c < kZc ? zg + 2 * c : yg + 2 * (c - kZc);
+          va[u] = __ldcg(src);
+          vb[u] = __ldcg(src + 1);
+        }
       }
     }
 #pragma unroll
@@ -746,18 +760,22 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     bv_body<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
   }
   NYS_MARK(kTrMid, 2);
-  // hand-off: the last B~ V block of a head merges Y; the second of {that
-  // block, the pseudoinverse block} forms W and raises the head's flag for
-  // the output kernel.  Counters: count[bh] B~ V blocks done, count[BH + bh]
-  // W inputs (Z, Y) in global memory, count[2 BH + bh] W stored.  Each
-  // count is taken by thread 0 between block barriers, with a fence on each
-  // side of the atomic: the barrier orders the block's stores before the
-  // first fence, the second fence orders the other block's stores (seen
-  // through the count) before the block's loads after the next barrier.
+  // hand-off.  Counts per head: count[bh] key-split blocks done,
+  // count[BH + bh] W inputs (merged Y, Z) in global memory, count[2 BH + bh]
+  // W stored (the output kernel's flag).  The last split block merges the
+  // partials at once; W is formed by whichever of {that block, the
+  // pseudoinverse block} comes second: if the pseudoinverse block has
+  // already counted in, the split block merges and forms W in one go (with
+  // Z copied in beside the partials, m <= 64); otherwise it stores Y and
+  // counts in, and the second to count forms W.  Each count is taken by
+  // thread 0 between block barriers, with a fence on each side of the
+  // atomic: the barrier orders the block's stores before the first fence,
+  // the second fence orders the other blocks' stores (seen through the
+  // count) before the block's loads after the next barrier.
   __shared__ uint32_t last;
   __shared__ volatile uint32_t w_abort;
-  if (t == 0) w_abort = 0;
   const int bh = is_pinv ? (int)blockIdx.x : (int)(blockIdx.x - prm.BH) / prm.splits;
+  uint32_t *cnt_w = prm.count + prm.BH + bh;
   auto count_in = [&](uint32_t *c, uint32_t target) {
     tc_fence_before();
     __syncthreads();
@@ -769,31 +787,45 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
   };
-  if (t == 0) test_delay(is_pinv ? 1 : 2);
+  if (t == 0) {
+    w_abort = 0;
+    test_delay(is_pinv ? 1 : 2);
+  }
+  const Abort wab{&w_abort, prm.err};
+  bool form = false, z_staged = is_pinv, y_staged = false, z_copy = false;
   if (is_pinv) {
-    if (t == 0) last = 1u;
-    __syncthreads();
+    count_in(cnt_w, 1u);
+    form = last;
   } else {
     count_in(prm.count + bh, (uint32_t)prm.splits - 1u);
-  }
-  if (last) {   // block-uniform
-    if (!is_pinv) {
+    if (last) {   // block-uniform
+      __shared__ uint32_t z_ready;
+      if (t == 0) z_ready = flag_acquire(cnt_w);
+      __syncthreads();
+      const bool direct = z_ready != 0;   // Z stored: this block forms W
+      z_copy = direct && MergeSmem<M>::kZ;
       NYS_MARK(kTrMid, 3);
-      merge_y<M>(prm, smem, bh, true, Abort{&w_abort, prm.err});
+      merge_y<M>(prm, smem, bh, true, wab, z_copy);
       NYS_MARK(kTrMid, 4);
-    }
-    count_in(prm.count + prm.BH + bh, 1u);
-    if (last) {
-      NYS_MARK(kTrMid, 5);
-      // this block's own result is in the W operands already
-      form_w<M>(prm, smem, bh, tmem, Abort{&w_abort, prm.err}, is_pinv, !is_pinv);
-      // form_w ends with a block barrier after every thread's stores
-      if (t == 0) {
-        fence_async_global();   // the output kernel reads W with a bulk copy
-        flag_release(prm.count + 2 * prm.BH + bh, 1u);
+      y_staged = true;
+      if (direct) {
+        form = true;
+      } else {
+        count_in(cnt_w, 1u);
+        form = last;
       }
-      NYS_MARK(kTrMid, 6);
     }
+  }
+  if (form) {   // block-uniform
+    NYS_MARK(kTrMid, 5);
+    form_w<M>(prm, smem, bh, tmem, wab, z_staged, y_staged,
+              z_copy ? (const float *)(smem + MergeSmem<M>::zf) : nullptr);
+    // form_w ends with a block barrier after every thread's stores
+    if (t == 0) {
+      fence_async_global();   // the output kernel reads W with a bulk copy
+      flag_release(prm.count + 2 * prm.BH + bh, 1u);
+    }
+    NYS_MARK(kTrMid, 6);
   }
   tc_fence_before();
   __syncthreads();

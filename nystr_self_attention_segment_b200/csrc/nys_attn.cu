@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 #include <utility>
 
 #include "common.cuh"
@@ -1217,16 +1218,24 @@ NYS_ATTN_API nys_status nys_test_timeout_probe(void *workspace, const nys_desc *
 // `reset` is set.  Synchronises the device.
 NYS_ATTN_API nys_status nys_debug_timeline(void *host, size_t cap, uint32_t *count, int reset) {
   if (!count) return NYS_ERR_INVALID_ARG;
+  std::vector<TraceRec> all(kTraceCap);
   if (cudaDeviceSynchronize() != cudaSuccess ||
-      cudaMemcpyFromSymbol(count, g_trace_n, sizeof(uint32_t)) != cudaSuccess)
+      cudaMemcpyFromSymbol(all.data(), g_trace, sizeof(TraceRec) * kTraceCap) != cudaSuccess)
     return NYS_ERR_CUDA;
-  size_t n = *count < (uint32_t)kTraceCap ? *count : (size_t)kTraceCap;
-  if (n > cap) n = cap;
-  if (host && n && cudaMemcpyFromSymbol(host, g_trace, n * sizeof(TraceRec)) != cudaSuccess)
-    return NYS_ERR_CUDA;
+  // the used slots, in slot order
+  uint32_t n = 0;
+  for (const TraceRec &r : all) {
+    if (r.ns == 0) continue;
+    if (host && n < cap) ((TraceRec *)host)[n] = r;
+    ++n;
+  }
+  *count = n;
   if (reset) {
-    const uint32_t zero = 0;
-    if (cudaMemcpyToSymbol(g_trace_n, &zero, sizeof(zero)) != cudaSuccess) return NYS_ERR_CUDA;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_trace) != cudaSuccess ||
+        cudaMemset(p, 0, sizeof(TraceRec) * kTraceCap) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
+      return NYS_ERR_CUDA;
   }
   return NYS_OK;
 }
