@@ -17,15 +17,18 @@
 // 128-key chunk, so every TMEM lane has work.  Per chunk:
 //   TMA  K and V chunks (128 x 64 bf16, zero past n),
 //   MMA  S = [Q~; ..; Q~] K_c^T       (M=128, N=128, K=64, operands in smem),
-//   softmax warpgroup: P = 2^(s - m_ref) as bf16 straight into TMEM (zero
-//        outside the row's key group), row sums in fp32,
+//   softmax: P = 2^(s - m_ref) as bf16 straight into TMEM (zero outside the
+//        row's key group), row sums in fp32,
 //   MMA  Y += P V_c                    (M=128, N=64, K=128, P read from TMEM,
 //        Y accumulated in TMEM).
-// Two softmax warpgroups take alternate chunks, each with its own TMEM
-// buffers, reference maxima and sums; the 2G states of a landmark are merged
-// in the block at the end, giving one partial per (block, landmark).
-// Warps: 0 TMA producer, 1 and 2 MMA issuers (one per softmax warpgroup;
-// warp 1 owns TMEM), 4-7 and 8-11 softmax.
+// m <= 64 (bv_body): two softmax warpgroups take alternate chunks, each with
+// its own TMEM buffers, reference maxima and sums; warps 0 TMA producer, 1
+// and 2 MMA issuers (one per softmax warpgroup), 4-7 and 8-11 softmax.
+// m = 128 (bv_body_split): both warpgroups work on every chunk, warpgroup h
+// on half h of each row's keys, with S and P double-buffered; warps 0 TMA
+// producer, 1 MMA issuer, 4-11 softmax.  Either way the states of a landmark
+// are merged in the block at the end, giving one partial per (block,
+// landmark); warp 1 owns TMEM.
 #pragma once
 
 #include "pinv_pow.cuh"
@@ -92,12 +95,14 @@ struct Params {
 // Softmax over the keys with a lazily updated reference maximum: P =
 // 2^(s - m_ref) with m_ref raised only when a chunk's maximum exceeds it by
 // more than kTau (log2 units), so P <= 2^kTau and the Y accumulator (in TMEM,
-// summed by the P V MMAs) is rescaled only then.  The two softmax
-// warpgroups take turns through their exponential-heavy section (named
-// barriers 2 and 3), so one computes while the other waits on its MMAs.
+// summed by the P V MMAs) is rescaled only then.  In bv_body (m <= 64) the
+// two softmax warpgroups take alternate chunks and turns through their
+// exponential sections (named barriers 2 and 3); in bv_body_split (m = 128)
+// they split every chunk's keys between them (named barrier 2: the halves'
+// maxima), so a chunk's softmax is half as long a chain.
 constexpr float kTau = 8.f;
-// Turn-taking of the two softmax warpgroups through their exponential
-// sections (1), or both at once (0).
+// Turn-taking of the two softmax warpgroups of bv_body through their
+// exponential sections (1), or both at once (0).
 #ifndef NYS_BV_TURNS
 #define NYS_BV_TURNS 1
 #endif
@@ -437,6 +442,354 @@ __device__ __forceinline__ void bv_body(const CUtensorMap *map_k, const CUtensor
   }
 }
 
+// The same with the softmax warpgroups splitting every chunk's keys (used
+// for m = 128, whose rows hold 128 keys of a chunk: one thread per row would
+// keep 128 scores in registers).
+template <int M>
+__device__ __forceinline__ void bv_body_split(const CUtensorMap *map_k, const CUtensorMap *map_v,
+                                        const Params &prm, uint8_t *smem, int bh, int split,
+                                        uint32_t tmem_in, bool wait_prev = false) {
+  constexpr int G = 128 / M;
+  const BvSmem L = bv_smem();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // keys [0, L): L = n, or the element's own length (an invalid one reads as
+  // 0 and leaves the split empty; the segment-mean kernel reports it)
+  int seq = prm.n;
+  if (prm.lens) {
+    seq = prm.lens[bh / prm.heads];
+    if (seq < M || seq > prm.n || (long)(M - 1) * ((seq + M - 1) / M) >= seq) seq = 0;
+  }
+  const int c_begin = (int)((long)split * prm.chunks_per_head / prm.splits);
+  const int c_end = min((int)((long)(split + 1) * prm.chunks_per_head / prm.splits),
+                        (seq + kChunk - 1) / kChunk);
+  const int nch = c_end > c_begin ? c_end - c_begin : 0;
+
+  uint64_t *bars = (uint64_t *)(smem + L.bars);
+  uint64_t *full = bars;                  // [kStages]
+  uint64_t *empty = bars + kStages;       // [kStages]
+  uint64_t *s_full = bars + 2 * kStages;  // [2] per softmax warpgroup
+  uint64_t *s_free = s_full + 2;
+  uint64_t *p_ready = s_free + 2;
+  uint64_t *y_full = p_ready + 2;
+  constexpr int kBars = 2 * kStages + 8;
+  uint32_t *tmem_slot = (uint32_t *)(bars + kBars);
+  volatile uint32_t *abort_flag = tmem_slot + 1;
+  const Abort ab{abort_flag, prm.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 256);
+      mbar_init(&p_ready[b], 256);
+      mbar_init(&y_full[b], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(map_k);
+    tma_prefetch_desc(map_v);
+  }
+  if (tmem_in != ~0u) {
+    if (threadIdx.x == 0) *tmem_slot = tmem_in;
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+  }
+  __syncthreads();   // barriers initialised
+  const int pre = nch < kStages ? nch : kStages;   // chunk loads issued up front
+  // K is read here for the last time in the pass (V again by the output
+  // kernel): its lines leave L2 first
+  const uint64_t last_use = policy_evict_first();
+  auto load_v = [&](int s, int k0) {
+    if (NYS_V_EVICT_FIRST)
+      tma_load_3d_hint(smem + L.v[s], map_v, &full[s], 0, k0, bh, last_use);
+    else
+      tma_load_3d(smem + L.v[s], map_v, &full[s], 0, k0, bh);
+  };
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < pre; ++i) {
+      const int k0 = (c_begin + i) * kChunk;
+      mbar_expect_tx(&full[i], 32768u);
+      tma_load_3d_hint(smem + L.k[i], map_k, &full[i], 0, k0, bh, last_use);
+      load_v(i, k0);
+    }
+  }
+  if (wait_prev) {
+    griddep_wait();
+    griddep_launch_dependents();
+    NYS_MARK(kTrMid, 1);
+  }
+  // A operand rows: row r holds landmark r % M (bf16, 128-byte swizzle)
+  if (threadIdx.x < 256) {
+    const float4 *qt = (const float4 *)(prm.q_land + (size_t)bh * M * 64);
+    const int row = threadIdx.x >> 1, half = threadIdx.x & 1;   // 4 chunks each
+    float4 a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = __ldcg(qt + (row % M) * 16 + half * 8 + u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      st_shared_v4(smem_u32(smem + L.q) + sw128_offset(row, half * 4 + u),
+                   pack_bf16(a[2 * u].x, a[2 * u].y), pack_bf16(a[2 * u].z, a[2 * u].w),
+                   pack_bf16(a[2 * u + 1].x, a[2 * u + 1].y),
+                   pack_bf16(a[2 * u + 1].z, a[2 * u + 1].w));
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM: S of chunk i in buffer i & 1 (columns 128 (i & 1), 128 wide), P of
+  // chunk i at 256 + 64 (i & 1) (bf16 pairs, 64 wide), Y at 384 (64 wide).
+  // Both softmax warpgroups work on every chunk: warpgroup h takes half h of
+  // each row's keys, the two halves of a row agree on the row's reference
+  // maximum through shared memory, and P V runs once both halves of P are in.
+  constexpr uint32_t kP = 256, kY = 384;
+  __shared__ float xmax[2][2][128];   // chunk parity, half, row: the halves' maxima
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = pre; i < nch; ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ab)) break;
+        const int k0 = (c_begin + i) * kChunk;
+        mbar_expect_tx(&full[s], 32768u);
+        tma_load_3d_hint(smem + L.k[s], map_k, &full[s], 0, k0, bh, last_use);
+        load_v(s, k0);
+      }
+      // consume the stage releases nobody else waits for, so that no
+      // tensor-core arrival is pending when the barriers are invalidated
+      for (int i = nch > kStages ? nch - kStages : 0; i < nch; ++i)
+        if (!mbar_wait(&empty[i % kStages], (i / kStages) & 1, ab)) break;
+    }
+  } else if (warp == 1) {
+    // MMA issuer: S of the next chunks as soon as their buffer has been read,
+    // P V of a chunk once both halves of its P are in TMEM
+    if (lane == 0) {
+      const uint32_t id_s = make_idesc(kFmtBF16, 128, 128, 0, 0);
+      const uint32_t id_y = make_idesc(kFmtBF16, 128, 64, 0, 1);
+      const uint64_t dq = make_sdesc(smem_u32(smem + L.q), 16, 1024);
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % kStages;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, ab)) return false;
+        tc_fence_after();
+        const uint64_t dk = make_sdesc(smem_u32(smem + L.k[s]), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem + 128 * (i & 1), dq + 2u * k, dk + 2u * k, id_s, k > 0);
+        mma_commit(&s_full[i & 1]);
+        return true;
+      };
+      bool ok = nch > 0 ? issue_s(0) : true;
+      if (ok && nch > 1) ok = issue_s(1);
+      for (int i = 0; i < nch && ok; ++i) {
+        const int s = i % kStages, b = i & 1, u = i >> 1;
+        if (!mbar_wait(&p_ready[b], u & 1, ab)) break;
+        tc_fence_after();
+        const uint64_t dv = make_sdesc(smem_u32(smem + L.v[s]), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts(tmem + kY, tmem + kP + 64 * b + 8 * k, dv + 128u * k, id_y,
+                      (i > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&y_full[b]);
+        mma_commit(&empty[s]);
+        if (i + 2 < nch) {
+          if (!mbar_wait(&s_free[b], u & 1, ab)) break;
+          ok = issue_s(i + 2);
+        }
+      }
+    }
+  }
+  // softmax warpgroups; their running states are kept for the merge below
+  constexpr int H = M / 2;                 // keys of a row per chunk and half
+  float run_max = -INFINITY, run_sum = 0.f;
+  float acc[32];                           // this half of the row's Y
+  const int h = (warp >= 8) ? 1 : 0;
+  const int r = threadIdx.x & 127;          // accumulator row == TMEM lane
+  const int j = r % M, g = r / M;           // landmark, key group
+  if (warp >= 4) {
+    const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    {   // P starts at zero: each row only ever writes its own keys
+      uint32_t z[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) z[e] = 0u;
+      tmem_st32(t_row + kP + 32 * h, z);
+      tmem_st32(t_row + kP + 64 + 32 * h, z);
+      tmem_st_wait();
+    }
+    // ok stays uniform over the 256 softmax threads: a failed wait is
+    // reported at the next exchange barrier, where every thread leaves the
+    // loop (a thread that left before it would leave the others waiting)
+    bool ok = true;
+    for (int i = 0; i < nch; ++i) {
+      const int b = i & 1, u = i >> 1;
+      const bool got = ok && mbar_wait(&s_full[b], u & 1, ab);
+      if (threadIdx.x == 128 && blockIdx.x == (unsigned)prm.BH && i < 32) NYS_MARK_T(kTrMid, 32 + i);
+      tc_fence_after();
+      float v[H];
+      const int key0 = (c_begin + i) * kChunk + g * M + h * H;
+      const int valid = max(0, min(H, seq - key0));   // keys of this half inside [0, L)
+      float hmax = -INFINITY;
+      if (got) {
+        const uint32_t t_s = t_row + 128 * b + g * M + h * H;
+        if constexpr (H >= 32) {
+#pragma unroll
+          for (int c = 0; c < H; c += 32) tmem_ld32(t_s + c, v + c);
+        } else {
+          tmem_ld16(t_s, v);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[b]);
+        float mx[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+        if (valid == H) {
+#pragma unroll
+          for (int c = 0; c < H; ++c) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < H; ++c)
+            if (c < valid) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
+        }
+        hmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      }
+      // the row's maximum over both halves (the same value in both threads)
+      xmax[b][h][r] = hmax;
+      if (named_barrier_or(2, 256, !got)) {
+        ok = false;
+        break;
+      }
+      const float cmax = fmaxf(hmax, xmax[b][h ^ 1][r]) * prm.scale_log2;
+      const bool up = cmax > run_max + kTau;
+      bool y_done = false;   // P V of chunk i - 1 (and so of i - 2) has completed
+      // warp-uniform, and the same in the two warps that share these rows
+      if (__any_sync(0xffffffffu, up)) {
+        // raise the reference of the rows that need it and rescale this half
+        // of their Y
+        const float m_new = up ? cmax : run_max;
+        const float alpha = (run_max == -INFINITY) ? 0.f : fast_exp2(run_max - m_new);
+        if (i > 0) {
+          if (!(ok = mbar_wait(&y_full[(i - 1) & 1], ((i - 1) >> 1) & 1, ab))) continue;
+          tc_fence_after();
+          y_done = true;
+          float y[32];
+          tmem_ld32(t_row + kY + 32 * h, y);
+          tmem_ld_wait();
+          uint32_t ys[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ys[c] = __float_as_uint(y[c] * alpha);
+          tmem_st32(t_row + kY + 32 * h, ys);
+          tmem_st_wait();
+        }
+        run_sum *= alpha;
+        run_max = m_new;
+      }
+      const float mref = run_max;
+      const bool none = (mref == -INFINITY);
+      float ps[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+      uint32_t pk[H / 2];
+      if (valid == H && !none) {
+#pragma unroll
+        for (int c = 0; c < H; c += 2) {
+          const float p0 = fast_exp2(fmaf(v[c], prm.scale_log2, -mref));
+          const float p1 = fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mref));
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < H; c += 2) {
+          const float p0 = (c < valid && !none) ? fast_exp2(fmaf(v[c], prm.scale_log2, -mref)) : 0.f;
+          const float p1 =
+              (c + 1 < valid && !none) ? fast_exp2(fmaf(v[c + 1], prm.scale_log2, -mref)) : 0.f;
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+      }
+      run_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      // P buffer b was read by P V of chunk i - 2
+      if (i >= 2 && !y_done) {
+        if (!(ok = mbar_wait(&y_full[b], ((i - 2) >> 1) & 1, ab))) continue;
+        tc_fence_after();
+      }
+      const uint32_t t_p = t_row + kP + 64 * b + g * (M / 2) + h * (H / 2);
+      if constexpr (H / 2 >= 16) {
+#pragma unroll
+        for (int c = 0; c < H / 2; c += 16) tmem_st16(t_p + c, pk + c);
+      } else {
+        tmem_st8(t_p, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[b]);
+      if (threadIdx.x == 128 && blockIdx.x == (unsigned)prm.BH && i < 32) NYS_MARK_T(kTrMid, 96 + i);
+    }
+    // the state: this half of the row's Y after the last P V
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+    if (ok && nch > 0 &&
+        mbar_wait(&y_full[(nch - 1) & 1], ((nch - 1) >> 1) & 1, ab)) {
+      tc_fence_after();
+      tmem_ld32(t_row + kY + 32 * h, acc);
+      tmem_ld_wait();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();   // pipeline drained: stage buffers are free for the merge
+  if (threadIdx.x == 0 && !*abort_flag)
+    for (int bb = 0; bb < kBars; ++bb) mbar_inval(bars + bb);
+  if (warp == 1 && tmem_in == ~0u) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  // In-block merge of the G key groups of every landmark (two halves each),
+  // in a fixed order.
+  float *st = (float *)(smem + L.k[0]);   // [2][128][66]: max, half sum, Y (this half's columns)
+  if (warp >= 4) {
+    float *o = st + (h * 128 + r) * 66;
+    o[0] = run_max;
+    o[1] = run_sum;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) o[2 + 32 * h + c] = acc[c];
+  }
+  __syncthreads();
+  if (warp >= 4 && h == 0 && g == 0) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < G; ++q) mx = fmaxf(mx, st[(q * M + j) * 66]);
+    float f[G], den = 0.f;
+#pragma unroll
+    for (int q = 0; q < G; ++q) {
+      const float m_q = st[(q * M + j) * 66];
+      f[q] = (mx == -INFINITY || m_q == -INFINITY) ? 0.f : fast_exp2(m_q - mx);
+      den = fmaf(st[(q * M + j) * 66 + 1] + st[(128 + q * M + j) * 66 + 1], f[q], den);
+    }
+    const size_t base = ((size_t)bh * prm.splits + split) * M + j;
+    prm.pmax[base] = mx;
+    prm.psum[base] = den;
+    float4 *dst = (float4 *)(prm.py + base * 64);
+#pragma unroll 4
+    for (int c4 = 0; c4 < 16; ++c4) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < G; ++q) {
+        // columns 4 c4 .. 4 c4 + 3 come from half (4 c4) / 32
+        const float *o = st + (((c4 >= 8) ? 128 : 0) + q * M + j) * 66 + 2 + 4 * c4;
+        a.x = fmaf(f[q], o[0], a.x);
+        a.y = fmaf(f[q], o[1], a.y);
+        a.z = fmaf(f[q], o[2], a.z);
+        a.w = fmaf(f[q], o[3], a.w);
+      }
+      dst[c4] = a;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ merge + W
 // The last B~ V block of a head (counted with an atomic) merges the head's S
 // partial states (m_s, l_s, Y_s) of every landmark into Y, in split order
@@ -757,7 +1110,10 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   } else {
     const int b = blockIdx.x - prm.BH;
     const int bh = b / prm.splits, split = b % prm.splits;
-    bv_body<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
+    if constexpr (M == 128)
+      bv_body_split<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
+    else
+      bv_body<M>(&map_k, &map_v, prm, smem, bh, split, tmem, true);
   }
   NYS_MARK(kTrMid, 2);
   // hand-off.  Counts per head: count[bh] key-split blocks done,
