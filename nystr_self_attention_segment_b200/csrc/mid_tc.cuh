@@ -1086,8 +1086,9 @@ mid_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CU
   // launched early (programmatic dependent launch): the bodies wait for the
   // previous kernel before they read the landmarks, and only then let the
   // next kernel launch.  So the next kernel starts after the segment-mean
-  // kernel has completed and may read K~ before its own wait; it waits for
-  // this whole grid before it reads anything this grid writes.
+  // kernel has completed and may read K~ at once; it reads a head's W after
+  // that head's W flag (count[2 BH + bh]) and waits for this whole grid only
+  // before it exits.
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
