@@ -28,12 +28,14 @@
 //              dK~ (total), D = rowsum(dY * Y)
 //   bwd_keys   per 64-key tile: B, dB, dS_B; dK, dV (with the conv part);
 //              block partials of dQ~
+//   bwd_dqt_total  dQ~ = dQ~_A + the key blocks' partials, in order
 //   bwd_dq     dQ += dQ~_{seg(i)} / count
 //   bwd_dconv  dw summed over the batch and the row blocks, in order
 // Every sum runs in a fixed order: results are bitwise reproducible.
 #pragma once
 
 #include "common.cuh"
+#include "simt.cuh"
 
 namespace nys {
 namespace bwd {
@@ -41,31 +43,7 @@ namespace bwd {
 constexpr int kThreads = 256;
 constexpr int kTile = 64;   // rows / keys per tile
 
-// acc[r][c] += sum_k A(i, k) B(k, j) for the outputs this thread owns:
-// i = ty + 16 r, j = tx + 16 c (ty = t / 16, tx = t % 16), i < M, j < N.
-// A(i, k) = A[i * sai + k * sak], B(k, j) = B[k * sbk + j * sbj].
-template <int RM, int RN>
-__device__ __forceinline__ void mm_acc(float (&acc)[RM][RN], const float *A, int sai, int sak,
-                                       const float *B, int sbk, int sbj, int K, int M, int N) {
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  for (int k = 0; k < K; ++k) {
-    float a[RM], b[RN];
-#pragma unroll
-    for (int r = 0; r < RM; ++r) {
-      const int i = ty + 16 * r;
-      a[r] = i < M ? A[i * sai + k * sak] : 0.f;
-    }
-#pragma unroll
-    for (int c = 0; c < RN; ++c) {
-      const int j = tx + 16 * c;
-      b[c] = j < N ? B[k * sbk + j * sbj] : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < RM; ++r)
-#pragma unroll
-      for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
-  }
-}
+// mm_acc (simt.cuh): the register-tiled block product every kernel here uses.
 
 template <int RM, int RN>
 __device__ __forceinline__ void zero(float (&acc)[RM][RN]) {
@@ -107,22 +85,25 @@ struct RowsParams {
 
 template <int M>
 struct RowsSmem {
-  // padded fp32 tiles
+  // padded fp32 tiles; the V halo is only read by the conv gradient, which
+  // runs before F and dS_F are formed, so they share their bytes (two
+  // blocks per SM at m <= 64)
   static constexpr int LD = 65, LM = M + 1;
+  static constexpr uint32_t kHalo = (kTile + 62) * LD * 4, kFD = 2 * kTile * LM * 4;
   static constexpr uint32_t kt = 0;                            // [M][LD]
   static constexpr uint32_t w = kt + M * LD * 4;               // [M][LD]
   static constexpr uint32_t q = w + M * LD * 4;                // [64][LD]
   static constexpr uint32_t g = q + kTile * LD * 4;            // [64][LD]
-  static constexpr uint32_t f = g + kTile * LD * 4;            // [64][LM]
+  static constexpr uint32_t vh = g + kTile * LD * 4;           // [64 + 62][LD] V halo, or
+  static constexpr uint32_t f = vh;                            // [64][LM]
   static constexpr uint32_t ds = f + kTile * LM * 4;           // [64][LM]
-  static constexpr uint32_t vh = ds + kTile * LM * 4;          // [64 + 62][LD] V halo
-  static constexpr uint32_t cw = vh + (kTile + 62) * LD * 4;   // [64]
+  static constexpr uint32_t cw = vh + (kHalo > kFD ? kHalo : kFD);   // [64]
   static constexpr uint32_t dwc = cw + 64 * 4;                 // [64] conv partial
   static constexpr uint32_t total = dwc + 64 * 4;
 };
 
 template <typename T, int M>
-__global__ void __launch_bounds__(kThreads) bwd_rows(const RowsParams p) {
+__global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_rows(const RowsParams p) {
   using S = RowsSmem<M>;
   constexpr int LD = S::LD, LM = S::LM;
   constexpr int RM = M / 16;   // dW / dK~ rows per thread (m x 64 outputs)
@@ -169,6 +150,20 @@ __global__ void __launch_bounds__(kThreads) bwd_rows(const RowsParams p) {
         vh[i] = (row >= 0 && row < n && c < d) ? to_f(V[(size_t)row * d + c]) : 0.f;
       }
     __syncthreads();
+    // conv kernel gradient: tap j gets sum_i sum_c dO_i,c V_{i+j-half},c
+    if (k > 0) {
+      const int warp = t >> 5, lane = t & 31;
+      for (int j = warp; j < k; j += 8) {
+        float acc = 0.f;
+        for (int e = lane; e < kTile * d; e += 32) {
+          const int r = e / d, c = e % d;
+          acc = fmaf(gs[r * LD + c], vh[(r + j) * LD + c], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) dwc[j] += acc;
+      }
+      __syncthreads();   // fs and ds overwrite the halo
+    }
     {   // logits S = Q K~^T (64 x m) into fs, dF = dO W^T into ds
       float a[4][RM], b[4][RM];
       zero(a);
@@ -224,19 +219,6 @@ __global__ void __launch_bounds__(kThreads) bwd_rows(const RowsParams p) {
     // dW += F^T dO, dK~ += dS_F^T Q (m x d, over the tile's rows)
     mm_acc(dW, fs, 1, LM, gs, LD, 1, kTile, m, d);
     mm_acc(dK, ds, 1, LM, qs, LD, 1, kTile, m, d);
-    // conv kernel gradient: tap j gets sum_i sum_c dO_i,c V_{i+j-half},c
-    if (k > 0) {
-      const int warp = t >> 5, lane = t & 31;
-      for (int j = warp; j < k; j += 8) {
-        float acc = 0.f;
-        for (int e = lane; e < kTile * d; e += 32) {
-          const int r = e / d, c = e % d;
-          acc = fmaf(gs[r * LD + c], vh[(r + j) * LD + c], acc);
-        }
-        acc = warp_sum(acc);
-        if (lane == 0) dwc[j] += acc;
-      }
-    }
   }
   // block partials
   const size_t pb = ((size_t)bh * p.R + blk) * m * d;
@@ -282,10 +264,34 @@ __device__ __forceinline__ void mm_block(float *C, int ldc, const float *A, int 
   __syncthreads();
 }
 
+// sum_{r < R} x[r * stride], added in order of r; four loads in flight.
+__device__ __forceinline__ float sum_parts(const float *x, size_t stride, int R) {
+  float s = 0.f;
+  int r = 0;
+  for (; r + 4 <= R; r += 4) {
+    const float v0 = x[r * stride], v1 = x[(r + 1) * stride], v2 = x[(r + 2) * stride],
+                v3 = x[(r + 3) * stride];
+    s += v0;
+    s += v1;
+    s += v2;
+    s += v3;
+  }
+  for (; r < R; ++r) s += x[r * stride];
+  return s;
+}
+
+// Row stride of bwd_head<M>'s matrices: m columns or the d <= 64 columns of
+// the m x d ones, plus one so that a column walk (the transposed operands)
+// falls in 32 different banks.
+template <int M>
+__host__ __device__ constexpr int head_ld() {
+  return (M > 64 ? M : 64) + 1;
+}
+
 // Bytes of the twelve matrices of bwd_head<M>.
 template <int M>
 __host__ __device__ constexpr size_t head_bytes() {
-  return (size_t)12 * M * (M > 64 ? M : 64) * 4;
+  return (size_t)12 * M * head_ld<M>() * 4;
 }
 
 template <int M>
@@ -293,9 +299,8 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   constexpr int RM = M / 16;
   extern __shared__ __align__(16) float smem_f[];
   const int bh = blockIdx.x, t = threadIdx.x;
-  // twelve M x LDH matrices (m <= M rows; row stride LDH holds m columns and
-  // the d <= 64 columns of the m x d ones)
-  constexpr int ld = M > 64 ? M : 64, kMat = M * ld;
+  // twelve M x ld matrices (m <= M rows)
+  constexpr int ld = head_ld<M>(), kMat = M * ld;
   const int m = p.m, d = p.d;
   float *base = p.use_smem ? smem_f : p.scratch + (size_t)bh * (head_bytes<M>() / 4);
   float *A = base, *Zj = A + kMat, *P = Zj + kMat, *T1 = P + kMat, *T2 = T1 + kMat,
@@ -305,8 +310,7 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   const size_t hd = (size_t)bh * m * d;
   for (int e = t; e < m * d; e += kThreads) {
     const int i = e / d, c = e % d;
-    float sw = 0.f;
-    for (int r = 0; r < p.R; ++r) sw += p.dw_part[((size_t)bh * p.R + r) * m * d + e];
+    const float sw = sum_parts(p.dw_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
     X[i * ld + c] = sw;
     Y2[i * ld + c] = p.y[hd + e];
   }
@@ -371,24 +375,35 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
     __syncthreads();
   }
   // Z0 = A^T c, c = 1 / (||A||_1 ||A||_inf): gradients through c and the
-  // maximising column / row (first index at ties)
+  // maximising column / row (first index at ties).  Column sums, row sums
+  // and the rows of dc = sum_ij dZ_ij A_ji run one per thread, each in index
+  // order; one thread then takes the maxima and adds the rows in order.
   __shared__ float red[4];
   __shared__ int arg[2];
+  __shared__ float cs[M], rs[M], dcr[M];
+  for (int u = t; u < 3 * m; u += kThreads) {
+    const int i = u % m;
+    float s = 0.f;
+    if (u < m) {
+      for (int r = 0; r < m; ++r) s += fabsf(A[r * ld + i]);
+      cs[i] = s;
+    } else if (u < 2 * m) {
+      for (int j = 0; j < m; ++j) s += fabsf(A[i * ld + j]);
+      rs[i] = s;
+    } else {
+      for (int j = 0; j < m; ++j) s = fmaf(dZ[i * ld + j], A[j * ld + i], s);
+      dcr[i] = s;
+    }
+  }
+  __syncthreads();
   if (t == 0) {
     float n1 = -1.f, ninf = -1.f, dc = 0.f;
     int jc = 0, ir = 0;
-    for (int j = 0; j < m; ++j) {
-      float cs = 0.f;
-      for (int i = 0; i < m; ++i) cs += fabsf(A[i * ld + j]);
-      if (cs > n1) { n1 = cs; jc = j; }
-    }
-    for (int i = 0; i < m; ++i) {
-      float rs = 0.f;
-      for (int j = 0; j < m; ++j) rs += fabsf(A[i * ld + j]);
-      if (rs > ninf) { ninf = rs; ir = i; }
-    }
+    for (int j = 0; j < m; ++j)
+      if (cs[j] > n1) { n1 = cs[j]; jc = j; }
     for (int i = 0; i < m; ++i)
-      for (int j = 0; j < m; ++j) dc = fmaf(dZ[i * ld + j], A[j * ld + i], dc);
+      if (rs[i] > ninf) { ninf = rs[i]; ir = i; }
+    for (int i = 0; i < m; ++i) dc += dcr[i];
     red[0] = 1.f / (n1 * ninf);
     red[1] = dc;
     red[2] = n1;
@@ -427,8 +442,7 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   mm_block<RM, 4>(X, ld, dP, 1, ld, T1, ld, 1, m, m, d, p.scale, 0.f);
   for (int e = t; e < m * d; e += kThreads) {
     const int i = e / d, c = e % d;
-    float s = 0.f;
-    for (int r = 0; r < p.R; ++r) s += p.dkt_part[((size_t)bh * p.R + r) * m * d + e];
+    const float s = sum_parts(p.dkt_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
     p.dkt[hd + e] = s + X[i * ld + c];
   }
 }
@@ -447,22 +461,26 @@ struct KeysParams {
 
 template <int M>
 struct KeysSmem {
+  // the dO halo is only read by conv^T, which runs (into registers) before
+  // B and dS_B are formed, so they share their bytes (two blocks per SM at
+  // m <= 64)
   static constexpr int LD = 65, LK = kTile + 1;
+  static constexpr uint32_t kHalo = (kTile + 62) * LD * 4, kBD = 2 * M * LK * 4;
   static constexpr uint32_t qt = 0;                              // [M][LD]
   static constexpr uint32_t dy = qt + M * LD * 4;                // [M][LD]
   static constexpr uint32_t ks = dy + M * LD * 4;                // [64][LD]
   static constexpr uint32_t vs = ks + kTile * LD * 4;            // [64][LD]
-  static constexpr uint32_t b = vs + kTile * LD * 4;             // [M][LK]
+  static constexpr uint32_t gh = vs + kTile * LD * 4;            // [64 + 62][LD] dO halo, or
+  static constexpr uint32_t b = gh;                              // [M][LK]
   static constexpr uint32_t db = b + M * LK * 4;                 // [M][LK]
-  static constexpr uint32_t gh = db + M * LK * 4;                // [64 + 62][LD] dO halo
-  static constexpr uint32_t cw = gh + (kTile + 62) * LD * 4;     // [64]
+  static constexpr uint32_t cw = gh + (kHalo > kBD ? kHalo : kBD);   // [64]
   static constexpr uint32_t lse = cw + 64 * 4;                   // [M]
   static constexpr uint32_t dd = lse + M * 4;                    // [M]
   static constexpr uint32_t total = dd + M * 4;
 };
 
 template <typename T, int M>
-__global__ void __launch_bounds__(kThreads) bwd_keys(const KeysParams p) {
+__global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const KeysParams p) {
   using S = KeysSmem<M>;
   constexpr int LD = S::LD, LK = S::LK, RM = M / 16;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -512,6 +530,23 @@ __global__ void __launch_bounds__(kThreads) bwd_keys(const KeysParams p) {
         gh[i] = (row >= 0 && row < n && c < d) ? to_f(G[(size_t)row * d + c]) : 0.f;
       }
     __syncthreads();
+    // conv^T(dO) for the tile's dV outputs: dV_row += w[tp] dO[row - tp + half]
+    float cv[4][4];
+    zero(cv);
+    if (k > 0) {
+      const int ty = t >> 4, tx = t & 15;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int key = ty + 16 * r, col = tx + 16 * c;
+          float gv = 0.f;
+          for (int tp = 0; tp < k; ++tp)
+            gv = fmaf(cw[tp], gh[(key + (k - 1) - tp) * LD + col], gv);
+          cv[r][c] = gv;
+        }
+      __syncthreads();   // bs and dbs overwrite the halo
+    }
     {   // B = 2^(s log2e Q~ K^T - lse) (m x 64), dB = dY V^T
       float a[RM][4], b[RM][4];
       zero(a);
@@ -548,11 +583,8 @@ __global__ void __launch_bounds__(kThreads) bwd_keys(const KeysParams p) {
             const int j = seg_of(row, l);
             const float gk =
                 p.scale * a[r][c] + __ldg(p.dkt + hd + j * d + col) / (float)seg_count(j, l, n);
-            float gv = b[r][c];
-            for (int tp = 0; tp < k; ++tp)   // dV_row += w[tp] dO[row - tp + half]
-              gv = fmaf(cw[tp], gh[(key + (k - 1) - tp) * LD + col], gv);
             dK[(size_t)row * d + col] = from_f<T>(gk);
-            dV[(size_t)row * d + col] = from_f<T>(gv);
+            dV[(size_t)row * d + col] = from_f<T>(b[r][c] + cv[r][c]);
           }
         }
     }
@@ -563,20 +595,24 @@ __global__ void __launch_bounds__(kThreads) bwd_keys(const KeysParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// dQ += dQ~_{seg(i)} / count: dQ~ = dQ~_A + the key blocks' partials in
-// order, recomputed by every block of the head.
+// dQ~ = dQ~_A + the key blocks' partials in order, in place of dQ~_A: one
+// thread per element of the head's m x d matrix.
+__global__ void __launch_bounds__(kThreads)
+bwd_dqt_total(float *dqt, const float *dqt_part, int md, int S2) {
+  const int bh = blockIdx.y, e = blockIdx.x * kThreads + threadIdx.x;
+  if (e >= md) return;
+  const float s = sum_parts(dqt_part + (size_t)bh * S2 * md + e, (size_t)md, S2);
+  dqt[(size_t)bh * md + e] += s;
+}
+
+// dQ += dQ~_{seg(i)} / count over the block's rows.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-bwd_dq(void *dQv, const float *dqt_a, const float *dqt_part, int n, int d, int m, int S2,
-       int rows_per_block) {
+bwd_dq(void *dQv, const float *dqt, int n, int d, int m, int rows_per_block) {
   extern __shared__ float dq[];   // [m][d]
   const int bh = blockIdx.y, t = threadIdx.x;
   const size_t hd = (size_t)bh * m * d;
-  for (int e = t; e < m * d; e += kThreads) {
-    float s = dqt_a[hd + e];
-    for (int r = 0; r < S2; ++r) s += dqt_part[((size_t)bh * S2 + r) * m * d + e];
-    dq[e] = s;
-  }
+  for (int e = t; e < m * d; e += kThreads) dq[e] = dqt[hd + e];
   __syncthreads();
   T *dQ = (T *)dQv + (size_t)bh * n * d;
   const int l = (n + m - 1) / m;

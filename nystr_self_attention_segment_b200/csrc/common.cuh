@@ -15,7 +15,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxIters = 64;
 constexpr int kMaxConvK = 63;
 constexpr int kNumSms = 148;       // streaming multiprocessors of a B200
-constexpr int kTargetCtas = 296;   // 2 x 148
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -55,6 +55,21 @@ bool is_empty(const nys_desc *desc) {
 }
 
 
+// Key splits per head of the SIMT B~ V pass (whole 64-key tiles each): one
+// wave of three blocks per SM, at most 64 (the merge keeps a weight per split
+// and row in shared memory); *keys_per_split gets the split length.
+int simt_key_splits(size_t BH, size_t n, int *keys_per_split) {
+  const int tile = kSimtKeyTile;
+  const int ntiles = (int)((n + tile - 1) / tile);
+  int splits = BH ? (int)((3 * kNumSms) / BH) : 1;
+  if (splits > 64) splits = 64;
+  if (splits > ntiles) splits = ntiles;
+  if (splits < 1) splits = 1;
+  const int tiles_per_split = (ntiles + splits - 1) / splits;
+  *keys_per_split = tiles_per_split * tile;
+  return (ntiles + tiles_per_split - 1) / tiles_per_split;
+}
+
 Layout make_layout(const nys_desc *desc, int m) {
   Layout L;
   memset(&L, 0, sizeof(L));
@@ -75,15 +90,7 @@ Layout make_layout(const nys_desc *desc, int m) {
     splits = per_head;
     L.keys_per_split = 0;
   } else {
-    // key splits of the SIMT B~ V pass: enough blocks to fill the GPU twice
-    const int tile = kSimtKeyTile;
-    int ntiles = (int)((n + tile - 1) / tile);
-    splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
-    if (splits > ntiles) splits = ntiles;
-    if (splits < 1) splits = 1;
-    int tiles_per_split = (ntiles + splits - 1) / splits;
-    splits = (ntiles + tiles_per_split - 1) / tiles_per_split;
-    L.keys_per_split = tiles_per_split * tile;
+    splits = simt_key_splits(BH, n, &L.keys_per_split);
     L.bv_ctas_per_head = 0;
   }
   L.splits = splits;
@@ -240,17 +247,18 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   {
     const int use_smem = m <= 64;
     size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
-    if (!allow_smem(pinv_simt, sm) ||
-        launch(pinv_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
+    auto kern = pinv_simt_for(m);
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
                kt, z, scratch, m, d, scale, iters, use_smem, (float *)nullptr,
                (float *)nullptr) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
   {
-    size_t sm = ((size_t)m * d + kSimtKeyTile * (d + 1) + kSimtKeyTile * d) * 4;
+    const size_t sm = bv_partial_simt_smem(m);
     dim3 grid(L.splits, BH);
-    auto kern = m <= 64 ? bv_partial_simt<T, 8> : bv_partial_simt<T, 16>;
+    auto kern = bv_partial_simt_for<T>(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, qt, K, V,
                pmax, psum, py, n, d, m, L.splits, L.keys_per_split, scale_log2, lens,
@@ -259,9 +267,10 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     mk.after(stream);
   }
   {
-    size_t sm = (size_t)m * d * 4;
-    if (!allow_smem(merge_w_simt, sm) ||
-        launch(merge_w_simt, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false,
+    const size_t sm = merge_w_smem(m, d, L.splits);
+    auto kern = merge_w_simt_for(m);
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false,
                pmax, psum, py, z, y, w, m, d, L.splits, (float *)nullptr) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
@@ -478,20 +487,16 @@ BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
   memset(&L, 0, sizeof(L));
   const size_t BH = (size_t)desc->batch * desc->heads;
   const size_t n = desc->seq_len, d = desc->head_dim;
-  const int tile = kSimtKeyTile;
-  const int ntiles = (int)((n + tile - 1) / tile);
-  int splits = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
-  if (splits > ntiles) splits = ntiles;
-  if (splits < 1) splits = 1;
-  const int tps = (ntiles + splits - 1) / splits;
-  L.S = (ntiles + tps - 1) / tps;
-  L.keys_per_split = tps * tile;
+  L.S = simt_key_splits(BH, n, &L.keys_per_split);
+  // row / key blocks per head: one wave of the resident blocks (two per SM
+  // for m <= 64, one for m = 128), so that no SM runs a tail of its own
+  L.mb = bwd_mbucket(m);
   const int t64 = (int)((n + bwd::kTile - 1) / bwd::kTile);
-  int r = BH ? (int)((kTargetCtas + BH - 1) / BH) : 1;
+  const int slots = kNumSms * (L.mb <= 64 ? 2 : 1);
+  int r = BH ? (int)(slots / BH) : 1;
   if (r > t64) r = t64;
   if (r < 1) r = 1;
   L.R = L.S2 = r;
-  L.mb = bwd_mbucket(m);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t at = off;
@@ -551,15 +556,16 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
   {
     const int use_smem = m <= 64;
     const size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
-    if (!allow_smem(pinv_simt, sm) ||
-        launch(pinv_simt, dim3(BH), dim3(256), sm, stream, false, (const float *)qt,
+    auto kern = pinv_simt_for(m);
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH), dim3(256), sm, stream, false, (const float *)qt,
                (const float *)kt, z, (float *)(ws + L.pscr), m, d, scale, iters, use_smem, a,
                zall) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
   {
-    const size_t sm = ((size_t)m * d + kSimtKeyTile * (d + 1) + kSimtKeyTile * d) * 4;
-    auto kern = m <= 64 ? bv_partial_simt<T, 8> : bv_partial_simt<T, 16>;
+    const size_t sm = bv_partial_simt_smem(m);
+    auto kern = bv_partial_simt_for<T>(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(L.S, BH), dim3(256), sm, stream, false, (const float *)qt, K, V, pmax,
                psum, py, n, d, m, L.S, L.keys_per_split, scale_log2, (const int *)nullptr,
@@ -567,9 +573,10 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
       return NYS_ERR_CUDA;
   }
   {
-    const size_t sm = (size_t)m * d * 4;
-    if (!allow_smem(merge_w_simt, sm) ||
-        launch(merge_w_simt, dim3(BH), dim3(256), sm, stream, false, (const float *)pmax,
+    const size_t sm = merge_w_smem(m, d, L.S);
+    auto kern = merge_w_simt_for(m);
+    if (!allow_smem(kern, sm) ||
+        launch(kern, dim3(BH), dim3(256), sm, stream, false, (const float *)pmax,
                (const float *)psum, (const float *)py, (const float *)z, y, w, m, d, L.S,
                lse) != cudaSuccess)
       return NYS_ERR_CUDA;
@@ -606,14 +613,17 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
         launch(kern, dim3(L.S2, BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
+  if (launch(bwd::bwd_dqt_total, dim3((m * d + bwd::kThreads - 1) / bwd::kThreads, BH),
+             dim3(bwd::kThreads), 0, stream, false, (float *)(ws + L.dqta),
+             (const float *)(ws + L.dqtp), m * d, L.S2) != cudaSuccess)
+    return NYS_ERR_CUDA;
   {
     const int rpb = 256;
     const size_t sm = (size_t)m * d * 4;
     auto kern = bwd::bwd_dq<T>;
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3((n + rpb - 1) / rpb, BH), dim3(bwd::kThreads), sm, stream, false,
-               (void *)dQ, (const float *)(ws + L.dqta), (const float *)(ws + L.dqtp), n, d, m,
-               L.S2, rpb) != cudaSuccess)
+               (void *)dQ, (const float *)(ws + L.dqta), n, d, m, rpb) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
   if (ck > 0 &&

@@ -56,18 +56,60 @@ __global__ void seg_means_scalar(const T *__restrict__ Q, const T *__restrict__ 
 }
 
 // ---------------------------------------------------------------------------
+// Register-tiled block product on 256 threads: acc[r][c] += sum_k A(i, k)
+// B(k, j) for the outputs this thread owns, i = ty + 16 r, j = tx + 16 c
+// (ty = t / 16, tx = t % 16), i < M, j < N, terms added in order of k.
+// A(i, k) = A[i * sai + k * sak], B(k, j) = B[k * sbk + j * sbj].
+template <int RM, int RN>
+__device__ __forceinline__ void mm_acc(float (&acc)[RM][RN], const float *A, int sai, int sak,
+                                       const float *B, int sbk, int sbj, int K, int M, int N) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float a[RM], b[RN];
+#pragma unroll
+    for (int r = 0; r < RM; ++r) {
+      const int i = ty + 16 * r;
+      a[r] = i < M ? A[i * sai + k * sak] : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < RN; ++c) {
+      const int j = tx + 16 * c;
+      b[c] = j < N ? B[k * sbk + j * sbj] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Landmark kernel A = softmax(Q~ K~^T / sqrt(d)) and its pseudoinverse by
 // Lemma 1 as printed: Z <- 1/4 Z (13I - AZ (15I - AZ (7I - AZ))), from
-// Z0 = A^T / (||A||_1 ||A||_inf).  One block per head; all five m x m fp32
-// matrices live in `mats` (shared memory when it fits, else the per-head
-// workspace scratch).
+// Z0 = A^T / (||A||_1 ||A||_inf).  One block of 256 threads per head; all
+// five m x m fp32 matrices live in `mats` (shared memory when it fits, else
+// the per-head workspace scratch).
+//
+// Products run register-tiled: thread (ty, tx) = (t / 16, t % 16) owns the
+// outputs (ty + 16 r, tx + 16 c), r, c < RM (m <= 16 RM), and adds each one's
+// terms in index order with fmaf.
+template <int RM>
 __device__ __forceinline__ void block_gemm(float *C, const float *X, const float *Y, int m) {
-  for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
-    int i = idx / m, j = idx % m;
-    float acc = 0.f;
-    for (int k = 0; k < m; ++k) acc = fmaf(X[i * m + k], Y[k * m + j], acc);
-    C[idx] = acc;
-  }
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[RM][RM];
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < RM; ++c) acc[r][c] = 0.f;
+  mm_acc(acc, X, m, 1, Y, m, 1, m, m, m);
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < RM; ++c) {
+      const int i = ty + 16 * r, j = tx + 16 * c;
+      if (i < m && j < m) C[i * m + j] = acc[r][c];
+    }
   __syncthreads();
 }
 
@@ -81,57 +123,75 @@ __device__ __forceinline__ void block_diag_minus(float *dst, const float *src, f
 
 // a_out, z_all (optional, for the backward pass): A [BH][m][m] and every
 // iterate Z0 .. Z_iters [BH][iters + 1][m][m].
-__global__ void pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt,
-                          float *__restrict__ Zout, float *__restrict__ scratch, int m, int d,
-                          float scale, int iters, int use_smem, float *__restrict__ a_out = nullptr,
-                          float *__restrict__ z_all = nullptr) {
+template <int RM>   // m <= 16 RM
+__global__ void __launch_bounds__(256)
+pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__restrict__ Zout,
+          float *__restrict__ scratch, int m, int d, float scale, int iters, int use_smem,
+          float *__restrict__ a_out = nullptr, float *__restrict__ z_all = nullptr) {
   extern __shared__ float smem[];
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x, t = threadIdx.x;
   float *mats = use_smem ? smem : scratch + (size_t)bh * 5 * m * m;
   float *A = mats, *Z = A + m * m, *P = Z + m * m, *T1 = P + m * m, *T2 = T1 + m * m;
   __shared__ float red[2];
+  __shared__ float nsum[2 * 16 * RM];   // column sums, then row sums
   const float *qt = Qt + (size_t)bh * m * d;
   const float *kt = Kt + (size_t)bh * m * d;
-
-  for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
-    int i = idx / m, j = idx % m;
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(qt[i * d + c], kt[j * d + c], acc);
-    A[idx] = acc * scale;
+  {   // logits, each a dot product over the features in order
+    const int ty = t >> 4, tx = t & 15;
+    float acc[RM][RM];
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int c = 0; c < RM; ++c) acc[r][c] = 0.f;
+    mm_acc(acc, qt, d, 1, kt, 1, d, d, m, m);
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int c = 0; c < RM; ++c) {
+        const int i = ty + 16 * r, j = tx + 16 * c;
+        if (i < m && j < m) A[i * m + j] = acc[r][c] * scale;
+      }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < m; i += blockDim.x) {        // row softmax
-    float mx = -INFINITY;
-    for (int j = 0; j < m; ++j) mx = fmaxf(mx, A[i * m + j]);
+  {   // row softmax, a warp per row
+    const int warp = t >> 5, lane = t & 31;
+    for (int i = warp; i < m; i += 8) {
+      float mx = -INFINITY;
+      for (int j = lane; j < m; j += 32) mx = fmaxf(mx, A[i * m + j]);
+      mx = warp_max(mx);
+      float s = 0.f;
+      for (int j = lane; j < m; j += 32) {
+        const float e = __expf(A[i * m + j] - mx);
+        A[i * m + j] = e;
+        s += e;
+      }
+      const float inv = 1.f / warp_sum(s);
+      for (int j = lane; j < m; j += 32) A[i * m + j] *= inv;
+    }
+  }
+  __syncthreads();
+  // ||A||_1 (max column sum) and ||A||_inf (max row sum): each sum in index
+  // order by its own thread, the maxima in order by one thread, so the
+  // result is deterministic.
+  for (int u = t; u < 2 * m; u += blockDim.x) {
     float s = 0.f;
-    for (int j = 0; j < m; ++j) {
-      float e = __expf(A[i * m + j] - mx);
-      A[i * m + j] = e;
-      s += e;
+    if (u < m) {
+      for (int i = 0; i < m; ++i) s += fabsf(A[i * m + u]);
+    } else {
+      for (int j = 0; j < m; ++j) s += fabsf(A[(u - m) * m + j]);
     }
-    float inv = 1.f / s;
-    for (int j = 0; j < m; ++j) A[i * m + j] *= inv;
+    nsum[u] = s;
   }
   __syncthreads();
-  // ||A||_1 (max column sum) and ||A||_inf (max row sum), sequential in a
-  // fixed order by one thread so the result is deterministic.
-  if (threadIdx.x == 0) {
+  if (t == 0) {
     float n1 = 0.f, ninf = 0.f;
-    for (int j = 0; j < m; ++j) {
-      float cs = 0.f;
-      for (int i = 0; i < m; ++i) cs += fabsf(A[i * m + j]);
-      n1 = fmaxf(n1, cs);
-    }
-    for (int i = 0; i < m; ++i) {
-      float rs = 0.f;
-      for (int j = 0; j < m; ++j) rs += fabsf(A[i * m + j]);
-      ninf = fmaxf(ninf, rs);
-    }
+    for (int j = 0; j < m; ++j) n1 = fmaxf(n1, nsum[j]);
+    for (int i = 0; i < m; ++i) ninf = fmaxf(ninf, nsum[m + i]);
     red[0] = 1.f / (n1 * ninf);
   }
   __syncthreads();
   const float c0 = red[0];
-  for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
+  for (int idx = t; idx < m * m; idx += blockDim.x) {
     int i = idx / m, j = idx % m;
     Z[idx] = A[j * m + i] * c0;
     if (a_out) a_out[(size_t)bh * m * m + idx] = A[idx];
@@ -139,53 +199,69 @@ __global__ void pinv_simt(const float *__restrict__ Qt, const float *__restrict_
   }
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
-    block_gemm(P, A, Z, m);               // AZ
+    block_gemm<RM>(P, A, Z, m);           // AZ
     block_diag_minus(T1, P, 7.f, m);      // 7I - AZ
-    block_gemm(T2, P, T1, m);             // AZ (7I - AZ)
+    block_gemm<RM>(T2, P, T1, m);         // AZ (7I - AZ)
     block_diag_minus(T1, T2, 15.f, m);    // 15I - ...
-    block_gemm(T2, P, T1, m);             // AZ (15I - ...)
+    block_gemm<RM>(T2, P, T1, m);         // AZ (15I - ...)
     block_diag_minus(T1, T2, 13.f, m);    // 13I - ...
-    block_gemm(T2, Z, T1, m);             // Z (13I - ...)
-    for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
+    block_gemm<RM>(T2, Z, T1, m);         // Z (13I - ...)
+    for (int idx = t; idx < m * m; idx += blockDim.x) {
       Z[idx] = 0.25f * T2[idx];
       if (z_all) z_all[((size_t)bh * (iters + 1) + it + 1) * m * m + idx] = 0.25f * T2[idx];
     }
     __syncthreads();
   }
   float *zo = Zout + (size_t)bh * m * m;
-  for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) zo[idx] = Z[idx];
+  for (int idx = t; idx < m * m; idx += blockDim.x) zo[idx] = Z[idx];
+}
+
+// pinv_simt for m landmarks (m <= 128)
+inline auto pinv_simt_for(int m) {
+  return m <= 32 ? pinv_simt<2> : (m <= 64 ? pinv_simt<4> : pinv_simt<8>);
 }
 
 // ---------------------------------------------------------------------------
 // B~ V over one split of the keys (Eq. 17): for every landmark row j, an
 // online softmax over the split's keys of s * q~_j . k_i, keeping the running
 // maximum (log2 units), the running sum and the unnormalised sum of p_i v_i.
-// Grid (splits, heads), 8 warps; warp w owns rows j = w, w+8, ...; lane owns
-// features lane and lane+32.
-constexpr int kSimtKeyTile = 32;
+// Grid (splits, heads), 256 threads; per 64-key tile the logits and the
+// P V product run register-tiled (thread (ty, tx) owns rows ty + 16 r and
+// keys / features tx + 16 c), and the 16 threads of a row reduce its tile
+// maximum and sum by shuffles.
+constexpr int kSimtKeyTile = 64;
+constexpr int kSimtLd = 65;   // padded rows of the tiles (d <= 64 or 64 keys)
 
-template <typename T, int kSimtMaxRowsPerWarp>   // m <= 8 * kSimtMaxRowsPerWarp
+template <int RM>   // m <= 16 RM
+__host__ __device__ constexpr size_t bv_partial_smem() {
+  return (size_t)(2 * 16 * RM + 2 * kSimtKeyTile) * kSimtLd * 4;
+}
+
+template <typename T, int RM>   // m <= 16 RM
 __global__ void __launch_bounds__(256)
 bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *__restrict__ V,
                 float *__restrict__ pmax, float *__restrict__ psum, float *__restrict__ py,
                 int n, int d, int m, int splits, int keys_per_split, float scale_log2,
                 const int *lens, int heads) {
+  constexpr int LD = kSimtLd, kT = kSimtKeyTile;
   extern __shared__ float smem[];
-  const int split = blockIdx.x, bh = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float *qs = smem;                            // [m][d]
-  float *ks = qs + m * d;                      // [32][d+1]
-  float *vs = ks + kSimtKeyTile * (d + 1);     // [32][d]
-  for (int i = threadIdx.x; i < m * d; i += blockDim.x) qs[i] = Qt[(size_t)bh * m * d + i];
-
-  float M[kSimtMaxRowsPerWarp], S[kSimtMaxRowsPerWarp], y0[kSimtMaxRowsPerWarp],
-      y1[kSimtMaxRowsPerWarp];
+  const int split = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int ty = t >> 4, tx = t & 15;
+  float *qs = smem;                 // [16 RM][LD] Q~ rows
+  float *ks = qs + 16 * RM * LD;    // [64][LD]
+  float *vs = ks + kT * LD;         // [64][LD]
+  float *ps = vs + kT * LD;         // [16 RM][LD] the tile's p (row j, key)
+  for (int i = t; i < 16 * RM * LD; i += 256) {
+    const int j = i / LD, c = i % LD;
+    qs[i] = (j < m && c < d) ? Qt[((size_t)bh * m + j) * d + c] : 0.f;
+  }
+  float Mx[RM], Sm[RM], y[RM][4];
 #pragma unroll
-  for (int r = 0; r < kSimtMaxRowsPerWarp; ++r) {
-    M[r] = -INFINITY;
-    S[r] = 0.f;
-    y0[r] = 0.f;
-    y1[r] = 0.f;
+  for (int r = 0; r < RM; ++r) {
+    Mx[r] = -INFINITY;
+    Sm[r] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) y[r][c] = 0.f;
   }
   // keys of the element: [0, L) (an invalid length reads as 0: no keys)
   const int L = seq_len_of(lens, bh, heads, n, m, nullptr);
@@ -193,90 +269,148 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
   const int k1 = min(L, k0 + keys_per_split);
   const T *Kh = K + (size_t)bh * n * d;
   const T *Vh = V + (size_t)bh * n * d;
-  for (int t0 = k0; t0 < k1; t0 += kSimtKeyTile) {
+  for (int t0 = k0; t0 < k1; t0 += kT) {
     __syncthreads();
-    for (int i = threadIdx.x; i < kSimtKeyTile * d; i += blockDim.x) {
-      int r = i / d, c = i % d;
-      int key = t0 + r;
-      float kv = 0.f, vv = 0.f;
-      if (key < k1) {
-        kv = to_f(Kh[(size_t)key * d + c]);
-        vv = to_f(Vh[(size_t)key * d + c]);
-      }
-      ks[r * (d + 1) + c] = kv;
-      vs[r * d + c] = vv;
+    for (int i = t; i < kT * LD; i += 256) {
+      const int r = i / LD, c = i % LD, key = t0 + r;
+      const bool in = key < k1 && c < d;
+      ks[i] = in ? to_f(Kh[(size_t)key * d + c]) : 0.f;
+      vs[i] = in ? to_f(Vh[(size_t)key * d + c]) : 0.f;
     }
     __syncthreads();
-    const bool valid = (t0 + lane) < k1;
+    float sc[RM][4];
 #pragma unroll
-    for (int r = 0; r < kSimtMaxRowsPerWarp; ++r) {
-      const int j = warp + 8 * r;
-      if (j >= m) break;
-      float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(qs[j * d + c], ks[lane * (d + 1) + c], acc);
-      float l2 = valid ? acc * scale_log2 : -INFINITY;
-      float mnew = fmaxf(M[r], warp_max(l2));
-      float alpha = exp2f(M[r] - mnew);        // 0 when M was -inf
-      float p = exp2f(l2 - mnew);
-      S[r] = S[r] * alpha + warp_sum(p);
-      float a0 = y0[r] * alpha, a1 = y1[r] * alpha;
-      for (int i = 0; i < kSimtKeyTile; ++i) {
-        float pi = __shfl_sync(0xffffffffu, p, i);
-        if (lane < d) a0 = fmaf(pi, vs[i * d + lane], a0);
-        if (lane + 32 < d) a1 = fmaf(pi, vs[i * d + lane + 32], a1);
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sc[r][c] = 0.f;
+    mm_acc(sc, qs, LD, 1, ks, 1, LD, d, 16 * RM, kT);
+#pragma unroll
+    for (int r = 0; r < RM; ++r) {
+      float l2[4], mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        l2[c] = t0 + tx + 16 * c < k1 ? sc[r][c] * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, l2[c]);
       }
-      y0[r] = a0;
-      y1[r] = a1;
-      M[r] = mnew;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mnew = fmaxf(Mx[r], mx);     // finite: the tile's first key is in range
+      const float alpha = exp2f(Mx[r] - mnew);  // 0 when Mx was -inf
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float p = exp2f(l2[c] - mnew);
+        ps[(ty + 16 * r) * LD + tx + 16 * c] = p;
+        sum += p;
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      Sm[r] = Sm[r] * alpha + sum;
+      Mx[r] = mnew;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) y[r][c] *= alpha;
     }
+    __syncthreads();
+    mm_acc(y, ps, LD, 1, vs, LD, 1, kT, 16 * RM, d);
   }
   const size_t base = ((size_t)bh * splits + split) * m;
 #pragma unroll
-  for (int r = 0; r < kSimtMaxRowsPerWarp; ++r) {
-    const int j = warp + 8 * r;
-    if (j >= m) break;
-    if (lane == 0) {
-      pmax[base + j] = M[r];
-      psum[base + j] = S[r];
+  for (int r = 0; r < RM; ++r) {
+    const int j = ty + 16 * r;
+    if (j >= m) continue;
+    if (tx == 0) {
+      pmax[base + j] = Mx[r];
+      psum[base + j] = Sm[r];
     }
-    if (lane < d) py[(base + j) * d + lane] = y0[r];
-    if (lane + 32 < d) py[(base + j) * d + lane + 32] = y1[r];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (tx + 16 * c < d) py[(base + j) * d + tx + 16 * c] = y[r][c];
   }
+}
+
+// bv_partial_simt for m landmarks (m <= 128)
+template <typename T>
+inline auto bv_partial_simt_for(int m) {
+  return m <= 32 ? bv_partial_simt<T, 2> : (m <= 64 ? bv_partial_simt<T, 4> : bv_partial_simt<T, 8>);
+}
+inline size_t bv_partial_simt_smem(int m) {
+  return m <= 32 ? bv_partial_smem<2>() : (m <= 64 ? bv_partial_smem<4>() : bv_partial_smem<8>());
 }
 
 // ---------------------------------------------------------------------------
 // Merge of the key splits in split order (Y = B~ V), then W = Z Y.  One block
-// per head.
-__global__ void merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
-                             const float *__restrict__ py, const float *__restrict__ Zg,
-                             float *__restrict__ Yg, float *__restrict__ Wg, int m, int d,
-                             int splits, float *__restrict__ lse2 = nullptr) {
-  extern __shared__ float ys[];   // [m][d]
-  const int bh = blockIdx.x;
+// of 256 threads per head: a thread per landmark row takes the row's maximum
+// and weights, every output then adds its splits in order, and W runs
+// register-tiled (m <= 16 RM).
+inline size_t merge_w_smem(int m, int d, int splits) {
+  return ((size_t)m * d + (size_t)m * m + (size_t)splits * m + m) * 4;
+}
+
+template <int RM>
+__global__ void __launch_bounds__(256)
+merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
+             const float *__restrict__ py, const float *__restrict__ Zg, float *__restrict__ Yg,
+             float *__restrict__ Wg, int m, int d, int splits, float *__restrict__ lse2 = nullptr) {
+  extern __shared__ float smem[];
+  const int bh = blockIdx.x, t = threadIdx.x;
+  float *ys = smem;                    // [m][d]
+  float *zs = ys + m * d;              // [m][m]
+  float *fac = zs + m * m;             // [splits][m]: 2^(max_s - max)
+  float *tot = fac + splits * m;       // [m]: the row's merged sum
   const size_t pb = (size_t)bh * splits * m;
-  for (int idx = threadIdx.x; idx < m * d; idx += blockDim.x) {
-    int j = idx / d, c = idx % d;
+  for (int j = t; j < m; j += 256) {
     float mx = -INFINITY;
     for (int s = 0; s < splits; ++s) mx = fmaxf(mx, pmax[pb + (size_t)s * m + j]);
-    float sum = 0.f, acc = 0.f;
+    float sum = 0.f;
     for (int s = 0; s < splits; ++s) {
-      float f = exp2f(pmax[pb + (size_t)s * m + j] - mx);
+      const float f = exp2f(pmax[pb + (size_t)s * m + j] - mx);
+      fac[s * m + j] = f;
       sum = fmaf(psum[pb + (size_t)s * m + j], f, sum);
-      acc = fmaf(py[(pb + (size_t)s * m + j) * d + c], f, acc);
     }
-    float y = acc / sum;
-    if (lse2 && c == 0) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
+    tot[j] = sum;
+    if (lse2) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
+  }
+  for (int e = t; e < m * m; e += 256) zs[e] = Zg[(size_t)bh * m * m + e];
+  __syncthreads();
+  for (int idx = t; idx < m * d; idx += 256) {
+    const int j = idx / d;
+    const float *src = py + pb * d + idx;
+    const size_t stride = (size_t)m * d;
+    float acc = 0.f;
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {   // four loads in flight, added in order
+      const float v0 = src[s * stride], v1 = src[(s + 1) * stride], v2 = src[(s + 2) * stride],
+                  v3 = src[(s + 3) * stride];
+      acc = fmaf(v0, fac[s * m + j], acc);
+      acc = fmaf(v1, fac[(s + 1) * m + j], acc);
+      acc = fmaf(v2, fac[(s + 2) * m + j], acc);
+      acc = fmaf(v3, fac[(s + 3) * m + j], acc);
+    }
+    for (; s < splits; ++s) acc = fmaf(src[s * stride], fac[s * m + j], acc);
+    const float y = acc / tot[j];
     ys[idx] = y;
     Yg[(size_t)bh * m * d + idx] = y;
   }
   __syncthreads();
-  const float *z = Zg + (size_t)bh * m * m;
-  for (int idx = threadIdx.x; idx < m * d; idx += blockDim.x) {
-    int j = idx / d, c = idx % d;
-    float acc = 0.f;
-    for (int k = 0; k < m; ++k) acc = fmaf(z[j * m + k], ys[k * d + c], acc);
-    Wg[(size_t)bh * m * d + idx] = acc;
-  }
+  float acc[RM][4];
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+  mm_acc(acc, zs, m, 1, ys, d, 1, m, m, d);
+  const int ty = t >> 4, tx = t & 15;
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = ty + 16 * r, col = tx + 16 * c;
+      if (j < m && col < d) Wg[((size_t)bh * m + j) * d + col] = acc[r][c];
+    }
+}
+
+// merge_w_simt for m landmarks (m <= 128)
+inline auto merge_w_simt_for(int m) {
+  return m <= 32 ? merge_w_simt<2> : (m <= 64 ? merge_w_simt<4> : merge_w_simt<8>);
 }
 
 // ---------------------------------------------------------------------------
