@@ -41,6 +41,7 @@ namespace nys {
 namespace bwd {
 
 constexpr int kThreads = 256;
+constexpr int kHeadThreads = 512;   // bwd_head: one block per head, twice the warps
 constexpr int kTile = 64;   // rows / keys per tile
 
 // mm_acc (simt.cuh): the register-tiled block product every kernel here uses.
@@ -83,12 +84,15 @@ struct RowsParams {
   float scale;
 };
 
+// Row stride of the 64-column tiles: 16-byte aligned rows, 4 mod 32 words.
+constexpr int kLd = 68;
+
 template <int M>
 struct RowsSmem {
-  // padded fp32 tiles; the V halo is only read by the conv gradient, which
+  // padded fp32 tiles (rows of 16-byte multiples, zero beyond the data); the V halo is only read by the conv gradient, which
   // runs before F and dS_F are formed, so they share their bytes (two
   // blocks per SM at m <= 64)
-  static constexpr int LD = 65, LM = M + 1;
+  static constexpr int LD = kLd, LM = M + 4;
   static constexpr uint32_t kHalo = (kTile + 62) * LD * 4, kFD = 2 * kTile * LM * 4;
   static constexpr uint32_t kt = 0;                            // [M][LD]
   static constexpr uint32_t w = kt + M * LD * 4;               // [M][LD]
@@ -99,22 +103,28 @@ struct RowsSmem {
   static constexpr uint32_t ds = f + kTile * LM * 4;           // [64][LM]
   static constexpr uint32_t cw = vh + (kHalo > kFD ? kHalo : kFD);   // [64]
   static constexpr uint32_t dwc = cw + 64 * 4;                 // [64] conv partial
-  static constexpr uint32_t total = dwc + 64 * 4;
+  static constexpr uint32_t cpart = dwc + 64 * 4;              // [64][2] the tile's tap halves
+  static constexpr uint32_t total = cpart + 128 * 4;
 };
+
+// Taps per thread of the conv gradient: 64 columns x ceil(k / kTapGroup)
+// groups fill the block once for k <= 36.
+constexpr int kTapGroup = 9;
 
 template <typename T, int M>
 __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_rows(const RowsParams p) {
   using S = RowsSmem<M>;
   constexpr int LD = S::LD, LM = S::LM;
-  constexpr int RM = M / 16;   // dW / dK~ rows per thread (m x 64 outputs)
+  constexpr int RM = M / 16;   // landmarks per thread (dW, dK~ rows; F, dF columns)
   extern __shared__ __align__(16) uint8_t smem[];
   float *kt = (float *)(smem + S::kt), *w = (float *)(smem + S::w);
   float *qs = (float *)(smem + S::q), *gs = (float *)(smem + S::g);
   float *fs = (float *)(smem + S::f), *ds = (float *)(smem + S::ds);
   float *vh = (float *)(smem + S::vh), *cw = (float *)(smem + S::cw);
-  float *dwc = (float *)(smem + S::dwc);
+  float *dwc = (float *)(smem + S::dwc), *cpart = (float *)(smem + S::cpart);
   const int blk = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int n = p.n, d = p.d, m = p.m, head = bh % p.heads;
+  const int d4 = round4(d), m4 = round4(m);
   const int k = p.conv_w ? p.conv_k : 0, half = (k - 1) / 2;
   const T *Q = (const T *)p.Q + (size_t)bh * n * d;
   const T *V = (const T *)p.V + (size_t)bh * n * d;
@@ -151,30 +161,63 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_rows(const Rows
       }
     __syncthreads();
     // conv kernel gradient: tap j gets sum_i sum_c dO_i,c V_{i+j-half},c
+    // (halo row i + j).  A thread takes one column c and kTapGroup taps
+    // j0 ..: down the rows it keeps the halo rows i + j0 .. in a sliding
+    // window of registers, so each row costs two loads; a warp's 32 columns
+    // are then summed by shuffles, and the two halves of 64 in order.
     if (k > 0) {
-      const int warp = t >> 5, lane = t & 31;
-      for (int j = warp; j < k; j += 8) {
-        float acc = 0.f;
-        for (int e = lane; e < kTile * d; e += 32) {
-          const int r = e / d, c = e % d;
-          acc = fmaf(gs[r * LD + c], vh[(r + j) * LD + c], acc);
+      const int hr = kTile + k - 1;   // halo rows loaded
+      const int items = ((k + kTapGroup - 1) / kTapGroup) * 64;
+      for (int u = t; u < items; u += kThreads) {
+        const int j0 = (u >> 6) * kTapGroup, c = u & 63;
+        float acc[kTapGroup], win[kTapGroup];
+#pragma unroll
+        for (int q = 0; q < kTapGroup; ++q) {
+          acc[q] = 0.f;
+          win[q] = j0 + q < hr ? vh[(j0 + q) * LD + c] : 0.f;
         }
-        acc = warp_sum(acc);
-        if (lane == 0) dwc[j] += acc;
+        for (int r = 0; r < kTile; ++r) {
+          const float g = gs[r * LD + c];
+#pragma unroll
+          for (int q = 0; q < kTapGroup; ++q) acc[q] = fmaf(g, win[q], acc[q]);
+#pragma unroll
+          for (int q = 0; q + 1 < kTapGroup; ++q) win[q] = win[q + 1];
+          const int nr = r + j0 + kTapGroup;   // the row entering the window
+          win[kTapGroup - 1] = nr < hr ? vh[nr * LD + c] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kTapGroup; ++q) {
+          const float v = warp_sum(acc[q]);
+          if ((t & 31) == 0 && j0 + q < k) cpart[(j0 + q) * 2 + ((u >> 5) & 1)] = v;
+        }
       }
-      __syncthreads();   // fs and ds overwrite the halo
+      __syncthreads();   // fs and ds overwrite the halo; cpart complete
+      if (t < k) dwc[t] += cpart[2 * t] + cpart[2 * t + 1];
     }
     {   // logits S = Q K~^T (64 x m) into fs, dF = dO W^T into ds
-      float a[4][RM], b[4][RM];
+      float a[4][RM];
       zero(a);
-      zero(b);
-      mm_acc(a, qs, LD, 1, kt, 1, LD, d, kTile, M);
-      mm_acc(b, gs, LD, 1, w, 1, LD, d, kTile, M);
-      store(a, fs, LM, kTile, m, p.scale);
-      store(b, ds, LM, kTile, m);
+      mm_vec<4, RM, false, false>(a, qs, LD, kt, LD, d4);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < RM; ++c) {
+          const int col = vec_col<RM, false>(c);
+          if (col < m) fs[vec_row<4>(r) * LM + col] = p.scale * a[r][c];
+        }
+      zero(a);
+      mm_vec<4, RM, false, false>(a, gs, LD, w, LD, d4);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < RM; ++c) {
+          const int col = vec_col<RM, false>(c);
+          if (col < m) ds[vec_row<4>(r) * LM + col] = a[r][c];
+        }
     }
     __syncthreads();
-    // row softmax of F and dS_F = F (dF - rowsum(dF F)): a warp per row
+    // row softmax of F and dS_F = F (dF - rowsum(dF F)): a warp per row;
+    // columns m .. m4 - 1 are zeroed for the products over the landmarks
     {
       const int warp = t >> 5, lane = t & 31;
       for (int r = warp; r < kTile; r += 8) {
@@ -200,30 +243,41 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_rows(const Rows
           const float f = fs[r * LM + j];
           ds[r * LM + j] = in ? f * (ds[r * LM + j] - dot) : 0.f;
         }
+        for (int j = m + lane; j < m4; j += 32) {
+          fs[r * LM + j] = 0.f;
+          ds[r * LM + j] = 0.f;
+        }
       }
     }
     __syncthreads();
     {   // dQ (F part) = s dS_F K~ (64 x d)
       float a[4][4];
       zero(a);
-      mm_acc(a, ds, LM, 1, kt, LD, 1, m, kTile, d);
-      const int ty = t >> 4, tx = t & 15;
+      mm_vec<4, 4, false, true>(a, ds, LM, kt, LD, m4);
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int row = r0 + ty + 16 * r, col = tx + 16 * c;
+          const int row = r0 + vec_row<4>(r), col = vec_col<4, true>(c);
           if (row < n && col < d) dQ[(size_t)row * d + col] = from_f<T>(p.scale * a[r][c]);
         }
     }
     // dW += F^T dO, dK~ += dS_F^T Q (m x d, over the tile's rows)
-    mm_acc(dW, fs, 1, LM, gs, LD, 1, kTile, m, d);
-    mm_acc(dK, ds, 1, LM, qs, LD, 1, kTile, m, d);
+    mm_vec<RM, 4, true, true>(dW, fs, LM, gs, LD, kTile);
+    mm_vec<RM, 4, true, true>(dK, ds, LM, qs, LD, kTile);
   }
   // block partials
   const size_t pb = ((size_t)bh * p.R + blk) * m * d;
-  store(dW, p.dw_part + pb, d, m, d);
-  store(dK, p.dkt_part + pb, d, m, d, p.scale);
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = vec_row<RM>(r), col = vec_col<4, true>(c);
+      if (j < m && col < d) {
+        p.dw_part[pb + (size_t)j * d + col] = dW[r][c];
+        p.dkt_part[pb + (size_t)j * d + col] = p.scale * dK[r][c];
+      }
+    }
   __syncthreads();
   if (t < k) p.dconv_part[((size_t)bh * p.R + blk) * k + t] = dwc[t];
 }
@@ -240,22 +294,23 @@ struct HeadParams {
   float scale;
 };
 
-// C = alpha op(A) op(B) (+ beta C) over m x m (or m x d) matrices with row
-// stride ld, all in one block; the product runs with every thread.
-template <int RM, int RN>
-__device__ __forceinline__ void mm_block(float *C, int ldc, const float *A, int sai, int sak,
-                                         const float *B, int sbk, int sbj, int K, int M, int N,
+// C = alpha A B (+ beta C) over m x m (or m x d) matrices with row stride
+// ld, all in one block; the product runs with every thread (mm_vec: A, B
+// stored k-major when AK, BK, else transposed; K4 = the inner size rounded
+// up to 4, over zero padding).
+template <int RM, int RN, bool AK, bool BK>
+__device__ __forceinline__ void mm_block(float *C, int ldc, const float *A, int lda,
+                                         const float *B, int ldb, int K4, int M, int N,
                                          float alpha, float beta) {
   float acc[RM][RN];
   zero(acc);
-  mm_acc(acc, A, sai, sak, B, sbk, sbj, K, M, N);
+  mm_vec<RM, RN, AK, BK>(acc, A, lda, B, ldb, K4);
   __syncthreads();   // C may alias an operand's previous contents
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
   for (int r = 0; r < RM; ++r)
 #pragma unroll
     for (int c = 0; c < RN; ++c) {
-      const int i = ty + 16 * r, j = tx + 16 * c;
+      const int i = vec_row<RM>(r), j = vec_col<RN, BK>(c);
       if (i < M && j < N) {
         float *o = C + i * ldc + j;
         *o = alpha * acc[r][c] + (beta != 0.f ? beta * *o : 0.f);
@@ -281,11 +336,10 @@ __device__ __forceinline__ float sum_parts(const float *x, size_t stride, int R)
 }
 
 // Row stride of bwd_head<M>'s matrices: m columns or the d <= 64 columns of
-// the m x d ones, plus one so that a column walk (the transposed operands)
-// falls in 32 different banks.
+// the m x d ones, plus four (16-byte rows, 4 mod 32 words).
 template <int M>
 __host__ __device__ constexpr int head_ld() {
-  return (M > 64 ? M : 64) + 1;
+  return (M > 64 ? M : 64) + 4;
 }
 
 // Bytes of the twelve matrices of bwd_head<M>.
@@ -295,26 +349,32 @@ __host__ __device__ constexpr size_t head_bytes() {
 }
 
 template <int M>
-__global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
-  constexpr int RM = M / 16;
+__global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
+  // 512 threads: products own rows ty * RR + r (ty < 32) and 16 column
+  // threads; m x m outputs take RM columns per thread
+  constexpr int RR = M / 32, RM = M / 16;
   extern __shared__ __align__(16) float smem_f[];
   const int bh = blockIdx.x, t = threadIdx.x;
   // twelve M x ld matrices (m <= M rows)
   constexpr int ld = head_ld<M>(), kMat = M * ld;
-  const int m = p.m, d = p.d;
+  const int m = p.m, d = p.d, m4 = round4(m), d4 = round4(d);
   float *base = p.use_smem ? smem_f : p.scratch + (size_t)bh * (head_bytes<M>() / 4);
   float *A = base, *Zj = A + kMat, *P = Zj + kMat, *T1 = P + kMat, *T2 = T1 + kMat,
         *T3 = T2 + kMat, *dZ = T3 + kMat, *dP = dZ + kMat, *dT = dP + kMat,
         *dA = dT + kMat, *X = dA + kMat, *Y2 = X + kMat;
+  // every matrix starts zero: rows m .. M - 1 and the columns past its own
+  // stay zero, which the products over m4 or d4 terms read
+  for (int e = t; e < 12 * kMat; e += kHeadThreads) base[e] = 0.f;
+  __syncthreads();
   // X: dW (m x d) then scratch; Y2: Y (m x d)
   const size_t hd = (size_t)bh * m * d;
-  for (int e = t; e < m * d; e += kThreads) {
+  for (int e = t; e < m * d; e += kHeadThreads) {
     const int i = e / d, c = e % d;
     const float sw = sum_parts(p.dw_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
     X[i * ld + c] = sw;
     Y2[i * ld + c] = p.y[hd + e];
   }
-  for (int e = t; e < m * m; e += kThreads) {
+  for (int e = t; e < m * m; e += kHeadThreads) {
     const int i = e / m, j = e % m;
     A[i * ld + j] = p.a[(size_t)bh * m * m + e];
     Zj[i * ld + j] = p.zs[((size_t)bh * (p.iters + 1) + p.iters) * m * m + e];
@@ -322,9 +382,9 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   }
   __syncthreads();
   // dZ = dW Y^T (m x m), dY = Z^T dW (m x d)
-  mm_block<RM, RM>(dZ, ld, X, ld, 1, Y2, 1, ld, d, m, m, 1.f, 0.f);
-  mm_block<RM, 4>(T1, ld, Zj, 1, ld, X, ld, 1, m, m, d, 1.f, 0.f);
-  for (int e = t; e < m * d; e += kThreads) {
+  mm_block<RR, RM, false, false>(dZ, ld, X, ld, Y2, ld, d4, m, m, 1.f, 0.f);
+  mm_block<RR, 4, true, true>(T1, ld, Zj, ld, X, ld, m4, m, d, 1.f, 0.f);
+  for (int e = t; e < m * d; e += kHeadThreads) {
     const int i = e / d, c = e % d;
     p.dy[hd + e] = T1[i * ld + c];
   }
@@ -337,41 +397,41 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   // Lemma 1 steps backwards: Z' = 1/4 Z T3, T3 = 13I - P T2, T2 = 15I - P T1,
   // T1 = 7I - P, P = A Z
   for (int j = p.iters - 1; j >= 0; --j) {
-    for (int e = t; e < m * m; e += kThreads)
+    for (int e = t; e < m * m; e += kHeadThreads)
       Zj[(e / m) * ld + e % m] = p.zs[((size_t)bh * (p.iters + 1) + j) * m * m + e];
     __syncthreads();
-    mm_block<RM, RM>(P, ld, A, ld, 1, Zj, ld, 1, m, m, m, 1.f, 0.f);            // P = A Z
-    for (int e = t; e < m * m; e += kThreads) {
+    mm_block<RR, RM, false, true>(P, ld, A, ld, Zj, ld, m4, m, m, 1.f, 0.f);            // P = A Z
+    for (int e = t; e < m * m; e += kHeadThreads) {
       const int i = e / m, c = e % m;
       T1[i * ld + c] = (i == c ? 7.f : 0.f) - P[i * ld + c];
     }
     __syncthreads();
-    mm_block<RM, RM>(T2, ld, P, ld, 1, T1, ld, 1, m, m, m, -1.f, 0.f);          // -P T1
-    for (int e = t; e < m * m; e += kThreads) {
+    mm_block<RR, RM, false, true>(T2, ld, P, ld, T1, ld, m4, m, m, -1.f, 0.f);          // -P T1
+    for (int e = t; e < m * m; e += kHeadThreads) {
       const int i = e / m, c = e % m;
       T2[i * ld + c] += (i == c ? 15.f : 0.f);
     }
     __syncthreads();
-    mm_block<RM, RM>(T3, ld, P, ld, 1, T2, ld, 1, m, m, m, -1.f, 0.f);          // -P T2
-    for (int e = t; e < m * m; e += kThreads) {
+    mm_block<RR, RM, false, true>(T3, ld, P, ld, T2, ld, m4, m, m, -1.f, 0.f);          // -P T2
+    for (int e = t; e < m * m; e += kHeadThreads) {
       const int i = e / m, c = e % m;
       T3[i * ld + c] += (i == c ? 13.f : 0.f);
     }
     __syncthreads();
-    mm_block<RM, RM>(dT, ld, Zj, 1, ld, dZ, ld, 1, m, m, m, 0.25f, 0.f);       // dT3 = 1/4 Z^T dZ
-    mm_block<RM, RM>(X, ld, dZ, ld, 1, T3, 1, ld, m, m, m, 0.25f, 0.f);        // dZ_prev = 1/4 dZ T3^T
-    mm_block<RM, RM>(dP, ld, dT, ld, 1, T2, 1, ld, m, m, m, -1.f, 0.f);        // dP = -dT3 T2^T
-    mm_block<RM, RM>(T3, ld, P, 1, ld, dT, ld, 1, m, m, m, -1.f, 0.f);         // dT2 = -P^T dT3
-    mm_block<RM, RM>(dP, ld, T3, ld, 1, T1, 1, ld, m, m, m, -1.f, 1.f);        // dP -= dT2 T1^T
-    mm_block<RM, RM>(dT, ld, P, 1, ld, T3, ld, 1, m, m, m, -1.f, 0.f);         // dT1 = -P^T dT2
-    for (int e = t; e < m * m; e += kThreads) {
+    mm_block<RR, RM, true, true>(dT, ld, Zj, ld, dZ, ld, m4, m, m, 0.25f, 0.f);       // dT3 = 1/4 Z^T dZ
+    mm_block<RR, RM, false, false>(X, ld, dZ, ld, T3, ld, m4, m, m, 0.25f, 0.f);        // dZ_prev = 1/4 dZ T3^T
+    mm_block<RR, RM, false, false>(dP, ld, dT, ld, T2, ld, m4, m, m, -1.f, 0.f);        // dP = -dT3 T2^T
+    mm_block<RR, RM, true, true>(T3, ld, P, ld, dT, ld, m4, m, m, -1.f, 0.f);         // dT2 = -P^T dT3
+    mm_block<RR, RM, false, false>(dP, ld, T3, ld, T1, ld, m4, m, m, -1.f, 1.f);        // dP -= dT2 T1^T
+    mm_block<RR, RM, true, true>(dT, ld, P, ld, T3, ld, m4, m, m, -1.f, 0.f);         // dT1 = -P^T dT2
+    for (int e = t; e < m * m; e += kHeadThreads) {
       const int i = e / m, c = e % m;
       dP[i * ld + c] -= dT[i * ld + c];                                          // dP -= dT1
     }
     __syncthreads();
-    mm_block<RM, RM>(dA, ld, dP, ld, 1, Zj, 1, ld, m, m, m, 1.f, 1.f);         // dA += dP Z^T
-    mm_block<RM, RM>(X, ld, A, 1, ld, dP, ld, 1, m, m, m, 1.f, 1.f);           // dZ_prev += A^T dP
-    for (int e = t; e < m * m; e += kThreads) dZ[(e / m) * ld + e % m] = X[(e / m) * ld + e % m];
+    mm_block<RR, RM, false, false>(dA, ld, dP, ld, Zj, ld, m4, m, m, 1.f, 1.f);         // dA += dP Z^T
+    mm_block<RR, RM, true, true>(X, ld, A, ld, dP, ld, m4, m, m, 1.f, 1.f);           // dZ_prev += A^T dP
+    for (int e = t; e < m * m; e += kHeadThreads) dZ[(e / m) * ld + e % m] = X[(e / m) * ld + e % m];
     __syncthreads();
   }
   // Z0 = A^T c, c = 1 / (||A||_1 ||A||_inf): gradients through c and the
@@ -381,7 +441,7 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   __shared__ float red[4];
   __shared__ int arg[2];
   __shared__ float cs[M], rs[M], dcr[M];
-  for (int u = t; u < 3 * m; u += kThreads) {
+  for (int u = t; u < 3 * m; u += kHeadThreads) {
     const int i = u % m;
     float s = 0.f;
     if (u < m) {
@@ -414,7 +474,7 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
   __syncthreads();
   {
     const float c = red[0], dc = red[1], n1 = red[2], ninf = red[3];
-    for (int e = t; e < m * m; e += kThreads) {
+    for (int e = t; e < m * m; e += kHeadThreads) {
       const int i = e / m, j = e % m;
       float g = dA[i * ld + j] + c * dZ[j * ld + i];
       if (j == arg[0]) g += -dc * c / n1 * (A[i * ld + j] > 0.f ? 1.f : (A[i * ld + j] < 0.f ? -1.f : 0.f));
@@ -430,17 +490,17 @@ __global__ void __launch_bounds__(kThreads) bwd_head(const HeadParams p) {
     for (int j = 0; j < m; ++j) dP[t * ld + j] = A[t * ld + j] * (dA[t * ld + j] - dot);
   }
   // Q~, K~ into T1, T2 (m x d)
-  for (int e = t; e < m * d; e += kThreads) {
+  for (int e = t; e < m * d; e += kHeadThreads) {
     const int i = e / d, c = e % d;
     T1[i * ld + c] = p.qt[hd + e];
     T2[i * ld + c] = p.kt[hd + e];
   }
   __syncthreads();
   // dQ~_A = s dS_A K~ ; dK~ = (F part) + s dS_A^T Q~
-  mm_block<RM, 4>(T3, ld, dP, ld, 1, T2, ld, 1, m, m, d, p.scale, 0.f);
-  for (int e = t; e < m * d; e += kThreads) p.dqt_a[hd + e] = T3[(e / d) * ld + e % d];
-  mm_block<RM, 4>(X, ld, dP, 1, ld, T1, ld, 1, m, m, d, p.scale, 0.f);
-  for (int e = t; e < m * d; e += kThreads) {
+  mm_block<RR, 4, false, true>(T3, ld, dP, ld, T2, ld, m4, m, d, p.scale, 0.f);
+  for (int e = t; e < m * d; e += kHeadThreads) p.dqt_a[hd + e] = T3[(e / d) * ld + e % d];
+  mm_block<RR, 4, true, true>(X, ld, dP, ld, T1, ld, m4, m, d, p.scale, 0.f);
+  for (int e = t; e < m * d; e += kHeadThreads) {
     const int i = e / d, c = e % d;
     const float s = sum_parts(p.dkt_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
     p.dkt[hd + e] = s + X[i * ld + c];
@@ -464,7 +524,7 @@ struct KeysSmem {
   // the dO halo is only read by conv^T, which runs (into registers) before
   // B and dS_B are formed, so they share their bytes (two blocks per SM at
   // m <= 64)
-  static constexpr int LD = 65, LK = kTile + 1;
+  static constexpr int LD = kLd, LK = kLd;
   static constexpr uint32_t kHalo = (kTile + 62) * LD * 4, kBD = 2 * M * LK * 4;
   static constexpr uint32_t qt = 0;                              // [M][LD]
   static constexpr uint32_t dy = qt + M * LD * 4;                // [M][LD]
@@ -492,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
   float *ddv = (float *)(smem + S::dd);
   const int blk = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const int n = p.n, d = p.d, m = p.m, head = bh % p.heads;
+  const int d4 = round4(d), m4 = round4(m);
   const int k = p.conv_w ? p.conv_k : 0, half = (k - 1) / 2;
   const int l = (n + m - 1) / m;
   const T *K = (const T *)p.K + (size_t)bh * n * d;
@@ -530,40 +591,42 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
         gh[i] = (row >= 0 && row < n && c < d) ? to_f(G[(size_t)row * d + c]) : 0.f;
       }
     __syncthreads();
-    // conv^T(dO) for the tile's dV outputs: dV_row += w[tp] dO[row - tp + half]
+    // conv^T(dO) for the tile's dV outputs (key vec_row<4>(r), column
+    // vec_col<4, true>(c)): dV_row += w[tp] dO[row - tp + half]
     float cv[4][4];
     zero(cv);
     if (k > 0) {
-      const int ty = t >> 4, tx = t & 15;
+      for (int tp = 0; tp < k; ++tp) {
+        const float wt = cw[tp];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 4; ++r) {
+          float g[4];
+          ld_vec<4>(g, gh + (vec_row<4>(r) + (k - 1) - tp) * LD + vec_col<4, true>(0));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int key = ty + 16 * r, col = tx + 16 * c;
-          float gv = 0.f;
-          for (int tp = 0; tp < k; ++tp)
-            gv = fmaf(cw[tp], gh[(key + (k - 1) - tp) * LD + col], gv);
-          cv[r][c] = gv;
+          for (int c = 0; c < 4; ++c) cv[r][c] = fmaf(wt, g[c], cv[r][c]);
         }
+      }
       __syncthreads();   // bs and dbs overwrite the halo
     }
-    {   // B = 2^(s log2e Q~ K^T - lse) (m x 64), dB = dY V^T
+    {   // B = 2^(s log2e Q~ K^T - lse) (m x 64), dB = dY V^T; rows m .. M - 1
+        // zeroed for the products over the landmarks
       float a[RM][4], b[RM][4];
       zero(a);
       zero(b);
-      mm_acc(a, qt, LD, 1, ks, 1, LD, d, m, kTile);
-      mm_acc(b, dy, LD, 1, vs, 1, LD, d, m, kTile);
-      const int ty = t >> 4, tx = t & 15;
+      mm_vec<RM, 4, false, false>(a, qt, LD, ks, LD, d4);
+      mm_vec<RM, 4, false, false>(b, dy, LD, vs, LD, d4);
 #pragma unroll
       for (int r = 0; r < RM; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int j = ty + 16 * r, key = tx + 16 * c;
+          const int j = vec_row<RM>(r), key = vec_col<4, false>(c);
+          float bv = 0.f, dbv = 0.f;
           if (j < m) {
-            const float bv = (k0 + key < n) ? exp2f(a[r][c] * p.scale_log2 - lse[j]) : 0.f;
-            bs[j * LK + key] = bv;
-            dbs[j * LK + key] = bv * (b[r][c] - ddv[j]);   // dS_B
+            bv = (k0 + key < n) ? exp2f(a[r][c] * p.scale_log2 - lse[j]) : 0.f;
+            dbv = bv * (b[r][c] - ddv[j]);   // dS_B
           }
+          bs[j * LK + key] = bv;
+          dbs[j * LK + key] = dbv;
         }
     }
     __syncthreads();
@@ -571,14 +634,13 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
       float a[4][4], b[4][4];
       zero(a);
       zero(b);
-      mm_acc(a, dbs, 1, LK, qt, LD, 1, m, kTile, d);
-      mm_acc(b, bs, 1, LK, dy, LD, 1, m, kTile, d);
-      const int ty = t >> 4, tx = t & 15;
+      mm_vec<4, 4, true, true>(a, dbs, LK, qt, LD, m4);
+      mm_vec<4, 4, true, true>(b, bs, LK, dy, LD, m4);
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int key = ty + 16 * r, col = tx + 16 * c, row = k0 + key;
+          const int col = vec_col<4, true>(c), row = k0 + vec_row<4>(r);
           if (row < n && col < d) {
             const int j = seg_of(row, l);
             const float gk =
@@ -589,9 +651,16 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
         }
     }
     // dQ~ += s dS_B K (m x d, over the tile's keys)
-    mm_acc(dq, dbs, LK, 1, ks, LD, 1, kTile, m, d);
+    mm_vec<RM, 4, false, true>(dq, dbs, LK, ks, LD, kTile);
   }
-  store(dq, p.dqt_part + ((size_t)bh * p.S2 + blk) * m * d, d, m, d, p.scale);
+  const size_t pb = ((size_t)bh * p.S2 + blk) * m * d;
+#pragma unroll
+  for (int r = 0; r < RM; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = vec_row<RM>(r), col = vec_col<4, true>(c);
+      if (j < m && col < d) p.dqt_part[pb + (size_t)j * d + col] = p.scale * dq[r][c];
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -605,23 +674,28 @@ bwd_dqt_total(float *dqt, const float *dqt_part, int md, int S2) {
   dqt[(size_t)bh * md + e] += s;
 }
 
-// dQ += dQ~_{seg(i)} / count over the block's rows.
+// dQ += dQ~_{seg(i)} / count over the block's rows: the m x d quotients
+// once into shared memory, then thread t takes column t % 64 of every
+// fourth row (d <= 64).
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_dq(void *dQv, const float *dqt, int n, int d, int m, int rows_per_block) {
   extern __shared__ float dq[];   // [m][d]
   const int bh = blockIdx.y, t = threadIdx.x;
   const size_t hd = (size_t)bh * m * d;
-  for (int e = t; e < m * d; e += kThreads) dq[e] = dqt[hd + e];
+  const int l = (n + m - 1) / m;
+  for (int e = t; e < m * d; e += kThreads) {
+    const int j = e / d;
+    dq[e] = dqt[hd + e] / (float)seg_count(j, l, n);
+  }
   __syncthreads();
   T *dQ = (T *)dQv + (size_t)bh * n * d;
-  const int l = (n + m - 1) / m;
   const int r0 = blockIdx.x * rows_per_block, r1 = min(n, r0 + rows_per_block);
-  for (int e = t; e < (r1 - r0) * d; e += kThreads) {
-    const int row = r0 + e / d, c = e % d;
-    const int j = seg_of(row, l);
+  const int c = t & 63;
+  if (c >= d) return;
+  for (int row = r0 + (t >> 6); row < r1; row += kThreads / 64) {
     const size_t o = (size_t)row * d + c;
-    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[j * d + c] / (float)seg_count(j, l, n));
+    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[seg_of(row, l) * d + c]);
   }
 }
 

@@ -112,7 +112,7 @@ Layout make_layout(const nys_desc *desc, int m) {
   L.pmax = take(BH * splits * m * 4);
   L.psum = take(BH * splits * m * 4);
   L.py = take(BH * splits * m * d * 4);
-  L.scratch = take(desc->dtype == NYS_F32 && m > 64 ? BH * 5 * m * m * 4 : 0);
+  L.scratch = take(desc->dtype == NYS_F32 && m > 64 ? BH * pinv_simt_mats_bytes(m) : 0);
   L.w_bf = take(desc->dtype == NYS_BF16 ? BH * m * 128 : 0);   // W as the bf16 P W operand
   L.total = off;
   return L;
@@ -246,7 +246,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   }
   {
     const int use_smem = m <= 64;
-    size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
+    size_t sm = use_smem ? pinv_simt_mats_bytes(m) : 0;
     auto kern = pinv_simt_for(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
@@ -268,10 +268,11 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   }
   {
     const size_t sm = merge_w_smem(m, d, L.splits);
-    auto kern = merge_w_simt_for(m);
+    auto kern = merge_w_simt;
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false,
-               pmax, psum, py, z, y, w, m, d, L.splits, (float *)nullptr) != cudaSuccess)
+        launch(kern, dim3(BH, (d + kMergeCols - 1) / kMergeCols), dim3(256),
+               launch_smem(mk.launched, sm), stream, false, pmax, psum, py, z, y, w, m, d,
+               L.splits, (float *)nullptr) != cudaSuccess)
       return NYS_ERR_CUDA;
     mk.after(stream);
   }
@@ -509,7 +510,7 @@ BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
   L.z = take(mm);
   L.a = take(mm);
   L.zall = take(mm * (iters + 1));
-  L.pscr = take(m > 64 ? 5 * mm : 0);
+  L.pscr = take(m > 64 ? BH * pinv_simt_mats_bytes(m) : 0);
   L.pmax = take(BH * L.S * m * 4);
   L.psum = take(BH * L.S * m * 4);
   L.py = take(BH * L.S * m * d * 4);
@@ -555,7 +556,7 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
   }
   {
     const int use_smem = m <= 64;
-    const size_t sm = use_smem ? (size_t)5 * m * m * 4 : 0;
+    const size_t sm = use_smem ? pinv_simt_mats_bytes(m) : 0;
     auto kern = pinv_simt_for(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH), dim3(256), sm, stream, false, (const float *)qt,
@@ -574,9 +575,10 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
   }
   {
     const size_t sm = merge_w_smem(m, d, L.S);
-    auto kern = merge_w_simt_for(m);
+    auto kern = merge_w_simt;
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(BH), dim3(256), sm, stream, false, (const float *)pmax,
+        launch(kern, dim3(BH, (d + kMergeCols - 1) / kMergeCols), dim3(256), sm, stream, false,
+               (const float *)pmax,
                (const float *)psum, (const float *)py, (const float *)z, y, w, m, d, L.S,
                lse) != cudaSuccess)
       return NYS_ERR_CUDA;
@@ -600,7 +602,7 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
     auto kern = bwd::bwd_head<MB>;
     const size_t sm = MB <= 64 ? bwd::head_bytes<MB>() : 0;
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
+        launch(kern, dim3(BH), dim3(bwd::kHeadThreads), sm, stream, false, p) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
   {

@@ -85,38 +85,127 @@ __device__ __forceinline__ void mm_acc(float (&acc)[RM][RN], const float *A, int
 }
 
 // ---------------------------------------------------------------------------
+// The same product from 16-byte shared-memory loads, for operands whose rows
+// are 16-byte aligned (row strides a multiple of 4 floats) and zero-padded
+// to K4, a multiple of 4.  Thread (ty, tx) owns rows ty * RM + r and
+// columns tx * RN + c when B is stored k-major (B(k, j) = B[k * ldb + j]),
+// else tx + 16 c (B(k, j) = B[j * ldb + k]); A(i, k) = A[k * lda + i] when
+// A is stored k-major, else A[i * lda + k].  Each k-step then costs one
+// load of A's rows and one of B's columns; a row stride of 4 mod 32 words
+// keeps the strided forms to the minimum number of bank wavefronts.
+template <int N>
+__device__ __forceinline__ void ld_vec(float (&v)[N], const float *p) {
+  if constexpr (N == 1) {
+    v[0] = p[0];
+  } else if constexpr (N == 2) {
+    const float2 x = *reinterpret_cast<const float2 *>(p);
+    v[0] = x.x, v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 x = *reinterpret_cast<const float4 *>(p + 4 * q);
+      v[4 * q] = x.x, v[4 * q + 1] = x.y, v[4 * q + 2] = x.z, v[4 * q + 3] = x.w;
+    }
+  }
+}
+
+template <int RM, int RN, bool AK, bool BK>
+__device__ __forceinline__ void mm_vec(float (&acc)[RM][RN], const float *A, int lda,
+                                       const float *B, int ldb, int K4) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  const float *a0 = AK ? A + ty * RM : A + ty * RM * lda;
+  const float *b0 = BK ? B + tx * RN : B + tx * ldb;
+  for (int k = 0; k < K4; k += 4) {
+    float a[4][RM], b[4][RN];
+    if constexpr (AK) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ld_vec<RM>(a[q], a0 + (k + q) * lda);
+    } else {
+#pragma unroll
+      for (int r = 0; r < RM; ++r) {
+        const float4 x = *reinterpret_cast<const float4 *>(a0 + r * lda + k);
+        a[0][r] = x.x, a[1][r] = x.y, a[2][r] = x.z, a[3][r] = x.w;
+      }
+    }
+    if constexpr (BK) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ld_vec<RN>(b[q], b0 + (k + q) * ldb);
+    } else {
+#pragma unroll
+      for (int c = 0; c < RN; ++c) {
+        const float4 x = *reinterpret_cast<const float4 *>(b0 + 16 * c * ldb + k);
+        b[0][c] = x.x, b[1][c] = x.y, b[2][c] = x.z, b[3][c] = x.w;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int r = 0; r < RM; ++r)
+#pragma unroll
+        for (int c = 0; c < RN; ++c) acc[r][c] = fmaf(a[q][r], b[q][c], acc[r][c]);
+  }
+}
+
+// The output row and column that mm_vec<RM, RN, *, BK> accumulates in
+// acc[r][c].
+template <int RM>
+__device__ __forceinline__ int vec_row(int r) {
+  return (threadIdx.x >> 4) * RM + r;
+}
+template <int RN, bool BK>
+__device__ __forceinline__ int vec_col(int c) {
+  return BK ? (threadIdx.x & 15) * RN + c : (threadIdx.x & 15) + 16 * c;
+}
+
+// k rounded up to a multiple of 4
+__host__ __device__ constexpr int round4(int k) { return (k + 3) & ~3; }
+
+// ---------------------------------------------------------------------------
 // Landmark kernel A = softmax(Q~ K~^T / sqrt(d)) and its pseudoinverse by
 // Lemma 1 as printed: Z <- 1/4 Z (13I - AZ (15I - AZ (7I - AZ))), from
 // Z0 = A^T / (||A||_1 ||A||_inf).  One block of 256 threads per head; all
 // five m x m fp32 matrices live in `mats` (shared memory when it fits, else
-// the per-head workspace scratch).
-//
-// Products run register-tiled: thread (ty, tx) = (t / 16, t % 16) owns the
-// outputs (ty + 16 r, tx + 16 c), r, c < RM (m <= 16 RM), and adds each one's
-// terms in index order with fmaf.
+// the per-head workspace scratch), each 16 RM rows (m <= 16 RM) of stride
+// 16 RM + 4, zero past row and column m: the products read whole rows and
+// columns of their 16 RM x 16 RM tiles.
+template <int RM>
+__host__ __device__ constexpr int pinv_ld() {
+  return 16 * RM + 4;
+}
+
+// bytes of pinv_simt<RM>'s five matrices
+template <int RM>
+__host__ __device__ constexpr size_t pinv_mats_bytes() {
+  return (size_t)5 * 16 * RM * pinv_ld<RM>() * 4;
+}
+
+// C = X Y (m x m, row stride ld), register-tiled on mm_vec: each output adds
+// its terms in index order with fmaf.
 template <int RM>
 __device__ __forceinline__ void block_gemm(float *C, const float *X, const float *Y, int m) {
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float acc[RM][RM];
+  constexpr int ld = pinv_ld<RM>(), RR = RM;
+  float acc[RR][RM];
 #pragma unroll
-  for (int r = 0; r < RM; ++r)
+  for (int r = 0; r < RR; ++r)
 #pragma unroll
     for (int c = 0; c < RM; ++c) acc[r][c] = 0.f;
-  mm_acc(acc, X, m, 1, Y, m, 1, m, m, m);
+  mm_vec<RR, RM, false, true>(acc, X, ld, Y, ld, round4(m));
 #pragma unroll
-  for (int r = 0; r < RM; ++r)
+  for (int r = 0; r < RR; ++r)
 #pragma unroll
     for (int c = 0; c < RM; ++c) {
-      const int i = ty + 16 * r, j = tx + 16 * c;
-      if (i < m && j < m) C[i * m + j] = acc[r][c];
+      const int i = vec_row<RR>(r), j = vec_col<RM, true>(c);
+      if (i < m && j < m) C[i * ld + j] = acc[r][c];
     }
   __syncthreads();
 }
 
-__device__ __forceinline__ void block_diag_minus(float *dst, const float *src, float c, int m) {
+// dst = c I - src (m x m, row stride ld)
+__device__ __forceinline__ void block_diag_minus(float *dst, const float *src, float c, int m,
+                                                 int ld) {
   for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
-    int i = idx / m, j = idx % m;
-    dst[idx] = (i == j ? c : 0.f) - src[idx];
+    const int i = idx / m, j = idx % m;
+    dst[i * ld + j] = (i == j ? c : 0.f) - src[i * ld + j];
   }
   __syncthreads();
 }
@@ -128,45 +217,61 @@ __global__ void __launch_bounds__(256)
 pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__restrict__ Zout,
           float *__restrict__ scratch, int m, int d, float scale, int iters, int use_smem,
           float *__restrict__ a_out = nullptr, float *__restrict__ z_all = nullptr) {
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
+  constexpr int ld = pinv_ld<RM>();
   const int bh = blockIdx.x, t = threadIdx.x;
-  float *mats = use_smem ? smem : scratch + (size_t)bh * 5 * m * m;
-  float *A = mats, *Z = A + m * m, *P = Z + m * m, *T1 = P + m * m, *T2 = T1 + m * m;
+  constexpr int mm = 16 * RM * ld;
+  float *mats = use_smem ? smem : scratch + (size_t)bh * (pinv_mats_bytes<RM>() / 4);
+  float *A = mats, *Z = A + mm, *P = Z + mm, *T1 = P + mm, *T2 = T1 + mm;
   __shared__ float red[2];
   __shared__ float nsum[2 * 16 * RM];   // column sums, then row sums
   const float *qt = Qt + (size_t)bh * m * d;
   const float *kt = Kt + (size_t)bh * m * d;
-  {   // logits, each a dot product over the features in order
+  for (int e = t; e < 5 * mm; e += blockDim.x) mats[e] = 0.f;
+  __syncthreads();
+  {   // logits, each a dot product over the features in order: thread
+      // (ty, tx) = (t / 16, t % 16) takes rows ty + 16 r, columns tx + 16 c
+    constexpr int RR = RM;
     const int ty = t >> 4, tx = t & 15;
-    float acc[RM][RM];
+    float acc[RR][RM];
 #pragma unroll
-    for (int r = 0; r < RM; ++r)
+    for (int r = 0; r < RR; ++r)
 #pragma unroll
       for (int c = 0; c < RM; ++c) acc[r][c] = 0.f;
-    mm_acc(acc, qt, d, 1, kt, 1, d, d, m, m);
+    for (int k = 0; k < d; ++k) {
+      float a[RR], b[RM];
 #pragma unroll
-    for (int r = 0; r < RM; ++r)
+      for (int r = 0; r < RR; ++r) a[r] = ty + 16 * r < m ? qt[(ty + 16 * r) * d + k] : 0.f;
+#pragma unroll
+      for (int c = 0; c < RM; ++c) b[c] = tx + 16 * c < m ? kt[(tx + 16 * c) * d + k] : 0.f;
+#pragma unroll
+      for (int r = 0; r < RR; ++r)
+#pragma unroll
+        for (int c = 0; c < RM; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < RR; ++r)
 #pragma unroll
       for (int c = 0; c < RM; ++c) {
         const int i = ty + 16 * r, j = tx + 16 * c;
-        if (i < m && j < m) A[i * m + j] = acc[r][c] * scale;
+        if (i < m && j < m) A[i * ld + j] = acc[r][c] * scale;
       }
   }
   __syncthreads();
   {   // row softmax, a warp per row
-    const int warp = t >> 5, lane = t & 31;
-    for (int i = warp; i < m; i += 8) {
+    const int warp = t >> 5, lane = t & 31, warps = blockDim.x >> 5;
+    for (int i = warp; i < m; i += warps) {
       float mx = -INFINITY;
-      for (int j = lane; j < m; j += 32) mx = fmaxf(mx, A[i * m + j]);
+      for (int j = lane; j < m; j += 32) mx = fmaxf(mx, A[i * ld + j]);
       mx = warp_max(mx);
       float s = 0.f;
       for (int j = lane; j < m; j += 32) {
-        const float e = __expf(A[i * m + j] - mx);
-        A[i * m + j] = e;
+        const float e = __expf(A[i * ld + j] - mx);
+        A[i * ld + j] = e;
         s += e;
       }
       const float inv = 1.f / warp_sum(s);
-      for (int j = lane; j < m; j += 32) A[i * m + j] *= inv;
+      for (int j = lane; j < m; j += 32) A[i * ld + j] *= inv;
     }
   }
   __syncthreads();
@@ -176,9 +281,9 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
   for (int u = t; u < 2 * m; u += blockDim.x) {
     float s = 0.f;
     if (u < m) {
-      for (int i = 0; i < m; ++i) s += fabsf(A[i * m + u]);
+      for (int i = 0; i < m; ++i) s += fabsf(A[i * ld + u]);
     } else {
-      for (int j = 0; j < m; ++j) s += fabsf(A[(u - m) * m + j]);
+      for (int j = 0; j < m; ++j) s += fabsf(A[(u - m) * ld + j]);
     }
     nsum[u] = s;
   }
@@ -192,33 +297,38 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
   __syncthreads();
   const float c0 = red[0];
   for (int idx = t; idx < m * m; idx += blockDim.x) {
-    int i = idx / m, j = idx % m;
-    Z[idx] = A[j * m + i] * c0;
-    if (a_out) a_out[(size_t)bh * m * m + idx] = A[idx];
-    if (z_all) z_all[(size_t)bh * (iters + 1) * m * m + idx] = A[j * m + i] * c0;
+    const int i = idx / m, j = idx % m;
+    Z[i * ld + j] = A[j * ld + i] * c0;
+    if (a_out) a_out[(size_t)bh * m * m + idx] = A[i * ld + j];
+    if (z_all) z_all[(size_t)bh * (iters + 1) * m * m + idx] = A[j * ld + i] * c0;
   }
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
-    block_gemm<RM>(P, A, Z, m);           // AZ
-    block_diag_minus(T1, P, 7.f, m);      // 7I - AZ
-    block_gemm<RM>(T2, P, T1, m);         // AZ (7I - AZ)
-    block_diag_minus(T1, T2, 15.f, m);    // 15I - ...
-    block_gemm<RM>(T2, P, T1, m);         // AZ (15I - ...)
-    block_diag_minus(T1, T2, 13.f, m);    // 13I - ...
-    block_gemm<RM>(T2, Z, T1, m);         // Z (13I - ...)
+    block_gemm<RM>(P, A, Z, m);               // AZ
+    block_diag_minus(T1, P, 7.f, m, ld);      // 7I - AZ
+    block_gemm<RM>(T2, P, T1, m);             // AZ (7I - AZ)
+    block_diag_minus(T1, T2, 15.f, m, ld);    // 15I - ...
+    block_gemm<RM>(T2, P, T1, m);             // AZ (15I - ...)
+    block_diag_minus(T1, T2, 13.f, m, ld);    // 13I - ...
+    block_gemm<RM>(T2, Z, T1, m);             // Z (13I - ...)
     for (int idx = t; idx < m * m; idx += blockDim.x) {
-      Z[idx] = 0.25f * T2[idx];
-      if (z_all) z_all[((size_t)bh * (iters + 1) + it + 1) * m * m + idx] = 0.25f * T2[idx];
+      const int i = idx / m, j = idx % m;
+      Z[i * ld + j] = 0.25f * T2[i * ld + j];
+      if (z_all)
+        z_all[((size_t)bh * (iters + 1) + it + 1) * m * m + idx] = 0.25f * T2[i * ld + j];
     }
     __syncthreads();
   }
   float *zo = Zout + (size_t)bh * m * m;
-  for (int idx = t; idx < m * m; idx += blockDim.x) zo[idx] = Z[idx];
+  for (int idx = t; idx < m * m; idx += blockDim.x) zo[idx] = Z[(idx / m) * ld + idx % m];
 }
 
-// pinv_simt for m landmarks (m <= 128)
+// pinv_simt for m landmarks (m <= 128), and the bytes of its matrices
 inline auto pinv_simt_for(int m) {
   return m <= 32 ? pinv_simt<2> : (m <= 64 ? pinv_simt<4> : pinv_simt<8>);
+}
+inline size_t pinv_simt_mats_bytes(int m) {
+  return m <= 32 ? pinv_mats_bytes<2>() : (m <= 64 ? pinv_mats_bytes<4>() : pinv_mats_bytes<8>());
 }
 
 // ---------------------------------------------------------------------------
@@ -226,11 +336,11 @@ inline auto pinv_simt_for(int m) {
 // online softmax over the split's keys of s * q~_j . k_i, keeping the running
 // maximum (log2 units), the running sum and the unnormalised sum of p_i v_i.
 // Grid (splits, heads), 256 threads; per 64-key tile the logits and the
-// P V product run register-tiled (thread (ty, tx) owns rows ty + 16 r and
-// keys / features tx + 16 c), and the 16 threads of a row reduce its tile
-// maximum and sum by shuffles.
+// P V product run register-tiled on mm_vec (thread (ty, tx) owns rows
+// ty * RM + r, keys tx + 16 c and features tx * 4 + c), and the 16 threads
+// of a row reduce its tile maximum and sum by shuffles.
 constexpr int kSimtKeyTile = 64;
-constexpr int kSimtLd = 65;   // padded rows of the tiles (d <= 64 or 64 keys)
+constexpr int kSimtLd = 68;   // row stride of the tiles (d <= 64 or 64 keys): 16-byte rows
 
 template <int RM>   // m <= 16 RM
 __host__ __device__ constexpr size_t bv_partial_smem() {
@@ -244,9 +354,9 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
                 int n, int d, int m, int splits, int keys_per_split, float scale_log2,
                 const int *lens, int heads) {
   constexpr int LD = kSimtLd, kT = kSimtKeyTile;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   const int split = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-  const int ty = t >> 4, tx = t & 15;
+  const int tx = t & 15, d4 = round4(d);
   float *qs = smem;                 // [16 RM][LD] Q~ rows
   float *ks = qs + 16 * RM * LD;    // [64][LD]
   float *vs = ks + kT * LD;         // [64][LD]
@@ -283,7 +393,7 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
     for (int r = 0; r < RM; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) sc[r][c] = 0.f;
-    mm_acc(sc, qs, LD, 1, ks, 1, LD, d, 16 * RM, kT);
+    mm_vec<RM, 4, false, false>(sc, qs, LD, ks, LD, d4);
 #pragma unroll
     for (int r = 0; r < RM; ++r) {
       float l2[4], mx = -INFINITY;
@@ -300,7 +410,7 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float p = exp2f(l2[c] - mnew);
-        ps[(ty + 16 * r) * LD + tx + 16 * c] = p;
+        ps[vec_row<RM>(r) * LD + vec_col<4, false>(c)] = p;
         sum += p;
       }
 #pragma unroll
@@ -311,20 +421,22 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
       for (int c = 0; c < 4; ++c) y[r][c] *= alpha;
     }
     __syncthreads();
-    mm_acc(y, ps, LD, 1, vs, LD, 1, kT, 16 * RM, d);
+    mm_vec<RM, 4, false, true>(y, ps, LD, vs, LD, kT);
   }
   const size_t base = ((size_t)bh * splits + split) * m;
 #pragma unroll
   for (int r = 0; r < RM; ++r) {
-    const int j = ty + 16 * r;
+    const int j = vec_row<RM>(r);
     if (j >= m) continue;
     if (tx == 0) {
       pmax[base + j] = Mx[r];
       psum[base + j] = Sm[r];
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      if (tx + 16 * c < d) py[(base + j) * d + tx + 16 * c] = y[r][c];
+    for (int c = 0; c < 4; ++c) {
+      const int col = vec_col<4, true>(c);
+      if (col < d) py[(base + j) * d + col] = y[r][c];
+    }
   }
 }
 
@@ -338,23 +450,26 @@ inline size_t bv_partial_simt_smem(int m) {
 }
 
 // ---------------------------------------------------------------------------
-// Merge of the key splits in split order (Y = B~ V), then W = Z Y.  One block
-// of 256 threads per head: a thread per landmark row takes the row's maximum
-// and weights, every output then adds its splits in order, and W runs
-// register-tiled (m <= 16 RM).
+// Merge of the key splits in split order (Y = B~ V), then W = Z Y.  Grid
+// (heads, column blocks of kMergeCols): a thread per landmark row takes the
+// row's maximum and split weights, every output of the block's columns then
+// adds its splits in order, and W's columns follow from Z and those of Y.
+constexpr int kMergeCols = 16;
+
 inline size_t merge_w_smem(int m, int d, int splits) {
-  return ((size_t)m * d + (size_t)m * m + (size_t)splits * m + m) * 4;
+  (void)d;
+  return ((size_t)m * kMergeCols + (size_t)m * m + (size_t)splits * m + m) * 4;
 }
 
-template <int RM>
 __global__ void __launch_bounds__(256)
 merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
              const float *__restrict__ py, const float *__restrict__ Zg, float *__restrict__ Yg,
              float *__restrict__ Wg, int m, int d, int splits, float *__restrict__ lse2 = nullptr) {
   extern __shared__ float smem[];
-  const int bh = blockIdx.x, t = threadIdx.x;
-  float *ys = smem;                    // [m][d]
-  float *zs = ys + m * d;              // [m][m]
+  const int bh = blockIdx.x, c0 = blockIdx.y * kMergeCols, t = threadIdx.x;
+  const int nc = min(kMergeCols, d - c0);
+  float *ys = smem;                    // [m][kMergeCols]
+  float *zs = ys + m * kMergeCols;     // [m][m]
   float *fac = zs + m * m;             // [splits][m]: 2^(max_s - max)
   float *tot = fac + splits * m;       // [m]: the row's merged sum
   const size_t pb = (size_t)bh * splits * m;
@@ -368,13 +483,14 @@ merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
       sum = fmaf(psum[pb + (size_t)s * m + j], f, sum);
     }
     tot[j] = sum;
-    if (lse2) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
+    if (lse2 && blockIdx.y == 0) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
   }
   for (int e = t; e < m * m; e += 256) zs[e] = Zg[(size_t)bh * m * m + e];
   __syncthreads();
-  for (int idx = t; idx < m * d; idx += 256) {
-    const int j = idx / d;
-    const float *src = py + pb * d + idx;
+  for (int idx = t; idx < m * kMergeCols; idx += 256) {
+    const int j = idx / kMergeCols, c = idx % kMergeCols;
+    if (c >= nc) continue;
+    const float *src = py + (pb + j) * d + c0 + c;
     const size_t stride = (size_t)m * d;
     float acc = 0.f;
     int s = 0;
@@ -389,28 +505,16 @@ merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
     for (; s < splits; ++s) acc = fmaf(src[s * stride], fac[s * m + j], acc);
     const float y = acc / tot[j];
     ys[idx] = y;
-    Yg[(size_t)bh * m * d + idx] = y;
+    Yg[((size_t)bh * m + j) * d + c0 + c] = y;
   }
   __syncthreads();
-  float acc[RM][4];
-#pragma unroll
-  for (int r = 0; r < RM; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-  mm_acc(acc, zs, m, 1, ys, d, 1, m, m, d);
-  const int ty = t >> 4, tx = t & 15;
-#pragma unroll
-  for (int r = 0; r < RM; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = ty + 16 * r, col = tx + 16 * c;
-      if (j < m && col < d) Wg[((size_t)bh * m + j) * d + col] = acc[r][c];
-    }
-}
-
-// merge_w_simt for m landmarks (m <= 128)
-inline auto merge_w_simt_for(int m) {
-  return m <= 32 ? merge_w_simt<2> : (m <= 64 ? merge_w_simt<4> : merge_w_simt<8>);
+  for (int idx = t; idx < m * kMergeCols; idx += 256) {
+    const int j = idx / kMergeCols, c = idx % kMergeCols;
+    if (c >= nc) continue;
+    float acc = 0.f;
+    for (int k = 0; k < m; ++k) acc = fmaf(zs[j * m + k], ys[k * kMergeCols + c], acc);
+    Wg[((size_t)bh * m + j) * d + c0 + c] = acc;
+  }
 }
 
 // ---------------------------------------------------------------------------
