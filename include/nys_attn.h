@@ -199,12 +199,16 @@ NYS_ATTN_API nys_status nys_attn_layer_check_error(void *workspace_dev, const ny
  * backward), each Lemma 1 step's products in reverse, Z0's norms (the
  * gradient goes to the maximising column and row) and the segment means.
  * Arithmetic is fp32 on the CUDA cores; for NYS_BF16 the gradients are
- * rounded to bf16 (dQ twice: its F~ part, then the landmark part added).
+ * rounded to bf16 (dQ and dK twice: their first part, then the landmark
+ * part added).
  *   workspace_dev            at least nys_attn_backward_workspace_size
  *                            bytes, 256-byte aligned, or NULL (allocated and
  *                            freed stream-ordered).
- * Shapes, validation, errors and determinism as for nys_attn_forward.
- * Ragged batches (nys_attn_forward_lens) have no backward here. */
+ * Shapes, validation, errors and determinism as for nys_attn_forward.  The
+ * key-tile kernel runs beside the per-head kernel and waits, bounded, for
+ * its dY; a wait that gives up writes NYS_ERR_TIMEOUT to the first 4 bytes
+ * of the workspace (uint32, cleared by every call).  Ragged batches
+ * (nys_attn_forward_lens) have no backward here. */
 NYS_ATTN_API nys_status nys_attn_backward_workspace_size(const nys_desc *desc, int num_landmarks,
                                                          int pinv_iters, int conv_k,
                                                          size_t *bytes);

@@ -26,16 +26,19 @@
 //              of dW, dK~ and dw
 //   bwd_head   per head: dW, dY, dZ, the Lemma 1 steps backwards, dA, dQ~_A,
 //              dK~ (total), D = rowsum(dY * Y)
-//   bwd_keys   per 64-key tile: B, dB, dS_B; dK, dV (with the conv part);
-//              block partials of dQ~
+//   bwd_keys   per 64-key tile: B, dB, dS_B; dK (without its dK~ part), dV
+//              (with the conv part); block partials of dQ~.  It starts
+//              while bwd_head runs (programmatic launch) and waits only for
+//              the head's dY and D flag
 //   bwd_dqt_total  dQ~ = dQ~_A + the key blocks' partials, in order
-//   bwd_dq     dQ += dQ~_{seg(i)} / count
+//   bwd_dqk    dQ += dQ~_{seg(i)} / count, dK += dK~_{seg(i)} / count
 //   bwd_dconv  dw summed over the batch and the row blocks, in order
 // Every sum runs in a fixed order: results are bitwise reproducible.
 #pragma once
 
 #include "common.cuh"
 #include "simt.cuh"
+#include "sm100.cuh"
 
 namespace nys {
 namespace bwd {
@@ -290,6 +293,7 @@ struct HeadParams {
   float *dy, *dqt_a, *dkt;           // [BH][m][d]
   float *dd;                         // [BH][m]: rowsum(dY * Y)
   float *scratch;                    // [BH][head_bytes] when the matrices do not fit smem
+  uint32_t *ready;                   // [BH]: set once dY and D of the head are stored
   int d, m, iters, R, use_smem;
   float scale;
 };
@@ -335,6 +339,45 @@ __device__ __forceinline__ float sum_parts(const float *x, size_t stride, int R)
   return s;
 }
 
+// out[e] = sum_{r < R} x[r * md + e] (+ add[e]) for the elements
+// e = t, t + kHeadThreads, ... < md of a bwd_head thread, each added in order
+// of r; 16 loads in flight per step.
+template <typename Store>
+__device__ __forceinline__ void head_sum_parts(const float *x, int md, int R, Store store) {
+  constexpr int kE = 8;
+  for (int e0 = threadIdx.x; e0 < md; e0 += kE * kHeadThreads) {
+    float acc[kE];
+#pragma unroll
+    for (int i = 0; i < kE; ++i) acc[i] = 0.f;
+    int r = 0;
+    for (; r + 2 <= R; r += 2) {
+      float v0[kE], v1[kE];
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        const int e = e0 + i * kHeadThreads;
+        v0[i] = e < md ? x[(size_t)r * md + e] : 0.f;
+        v1[i] = e < md ? x[(size_t)(r + 1) * md + e] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        acc[i] += v0[i];
+        acc[i] += v1[i];
+      }
+    }
+    for (; r < R; ++r)
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        const int e = e0 + i * kHeadThreads;
+        acc[i] += e < md ? x[(size_t)r * md + e] : 0.f;
+      }
+#pragma unroll
+    for (int i = 0; i < kE; ++i) {
+      const int e = e0 + i * kHeadThreads;
+      if (e < md) store(e, acc[i]);
+    }
+  }
+}
+
 // Row stride of bwd_head<M>'s matrices: m columns or the d <= 64 columns of
 // the m x d ones, plus four (16-byte rows, 4 mod 32 words).
 template <int M>
@@ -368,12 +411,9 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
   __syncthreads();
   // X: dW (m x d) then scratch; Y2: Y (m x d)
   const size_t hd = (size_t)bh * m * d;
-  for (int e = t; e < m * d; e += kHeadThreads) {
-    const int i = e / d, c = e % d;
-    const float sw = sum_parts(p.dw_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
-    X[i * ld + c] = sw;
-    Y2[i * ld + c] = p.y[hd + e];
-  }
+  head_sum_parts(p.dw_part + (size_t)bh * p.R * m * d, m * d, p.R,
+                 [&](int e, float v) { X[(e / d) * ld + e % d] = v; });
+  for (int e = t; e < m * d; e += kHeadThreads) Y2[(e / d) * ld + e % d] = p.y[hd + e];
   for (int e = t; e < m * m; e += kHeadThreads) {
     const int i = e / m, j = e % m;
     A[i * ld + j] = p.a[(size_t)bh * m * m + e];
@@ -394,6 +434,10 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
     p.dd[(size_t)bh * m + t] = s;
   }
   __syncthreads();
+  // dY and D are all bwd_keys reads of this kernel's results: publish them,
+  // and let bwd_keys start on the SMs this kernel leaves free
+  if (t == 0) sm100::flag_release(p.ready + bh, 1u);
+  sm100::griddep_launch_dependents();
   // Lemma 1 steps backwards: Z' = 1/4 Z T3, T3 = 13I - P T2, T2 = 15I - P T1,
   // T1 = 7I - P, P = A Z
   for (int j = p.iters - 1; j >= 0; --j) {
@@ -500,19 +544,18 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
   mm_block<RR, 4, false, true>(T3, ld, dP, ld, T2, ld, m4, m, d, p.scale, 0.f);
   for (int e = t; e < m * d; e += kHeadThreads) p.dqt_a[hd + e] = T3[(e / d) * ld + e % d];
   mm_block<RR, 4, true, true>(X, ld, dP, ld, T1, ld, m4, m, d, p.scale, 0.f);
-  for (int e = t; e < m * d; e += kHeadThreads) {
-    const int i = e / d, c = e % d;
-    const float s = sum_parts(p.dkt_part + (size_t)bh * p.R * m * d + e, (size_t)m * d, p.R);
-    p.dkt[hd + e] = s + X[i * ld + c];
-  }
+  head_sum_parts(p.dkt_part + (size_t)bh * p.R * m * d, m * d, p.R,
+                 [&](int e, float v) { p.dkt[hd + e] = v + X[(e / d) * ld + e % d]; });
 }
 
 // ---------------------------------------------------------------------------
 struct KeysParams {
   const void *K, *V, *G;        // [BH][n][d] (T)
-  const float *qt, *dy, *dkt;   // [BH][m][d]
+  const float *qt, *dy;         // [BH][m][d]
   const float *lse2, *dd;       // [BH][m]: log2-sum-exp of B~'s scaled logits, rowsum(dY Y)
   const float *conv_w;          // [H][k] or null
+  const uint32_t *ready;        // [BH]: bwd_head's flag for dY and D
+  uint32_t *err;                // workspace error word
   void *dK, *dV;                // [BH][n][d] (T)
   float *dqt_part;              // [BH][S2][m][d]
   int n, d, m, heads, conv_k, S2;
@@ -554,13 +597,25 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
   const int n = p.n, d = p.d, m = p.m, head = bh % p.heads;
   const int d4 = round4(d), m4 = round4(m);
   const int k = p.conv_w ? p.conv_k : 0, half = (k - 1) / 2;
-  const int l = (n + m - 1) / m;
   const T *K = (const T *)p.K + (size_t)bh * n * d;
   const T *V = (const T *)p.V + (size_t)bh * n * d;
   const T *G = (const T *)p.G + (size_t)bh * n * d;
   T *dK = (T *)p.dK + (size_t)bh * n * d;
   T *dV = (T *)p.dV + (size_t)bh * n * d;
   const size_t hd = (size_t)bh * m * d;
+  // this kernel may start while bwd_head runs: wait (bounded) for the head's
+  // dY and D; on a timeout (recorded in the error word) the block leaves
+  __shared__ uint32_t abort_flag;
+  if (t == 0) {
+    abort_flag = 0u;
+    const sm100::Abort ab{&abort_flag, p.err};
+    sm100::flag_wait(p.ready + bh, ab, sm100::kWaitLimitCycles);
+  }
+  __syncthreads();
+  if (abort_flag) {
+    if (t == 0) sm100::griddep_wait();
+    return;
+  }
   for (int i = t; i < M * LD; i += kThreads) {
     const int j = i / LD, c = i % LD;
     const bool in = j < m && c < d;
@@ -630,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
         }
     }
     __syncthreads();
-    {   // dK = s dS_B^T Q~ + dK~_seg / count ; dV = B^T dY + conv^T(dO)
+    {   // dK = s dS_B^T Q~ (bwd_dqk adds dK~_seg / count) ; dV = B^T dY + conv^T(dO)
       float a[4][4], b[4][4];
       zero(a);
       zero(b);
@@ -642,10 +697,7 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
         for (int c = 0; c < 4; ++c) {
           const int col = vec_col<4, true>(c), row = k0 + vec_row<4>(r);
           if (row < n && col < d) {
-            const int j = seg_of(row, l);
-            const float gk =
-                p.scale * a[r][c] + __ldg(p.dkt + hd + j * d + col) / (float)seg_count(j, l, n);
-            dK[(size_t)row * d + col] = from_f<T>(gk);
+            dK[(size_t)row * d + col] = from_f<T>(p.scale * a[r][c]);
             dV[(size_t)row * d + col] = from_f<T>(b[r][c] + cv[r][c]);
           }
         }
@@ -661,6 +713,8 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
       const int j = vec_row<RM>(r), col = vec_col<4, true>(c);
       if (j < m && col < d) p.dqt_part[pb + (size_t)j * d + col] = p.scale * dq[r][c];
     }
+  // complete only after bwd_head, whose other results the next kernels read
+  if (t == 0) sm100::griddep_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -674,28 +728,34 @@ bwd_dqt_total(float *dqt, const float *dqt_part, int md, int S2) {
   dqt[(size_t)bh * md + e] += s;
 }
 
-// dQ += dQ~_{seg(i)} / count over the block's rows: the m x d quotients
-// once into shared memory, then thread t takes column t % 64 of every
-// fourth row (d <= 64).
+// dQ += dQ~_{seg(i)} / count and dK += dK~_{seg(i)} / count over the block's
+// rows: the m x d quotients once into shared memory, then thread t takes
+// column t % 64 of every fourth row (d <= 64).
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-bwd_dq(void *dQv, const float *dqt, int n, int d, int m, int rows_per_block) {
-  extern __shared__ float dq[];   // [m][d]
+bwd_dqk(void *dQv, void *dKv, const float *dqt, const float *dkt, int n, int d, int m,
+        int rows_per_block) {
+  extern __shared__ float quot[];   // [2][m][d]
+  float *dq = quot, *dk = quot + m * d;
   const int bh = blockIdx.y, t = threadIdx.x;
   const size_t hd = (size_t)bh * m * d;
   const int l = (n + m - 1) / m;
   for (int e = t; e < m * d; e += kThreads) {
-    const int j = e / d;
-    dq[e] = dqt[hd + e] / (float)seg_count(j, l, n);
+    const float cnt = (float)seg_count(e / d, l, n);
+    dq[e] = dqt[hd + e] / cnt;
+    dk[e] = dkt[hd + e] / cnt;
   }
   __syncthreads();
   T *dQ = (T *)dQv + (size_t)bh * n * d;
+  T *dK = (T *)dKv + (size_t)bh * n * d;
   const int r0 = blockIdx.x * rows_per_block, r1 = min(n, r0 + rows_per_block);
   const int c = t & 63;
   if (c >= d) return;
   for (int row = r0 + (t >> 6); row < r1; row += kThreads / 64) {
     const size_t o = (size_t)row * d + c;
-    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[seg_of(row, l) * d + c]);
+    const int q = seg_of(row, l) * d + c;
+    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[q]);
+    dK[o] = from_f<T>(to_f(dK[o]) + dk[q]);
   }
 }
 

@@ -260,7 +260,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
     dim3 grid(L.splits, BH);
     auto kern = bv_partial_simt_for<T>(m);
     if (!allow_smem(kern, sm) ||
-        launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, false, qt, K, V,
+        launch(kern, grid, dim3(256), launch_smem(mk.launched, sm), stream, true, qt, K, V,
                pmax, psum, py, n, d, m, L.splits, L.keys_per_split, scale_log2, lens,
                heads) != cudaSuccess)
       return NYS_ERR_CUDA;
@@ -477,7 +477,7 @@ nys_status launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const gemm:
 // Backward pass: workspace layout and launch sequence (bwd_simt.cuh).
 struct BwdLayout {
   size_t qt, kt, z, a, zall, pscr, pmax, psum, py, y, w, lse, dwp, dktp, dcp, dy, dqta, dkt,
-      dd, hscr, dqtp, err, total;
+      dd, hscr, dqtp, err, ready, total;
   int S, keys_per_split, R, S2, mb;
 };
 
@@ -493,11 +493,18 @@ BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
   // for m <= 64, one for m = 128), so that no SM runs a tail of its own
   L.mb = bwd_mbucket(m);
   const int t64 = (int)((n + bwd::kTile - 1) / bwd::kTile);
-  const int slots = kNumSms * (L.mb <= 64 ? 2 : 1);
-  int r = BH ? (int)(slots / BH) : 1;
+  const int per_sm = L.mb <= 64 ? 2 : 1;
+  int r = BH ? (int)(kNumSms * per_sm / BH) : 1;
   if (r > t64) r = t64;
   if (r < 1) r = 1;
-  L.R = L.S2 = r;
+  L.R = r;
+  // key blocks run beside bwd_head, one block per head on its own SM: one
+  // wave on the SMs it leaves
+  const int free_sms = BH < (size_t)kNumSms ? kNumSms - (int)BH : kNumSms;
+  int s2 = BH ? (int)(free_sms * per_sm / BH) : 1;
+  if (s2 > t64) s2 = t64;
+  if (s2 < 1) s2 = 1;
+  L.S2 = s2;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t at = off;
@@ -505,6 +512,10 @@ BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
     return at;
   };
   const size_t md = BH * m * d * 4, mm = BH * m * m * 4;
+  // the error word first (offset 0), then bwd_head's per-head flags; one
+  // memset per call clears both
+  L.err = take(256);
+  L.ready = take(BH * 4);
   L.qt = take(md);
   L.kt = take(md);
   L.z = take(mm);
@@ -526,7 +537,6 @@ BwdLayout make_bwd_layout(const nys_desc *desc, int m, int iters, int conv_k) {
   L.dd = take(BH * m * 4);
   L.hscr = take(L.mb > 64 ? BH * bwd::head_bytes<128>() : 0);
   L.dqtp = take(md * L.S2);
-  L.err = take(256);
   L.total = off;
   return L;
 }
@@ -568,7 +578,7 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
     const size_t sm = bv_partial_simt_smem(m);
     auto kern = bv_partial_simt_for<T>(m);
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(L.S, BH), dim3(256), sm, stream, false, (const float *)qt, K, V, pmax,
+        launch(kern, dim3(L.S, BH), dim3(256), sm, stream, true, (const float *)qt, K, V, pmax,
                psum, py, n, d, m, L.S, L.keys_per_split, scale_log2, (const int *)nullptr,
                H) != cudaSuccess)
       return NYS_ERR_CUDA;
@@ -598,7 +608,8 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
     const bwd::HeadParams p{(const float *)(ws + L.dwp), (const float *)(ws + L.dktp), qt, kt, y,
                             a, zall, (float *)(ws + L.dy), (float *)(ws + L.dqta),
                             (float *)(ws + L.dkt), (float *)(ws + L.dd),
-                            (float *)(ws + L.hscr), d, m, iters, L.R, MB <= 64 ? 1 : 0, scale};
+                            (float *)(ws + L.hscr), (uint32_t *)(ws + L.ready), d, m, iters,
+                            L.R, MB <= 64 ? 1 : 0, scale};
     auto kern = bwd::bwd_head<MB>;
     const size_t sm = MB <= 64 ? bwd::head_bytes<MB>() : 0;
     if (!allow_smem(kern, sm) ||
@@ -606,13 +617,16 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
       return NYS_ERR_CUDA;
   }
   {
-    const bwd::KeysParams p{K, V, dO, qt, (const float *)(ws + L.dy), (const float *)(ws + L.dkt),
-                            lse, (const float *)(ws + L.dd), conv_w, dK, dV,
+    // programmatic launch: the key tiles run beside bwd_head once every
+    // head has published dY and D
+    const bwd::KeysParams p{K, V, dO, qt, (const float *)(ws + L.dy), lse,
+                            (const float *)(ws + L.dd), conv_w,
+                            (const uint32_t *)(ws + L.ready), err, dK, dV,
                             (float *)(ws + L.dqtp), n, d, m, H, ck, L.S2, scale, scale_log2};
     auto kern = bwd::bwd_keys<T, MB>;
     const size_t sm = bwd::KeysSmem<MB>::total;
     if (!allow_smem(kern, sm) ||
-        launch(kern, dim3(L.S2, BH), dim3(bwd::kThreads), sm, stream, false, p) != cudaSuccess)
+        launch(kern, dim3(L.S2, BH), dim3(bwd::kThreads), sm, stream, true, p) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
   if (launch(bwd::bwd_dqt_total, dim3((m * d + bwd::kThreads - 1) / bwd::kThreads, BH),
@@ -621,11 +635,12 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
     return NYS_ERR_CUDA;
   {
     const int rpb = 256;
-    const size_t sm = (size_t)m * d * 4;
-    auto kern = bwd::bwd_dq<T>;
+    const size_t sm = (size_t)2 * m * d * 4;
+    auto kern = bwd::bwd_dqk<T>;
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3((n + rpb - 1) / rpb, BH), dim3(bwd::kThreads), sm, stream, false,
-               (void *)dQ, (const float *)(ws + L.dqta), n, d, m, rpb) != cudaSuccess)
+               (void *)dQ, (void *)dK, (const float *)(ws + L.dqta),
+               (const float *)(ws + L.dkt), n, d, m, rpb) != cudaSuccess)
       return NYS_ERR_CUDA;
   }
   if (ck > 0 &&
@@ -920,7 +935,9 @@ NYS_ATTN_API nys_status nys_attn_backward(const void *Q, const void *K, const vo
     if (cudaMallocAsync((void **)&ws, L.total, stream) != cudaSuccess) return NYS_ERR_CUDA;
     owned = true;
   }
-  if (cudaMemsetAsync(ws + L.err, 0, 256, stream) != cudaSuccess) st = NYS_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.err, 0, L.ready - L.err + (size_t)desc->batch * desc->heads * 4,
+                      stream) != cudaSuccess)
+    st = NYS_ERR_CUDA;
   if (st == NYS_OK) {
     const int mb = L.mb;
     if (desc->dtype == NYS_F32) {

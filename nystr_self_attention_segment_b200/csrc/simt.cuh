@@ -9,6 +9,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace nys {
 
@@ -227,6 +228,9 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
   __shared__ float nsum[2 * 16 * RM];   // column sums, then row sums
   const float *qt = Qt + (size_t)bh * m * d;
   const float *kt = Kt + (size_t)bh * m * d;
+  // the B~ V partials that follow read nothing of this kernel: they may run
+  // beside it (programmatic launch)
+  sm100::griddep_launch_dependents();
   for (int e = t; e < 5 * mm; e += blockDim.x) mats[e] = 0.f;
   __syncthreads();
   {   // logits, each a dot product over the features in order: thread
@@ -438,6 +442,9 @@ bv_partial_simt(const float *__restrict__ Qt, const T *__restrict__ K, const T *
       if (col < d) py[(base + j) * d + col] = y[r][c];
     }
   }
+  // launched beside pinv_simt: complete only after it, whose Z the merge
+  // reads
+  if (t == 0) sm100::griddep_wait();
 }
 
 // bv_partial_simt for m landmarks (m <= 128)

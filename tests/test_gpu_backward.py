@@ -5,7 +5,8 @@ Normwise error per head and per gradient, max|gpu - oracle| / max|oracle|:
 the gradients are computed in fp32 on the CUDA cores from the same rounded
 inputs, so the fp32 path is held to 1e-3 (the six Lemma 1 steps are
 differentiated in fp32: their products amplify rounding by the conditioning
-of A) and the bf16 path to 2e-2 (bf16 rounding of the gradients, dQ twice)."""
+of A) and the bf16 path to 2e-2 (bf16 rounding of the gradients, dQ and dK
+twice)."""
 import numpy as np
 import pytest
 
