@@ -71,6 +71,28 @@ __device__ __forceinline__ void store(const float (&acc)[RM][RN], float *C, int 
     }
 }
 
+// dst[r * LD + c] = X[row0 + r][c] as fp32 for r < rows, c < LD: zero for
+// rows outside [0, n) and columns past d.  Eight loads in flight per thread.
+template <int LD, typename T>
+__device__ __forceinline__ void load_tile(float *dst, const T *X, int row0, int rows, int n,
+                                          int d) {
+  constexpr int kU = 8;
+  const int total = rows * LD;
+  for (int i0 = threadIdx.x; i0 < total; i0 += kU * kThreads) {
+    float v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * kThreads, r = i / LD, c = i % LD, row = row0 + r;
+      v[u] = (i < total && row >= 0 && row < n && c < d) ? to_f(X[(size_t)row * d + c]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = i0 + u * kThreads;
+      if (i < total) dst[i] = v[u];
+    }
+  }
+}
+
 // segment of token i, and its token count, for l = ceil(L / m)
 __device__ __forceinline__ int seg_of(int i, int l) { return i / l; }
 __device__ __forceinline__ int seg_count(int j, int l, int L) { return min(l, L - j * l); }
@@ -378,6 +400,28 @@ __device__ __forceinline__ void head_sum_parts(const float *x, int md, int R, St
   }
 }
 
+// dst[(e / cols) * ld + e % cols] = src[e] for e < rows * cols (a row-major
+// matrix into the padded layout), by a bwd_head thread; eight loads in
+// flight.
+__device__ __forceinline__ void head_copy(float *dst, int ld, const float *src, int rows,
+                                          int cols) {
+  constexpr int kU = 8;
+  const int total = rows * cols;
+  for (int e0 = threadIdx.x; e0 < total; e0 += kU * kHeadThreads) {
+    float v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int e = e0 + u * kHeadThreads;
+      v[u] = e < total ? src[e] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int e = e0 + u * kHeadThreads;
+      if (e < total) dst[(e / cols) * ld + e % cols] = v[u];
+    }
+  }
+}
+
 // Row stride of bwd_head<M>'s matrices: m columns or the d <= 64 columns of
 // the m x d ones, plus four (16-byte rows, 4 mod 32 words).
 template <int M>
@@ -413,13 +457,9 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
   const size_t hd = (size_t)bh * m * d;
   head_sum_parts(p.dw_part + (size_t)bh * p.R * m * d, m * d, p.R,
                  [&](int e, float v) { X[(e / d) * ld + e % d] = v; });
-  for (int e = t; e < m * d; e += kHeadThreads) Y2[(e / d) * ld + e % d] = p.y[hd + e];
-  for (int e = t; e < m * m; e += kHeadThreads) {
-    const int i = e / m, j = e % m;
-    A[i * ld + j] = p.a[(size_t)bh * m * m + e];
-    Zj[i * ld + j] = p.zs[((size_t)bh * (p.iters + 1) + p.iters) * m * m + e];
-    dA[i * ld + j] = 0.f;
-  }
+  head_copy(Y2, ld, p.y + hd, m, d);
+  head_copy(A, ld, p.a + (size_t)bh * m * m, m, m);
+  head_copy(Zj, ld, p.zs + ((size_t)bh * (p.iters + 1) + p.iters) * m * m, m, m);
   __syncthreads();
   // dZ = dW Y^T (m x m), dY = Z^T dW (m x d)
   mm_block<RR, RM, false, false>(dZ, ld, X, ld, Y2, ld, d4, m, m, 1.f, 0.f);
@@ -441,8 +481,7 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
   // Lemma 1 steps backwards: Z' = 1/4 Z T3, T3 = 13I - P T2, T2 = 15I - P T1,
   // T1 = 7I - P, P = A Z
   for (int j = p.iters - 1; j >= 0; --j) {
-    for (int e = t; e < m * m; e += kHeadThreads)
-      Zj[(e / m) * ld + e % m] = p.zs[((size_t)bh * (p.iters + 1) + j) * m * m + e];
+    head_copy(Zj, ld, p.zs + ((size_t)bh * (p.iters + 1) + j) * m * m, m, m);
     __syncthreads();
     mm_block<RR, RM, false, true>(P, ld, A, ld, Zj, ld, m4, m, m, 1.f, 0.f);            // P = A Z
     for (int e = t; e < m * m; e += kHeadThreads) {
@@ -534,11 +573,8 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
     for (int j = 0; j < m; ++j) dP[t * ld + j] = A[t * ld + j] * (dA[t * ld + j] - dot);
   }
   // Q~, K~ into T1, T2 (m x d)
-  for (int e = t; e < m * d; e += kHeadThreads) {
-    const int i = e / d, c = e % d;
-    T1[i * ld + c] = p.qt[hd + e];
-    T2[i * ld + c] = p.kt[hd + e];
-  }
+  head_copy(T1, ld, p.qt + hd, m, d);
+  head_copy(T2, ld, p.kt + hd, m, d);
   __syncthreads();
   // dQ~_A = s dS_A K~ ; dK~ = (F part) + s dS_A^T Q~
   mm_block<RR, 4, false, true>(T3, ld, dP, ld, T2, ld, m4, m, d, p.scale, 0.f);
@@ -634,17 +670,10 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_keys(const Keys
   for (int tile = tb; tile < te; ++tile) {
     const int k0 = tile * kTile;
     __syncthreads();
-    for (int i = t; i < kTile * LD; i += kThreads) {
-      const int r = i / LD, c = i % LD, row = k0 + r;
-      const bool in = row < n && c < d;
-      ks[i] = in ? to_f(K[(size_t)row * d + c]) : 0.f;
-      vs[i] = in ? to_f(V[(size_t)row * d + c]) : 0.f;
-    }
+    load_tile<LD>(ks, K, k0, kTile, n, d);
+    load_tile<LD>(vs, V, k0, kTile, n, d);
     if (k > 0)   // dO rows k0 + half - (k - 1) .. k0 + 63 + half: conv^T
-      for (int i = t; i < (kTile + k - 1) * LD; i += kThreads) {
-        const int r = i / LD, c = i % LD, row = k0 + half - (k - 1) + r;
-        gh[i] = (row >= 0 && row < n && c < d) ? to_f(G[(size_t)row * d + c]) : 0.f;
-      }
+      load_tile<LD>(gh, G, k0 + half - (k - 1), kTile + k - 1, n, d);
     __syncthreads();
     // conv^T(dO) for the tile's dV outputs (key vec_row<4>(r), column
     // vec_col<4, true>(c)): dV_row += w[tp] dO[row - tp + half]
@@ -740,10 +769,23 @@ bwd_dqk(void *dQv, void *dKv, const float *dqt, const float *dkt, int n, int d, 
   const int bh = blockIdx.y, t = threadIdx.x;
   const size_t hd = (size_t)bh * m * d;
   const int l = (n + m - 1) / m;
-  for (int e = t; e < m * d; e += kThreads) {
-    const float cnt = (float)seg_count(e / d, l, n);
-    dq[e] = dqt[hd + e] / cnt;
-    dk[e] = dkt[hd + e] / cnt;
+  for (int e0 = t; e0 < m * d; e0 += 4 * kThreads) {   // four elements' loads in flight
+    float vq[4], vk[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * kThreads;
+      vq[u] = e < m * d ? dqt[hd + e] : 0.f;
+      vk[u] = e < m * d ? dkt[hd + e] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * kThreads;
+      if (e < m * d) {
+        const float cnt = (float)seg_count(e / d, l, n);
+        dq[e] = vq[u] / cnt;
+        dk[e] = vk[u] / cnt;
+      }
+    }
   }
   __syncthreads();
   T *dQ = (T *)dQv + (size_t)bh * n * d;
@@ -751,11 +793,26 @@ bwd_dqk(void *dQv, void *dKv, const float *dqt, const float *dkt, int n, int d, 
   const int r0 = blockIdx.x * rows_per_block, r1 = min(n, r0 + rows_per_block);
   const int c = t & 63;
   if (c >= d) return;
-  for (int row = r0 + (t >> 6); row < r1; row += kThreads / 64) {
-    const size_t o = (size_t)row * d + c;
-    const int q = seg_of(row, l) * d + c;
-    dQ[o] = from_f<T>(to_f(dQ[o]) + dq[q]);
-    dK[o] = from_f<T>(to_f(dK[o]) + dk[q]);
+  constexpr int kStep = kThreads / 64, kU = 8;   // rows per pass; passes in flight
+  for (int row0 = r0 + (t >> 6); row0 < r1; row0 += kStep * kU) {
+    float gq[kU], gk[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int row = row0 + u * kStep;
+      const size_t o = (size_t)row * d + c;
+      gq[u] = row < r1 ? to_f(dQ[o]) : 0.f;
+      gk[u] = row < r1 ? to_f(dK[o]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int row = row0 + u * kStep;
+      if (row < r1) {
+        const size_t o = (size_t)row * d + c;
+        const int q = seg_of(row, l) * d + c;
+        dQ[o] = from_f<T>(gq[u] + dq[q]);
+        dK[o] = from_f<T>(gk[u] + dk[q]);
+      }
+    }
   }
 }
 

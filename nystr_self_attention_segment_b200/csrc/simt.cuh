@@ -465,7 +465,7 @@ constexpr int kMergeCols = 16;
 
 inline size_t merge_w_smem(int m, int d, int splits) {
   (void)d;
-  return ((size_t)m * kMergeCols + (size_t)m * m + (size_t)splits * m + m) * 4;
+  return ((size_t)m * kMergeCols + (size_t)m * m + 2 * (size_t)splits * m + m) * 4;
 }
 
 __global__ void __launch_bounds__(256)
@@ -477,17 +477,23 @@ merge_w_simt(const float *__restrict__ pmax, const float *__restrict__ psum,
   const int nc = min(kMergeCols, d - c0);
   float *ys = smem;                    // [m][kMergeCols]
   float *zs = ys + m * kMergeCols;     // [m][m]
-  float *fac = zs + m * m;             // [splits][m]: 2^(max_s - max)
-  float *tot = fac + splits * m;       // [m]: the row's merged sum
+  float *fac = zs + m * m;             // [splits][m]: the split maxima, then 2^(max_s - max)
+  float *sms = fac + splits * m;       // [splits][m]: the split sums
+  float *tot = sms + splits * m;       // [m]: the row's merged sum
   const size_t pb = (size_t)bh * splits * m;
+  for (int e = t; e < splits * m; e += 256) {
+    fac[e] = pmax[pb + e];
+    sms[e] = psum[pb + e];
+  }
+  __syncthreads();
   for (int j = t; j < m; j += 256) {
     float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, pmax[pb + (size_t)s * m + j]);
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, fac[s * m + j]);
     float sum = 0.f;
     for (int s = 0; s < splits; ++s) {
-      const float f = exp2f(pmax[pb + (size_t)s * m + j] - mx);
+      const float f = exp2f(fac[s * m + j] - mx);
       fac[s * m + j] = f;
-      sum = fmaf(psum[pb + (size_t)s * m + j], f, sum);
+      sum = fmaf(sms[s * m + j], f, sum);
     }
     tot[j] = sum;
     if (lse2 && blockIdx.y == 0) lse2[(size_t)bh * m + j] = mx + log2f(sum);   // backward pass
