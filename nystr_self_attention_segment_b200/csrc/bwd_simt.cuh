@@ -316,6 +316,7 @@ struct HeadParams {
   float *dd;                         // [BH][m]: rowsum(dY * Y)
   float *scratch;                    // [BH][head_bytes] when the matrices do not fit smem
   uint32_t *ready;                   // [BH]: set once dY and D of the head are stored
+  int publish;                       // 1: set `ready` (0 only in a test of the wait)
   int d, m, iters, R, use_smem;
   float scale;
 };
@@ -476,7 +477,7 @@ __global__ void __launch_bounds__(kHeadThreads) bwd_head(const HeadParams p) {
   __syncthreads();
   // dY and D are all bwd_keys reads of this kernel's results: publish them,
   // and let bwd_keys start on the SMs this kernel leaves free
-  if (t == 0) sm100::flag_release(p.ready + bh, 1u);
+  if (t == 0 && p.publish) sm100::flag_release(p.ready + bh, 1u);
   sm100::griddep_launch_dependents();
   // Lemma 1 steps backwards: Z' = 1/4 Z T3, T3 = 13I - P T2, T2 = 15I - P T1,
   // T1 = 7I - P, P = A Z

@@ -153,7 +153,20 @@ struct Marks {
 // index in the next forward call asks for more dynamic shared memory than a
 // block may have, so that the launch is refused and nothing of it runs.
 int g_fail_launch = -1;
+// Test builds only: while set, bwd_head never publishes its dY / D flag, so
+// that bwd_keys' bounded wait runs out.
+bool g_hold_head_flag = false;
 #endif
+
+// Whether bwd_head publishes its per-head flag (always, outside the test
+// build).
+int head_publishes() {
+#if defined(NYS_TEST_HOOKS) && NYS_TEST_HOOKS
+  return g_hold_head_flag ? 0 : 1;
+#else
+  return 1;
+#endif
+}
 
 // Dynamic shared memory of launch `idx` of a call (a test build may make one
 // launch impossible, see above).
@@ -608,8 +621,8 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
     const bwd::HeadParams p{(const float *)(ws + L.dwp), (const float *)(ws + L.dktp), qt, kt, y,
                             a, zall, (float *)(ws + L.dy), (float *)(ws + L.dqta),
                             (float *)(ws + L.dkt), (float *)(ws + L.dd),
-                            (float *)(ws + L.hscr), (uint32_t *)(ws + L.ready), d, m, iters,
-                            L.R, MB <= 64 ? 1 : 0, scale};
+                            (float *)(ws + L.hscr), (uint32_t *)(ws + L.ready),
+                            head_publishes(), d, m, iters, L.R, MB <= 64 ? 1 : 0, scale};
     auto kern = bwd::bwd_head<MB>;
     const size_t sm = MB <= 64 ? bwd::head_bytes<MB>() : 0;
     if (!allow_smem(kern, sm) ||
@@ -1215,8 +1228,15 @@ NYS_ATTN_API nys_status nys_attn_launch_names(const nys_desc *desc, int m, char 
 //                              cycles; the bounded wait gives up, records
 //                              NYS_ERR_TIMEOUT in the workspace error word and
 //                              the block returns.  No copy or MMA is in flight
-//                              when it gives up.
+//                              when it gives up;
+//  nys_test_hold_head_flag(on) while on, the backward's per-head kernel does
+//                              not publish dY / D, so every key block's
+//                              bounded flag wait (about 0.2 s) gives up and
+//                              records NYS_ERR_TIMEOUT in the backward
+//                              workspace's first word.
 NYS_ATTN_API void nys_test_fail_launch(int idx) { g_fail_launch = idx; }
+
+NYS_ATTN_API void nys_test_hold_head_flag(int on) { g_hold_head_flag = on != 0; }
 
 // nys_test_w_order(mode): 1 delays every pseudoinverse block, 2 every
 // Y-merging block, before it reports its W input (0: no delay), so that the

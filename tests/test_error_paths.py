@@ -1,5 +1,5 @@
 """Error paths of the C ABI on the GPU, through the test build of the library
-(libnys_attn_test.so: the same sources with two test-only entry points).
+(libnys_attn_test.so: the same sources with test-only entry points).
 
 - A launch that the runtime refuses (one launch of the call asks for more
   dynamic shared memory than a block may have) returns NYS_ERR_CUDA at once:
@@ -8,9 +8,13 @@
 - A bounded device wait that runs out (an mbarrier nothing completes, with a
   short limit, no copy or MMA in flight) records NYS_ERR_TIMEOUT in the
   workspace error word; nys_attn_check_error reports it once and clears it.
+- The backward's key blocks wait (bounded) on a flag of the per-head kernel;
+  with the flag held back the wait gives up, NYS_ERR_TIMEOUT lands in the
+  backward workspace's first word, and the next call recovers.
 
 Nothing here faults or hangs the GPU: the refused launch never starts, and
-the wait gives up after about a millisecond."""
+the waits give up after about a millisecond (the probe) or 0.2 s (the key
+blocks)."""
 import ctypes
 
 import numpy as np
@@ -48,7 +52,7 @@ def _test_lib():
 def test_hooks_exist_only_in_the_test_build():
     lib = _test_lib()
     prod = nys.load()
-    for name in ("nys_test_fail_launch", "nys_test_timeout_probe"):
+    for name in ("nys_test_fail_launch", "nys_test_timeout_probe", "nys_test_hold_head_flag"):
         assert hasattr(lib, name)
         assert not hasattr(prod, name)
 
@@ -158,3 +162,60 @@ def test_w_is_the_same_whichever_block_forms_it(name):
         lib.nys_test_w_order(0)
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
     assert np.array_equal(outs[2], want)
+
+
+@pytest.mark.gpu
+def test_backward_key_wait_that_runs_out_reports_timeout_and_next_call_recovers():
+    # The backward's key-tile kernel starts beside the per-head kernel and
+    # waits (bounded, about 0.2 s) for the head's dY / D flag.  The test build
+    # can hold that flag back: every key block's wait then gives up, records
+    # NYS_ERR_TIMEOUT in the workspace's first word and leaves.  The next call
+    # (flag published again) must clear the word and give the same gradients
+    # as before, bit for bit.
+    t = torch()
+    lib = _test_lib()
+    lib.nys_test_hold_head_flag.restype = None
+    lib.nys_test_hold_head_flag.argtypes = [ctypes.c_int]
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    D = ctypes.POINTER(_lib.nys_desc)
+    lib.nys_attn_backward_workspace_size.restype = I
+    lib.nys_attn_backward_workspace_size.argtypes = [D, I, I, I, ctypes.POINTER(S)]
+    lib.nys_attn_backward.restype = I
+    lib.nys_attn_backward.argtypes = [P, P, P, D, I, I, P, I, P, P, P, P, P, P, S, P]
+    shape, m, ck = (1, 2, 512, 64), 64, 33
+    x = make_custom(shape, BF16, seed=5, conv_k=ck)
+    _, _, (Q, K, V, cw) = run(x, BF16, m)
+    G = t.randn(shape, device="cuda", generator=t.Generator(device="cuda").manual_seed(5))
+    G = G.to(t.bfloat16)
+    desc = _lib.make_desc(_lib.NYS_BF16, *shape)
+    wsb = ctypes.c_size_t(0)
+    assert lib.nys_attn_backward_workspace_size(ctypes.byref(desc), m, 6, ck,
+                                                ctypes.byref(wsb)) == 0
+    buf = t.zeros(wsb.value + 256, dtype=t.uint8, device="cuda")
+    off = (-buf.data_ptr()) % 256
+    ws = buf.data_ptr() + off
+
+    def backward():
+        dQ, dK, dV = t.empty_like(Q), t.empty_like(Q), t.empty_like(Q)
+        dcw = t.empty_like(cw)
+        st = lib.nys_attn_backward(Q.data_ptr(), K.data_ptr(), V.data_ptr(), ctypes.byref(desc),
+                                   m, 6, cw.data_ptr(), ck, G.data_ptr(), dQ.data_ptr(),
+                                   dK.data_ptr(), dV.data_ptr(), dcw.data_ptr(),
+                                   ctypes.c_void_p(ws), ctypes.c_size_t(wsb.value), _stream())
+        t.cuda.synchronize()
+        word = int(buf[off:off + 4].cpu().numpy().view(np.uint32)[0])
+        return st, word, (dQ, dK, dV, dcw)
+
+    st, word, want = backward()
+    assert st == 0 and word == 0
+    try:
+        lib.nys_test_hold_head_flag(1)
+        st, word, _ = backward()
+    finally:
+        lib.nys_test_hold_head_flag(0)
+    assert st == 0
+    assert _lib.STATUS_NAMES[word] == "NYS_ERR_TIMEOUT"
+    st, word, got = backward()
+    assert st == 0 and word == 0
+    for a, b in zip(got, want):
+        assert t.equal(a, b)
