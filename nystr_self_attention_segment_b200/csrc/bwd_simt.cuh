@@ -72,10 +72,36 @@ __device__ __forceinline__ void store(const float (&acc)[RM][RN], float *C, int 
 }
 
 // dst[r * LD + c] = X[row0 + r][c] as fp32 for r < rows, c < LD: zero for
-// rows outside [0, n) and columns past d.  Eight loads in flight per thread.
+// rows outside [0, n) and columns past d.  bf16 rows of a multiple of 8
+// features (16-byte aligned: the inputs are) move as 16-byte loads of eight
+// values; otherwise eight scalar loads in flight per thread.
 template <int LD, typename T>
 __device__ __forceinline__ void load_tile(float *dst, const T *X, int row0, int rows, int n,
                                           int d) {
+  if constexpr (sizeof(T) == 2) {
+    if ((d & 7) == 0) {
+      const int cpr = d >> 3, total = rows * cpr;   // 16-byte chunks per row, in all
+      for (int u = threadIdx.x; u < total; u += kThreads) {
+        const int r = u / cpr, c8 = (u - r * cpr) * 8, row = row0 + r;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row >= 0 && row < n) v = *reinterpret_cast<const uint4 *>(X + (size_t)row * d + c8);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+        float4 lo, hi;
+        float2 f;
+        f = __bfloat1622float2(h[0]); lo.x = f.x; lo.y = f.y;
+        f = __bfloat1622float2(h[1]); lo.z = f.x; lo.w = f.y;
+        f = __bfloat1622float2(h[2]); hi.x = f.x; hi.y = f.y;
+        f = __bfloat1622float2(h[3]); hi.z = f.x; hi.w = f.y;
+        *reinterpret_cast<float4 *>(dst + r * LD + c8) = lo;
+        *reinterpret_cast<float4 *>(dst + r * LD + c8 + 4) = hi;
+      }
+      for (int u = threadIdx.x; u < rows * (LD - d); u += kThreads) {   // the padding
+        const int r = u / (LD - d);
+        dst[r * LD + d + (u - r * (LD - d))] = 0.f;
+      }
+      return;
+    }
+  }
   constexpr int kU = 8;
   const int total = rows * LD;
   for (int i0 = threadIdx.x; i0 < total; i0 += kU * kThreads) {
@@ -173,17 +199,23 @@ __global__ void __launch_bounds__(kThreads, M <= 64 ? 2 : 1) bwd_rows(const Rows
   for (int tile = tb; tile < te; ++tile) {
     const int r0 = tile * kTile;
     __syncthreads();
-    for (int i = t; i < kTile * LD; i += kThreads) {
-      const int r = i / LD, c = i % LD, row = r0 + r;
-      const bool in = row < n && c < d;
-      qs[i] = in ? to_f(Q[(size_t)row * d + c]) : 0.f;
-      gs[i] = in ? to_f(G[(size_t)row * d + c]) : 0.f;
-    }
-    if (k > 0)
-      for (int i = t; i < (kTile + k - 1) * LD; i += kThreads) {
-        const int r = i / LD, c = i % LD, row = r0 - half + r;
-        vh[i] = (row >= 0 && row < n && c < d) ? to_f(V[(size_t)row * d + c]) : 0.f;
+    if (sizeof(T) == 2 && (d & 7) == 0) {
+      load_tile<LD>(qs, Q, r0, kTile, n, d);
+      load_tile<LD>(gs, G, r0, kTile, n, d);
+      if (k > 0) load_tile<LD>(vh, V, r0 - half, kTile + k - 1, n, d);
+    } else {
+      for (int i = t; i < kTile * LD; i += kThreads) {
+        const int r = i / LD, c = i % LD, row = r0 + r;
+        const bool in = row < n && c < d;
+        qs[i] = in ? to_f(Q[(size_t)row * d + c]) : 0.f;
+        gs[i] = in ? to_f(G[(size_t)row * d + c]) : 0.f;
       }
+      if (k > 0)
+        for (int i = t; i < (kTile + k - 1) * LD; i += kThreads) {
+          const int r = i / LD, c = i % LD, row = r0 - half + r;
+          vh[i] = (row >= 0 && row < n && c < d) ? to_f(V[(size_t)row * d + c]) : 0.f;
+        }
+    }
     __syncthreads();
     // conv kernel gradient: tap j gets sum_i sum_c dO_i,c V_{i+j-half},c
     // (halo row i + j).  A thread takes one column c and kTapGroup taps
