@@ -71,54 +71,6 @@ __device__ __forceinline__ void store(const float (&acc)[RM][RN], float *C, int 
     }
 }
 
-// dst[r * LD + c] = X[row0 + r][c] as fp32 for r < rows, c < LD: zero for
-// rows outside [0, n) and columns past d.  bf16 rows of a multiple of 8
-// features (16-byte aligned: the inputs are) move as 16-byte loads of eight
-// values; otherwise eight scalar loads in flight per thread.
-template <int LD, typename T>
-__device__ __forceinline__ void load_tile(float *dst, const T *X, int row0, int rows, int n,
-                                          int d) {
-  if constexpr (sizeof(T) == 2) {
-    if ((d & 7) == 0) {
-      const int cpr = d >> 3, total = rows * cpr;   // 16-byte chunks per row, in all
-      for (int u = threadIdx.x; u < total; u += kThreads) {
-        const int r = u / cpr, c8 = (u - r * cpr) * 8, row = row0 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row >= 0 && row < n) v = *reinterpret_cast<const uint4 *>(X + (size_t)row * d + c8);
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
-        float4 lo, hi;
-        float2 f;
-        f = __bfloat1622float2(h[0]); lo.x = f.x; lo.y = f.y;
-        f = __bfloat1622float2(h[1]); lo.z = f.x; lo.w = f.y;
-        f = __bfloat1622float2(h[2]); hi.x = f.x; hi.y = f.y;
-        f = __bfloat1622float2(h[3]); hi.z = f.x; hi.w = f.y;
-        *reinterpret_cast<float4 *>(dst + r * LD + c8) = lo;
-        *reinterpret_cast<float4 *>(dst + r * LD + c8 + 4) = hi;
-      }
-      for (int u = threadIdx.x; u < rows * (LD - d); u += kThreads) {   // the padding
-        const int r = u / (LD - d);
-        dst[r * LD + d + (u - r * (LD - d))] = 0.f;
-      }
-      return;
-    }
-  }
-  constexpr int kU = 8;
-  const int total = rows * LD;
-  for (int i0 = threadIdx.x; i0 < total; i0 += kU * kThreads) {
-    float v[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = i0 + u * kThreads, r = i / LD, c = i % LD, row = row0 + r;
-      v[u] = (i < total && row >= 0 && row < n && c < d) ? to_f(X[(size_t)row * d + c]) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = i0 + u * kThreads;
-      if (i < total) dst[i] = v[u];
-    }
-  }
-}
-
 // segment of token i, and its token count, for l = ceil(L / m)
 __device__ __forceinline__ int seg_of(int i, int l) { return i / l; }
 __device__ __forceinline__ int seg_count(int j, int l, int L) { return min(l, L - j * l); }
