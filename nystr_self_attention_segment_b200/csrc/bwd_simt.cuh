@@ -776,6 +776,41 @@ bwd_dqk(void *dQv, void *dKv, const float *dqt, const float *dkt, int n, int d, 
   T *dQ = (T *)dQv + (size_t)bh * n * d;
   T *dK = (T *)dKv + (size_t)bh * n * d;
   const int r0 = blockIdx.x * rows_per_block, r1 = min(n, r0 + rows_per_block);
+  if constexpr (sizeof(T) == 2) {
+    if ((d & 7) == 0) {   // bf16 rows of 16-byte chunks: eight values per load
+      const int cpr = d >> 3;
+      constexpr int kU = 4;
+      for (int u0 = t; u0 < (r1 - r0) * cpr; u0 += kU * kThreads) {
+        uint4 vq[kU], vk[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = u0 + u * kThreads, row = r0 + i / cpr, c8 = (i % cpr) * 8;
+          vq[u] = vk[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (row < r1) {
+            vq[u] = *reinterpret_cast<const uint4 *>(dQ + (size_t)row * d + c8);
+            vk[u] = *reinterpret_cast<const uint4 *>(dK + (size_t)row * d + c8);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i = u0 + u * kThreads, row = r0 + i / cpr, c8 = (i % cpr) * 8;
+          if (row >= r1) continue;
+          const int q = seg_of(row, l) * d + c8;
+          __nv_bfloat162 *hq = reinterpret_cast<__nv_bfloat162 *>(&vq[u]);
+          __nv_bfloat162 *hk = reinterpret_cast<__nv_bfloat162 *>(&vk[u]);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 a = __bfloat1622float2(hq[h]), b = __bfloat1622float2(hk[h]);
+            hq[h] = __floats2bfloat162_rn(a.x + dq[q + 2 * h], a.y + dq[q + 2 * h + 1]);
+            hk[h] = __floats2bfloat162_rn(b.x + dk[q + 2 * h], b.y + dk[q + 2 * h + 1]);
+          }
+          *reinterpret_cast<uint4 *>(dQ + (size_t)row * d + c8) = vq[u];
+          *reinterpret_cast<uint4 *>(dK + (size_t)row * d + c8) = vk[u];
+        }
+      }
+      return;
+    }
+  }
   const int c = t & 63;
   if (c >= d) return;
   constexpr int kStep = kThreads / 64, kU = 8;   // rows per pass; passes in flight

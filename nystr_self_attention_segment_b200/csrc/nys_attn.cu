@@ -570,7 +570,16 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
   const int ck = conv_w ? conv_k : 0;
   // the forward's landmark steps, keeping A, every Z iterate and B~'s
   // log-sum-exp
-  {
+  if constexpr (sizeof(T) == 2) {
+    if (d == 64) {   // the bf16 path's streaming segment means
+      const segm::Shape sh{n, m, H, nullptr};
+      if (launch(segm::seg_means_bf16, dim3(m, BH, 2), dim3(segm::threads_for(n, m)), 0, stream,
+                 false, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, qt, kt, sh,
+                 err) != cudaSuccess)
+        return NYS_ERR_CUDA;
+    }
+  }
+  if (sizeof(T) != 2 || d != 64) {
     long total = (long)BH * m * d;
     if (launch(seg_means_scalar<T>, dim3((unsigned)((total + 255) / 256), 2), dim3(256), 0,
                stream, false, Q, K, qt, kt, BH, n, d, m, (const int *)nullptr, H,
