@@ -259,7 +259,7 @@ nys_status launch_simt(const T *Q, const T *K, const T *V, const nys_desc *desc,
   }
   {
     const int use_smem = m <= 64;
-    size_t sm = use_smem ? pinv_simt_mats_bytes(m) : 0;
+    size_t sm = pinv_simt_smem(m);
     auto kern = pinv_simt_for(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH), dim3(256), launch_smem(mk.launched, sm), stream, false, qt,
@@ -588,7 +588,7 @@ nys_status launch_bwd(const T *Q, const T *K, const T *V, const nys_desc *desc, 
   }
   {
     const int use_smem = m <= 64;
-    const size_t sm = use_smem ? pinv_simt_mats_bytes(m) : 0;
+    const size_t sm = pinv_simt_smem(m);
     auto kern = pinv_simt_for(m);
     if (!allow_smem(kern, sm) ||
         launch(kern, dim3(BH), dim3(256), sm, stream, false, (const float *)qt,

@@ -271,8 +271,11 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
   constexpr int ld = pinv_ld<RM>();
   const int bh = blockIdx.x, t = threadIdx.x;
   constexpr int mm = 16 * RM * ld;
+  // all five in shared memory, or (m > 64) A and Z in the scratch and the
+  // three the products write in shared memory
   float *mats = use_smem ? smem : scratch + (size_t)bh * (pinv_mats_bytes<RM>() / 4);
-  float *A = mats, *Z = A + mm, *P = Z + mm, *T1 = P + mm, *T2 = T1 + mm;
+  float *A = mats, *Z = A + mm;
+  float *P = use_smem ? Z + mm : smem, *T1 = P + mm, *T2 = T1 + mm;
   __shared__ float red[2];
   __shared__ float nsum[2 * 16 * RM];   // column sums, then row sums
   const float *qt = Qt + (size_t)bh * m * d;
@@ -280,7 +283,8 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
   // the B~ V partials that follow read nothing of this kernel: they may run
   // beside it (programmatic launch)
   sm100::griddep_launch_dependents();
-  for (int e = t; e < 5 * mm; e += blockDim.x) mats[e] = 0.f;
+  for (int e = t; e < 2 * mm; e += blockDim.x) A[e] = 0.f;   // A, Z
+  for (int e = t; e < 3 * mm; e += blockDim.x) P[e] = 0.f;   // P, T1, T2
   __syncthreads();
   {   // logits, each a dot product over the features in order: thread
       // (ty, tx) = (t / 16, t % 16) takes rows ty + 16 r, columns tx + 16 c
@@ -379,6 +383,11 @@ pinv_simt(const float *__restrict__ Qt, const float *__restrict__ Kt, float *__r
 // pinv_simt for m landmarks (m <= 128), and the bytes of its matrices
 inline auto pinv_simt_for(int m) {
   return m <= 32 ? pinv_simt<2> : (m <= 64 ? pinv_simt<4> : pinv_simt<8>);
+}
+// dynamic shared memory of pinv_simt for m landmarks: all five matrices for
+// m <= 64, else the three the products write
+inline size_t pinv_simt_smem(int m) {
+  return m <= 32 ? pinv_mats_bytes<2>() : (m <= 64 ? pinv_mats_bytes<4>() : pinv_mats_bytes<8>() / 5 * 3);
 }
 inline size_t pinv_simt_mats_bytes(int m) {
   return m <= 32 ? pinv_mats_bytes<2>() : (m <= 64 ? pinv_mats_bytes<4>() : pinv_mats_bytes<8>());
